@@ -1,0 +1,475 @@
+"""Pins for the fp64 oracle: each test ties a part of the oracle to something
+other than itself -- values the pages print, closed forms, special cases that
+reduce to a textbook or library result, invariants, or brute force on tiny
+inputs. Chosen so a dropped term, a wrong sign or index, or a transposed
+operand in the oracle fails at least one of them.
+"""
+
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+from oracle import moe_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def rng(seed=0):
+    return np.random.default_rng(seed)
+
+
+def rand_expert(r, H, I, scale=0.3):
+    return (r.normal(0, scale, (I, H)), r.normal(0, scale, (I, H)), r.normal(0, scale, (I, H)))
+
+
+# ---------------------------------------------------------------- bf16 / int4
+
+
+def test_bf16_round_matches_library_for_fp32_inputs():
+    # For values exactly representable in fp32, nearest-even rounding to bf16
+    # must equal torch's fp32 -> bf16 conversion (a library routine).
+    torch = pytest.importorskip("torch")
+    r = rng(1)
+    x = np.concatenate([r.normal(0, 1, 4000), r.normal(0, 1e-3, 1000), r.normal(0, 300, 1000)])
+    x = x.astype(np.float32)
+    # include exact halfway cases: 1 + 2^-8 (ties to 1), 1 + 3*2^-8 (ties up to 1 + 2^-6)
+    x = np.concatenate([x, np.array([1 + 2 ** -8, 1 + 3 * 2 ** -8, -(1 + 2 ** -8), 2.0 ** -126 * 1.5],
+                                    dtype=np.float32)])
+    ours = O.f64_to_bf16_bits_rne(x.astype(np.float64))
+    ref = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().astype(np.uint16)
+    assert np.array_equal(ours, ref)
+    assert O.bf16_round(np.array([1 + 2 ** -8]))[0] == 1.0
+    assert O.bf16_round(np.array([1 + 3 * 2 ** -8]))[0] == 1 + 2 ** -6
+
+
+def test_bf16_decode_known_patterns():
+    bits = np.array([0x3F80, 0xBF80, 0x4000, 0x0000, 0x3F81, 0x4300], dtype=np.uint16)
+    vals = O.bf16_bits_to_f64(bits)
+    assert vals.tolist() == [1.0, -1.0, 2.0, 0.0, 1.0 + 2 ** -7, 128.0]
+
+
+def test_int4_unpack_known_bytes():
+    # element 2i = low nibble, 2i+1 = high nibble, two's complement
+    packed = np.array([[0x80, 0x7F, 0x12, 0xF0]], dtype=np.uint8)
+    assert O.int4_unpack(packed).tolist() == [[0, -8, -1, 7, 2, 1, 0, -1]]
+
+
+def test_int4_dequant_group_boundaries():
+    I, H = 128, 128
+    codes = np.full((I, H // 2), 0x11, dtype=np.uint8)  # every element q = 1
+    s_rows = np.arange(1, I * (H // 64) + 1, dtype=np.float64).reshape(I, H // 64)
+    W = O.dequant_rows_int4(codes, s_rows)
+    assert W[5, 63] == s_rows[5, 0] and W[5, 64] == s_rows[5, 1]
+    s_down = np.arange(1, (I // 64) * H + 1, dtype=np.float64).reshape(I // 64, H)
+    Dt = O.dequant_down_t_int4(codes, s_down)
+    assert Dt[63, 7] == s_down[0, 7] and Dt[64, 7] == s_down[1, 7]
+    codes2 = np.full((I, H // 2), 0x9F, dtype=np.uint8)  # low -1, high -7
+    W2 = O.dequant_rows_int4(codes2, np.ones((I, H // 64)))
+    assert W2[0, 0] == -1 and W2[0, 1] == -7
+
+
+# ---------------------------------------------------------------- SiLU
+
+
+def test_silu_identities():
+    z = np.linspace(-20, 20, 401)
+    s = O.silu(z)
+    assert O.silu(np.array([0.0]))[0] == 0.0
+    # z*sigmoid(z) - (-z)*sigmoid(-z) = z (sigmoid(z) + sigmoid(-z) = 1)
+    assert np.allclose(s - O.silu(-z), z, atol=1e-12)
+    assert abs(O.silu(np.array([40.0]))[0] - 40.0) < 1e-12
+    h = 1e-6
+    assert abs((O.silu(np.array([h]))[0] - O.silu(np.array([-h]))[0]) / (2 * h) - 0.5) < 1e-9
+    assert abs(O.silu(np.array([1.0]))[0] - 1.0 / (1.0 + math.exp(-1.0))) < 1e-15
+
+
+# ---------------------------------------------------------------- router / top-k
+
+
+def test_topk_set_is_best_subset_bruteforce():
+    r = rng(2)
+    for E in range(2, 9):
+        for k in range(1, E + 1):
+            x = r.normal(0, 1, 6)
+            R = r.normal(0, 1, (E, 6))
+            ids, w, logits, _ = O.route_topk(x, R, k)
+            best = max(itertools.combinations(range(E), k), key=lambda S: sum(logits[list(S)]))
+            assert set(ids.tolist()) == set(best)
+            assert all(logits[ids[i]] >= logits[ids[i + 1]] for i in range(k - 1))
+
+
+def test_topk_ties_go_to_lowest_index():
+    R = np.zeros((7, 4))
+    ids, w, logits, margin = O.route_topk(np.ones(4), R, 3)
+    assert ids.tolist() == [0, 1, 2]
+    assert np.allclose(w, 1 / 3)
+    assert margin == 0.0
+    R2 = np.zeros((6, 2))
+    R2[:, 0] = [1, 3, 3, 2, 3, 0]
+    ids2, _, _, _ = O.route_topk(np.array([1.0, 0.0]), R2, 4)
+    assert ids2.tolist() == [1, 2, 4, 3]
+
+
+def test_topk_decision_taken_in_fp32():
+    # two logits that differ only below fp32 resolution tie in fp32 -> lower index
+    R = np.array([[1.0, 0.0], [1.0 + 1e-12, 0.0]])
+    ids, _, logits, _ = O.route_topk(np.array([1.0, 0.0]), R, 1)
+    assert logits[1] > logits[0] and ids.tolist() == [0]
+
+
+def test_two_expert_weights_are_logistic():
+    # softmax restricted to two experts: w_1 = sigmoid(l_1 - l_2) (textbook identity)
+    r = rng(3)
+    for _ in range(20):
+        x = r.normal(0, 1, 5)
+        R = r.normal(0, 1, (9, 5))
+        ids, w, logits, _ = O.route_topk(x, R, 2)
+        d = logits[ids[0]] - logits[ids[1]]
+        assert abs(w[0] - 1 / (1 + math.exp(-d))) < 1e-14
+        assert abs(w.sum() - 1) < 1e-15
+
+
+def test_router_onehot_rows_closed_form():
+    H, E = 16, 5
+    cols = [3, 0, 11, 7, 3]
+    c = [2.0, -1.0, 0.5, 3.0, -4.0]
+    R = np.zeros((E, H))
+    for e in range(E):
+        R[e, cols[e]] = c[e]
+    x = np.arange(1, H + 1, dtype=np.float64)
+    logits = O.router_logits(x, R)
+    assert logits.tolist() == [c[e] * x[cols[e]] for e in range(E)]
+
+
+def test_margin_is_gap_at_boundary():
+    R = np.array([[5.0], [1.0], [4.0], [2.0]])
+    ids, _, _, margin = O.route_topk(np.array([1.0]), R, 2)
+    assert ids.tolist() == [0, 2] and margin == 2.0
+    _, _, _, m_all = O.route_topk(np.array([1.0]), R, 4)
+    assert m_all == math.inf
+
+
+def test_tie_positions_flags_only_near_ties():
+    logits = np.array([1.0, 0.5, 0.5 + 5e-6, -1.0])
+    ids = O.topk_order(logits, 2)
+    assert ids.tolist() == [0, 2]
+    assert O.tie_positions(logits, ids) == {1}
+
+
+# ---------------------------------------------------------------- experts
+
+
+def perm_expert(H, I, a, b, p1, p2, p3):
+    G = np.zeros((I, H)); V = np.zeros((I, H)); Dt = np.zeros((I, H))
+    for i in range(I):
+        G[i, p1[i]] = a
+        V[i, p2[i]] = b
+        Dt[i, p3[i]] = 1.0
+    return G, V, Dt
+
+
+def test_swiglu_expert_permutation_closed_form():
+    # G = a P1, V = b P2, D^T rows one-hot at p3: y[p3(j)] = silu(a x[p1 j]) * b x[p2 j]
+    r = rng(4)
+    for H, I in [(8, 8), (12, 5)]:
+        p1 = r.permutation(H)[:I]; p2 = r.permutation(H)[:I]; p3 = r.permutation(H)[:I]
+        a, b = 0.7, -1.3
+        x = r.normal(0, 1, H)
+        y = O.swiglu_expert(x, *perm_expert(H, I, a, b, p1, p2, p3))
+        want = np.zeros(H)
+        for j in range(I):
+            z = a * x[p1[j]]
+            want[p3[j]] = z / (1 + math.exp(-z)) * (b * x[p2[j]])
+        assert np.allclose(y, want, rtol=0, atol=1e-14)
+
+
+def test_expert_is_linear_in_down_and_gate_up_roles_differ():
+    r = rng(5)
+    H, I = 16, 8
+    G, V, Dt = rand_expert(r, H, I)
+    x = r.normal(0, 1, H)
+    y = O.swiglu_expert(x, G, V, Dt)
+    assert np.allclose(O.swiglu_expert(x, G, V, 3 * Dt), 3 * y, atol=1e-13)
+    assert np.all(O.swiglu_expert(x, G, V, 0 * Dt) == 0)
+    # gate passes through phi, up does not: swapping them changes the result
+    assert not np.allclose(O.swiglu_expert(x, V, G, Dt), y)
+    # V = 0 kills the output (a_j = phi(g) * 0)
+    assert np.all(O.swiglu_expert(x, G, 0 * V, Dt) == 0)
+
+
+def make_layer(r, H, E, I, scale=0.3):
+    experts = [rand_expert(r, H, I, scale) for _ in range(E)]
+    R = r.normal(0, 1, (E, H))
+    return R, experts
+
+
+def test_k_equals_E_is_dense_softmax_mixture():
+    r = rng(6)
+    for H, E, I in [(16, 4, 8), (24, 7, 5)]:
+        R, ex = make_layer(r, H, E, I)
+        x = r.normal(0, 1, H)
+        y, ids, w, logits, _ = O.moe_layer(x, R, lambda e: ex[e], E)
+        dense = O.dense_mixture(x, R, lambda e: ex[e], E)
+        assert np.allclose(y, dense, rtol=1e-12, atol=1e-14)
+        assert np.allclose(w, O.softmax(logits)[ids], rtol=1e-14)
+
+
+def test_k1_selects_argmax_expert_with_weight_one():
+    r = rng(7)
+    R, ex = make_layer(r, 16, 6, 8)
+    x = r.normal(0, 1, 16)
+    y, ids, w, logits, _ = O.moe_layer(x, R, lambda e: ex[e], 1)
+    e = int(np.argmax(logits))
+    assert ids.tolist() == [e] and w.tolist() == [1.0]
+    assert np.array_equal(y, O.swiglu_expert(x, *ex[e]))
+
+
+def test_expert_relabelling_invariance():
+    # Relabel experts by a permutation pi (router rows and weights together):
+    # y is unchanged and ids are relabelled. Catches slot/id mix-ups.
+    r = rng(8)
+    H, E, I, k = 16, 8, 4, 3
+    R, ex = make_layer(r, H, E, I)
+    x = r.normal(0, 1, H)
+    y, ids, w, _, _ = O.moe_layer(x, R, lambda e: ex[e], k)
+    pi = r.permutation(E)  # new expert e' holds old expert pi[e']
+    y2, ids2, w2, _, _ = O.moe_layer(x, R[pi], lambda e: ex[pi[e]], k)
+    assert np.allclose(y, y2, atol=1e-13)
+    assert [int(pi[e]) for e in ids2] == ids.tolist()
+    assert np.allclose(w, w2)
+
+
+def test_shared_expert_is_added_with_unit_weight():
+    r = rng(9)
+    H, E, I = 16, 5, 4
+    R, ex = make_layer(r, H, E, I)
+    sh = rand_expert(r, H, 6)
+    x = r.normal(0, 1, H)
+    y0, *_ = O.moe_layer(x, R, lambda e: ex[e], 2)
+    y1, *_ = O.moe_layer(x, R, lambda e: ex[e], 2, shared=sh)
+    assert np.allclose(y1 - y0, O.swiglu_expert(x, *sh), atol=1e-13)
+
+
+def test_residual_keeps_bf16_input_when_y_zero():
+    x = O.bf16_round(rng(10).normal(0, 1, 64))
+    assert np.array_equal(O.residual_bf16(x, np.zeros(64)), x)
+    # 1 + 2^-9 is below half an ulp of bf16 at 1: rounds back to 1
+    assert O.residual_bf16(np.array([1.0]), np.array([2 ** -9]))[0] == 1.0
+
+
+def test_linear_experts_closed_forms():
+    r = rng(11)
+    H = 10
+    x = r.normal(0, 1, H)
+    c = [0.5, -2.0, 3.0, 1.5]
+    y = O.linear_experts(x, lambda e: c[e] * np.eye(H), [2, 0, 3], [1.0, 1.0, 0.25])
+    assert np.allclose(y, (3.0 + 0.5 + 0.25 * 1.5) * x, atol=1e-14)
+    P = np.zeros((H, H)); perm = r.permutation(H)
+    P[np.arange(H), perm] = 1.0  # (P x)[i] = x[perm[i]]
+    y2 = O.linear_experts(x, lambda e: P, [0], [1.0])
+    assert np.array_equal(y2, x[perm])
+
+
+# ---------------------------------------------------------------- touched experts
+
+
+def test_touched_formula_matches_printed_theory_column():
+    g = golden("touched_batch_sweep.json")
+    for B, printed in zip(g["batch"], g["theory_printed"]):
+        assert round(O.expected_touched(g["E"], g["k"], B), 1) == printed
+
+
+def test_touched_worked_example_printed_values():
+    g = golden("touched_batch_sweep.json")
+    we = g["worked_example"]
+    q = 1 - g["k"] / g["E"]
+    assert round(q, 3) == we["p_not_chosen_by_one_token"]
+    assert round(q ** we["B"], 2) == we["p_not_chosen_by_16_tokens"]
+    assert round(1 - q ** we["B"], 2) == we["p_touched"]
+
+
+def test_half_touch_batch_printed_is_small_p_approximation():
+    g = golden("touched_batch_sweep.json")
+    approx = O.half_touch_batch_small_p(g["E"], g["k"])
+    exact = O.half_touch_batch_exact(g["E"], g["k"])
+    assert round(approx, 1) == g["half_touch_batch_printed"]
+    assert abs(exact - 14.44) < 0.01
+    assert abs((1 - g["k"] / g["E"]) ** exact - 0.5) < 1e-12
+
+
+def test_touched_monte_carlo_within_sampling_error():
+    g = golden("touched_batch_sweep.json")
+    E, k = g["E"], g["k"]
+    r = rng(12)
+    draws = 2000
+    for B in g["batch"]:
+        counts = np.empty(draws)
+        for t in range(draws):
+            ids = np.stack([r.permutation(E)[:k] for _ in range(B)])
+            counts[t] = O.touched_experts(ids, E)[0]
+        theory = O.expected_touched(E, k, B)
+        # standard error: the sample's, floored by the independent-indicator
+        # bound sqrt(E p (1-p) / draws) with p = P(an expert is missed)
+        p_miss = (1 - k / E) ** B
+        se = max(counts.std(ddof=1), math.sqrt(E * p_miss * (1 - p_miss))) / math.sqrt(draws)
+        assert abs(counts.mean() - theory) <= 4 * se + 1e-12, (B, counts.mean(), theory)
+        if B == 1:
+            assert np.all(counts == k)
+
+
+def test_touched_counting_sort_bruteforce():
+    r = rng(13)
+    for B, k, E in [(1, 2, 16), (5, 3, 8), (8, 8, 256), (16, 3, 64)]:
+        ids = np.stack([r.permutation(E)[:k] for _ in range(B)])
+        count, bitmap, offsets, pairs = O.touched_experts(ids, E)
+        flat = ids.reshape(-1)
+        assert count == len(set(flat.tolist()))
+        assert offsets[0] == 0 and offsets[-1] == B * k
+        assert np.all(np.diff(offsets) >= 0)
+        assert sorted(pairs.tolist()) == list(range(B * k))
+        for e in range(E):
+            seg = pairs[offsets[e]:offsets[e + 1]]
+            assert np.all(np.diff(seg) > 0)
+            assert all(flat[p] == e for p in seg)
+            bit = (int(bitmap[e // 32]) >> (e % 32)) & 1
+            assert bit == (1 if len(seg) else 0)
+
+
+# ---------------------------------------------------------------- channel-sparse
+
+
+def test_sector_example_from_fig2c():
+    g = golden("sector_example.json")
+    # 80 needed bytes as four 20-byte pieces, each in its own 32-byte sector
+    ranges = [(0, 20), (70, 90), (128, 148), (300, 320)]
+    assert sum(hi - lo for lo, hi in ranges) == g["bytes_needed"]
+    n = O.sectors_touched(ranges)
+    assert n == g["sectors_touched"]
+    assert n * g["sector_bytes"] == g["bytes_charged"]
+    # the same 80 bytes packed at a sector boundary need 3 sectors
+    assert O.sectors_touched([(0, 80)]) == 3
+    assert O.sectors_touched([(31, 33)]) == 2
+    assert O.sectors_touched([(0, 10), (5, 20)]) == 1
+
+
+def test_sectors_of_aligned_channel_major_rows():
+    H, I = 2048, 768
+    kept = [0, 1, 5, 767, 768, 6143]
+    ranges = O.channel_major_ranges(kept, H)
+    assert O.sectors_touched(ranges) == 384 * len(kept)
+    # an unaligned base straddles one extra sector per non-adjacent run
+    assert O.sectors_touched(O.channel_major_ranges([0, 1], H, base=16)) == 2 * 384 + 1
+
+
+def test_channel_select_bruteforce_and_ties():
+    r = rng(14)
+    E, I = 5, 3
+    for keep in range(0, 7):
+        S = r.normal(0, 1, (E, I))
+        ids = [4, 1]
+        kept = O.channel_topk_select(S, ids, keep)
+        cand = [e * I + c for e in ids for c in range(I)]
+        best = max(itertools.combinations(cand, keep),
+                   key=lambda T: sum(S[j // I, j % I] for j in T)) if keep else ()
+        assert set(kept.tolist()) == set(best)
+    T = np.zeros((4, 2))
+    assert O.channel_topk_select(T, [3, 1], 3).tolist() == [2, 3, 6]
+
+
+def channel_view(ex, I):
+    return lambda e, c: np.stack([ex[e][0][c], ex[e][1][c], ex[e][2][c]])
+
+
+def test_channel_keep_all_equals_planar_experts():
+    r = rng(15)
+    H, E, I, k = 16, 6, 5, 3
+    R, ex = make_layer(r, H, E, I)
+    x = r.normal(0, 1, H)
+    ids, w, _, _ = O.route_topk(x, R, k)
+    S = np.abs(r.normal(0, 1, (E, I)))
+    kept = O.channel_topk_select(S, ids, k * I)
+    y_sparse = O.channel_sparse_forward(x, channel_view(ex, I), ids, w, kept, I)
+    y_planar = O.moe_experts_given(x, lambda e: ex[e], ids, w)
+    assert np.allclose(y_sparse, y_planar, rtol=1e-12, atol=1e-14)
+    y0 = O.channel_sparse_forward(x, channel_view(ex, I), ids, w, [], I)
+    assert np.all(y0 == 0)
+
+
+def test_channel_partial_keep_equals_masked_planar():
+    # keeping a subset equals the planar expert with the dropped channels'
+    # down rows zeroed
+    r = rng(16)
+    H, E, I, k = 12, 4, 6, 2
+    R, ex = make_layer(r, H, E, I)
+    x = r.normal(0, 1, H)
+    ids, w, _, _ = O.route_topk(x, R, k)
+    S = np.abs(r.normal(0, 1, (E, I)))
+    kept = O.channel_topk_select(S, ids, 5)
+    keep_set = set(kept.tolist())
+
+    def masked(e):
+        G, V, Dt = ex[e]
+        Dm = Dt.copy()
+        for c in range(I):
+            if e * I + c not in keep_set:
+                Dm[c] = 0
+        return G, V, Dm
+    y = O.channel_sparse_forward(x, channel_view(ex, I), ids, w, kept, I)
+    assert np.allclose(y, O.moe_experts_given(x, masked, ids, w), atol=1e-13)
+
+
+# ---------------------------------------------------------------- bytes / ceilings
+
+
+def test_decode_ceilings_match_moe_promise():
+    g = golden("decode_ceilings.json")
+    gb = g["gb_per_token"]["Qwen3.5-35B-A3B-4bit"]
+    fr = []
+    for m, bw in g["achieved_gbs"].items():
+        c = O.decode_ceiling(bw, gb)
+        assert round(c) == g["moe_ceiling_printed"][m]
+        fr.append(100 * g["moe_measured_printed"][m] / c)
+    lo, hi = g["moe_fraction_range_printed_pct"]
+    assert round(min(fr)) == lo and round(max(fr)) == hi
+    big = g["large_moe_example"]
+    assert round(O.decode_ceiling(big["achieved_gbs"], big["gb_per_token"])) == big["tok_s_printed"]
+
+
+def test_beam_memory_table():
+    g = golden("beam_memory.json")
+    assert round(O.param_bytes(g["total_params"], 16) / 1e9) == g["bf16"]["resident_gb_printed"]
+    assert round(O.param_bytes(g["active_params"], 16) / 1e9) == g["bf16"]["per_token_gb_printed"]
+    assert abs(O.param_bytes(g["total_params"], 4) / 1e9 - g["int4"]["resident_gb_printed"]) <= 0.5
+    assert O.param_bytes(g["active_params"], 4) / 1e9 == g["int4"]["per_token_gb_printed"]
+    assert round(100 * g["active_params"] / g["total_params"], 1) == g["active_ratio_pct_printed"]
+
+
+def test_reader_layer_bytes_vs_table7():
+    g = golden("reader_shapes.json")
+    q = g["table3"]["Qwen3-Thinking"]
+    assert q["k"] * q["I"] == g["candidates_per_layer_printed"]
+    routed = q["k"] * O.swiglu_expert_bytes(q["H"], q["I"])
+    assert routed == 75_497_472
+    # the profiler's cold-cache figure (router excluded) is within 0.2% of the count
+    assert abs(routed / 1e6 - g["table7_full_model_mb"]["1"]) / g["table7_full_model_mb"]["1"] < 2e-3
+    # real routing touches no more experts than the uniform-routing bound
+    for B in (4, 8):
+        bound = O.expected_touched(q["E"], q["k"], B) * O.swiglu_expert_bytes(q["H"], q["I"]) / 1e6
+        assert g["table7_full_model_mb"][str(B)] <= bound
+
+
+def test_layer_bytes_closed_forms():
+    # A3B-like layer: 8 routed + shared (I=512) + 256x2048 router, bf16
+    assert O.layer_bytes_b1(2048, 256, 512, 8, I_shared=512) == 57_671_680
+    assert O.swiglu_expert_bytes(2048, 512, "int4") == 1_671_168
+    assert O.layer_bytes_b1(2048, 256, 512, 8, I_shared=512, wtype="int4") == 20_709_376
+    assert O.layer_bytes_b1(512, 16, 256, 2) == 1_589_248
