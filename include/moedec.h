@@ -1,0 +1,198 @@
+/*
+ * libmoedec -- routed mixture-of-experts feed-forward layer at decode time,
+ * for NVIDIA B200 (sm_100a). Plain C ABI: device pointers, sizes, a CUDA
+ * stream; no C++ or framework types cross this boundary.
+ *
+ * The operation (pages cited by title and section):
+ *  - Router: logits = W_r x over E experts, softmax, top-k; a learned router
+ *    picks k experts per token and layer ("MoE 입문: 36B 모델이 27B보다 6배
+ *    빨랐던 이유", section "누가 8명을 고르나요"; "Mixture of Experts Changes
+ *    the Arithmetic", "Two Numbers Instead of One": 8 of 256).
+ *  - Expert = gated MLP. Channel j owns row j of the gate G_e, row j of the
+ *    up V_e and column j of the down D_e; a_j = phi(g_j.x)(v_j.x); the routed
+ *    output is the router-weighted sum of a_j d_j (review of arXiv:2610.37386,
+ *    "배경: 채널과 유지 규칙"). phi = SiLU (SwiGLU).
+ *  - Optional always-on shared expert ("Mixture of Experts Changes the
+ *    Arithmetic", checkpoint table: "256, 8 (+1 shared)").
+ *  - Channel-sparse top-k keep rule with 32-byte sector charging (same review,
+ *    keep-rule table, Fig. 2(c), and "2단계": one top-k across all of the
+ *    token's routed experts; down projection stored transposed).
+ *  - Touched experts at batch B ~ E[1-(1-k/E)^B] ("5,010억 개 중 230억 개만
+ *    켠다 — 4.6% 의 산수", §2 핵심 개념 and "둘째 식 — 배치의 함정").
+ *
+ * Conventions for every call:
+ *  - Pointers named x, y, ids, w, ... and every weight pointer are CUDA DEVICE
+ *    pointers owned by the caller; the library never allocates or frees
+ *    device memory. Descriptor structs (moe_layer_desc) live in HOST memory
+ *    and are read during the call only.
+ *  - Every device pointer must be 16-byte aligned.
+ *  - Calls are asynchronous on `stream` (NULL = the legacy default stream).
+ *    Outputs are valid after the stream is synchronised.
+ *  - Host-side argument errors return MOE_ERR_INVALID / MOE_ERR_UNSUPPORTED
+ *    before anything is launched. CUDA launch errors return MOE_ERR_CUDA.
+ *    Errors found on the device (a wait that ran out of its time budget,
+ *    expert ids out of range or repeated) are written to the workspace
+ *    status word and read with moe_get_status(); kernels never trap.
+ *  - A workspace is owned by one stream at a time: calls that share a
+ *    workspace must not run concurrently.
+ *  - bf16 is IEEE binary32's upper half; int32/float are 4 bytes.
+ *
+ * Layouts (row-major, innermost dimension last):
+ *  - x: [B, H] bf16.  y: [B, H] fp32 (overwritten).
+ *  - router: [E, H] bf16.
+ *  - PLANAR bf16 experts: gate, up, down_t each [E, I, H]; down_t[e, j, :] is
+ *    column j of D_e (the down projection stored transposed).
+ *  - PLANAR int4 (MOE_W_INT4_G64) experts: codes packed two per byte, element
+ *    2i in the low nibble, two's complement in [-8, 7], value = q * s with one
+ *    bf16 scale per 64 consecutive INPUT elements:
+ *      gate/up codes [E, I, H/2] u8, gate_s/up_s [E, I, H/64] bf16;
+ *      down_t codes [E, I, H/2] u8, down_s [E, I/64, H] bf16 (the down
+ *      projection's input is the channel index j, so its groups run along I).
+ *  - CHANNEL_MAJOR bf16 experts: gate = [E, I, 3, H]: for channel (e, c) the
+ *    gate row, up row and down column are contiguous (3*H*2 bytes); up and
+ *    down_t are NULL.
+ *  - LINEAR experts: gate = [E, H, H] (one H x H matrix per expert, output
+ *    row-major); E_e(x) = W_e x.
+ *  - Shared expert (SwiGLU, bf16, PLANAR): sh_gate, sh_up, sh_down_t each
+ *    [I_shared, H]; all NULL / I_shared = 0 for none.
+ */
+#ifndef MOEDEC_H
+#define MOEDEC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOEDEC_ABI_VERSION 1
+
+typedef struct CUstream_st* moe_stream_t; /* a cudaStream_t */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID = 1,     /* bad argument, or invalid expert ids found on the device */
+  MOE_ERR_UNSUPPORTED = 2, /* valid but outside what this build implements */
+  MOE_ERR_CUDA = 3,        /* a CUDA runtime call failed */
+  MOE_ERR_TIMEOUT = 4      /* a device-side wait ran out of its time budget */
+} moe_status;
+
+typedef enum { MOE_W_BF16 = 0, MOE_W_INT4_G64 = 1 } moe_wtype;
+typedef enum { MOE_EXPERT_SWIGLU = 0, MOE_EXPERT_LINEAR = 1 } moe_ekind;
+typedef enum { MOE_LAYOUT_PLANAR = 0, MOE_LAYOUT_CHANNEL_MAJOR = 1 } moe_layout;
+
+/* One MoE layer's shape and weights (host struct, device pointers). */
+typedef struct {
+  int32_t H;      /* hidden size; multiple of 64 (of 512 for int4)           */
+  int32_t E;      /* routed experts, 1..1024                                   */
+  int32_t I;      /* expert intermediate size (channels); multiple of 64 for int4 */
+  int32_t k;      /* experts per token, 1..min(E, 32)                          */
+  int32_t kind;   /* moe_ekind                                                 */
+  int32_t wtype;  /* moe_wtype                                                 */
+  int32_t layout; /* moe_layout                                                */
+  int32_t I_shared; /* shared-expert intermediate size, 0 = no shared expert  */
+  const void* router;          /* [E, H] bf16; may be NULL when ids are given */
+  const void* gate;            /* see Layouts above                           */
+  const void* up;
+  const void* down_t;
+  const void* gate_s;          /* int4 scales, else NULL                      */
+  const void* up_s;
+  const void* down_s;
+  const void* sh_gate;         /* shared expert, bf16 [I_shared, H] each      */
+  const void* sh_up;
+  const void* sh_down_t;
+} moe_layer_desc;
+
+/* ABI version compiled into the library (MOEDEC_ABI_VERSION). */
+int moe_abi_version(void);
+
+/* Text for a status code (static storage, never NULL). */
+const char* moe_status_string(moe_status s);
+
+/* Bytes of device workspace needed by any call below on layers of this shape
+ * at batch B (B tokens decoded together). 0 if the descriptor or B is
+ * invalid. The caller allocates it (16-byte aligned) and must clear it once
+ * with moe_workspace_init() before the first call. */
+size_t moe_workspace_bytes(const moe_layer_desc* desc, int32_t B);
+
+/* Clear a workspace (status word, barrier counters): once after allocation,
+ * and again after any call reported MOE_ERR_TIMEOUT. Asynchronous on stream. */
+moe_status moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Read (and keep) the device status word of a workspace. Synchronises
+ * `stream`. Returns MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_INVALID (bad ids). */
+moe_status moe_get_status(const void* ws, moe_stream_t stream);
+
+/* Router only: for each token b, logits = router @ x[b] (fp32 accumulate),
+ * ids[b, :] = the k experts with the largest logits in descending order,
+ * ties to the lowest index; w[b, i] = softmax over all E logits restricted to
+ * the chosen k and renormalised (= exp(l_i) / sum_{j chosen} exp(l_j)).
+ * margin_opt[b] = (k-th largest logit) - ((k+1)-th largest), +inf if k == E.
+ *   x [B, H] bf16; router [E, H] bf16; ids [B, k] int32; w [B, k] fp32;
+ *   margin_opt [B] fp32 or NULL. 1 <= B <= 256, H % 64 == 0, E <= 1024. */
+moe_status moe_route_topk(const void* x, const void* router, int32_t B, int32_t H,
+                          int32_t E, int32_t k, int32_t* ids, float* w, float* margin_opt,
+                          void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Routed experts only (no router, no shared expert, no residual):
+ *   y[b] = sum_i w[b, i] * E_{ids[b, i]}(x[b]).
+ * SWIGLU: E_e(x) = D_e (silu(G_e x) * (V_e x)); LINEAR: E_e(x) = W_e x.
+ * ids [B, k] int32 (distinct per token, < E; checked on the device),
+ * w [B, k] fp32, y [B, H] fp32 overwritten.
+ * SWIGLU PLANAR (bf16 or int4): 1 <= B <= 8. LINEAR bf16: 1 <= B <= 256. */
+moe_status moe_expert_forward(const moe_layer_desc* desc, const void* x, int32_t B,
+                              const int32_t* ids, const float* w, float* y,
+                              void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* One full layer: router, top-k, routed SwiGLU experts, shared expert:
+ *   y[b] = sum_i w[b,i] E_{ids[b,i]}(x[b]) + E_shared(x[b]);
+ * x_next_opt [B, H] bf16 = bf16_rne(x + y) (attention-free residual) or NULL;
+ * ids_out_opt [B, k], w_out_opt [B, k] or NULL. SWIGLU PLANAR, 1 <= B <= 8.
+ * One persistent launch; no per-expert dispatch. */
+moe_status moe_layer_forward(const moe_layer_desc* desc, const void* x, int32_t B, float* y,
+                             void* x_next_opt, int32_t* ids_out_opt, float* w_out_opt,
+                             void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* L layers in one persistent launch: x_{l+1} = bf16_rne(x_l + y_l) with y_l
+ * the full layer output above. layers[L] share H, E, I, k, kind, wtype,
+ * layout and I_shared (weights differ). x_out [B, H] bf16 = x_L.
+ * Optional histories for per-layer checking (NULL to skip):
+ *   x_hist [L+1, B, H] bf16 (x_0 .. x_L), y_hist [L, B, H] fp32,
+ *   ids_hist [L, B, k] int32, w_hist [L, B, k] fp32.
+ * 1 <= L <= 64, 1 <= B <= 8. */
+moe_status moe_stack_forward(const moe_layer_desc* layers, int32_t L, const void* x, int32_t B,
+                             void* x_out, void* x_hist_opt, float* y_hist_opt,
+                             int32_t* ids_hist_opt, float* w_hist_opt,
+                             void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Channel-sparse routed experts (CHANNEL_MAJOR bf16 SWIGLU, batch 1 per
+ * call row): for token b the candidates are the k*I channels (e, c) of its
+ * routed experts e = ids[b, :], indexed e*I + c. Keep the `keep` largest
+ * scores[b, e, c] (ties to the lowest index); dropped channels are not read
+ * and contribute 0:  y[b] = sum_{kept (e,c)} w_e a_{e,c} d_{e,c}.
+ *   scores [B, E, I] fp32 (only the routed rows are read);
+ *   kept_opt [B, keep] int32 = kept indices in ascending order, or NULL;
+ *   sectors [B] uint64 = distinct 32-byte sectors of routed-expert weights
+ *   the kernel read for that token. 0 <= keep <= k*I, 1 <= B <= 8. */
+moe_status moe_channel_topk_forward(const moe_layer_desc* desc, const void* x, int32_t B,
+                                    const int32_t* ids, const float* w, const float* scores,
+                                    int32_t keep, float* y, int32_t* kept_opt,
+                                    unsigned long long* sectors,
+                                    void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Touched experts of a batch: the union of the B tokens' expert sets.
+ *   ids [B, k] int32 (distinct per token, < E); count [1] int32 = |union|;
+ *   bitmap_opt [ceil(E/32)] uint32, bit e set iff expert e is touched;
+ *   offsets_opt [E+1] int32 exclusive prefix sum of per-expert pair counts;
+ *   pairs_opt [B*k] int32: pairs[offsets[e] .. offsets[e+1]) are the pair
+ *   indices b*k + s with ids[b, s] == e, ascending (a stable counting sort).
+ * 1 <= B <= 256, 1 <= k <= 32, E <= 1024. Invalid ids set count = -1. */
+moe_status moe_touched_experts(const int32_t* ids, int32_t B, int32_t k, int32_t E,
+                               int32_t* count, uint32_t* bitmap_opt, int32_t* offsets_opt,
+                               int32_t* pairs_opt, moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOEDEC_H */

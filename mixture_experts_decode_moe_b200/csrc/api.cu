@@ -1,0 +1,439 @@
+// libmoedec C ABI: argument validation, launch planning and launches.
+//
+// The definitions of each operation (and the passages of the pages they
+// follow) are documented in include/moedec.h.
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+
+#include "small_kernels.cuh"
+
+using namespace moedec;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t v, size_t a = kAlign) { return (v + a - 1) / a * a; }
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Workspace parts (byte offsets).
+struct WsLayout {
+  size_t logits, yacc, total;
+};
+
+inline WsLayout ws_layout(int B, int H, int E) {
+  WsLayout w;
+  size_t off = sizeof(WsControl);
+  w.logits = off;
+  off = align_up(off + (size_t)B * E * sizeof(float));
+  w.yacc = off;
+  off = align_up(off + 2 * (size_t)B * H * sizeof(float));
+  w.total = off;
+  return w;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+int max_dyn_smem() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+bool valid_shape(const moe_layer_desc* d) {
+  if (d == nullptr) return false;
+  if (d->H <= 0 || d->E <= 0 || d->I <= 0 || d->k <= 0) return false;
+  if (d->E > kMaxE || d->k > kMaxK || d->k > d->E) return false;
+  if (d->H % 64 != 0) return false;
+  if (d->kind != MOE_EXPERT_SWIGLU && d->kind != MOE_EXPERT_LINEAR) return false;
+  if (d->wtype != MOE_W_BF16 && d->wtype != MOE_W_INT4_G64) return false;
+  if (d->layout != MOE_LAYOUT_PLANAR && d->layout != MOE_LAYOUT_CHANNEL_MAJOR) return false;
+  if (d->wtype == MOE_W_INT4_G64 && (d->H % 512 != 0 || d->I % 64 != 0)) return false;
+  if (d->I_shared < 0) return false;
+  return true;
+}
+
+// Weights present and aligned for a SwiGLU layer of this descriptor.
+moe_status check_weights(const moe_layer_desc* d, bool need_router) {
+  if (need_router && (d->router == nullptr || !aligned16(d->router))) return MOE_ERR_INVALID;
+  if (d->gate == nullptr || !aligned16(d->gate)) return MOE_ERR_INVALID;
+  if (d->kind == MOE_EXPERT_SWIGLU && d->layout == MOE_LAYOUT_PLANAR) {
+    if (d->up == nullptr || d->down_t == nullptr || !aligned16(d->up) || !aligned16(d->down_t))
+      return MOE_ERR_INVALID;
+    if (d->wtype == MOE_W_INT4_G64) {
+      if (!d->gate_s || !d->up_s || !d->down_s || !aligned16(d->gate_s) || !aligned16(d->up_s) ||
+          !aligned16(d->down_s))
+        return MOE_ERR_INVALID;
+    }
+  }
+  if (d->I_shared > 0) {
+    if (!d->sh_gate || !d->sh_up || !d->sh_down_t || !aligned16(d->sh_gate) || !aligned16(d->sh_up) ||
+        !aligned16(d->sh_down_t))
+      return MOE_ERR_INVALID;
+  }
+  return MOE_OK;
+}
+
+// Launch plan for the persistent decode kernel.
+struct Plan {
+  int bmax, nch, nch_sh, rows_per_job, stage_bytes, nstages;
+  int off_x, off_lg, off_dots, off_hs, off_keys, off_kept, off_bar, smem_bytes;
+};
+
+constexpr int kStaticSmemReserve = 16 * 1024;  // RouteSmem and friends
+
+bool make_plan(const moe_layer_desc* d, int B, int mode, int keep, Plan* pl) {
+  const int H = d->H, rowb = 2 * H;
+  pl->bmax = (B <= 1) ? 1 : kMaxB;
+  const int budget = max_dyn_smem() - kStaticSmemReserve;
+  if (budget <= 0) return false;
+  // fixed parts
+  const int x_bytes = (int)align_up((size_t)B * H * 2, 128);
+  const int lg_bytes = (mode == MODE_LAYERS) ? (int)align_up((size_t)B * d->E * 4, 128) : 0;
+  const bool cm = d->layout == MOE_LAYOUT_CHANNEL_MAJOR;
+  const int keys_bytes = cm ? (int)align_up((size_t)d->k * d->I * 4, 128) : 0;
+  const int kept_bytes = cm ? (int)align_up((size_t)std::max(keep, 1) * 4, 128) : 0;
+  // shared-expert jobs (bf16 planar) and router rows
+  int nch_sh = std::max(1, std::min(64, (48 * 1024) / (3 * rowb)));
+  int rows_per_job = std::max(1, std::min(8, (48 * 1024) / rowb));
+  for (int nstages_target : {4, 3, 2}) {
+    // routed-job channels per stage
+    int nch, routed_bytes;
+    if (cm || d->wtype == MOE_W_BF16) {
+      nch = std::max(1, std::min(64, (48 * 1024) / (3 * rowb)));
+      routed_bytes = nch * 3 * rowb;
+    } else {
+      const int per_ch = 3 * (H / 2) + 2 * (H / 32);
+      nch = 64;
+      while (nch > 1 && nch * per_ch + rowb > 56 * 1024) nch >>= 1;
+      routed_bytes = nch * per_ch + rowb;
+    }
+    for (;;) {
+      int stage = std::max(routed_bytes, rows_per_job * rowb);
+      if (d->I_shared > 0) stage = std::max(stage, 3 * nch_sh * rowb);
+      stage = (int)align_up(stage, 128);
+      const int nchmax = std::max(nch, nch_sh);
+      const int dots_bytes = (int)align_up((size_t)2 * nchmax * pl->bmax * 4, 128);
+      const int hs_bytes = (int)align_up((size_t)nchmax * pl->bmax * 4, 128);
+      const int fixed = x_bytes + lg_bytes + dots_bytes + hs_bytes + keys_bytes + kept_bytes + 128;
+      const int nst = std::min(8, (budget - fixed) / stage);
+      if (nst >= nstages_target) {
+        pl->nch = nch;
+        pl->nch_sh = nch_sh;
+        pl->rows_per_job = rows_per_job;
+        pl->stage_bytes = stage;
+        pl->nstages = nst;
+        int off = nst * stage;
+        pl->off_x = off; off += x_bytes;
+        pl->off_lg = off; off += lg_bytes;
+        pl->off_dots = off; off += dots_bytes;
+        pl->off_hs = off; off += hs_bytes;
+        pl->off_keys = off; off += keys_bytes;
+        pl->off_kept = off; off += kept_bytes;
+        pl->off_bar = off; off += 128;
+        pl->smem_bytes = off;
+        return true;
+      }
+      // shrink the stages and retry
+      if (nch > 1 && (cm || d->wtype == MOE_W_BF16)) {
+        nch = std::max(1, nch / 2);
+        routed_bytes = nch * 3 * rowb;
+      } else if (nch > 1) {
+        const int per_ch = 3 * (H / 2) + 2 * (H / 32);
+        nch >>= 1;
+        routed_bytes = nch * per_ch + rowb;
+      } else {
+        break;
+      }
+      nch_sh = std::max(1, std::min(nch_sh, std::max(1, routed_bytes / (3 * rowb))));
+      rows_per_job = std::max(1, std::min(rows_per_job, routed_bytes / rowb));
+    }
+  }
+  return false;
+}
+
+template <int BMAX, int WT, int LAYOUT>
+cudaError_t launch_decode_t(const DecodeParams& p, int grid, cudaStream_t s) {
+  auto kern = decode_kernel<BMAX, WT, LAYOUT>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem_bytes);
+  if (err != cudaSuccess) return err;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = p.smem_bytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, p);
+}
+
+moe_status launch_decode(const DecodeParams& p, int bmax, cudaStream_t s) {
+  const int grid = sm_count();
+  if (grid <= 0) return MOE_ERR_CUDA;
+  cudaError_t err;
+  if (p.layout == MOE_LAYOUT_CHANNEL_MAJOR) {
+    if (bmax != 1) return MOE_ERR_UNSUPPORTED;
+    err = launch_decode_t<1, MOE_W_BF16, MOE_LAYOUT_CHANNEL_MAJOR>(p, grid, s);
+  } else if (p.wtype == MOE_W_BF16) {
+    err = (bmax == 1) ? launch_decode_t<1, MOE_W_BF16, MOE_LAYOUT_PLANAR>(p, grid, s)
+                      : launch_decode_t<kMaxB, MOE_W_BF16, MOE_LAYOUT_PLANAR>(p, grid, s);
+  } else {
+    err = (bmax == 1) ? launch_decode_t<1, MOE_W_INT4_G64, MOE_LAYOUT_PLANAR>(p, grid, s)
+                      : launch_decode_t<kMaxB, MOE_W_INT4_G64, MOE_LAYOUT_PLANAR>(p, grid, s);
+  }
+  return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+void fill_layer(LayerW* lw, const moe_layer_desc* d) {
+  lw->router = static_cast<const uint8_t*>(d->router);
+  lw->gate = static_cast<const uint8_t*>(d->gate);
+  lw->up = static_cast<const uint8_t*>(d->up);
+  lw->down = static_cast<const uint8_t*>(d->down_t);
+  lw->gate_s = static_cast<const uint8_t*>(d->gate_s);
+  lw->up_s = static_cast<const uint8_t*>(d->up_s);
+  lw->down_s = static_cast<const uint8_t*>(d->down_s);
+  lw->sh_gate = static_cast<const uint8_t*>(d->sh_gate);
+  lw->sh_up = static_cast<const uint8_t*>(d->sh_up);
+  lw->sh_down = static_cast<const uint8_t*>(d->sh_down_t);
+  lw->scores = nullptr;
+}
+
+void fill_common(DecodeParams* p, const moe_layer_desc* d, int B, const Plan& pl, void* ws) {
+  std::memset(p, 0, sizeof(*p));
+  p->B = B;
+  p->H = d->H;
+  p->E = d->E;
+  p->I = d->I;
+  p->k = d->k;
+  p->I_sh = d->I_shared;
+  p->wtype = d->wtype;
+  p->layout = d->layout;
+  p->nch = pl.nch;
+  p->nch_sh = pl.nch_sh;
+  p->rows_per_job = pl.rows_per_job;
+  p->nstages = pl.nstages;
+  p->stage_bytes = pl.stage_bytes;
+  p->off_x = pl.off_x;
+  p->off_lg = pl.off_lg;
+  p->off_dots = pl.off_dots;
+  p->off_hs = pl.off_hs;
+  p->off_keys = pl.off_keys;
+  p->off_kept = pl.off_kept;
+  p->off_bar = pl.off_bar;
+  p->smem_bytes = pl.smem_bytes;
+  const WsLayout w = ws_layout(B, d->H, d->E);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  p->ctl = reinterpret_cast<WsControl*>(base);
+  p->logits = reinterpret_cast<float*>(base + w.logits);
+  p->yacc = reinterpret_cast<float*>(base + w.yacc);
+}
+
+bool same_shape(const moe_layer_desc* a, const moe_layer_desc* b) {
+  return a->H == b->H && a->E == b->E && a->I == b->I && a->k == b->k && a->kind == b->kind &&
+         a->wtype == b->wtype && a->layout == b->layout && a->I_shared == b->I_shared;
+}
+
+}  // namespace
+
+extern "C" {
+
+int moe_abi_version(void) { return MOEDEC_ABI_VERSION; }
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID: return "invalid argument or expert ids";
+    case MOE_ERR_UNSUPPORTED: return "unsupported shape or mode";
+    case MOE_ERR_CUDA: return "CUDA runtime error";
+    case MOE_ERR_TIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+size_t moe_workspace_bytes(const moe_layer_desc* d, int32_t B) {
+  if (!valid_shape(d) || B < 1 || B > 256) return 0;
+  return ws_layout(B, d->H, d->E).total;
+}
+
+moe_status moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t stream) {
+  if (ws == nullptr || !aligned16(ws) || ws_bytes < sizeof(WsControl)) return MOE_ERR_INVALID;
+  return cudaMemsetAsync(ws, 0, ws_bytes, (cudaStream_t)stream) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status moe_get_status(const void* ws, moe_stream_t stream) {
+  if (ws == nullptr) return MOE_ERR_INVALID;
+  uint32_t st = 0;
+  if (cudaMemcpyAsync(&st, ws, sizeof(st), cudaMemcpyDeviceToHost, (cudaStream_t)stream) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return MOE_ERR_CUDA;
+  return (moe_status)st;
+}
+
+moe_status moe_route_topk(const void* x, const void* router, int32_t B, int32_t H, int32_t E, int32_t k,
+                          int32_t* ids, float* w, float* margin_opt, void* ws, size_t ws_bytes,
+                          moe_stream_t stream) {
+  if (!x || !router || !ids || !w || !ws) return MOE_ERR_INVALID;
+  if (B < 1 || B > 256 || H < 64 || H % 64 || E < 1 || E > kMaxE || k < 1 || k > kMaxK || k > E)
+    return MOE_ERR_INVALID;
+  if (!aligned16(x) || !aligned16(router) || !aligned16(ws)) return MOE_ERR_INVALID;
+  if (H > 8192) return MOE_ERR_UNSUPPORTED;
+  const WsLayout wl = ws_layout(B, H, E);
+  if (ws_bytes < wl.total) return MOE_ERR_INVALID;
+  float* logits = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + wl.logits);
+  cudaStream_t s = (cudaStream_t)stream;
+  const size_t sm1 = (size_t)kMaxB * H * 2;
+  if (sm1 > 48 * 1024 &&
+      cudaFuncSetAttribute(router_logits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1) !=
+          cudaSuccess)
+    return MOE_ERR_CUDA;
+  router_logits_kernel<<<dim3((E + kWarps - 1) / kWarps, (B + kMaxB - 1) / kMaxB), kThreads, sm1, s>>>(
+      static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(router), B, H, E, logits);
+  const size_t sm2 = (size_t)kWarps * E * 4;
+  topk_kernel<<<(B + kWarps - 1) / kWarps, kThreads, sm2, s>>>(logits, B, E, k, ids, w, margin_opt);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status moe_touched_experts(const int32_t* ids, int32_t B, int32_t k, int32_t E, int32_t* count,
+                               uint32_t* bitmap_opt, int32_t* offsets_opt, int32_t* pairs_opt,
+                               moe_stream_t stream) {
+  if (!ids || !count) return MOE_ERR_INVALID;
+  if (B < 1 || B > 256 || k < 1 || k > kMaxK || E < 1 || E > kMaxE || k > E) return MOE_ERR_INVALID;
+  touched_kernel<<<1, kThreads, 0, (cudaStream_t)stream>>>(ids, B, k, E, count, bitmap_opt, offsets_opt,
+                                                           pairs_opt);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status moe_expert_forward(const moe_layer_desc* d, const void* x, int32_t B, const int32_t* ids,
+                              const float* w, float* y, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  if (!valid_shape(d) || !x || !ids || !w || !y || !ws) return MOE_ERR_INVALID;
+  if (!aligned16(x) || !aligned16(y) || !aligned16(ws) || B < 1 || B > 256) return MOE_ERR_INVALID;
+  if (ws_bytes < moe_workspace_bytes(d, B)) return MOE_ERR_INVALID;
+  if (d->kind != MOE_EXPERT_SWIGLU || d->layout != MOE_LAYOUT_PLANAR) return MOE_ERR_UNSUPPORTED;
+  if (B > kMaxB || d->H > 2048) return MOE_ERR_UNSUPPORTED;
+  moe_status st = check_weights(d, false);
+  if (st != MOE_OK) return st;
+  Plan pl;
+  if (!make_plan(d, B, MODE_EXPERTS, 0, &pl)) return MOE_ERR_UNSUPPORTED;
+  DecodeParams p;
+  fill_common(&p, d, B, pl, ws);
+  p.L = 1;
+  p.mode = MODE_EXPERTS;
+  p.I_sh = 0;
+  p.x_in = static_cast<const uint16_t*>(x);
+  p.y_out = y;
+  p.ids_in = ids;
+  p.w_in = w;
+  fill_layer(&p.layer[0], d);
+  return launch_decode(p, pl.bmax, (cudaStream_t)stream);
+}
+
+moe_status moe_stack_forward(const moe_layer_desc* layers, int32_t L, const void* x, int32_t B, void* x_out,
+                             void* x_hist_opt, float* y_hist_opt, int32_t* ids_hist_opt, float* w_hist_opt,
+                             void* ws, size_t ws_bytes, moe_stream_t stream) {
+  if (layers == nullptr || L < 1 || L > kMaxLayers || !x || !ws) return MOE_ERR_INVALID;
+  const moe_layer_desc* d = &layers[0];
+  if (!valid_shape(d) || B < 1 || B > 256) return MOE_ERR_INVALID;
+  if (!aligned16(x) || !aligned16(ws) || (x_out && !aligned16(x_out)) || (x_hist_opt && !aligned16(x_hist_opt)) ||
+      (y_hist_opt && !aligned16(y_hist_opt)))
+    return MOE_ERR_INVALID;
+  if ((ids_hist_opt == nullptr) != (w_hist_opt == nullptr)) return MOE_ERR_INVALID;
+  if (ws_bytes < moe_workspace_bytes(d, B)) return MOE_ERR_INVALID;
+  if (d->kind != MOE_EXPERT_SWIGLU || d->layout != MOE_LAYOUT_PLANAR) return MOE_ERR_UNSUPPORTED;
+  if (B > kMaxB || d->H > 2048) return MOE_ERR_UNSUPPORTED;
+  for (int l = 0; l < L; ++l) {
+    if (!same_shape(&layers[l], d)) return MOE_ERR_INVALID;
+    moe_status st = check_weights(&layers[l], true);
+    if (st != MOE_OK) return st;
+  }
+  Plan pl;
+  if (!make_plan(d, B, MODE_LAYERS, 0, &pl)) return MOE_ERR_UNSUPPORTED;
+  DecodeParams p;
+  fill_common(&p, d, B, pl, ws);
+  p.L = L;
+  p.mode = MODE_LAYERS;
+  p.x_in = static_cast<const uint16_t*>(x);
+  p.x_out = static_cast<uint16_t*>(x_out);
+  p.x_hist = static_cast<uint16_t*>(x_hist_opt);
+  p.y_hist = y_hist_opt;
+  p.ids_out = ids_hist_opt;
+  p.w_out = w_hist_opt;
+  for (int l = 0; l < L; ++l) fill_layer(&p.layer[l], &layers[l]);
+  return launch_decode(p, pl.bmax, (cudaStream_t)stream);
+}
+
+moe_status moe_layer_forward(const moe_layer_desc* d, const void* x, int32_t B, float* y, void* x_next_opt,
+                             int32_t* ids_out_opt, float* w_out_opt, void* ws, size_t ws_bytes,
+                             moe_stream_t stream) {
+  if (!y || !aligned16(y)) return MOE_ERR_INVALID;
+  if (!valid_shape(d) || B < 1 || B > 256) return MOE_ERR_INVALID;
+  if (d->kind != MOE_EXPERT_SWIGLU || d->layout != MOE_LAYOUT_PLANAR) return MOE_ERR_UNSUPPORTED;
+  if (B > kMaxB || d->H > 2048) return MOE_ERR_UNSUPPORTED;
+  if ((ids_out_opt == nullptr) != (w_out_opt == nullptr)) return MOE_ERR_INVALID;
+  if (!x || !ws || !aligned16(x) || !aligned16(ws) || (x_next_opt && !aligned16(x_next_opt)))
+    return MOE_ERR_INVALID;
+  if (ws_bytes < moe_workspace_bytes(d, B)) return MOE_ERR_INVALID;
+  moe_status st = check_weights(d, true);
+  if (st != MOE_OK) return st;
+  Plan pl;
+  if (!make_plan(d, B, MODE_LAYERS, 0, &pl)) return MOE_ERR_UNSUPPORTED;
+  DecodeParams p;
+  fill_common(&p, d, B, pl, ws);
+  p.L = 1;
+  p.mode = MODE_LAYERS;
+  p.x_in = static_cast<const uint16_t*>(x);
+  p.x_out = static_cast<uint16_t*>(x_next_opt);
+  p.y_out = y;
+  p.ids_out = ids_out_opt;
+  p.w_out = w_out_opt;
+  fill_layer(&p.layer[0], d);
+  return launch_decode(p, pl.bmax, (cudaStream_t)stream);
+}
+
+moe_status moe_channel_topk_forward(const moe_layer_desc* d, const void* x, int32_t B, const int32_t* ids,
+                                    const float* w, const float* scores, int32_t keep, float* y,
+                                    int32_t* kept_opt, unsigned long long* sectors, void* ws, size_t ws_bytes,
+                                    moe_stream_t stream) {
+  if (!valid_shape(d) || !x || !ids || !w || !scores || !y || !sectors || !ws) return MOE_ERR_INVALID;
+  if (B < 1 || B > kMaxB) return MOE_ERR_INVALID;
+  if (d->kind != MOE_EXPERT_SWIGLU || d->layout != MOE_LAYOUT_CHANNEL_MAJOR || d->wtype != MOE_W_BF16)
+    return MOE_ERR_INVALID;
+  if (keep < 0 || keep > d->k * d->I) return MOE_ERR_INVALID;
+  if ((long long)d->k * d->I > kMaxCand || d->H > 2048) return MOE_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(y) || !aligned16(ws) || !aligned16(d->gate)) return MOE_ERR_INVALID;
+  if (ws_bytes < moe_workspace_bytes(d, 1)) return MOE_ERR_INVALID;
+  Plan pl;
+  if (!make_plan(d, 1, MODE_EXPERTS, keep, &pl)) return MOE_ERR_UNSUPPORTED;
+  // tokens run one after another through the same workspace
+  for (int b = 0; b < B; ++b) {
+    DecodeParams p;
+    fill_common(&p, d, 1, pl, ws);
+    p.L = 1;
+    p.mode = MODE_EXPERTS;
+    p.I_sh = 0;
+    p.keep = keep;
+    p.x_in = static_cast<const uint16_t*>(x) + (size_t)b * d->H;
+    p.y_out = y + (size_t)b * d->H;
+    p.ids_in = ids + (size_t)b * d->k;
+    p.w_in = w + (size_t)b * d->k;
+    p.kept_out = kept_opt ? kept_opt + (size_t)b * keep : nullptr;
+    p.sectors_out = sectors + b;
+    fill_layer(&p.layer[0], d);
+    p.layer[0].scores = scores + (size_t)b * d->E * d->I;
+    moe_status st = launch_decode(p, 1, (cudaStream_t)stream);
+    if (st != MOE_OK) return st;
+  }
+  return MOE_OK;
+}
+
+}  // extern "C"

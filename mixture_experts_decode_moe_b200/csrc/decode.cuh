@@ -1,0 +1,186 @@
+// Persistent decode kernel: router -> top-k -> routed SwiGLU experts (+ shared
+// expert) -> router-weighted sum -> residual, for L layers in ONE cooperative
+// launch with one CTA per SM.
+//
+// What it computes (pages cited by title and section):
+//  * router GEMV, softmax, top-k ("MoE 입문: 36B 모델이 27B보다 6배 빨랐던
+//    이유", "누가 8명을 고르나요"); ties go to the lowest expert index;
+//  * channel j of expert e: a_j = phi(g_j.x)(v_j.x), phi = SiLU, output
+//    += w_e a_j d_j (review of arXiv:2610.37386, "배경: 채널과 유지 규칙");
+//  * the shared expert every token touches, weight 1 ("Mixture of Experts
+//    Changes the Arithmetic", "Two Numbers Instead of One");
+//  * channel-sparse: one top-k over all routed experts' channels by a
+//    given score, only kept channels are read (same review, keep-rule table,
+//    "2단계", Fig. 2(c) for the 32-byte sector charge).
+//
+// How (B200 design):
+//  * the work unit is a run of up to `nch` consecutive channels of one
+//    expert: its gate rows, up rows and transposed-down rows are three
+//    contiguous byte ranges, fetched by 1-D bulk copies (TMA) into a ring of
+//    shared-memory stages with an L2 evict-first hint; one thread issues,
+//    all 256 compute; the ring keeps several stages in flight per SM;
+//  * each CTA owns a contiguous slice of (router rows, shared channels,
+//    routed channels); its partial y stays in registers and is added to an
+//    fp32 accumulator in L2 with vector reductions;
+//  * two grid-wide barriers per layer: after the router logits, and after
+//    the partial sums. Shared-expert work runs between the router's arrival
+//    and the top-k, and the next layer's router/shared weights are fetched
+//    into the ring while the current layer drains.
+#pragma once
+
+#include "common.cuh"
+
+namespace moedec {
+
+constexpr int kMaxLayers = 64;
+constexpr int kMaxB = 8;
+constexpr int kMaxK = 32;
+constexpr int kMaxE = 1024;
+constexpr int kMaxCand = 8192;  // channel-sparse candidates per token (k*I)
+
+enum DecodeMode : int { MODE_EXPERTS = 0, MODE_LAYERS = 1 };
+
+struct LayerW {
+  const uint8_t* router;  // [E, H] bf16
+  const uint8_t* gate;    // planar [E, I, H] bf16 | int4 codes [E, I, H/2] | channel-major [E, I, 3, H]
+  const uint8_t* up;
+  const uint8_t* down;    // transposed down, same shape as gate (planar)
+  const uint8_t* gate_s;  // int4 scales [E, I, H/64] bf16
+  const uint8_t* up_s;
+  const uint8_t* down_s;  // int4 [E, I/64, H] bf16
+  const uint8_t* sh_gate; // shared expert bf16 [I_sh, H]
+  const uint8_t* sh_up;
+  const uint8_t* sh_down;
+  const float* scores;    // channel-sparse scores [B, E, I] fp32
+};
+
+struct DecodeParams {
+  int L, B, H, E, I, k, I_sh;
+  int mode;     // DecodeMode
+  int wtype;    // MOE_W_BF16 / MOE_W_INT4_G64
+  int layout;   // MOE_LAYOUT_PLANAR / MOE_LAYOUT_CHANNEL_MAJOR
+  int keep;     // channel-sparse keep count
+  int nch;      // channels per job (routed); shared jobs use nch_sh
+  int nch_sh;
+  int rows_per_job;  // router rows per job
+  int nstages;
+  int stage_bytes;
+  // shared-memory carve-up (byte offsets from the dynamic smem base)
+  int off_x, off_lg, off_dots, off_hs, off_route, off_keys, off_kept, off_bar, smem_bytes;
+  // io
+  const uint16_t* x_in;   // [B, H]
+  uint16_t* x_out;        // [B, H] final x (or null)
+  uint16_t* x_hist;       // [L+1, B, H] (or null)
+  float* y_out;           // [B, H] last layer's y (or null)
+  float* y_hist;          // [L, B, H] (or null)
+  const int32_t* ids_in;  // MODE_EXPERTS: [B, k]
+  const float* w_in;
+  int32_t* ids_out;       // [L, B, k] (or null)
+  float* w_out;
+  int32_t* kept_out;      // channel-sparse [B, keep] (or null)
+  unsigned long long* sectors_out;  // channel-sparse [B] (or null)
+  WsControl* ctl;
+  float* logits;          // ws [B, E]
+  float* yacc;            // ws [2, B, H]
+  LayerW layer[kMaxLayers];
+};
+
+// Per-CTA routing state in shared memory.
+struct RouteSmem {
+  int U;                     // routed units (touched experts, ascending)
+  int ncand;                 // channel-sparse: number of kept channels
+  int unit_e[kMaxB * kMaxK];
+  uint32_t unit_mask[kMaxB * kMaxK];
+  float unit_w[kMaxB * kMaxK][kMaxB];
+  uint32_t bitmap[kMaxE / 32];
+  int rank_base[kMaxE / 32];
+  int ids[kMaxB][kMaxK];
+  float w[kMaxB][kMaxK];
+  float wmap_unit[kMaxK];    // channel-sparse (B = 1): weight per unit
+  uint32_t hist[256];
+  int scan[kThreads];
+  int sel_prefix, sel_rank;
+  unsigned long long sectors;
+};
+
+enum JobType : int { JOB_ROUTER = 0, JOB_SHARED = 1, JOB_ROUTED = 2, JOB_END = 3 };
+
+struct Job {
+  int type;
+  int layer;
+  int u;    // routed: unit index; channel-sparse: position in the kept list
+  int c0;   // first row / channel
+  int n;    // rows / channels
+};
+
+// Walks one CTA's job sequence: for each layer, its router rows, then its
+// shared channels, then its routed channels (known only after top-k).
+struct JobCursor {
+  int layer;
+  int type;
+  long long t;    // cursor inside the current type's range
+  long long t1;   // end of the range
+
+  __device__ void begin_layer(const DecodeParams& p, int l) {
+    layer = l;
+    type = JOB_ROUTER;
+    set_range(p);
+  }
+  __device__ void set_range(const DecodeParams& p) {
+    const long long G = gridDim.x, c = blockIdx.x;
+    for (;;) {
+      if (type == JOB_ROUTER) {
+        if (p.mode == MODE_LAYERS && p.layer[layer].router != nullptr) {
+          t = c * p.E / G; t1 = (c + 1) * p.E / G;
+          if (t < t1) return;
+        }
+        type = JOB_SHARED;
+      }
+      if (type == JOB_SHARED) {
+        if (p.mode == MODE_LAYERS && p.I_sh > 0) {
+          t = c * p.I_sh / G; t1 = (c + 1) * p.I_sh / G;
+          if (t < t1) return;
+        }
+        type = JOB_ROUTED;
+        t = -1; t1 = -1;  // set once the routing is known
+        return;
+      }
+      return;
+    }
+  }
+  // Routed range of this CTA once the number of routed channels R is known.
+  __device__ void set_routed(long long R) {
+    const long long G = gridDim.x, c = blockIdx.x;
+    t = c * R / G; t1 = (c + 1) * R / G;
+  }
+  __device__ bool routed_known() const { return !(type == JOB_ROUTED && t1 < 0); }
+};
+
+__device__ __forceinline__ long long llmin(long long a, long long b) { return a < b ? a : b; }
+
+__device__ __forceinline__ float silu_f(float z) { return z / (1.0f + expf(-z)); }
+
+// dot of 8 bf16 weights with 8 bf16 activations
+__device__ __forceinline__ float dot8_bf16(const uint4& wv, const uint4& xv) {
+  float a = bf16_lo(wv.x) * bf16_lo(xv.x);
+  a = fmaf(bf16_hi(wv.x), bf16_hi(xv.x), a);
+  a = fmaf(bf16_lo(wv.y), bf16_lo(xv.y), a);
+  a = fmaf(bf16_hi(wv.y), bf16_hi(xv.y), a);
+  a = fmaf(bf16_lo(wv.z), bf16_lo(xv.z), a);
+  a = fmaf(bf16_hi(wv.z), bf16_hi(xv.z), a);
+  a = fmaf(bf16_lo(wv.w), bf16_lo(xv.w), a);
+  a = fmaf(bf16_hi(wv.w), bf16_hi(xv.w), a);
+  return a;
+}
+
+// int4: two's-complement nibble j of word w (elements 8m..8m+7 of a row live
+// in one 32-bit word, element 2i in the low nibble of byte i) -> float q.
+// (w ^ 0x88888888) turns q into q + 8 in [0, 15]; OR-ing that into the
+// mantissa of 2^23 gives 2^23 + q + 8 exactly; subtracting 2^23 + 8 leaves q.
+__device__ __forceinline__ void int4x8_to_f(uint32_t w, float* q) {
+  const uint32_t t = w ^ 0x88888888u;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) q[j] = __uint_as_float(0x4B000000u | ((t >> (4 * j)) & 0xFu)) - 8388616.0f;
+}
+
+}  // namespace moedec
