@@ -271,7 +271,8 @@ def run_ours(args):
     torch.cuda.synchronize()
 
     def step(i):
-        M.moe_stack_forward(descs, xs[i % w["tokens"]:][:B], x_out, ws, stream=stream)
+        M.moe_stack_forward(descs, xs[i % w["tokens"]:][:B], x_out, ws, flags=M.MOE_STACK_PRE_RMSNORM,
+                            stream=stream)
 
     for i in range(args.warmup):
         step(i)
@@ -314,7 +315,7 @@ def run_ours(args):
     for i in range(args.steps):
         j = (args.warmup + i) % w["tokens"]
         x_dev.copy_(x_host[j:j + B], non_blocking=True)
-        M.moe_stack_forward(descs, x_dev, x_out, ws, stream=stream)
+        M.moe_stack_forward(descs, x_dev, x_out, ws, flags=M.MOE_STACK_PRE_RMSNORM, stream=stream)
         out_host.copy_(x_out, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()

@@ -154,15 +154,23 @@ moe_status moe_layer_forward(const moe_layer_desc* desc, const void* x, int32_t 
                              void* x_next_opt, int32_t* ids_out_opt, float* w_out_opt,
                              void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* Stack option: normalise each layer's MoE input, u_l = bf16_rne(x_l /
+ * sqrt(mean(x_l^2) + 1e-6)) (unit weight); the residual stays x_l + y_l. */
+#define MOE_STACK_PRE_RMSNORM 1u
+
 /* L layers in one persistent launch: x_{l+1} = bf16_rne(x_l + y_l) with y_l
- * the full layer output above. layers[L] share H, E, I, k, kind, wtype,
- * layout and I_shared (weights differ). x_out [B, H] bf16 = x_L.
+ * the full layer output above, computed on u_l = x_l, or on the RMS-normalised
+ * x_l when flags has MOE_STACK_PRE_RMSNORM (transformer blocks normalise the
+ * feed-forward input; the pages give the depth of the stack only, and without
+ * a norm a stack of random N(0, 0.02) SwiGLU layers overflows fp32 within
+ * ~25 layers). layers[L] share H, E, I, k, kind, wtype, layout and I_shared
+ * (weights differ). x_out [B, H] bf16 = x_L.
  * Optional histories for per-layer checking (NULL to skip):
  *   x_hist [L+1, B, H] bf16 (x_0 .. x_L), y_hist [L, B, H] fp32,
  *   ids_hist [L, B, k] int32, w_hist [L, B, k] fp32.
  * 1 <= L <= 64, 1 <= B <= 8. */
 moe_status moe_stack_forward(const moe_layer_desc* layers, int32_t L, const void* x, int32_t B,
-                             void* x_out, void* x_hist_opt, float* y_hist_opt,
+                             uint32_t flags, void* x_out, void* x_hist_opt, float* y_hist_opt,
                              int32_t* ids_hist_opt, float* w_hist_opt,
                              void* ws, size_t ws_bytes, moe_stream_t stream);
 

@@ -82,92 +82,62 @@ moe_status check_weights(const moe_layer_desc* d, bool need_router) {
   return MOE_OK;
 }
 
-// Launch plan for the persistent decode kernel.
-struct Plan {
-  int bmax, nch, nch_sh, rows_per_job, stage_bytes, nstages;
-  int off_x, off_lg, off_dots, off_hs, off_keys, off_kept, off_bar, smem_bytes;
-};
-
-constexpr int kStaticSmemReserve = 16 * 1024;  // RouteSmem and friends
-
-bool make_plan(const moe_layer_desc* d, int B, int mode, int keep, Plan* pl) {
-  const int H = d->H, rowb = 2 * H;
-  pl->bmax = (B <= 1) ? 1 : kMaxB;
-  const int budget = max_dyn_smem() - kStaticSmemReserve;
-  if (budget <= 0) return false;
-  // fixed parts
-  const int x_bytes = (int)align_up((size_t)B * H * 2, 128);
-  const int lg_bytes = (mode == MODE_LAYERS) ? (int)align_up((size_t)B * d->E * 4, 128) : 0;
-  const bool cm = d->layout == MOE_LAYOUT_CHANNEL_MAJOR;
-  const int keys_bytes = cm ? (int)align_up((size_t)d->k * d->I * 4, 128) : 0;
-  const int kept_bytes = cm ? (int)align_up((size_t)std::max(keep, 1) * 4, 128) : 0;
-  // shared-expert jobs (bf16 planar) and router rows
-  int nch_sh = std::max(1, std::min(64, (48 * 1024) / (3 * rowb)));
-  int rows_per_job = std::max(1, std::min(8, (48 * 1024) / rowb));
-  for (int nstages_target : {4, 3, 2}) {
-    // routed-job channels per stage
-    int nch, routed_bytes;
-    if (cm || d->wtype == MOE_W_BF16) {
-      nch = std::max(1, std::min(64, (48 * 1024) / (3 * rowb)));
-      routed_bytes = nch * 3 * rowb;
-    } else {
-      const int per_ch = 3 * (H / 2) + 2 * (H / 32);
-      nch = 64;
-      while (nch > 1 && nch * per_ch + rowb > 56 * 1024) nch >>= 1;
-      routed_bytes = nch * per_ch + rowb;
-    }
-    for (;;) {
-      int stage = std::max(routed_bytes, rows_per_job * rowb);
-      if (d->I_shared > 0) stage = std::max(stage, 3 * nch_sh * rowb);
-      stage = (int)align_up(stage, 128);
-      const int nchmax = std::max(nch, nch_sh);
-      const int dots_bytes = (int)align_up((size_t)2 * nchmax * pl->bmax * 4, 128);
-      const int hs_bytes = (int)align_up((size_t)nchmax * pl->bmax * 4, 128);
-      const int fixed = x_bytes + lg_bytes + dots_bytes + hs_bytes + keys_bytes + kept_bytes + 128;
-      const int nst = std::min(8, (budget - fixed) / stage);
-      if (nst >= nstages_target) {
-        pl->nch = nch;
-        pl->nch_sh = nch_sh;
-        pl->rows_per_job = rows_per_job;
-        pl->stage_bytes = stage;
-        pl->nstages = nst;
-        int off = nst * stage;
-        pl->off_x = off; off += x_bytes;
-        pl->off_lg = off; off += lg_bytes;
-        pl->off_dots = off; off += dots_bytes;
-        pl->off_hs = off; off += hs_bytes;
-        pl->off_keys = off; off += keys_bytes;
-        pl->off_kept = off; off += kept_bytes;
-        pl->off_bar = off; off += 128;
-        pl->smem_bytes = off;
-        return true;
-      }
-      // shrink the stages and retry
-      if (nch > 1 && (cm || d->wtype == MOE_W_BF16)) {
-        nch = std::max(1, nch / 2);
-        routed_bytes = nch * 3 * rowb;
-      } else if (nch > 1) {
-        const int per_ch = 3 * (H / 2) + 2 * (H / 32);
-        nch >>= 1;
-        routed_bytes = nch * per_ch + rowb;
-      } else {
-        break;
-      }
-      nch_sh = std::max(1, std::min(nch_sh, std::max(1, routed_bytes / (3 * rowb))));
-      rows_per_job = std::max(1, std::min(rows_per_job, routed_bytes / rowb));
-    }
-  }
-  return false;
+// Channels per job (template NCH): 8 for bf16 planar batch-1 decoding (96 KB
+// jobs, two stages), 4 otherwise.
+inline int pick_nch(const moe_layer_desc* d, int B) {
+  return (B == 1 && d->wtype == MOE_W_BF16 && d->layout == MOE_LAYOUT_PLANAR) ? 8 : 4;
 }
 
-template <int BMAX, int WT, int LAYOUT>
-cudaError_t launch_decode_t(const DecodeParams& p, int grid, cudaStream_t s) {
-  auto kern = decode_kernel<BMAX, WT, LAYOUT>;
-  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem_bytes);
+// Shared-memory carve-up of the persistent decode kernel: as many ring stages
+// as fit next to the fixed tiles, given the kernel's static shared memory.
+bool plan_smem(DecodeParams* p, int static_bytes) {
+  const int H = p->H, rowb = 2 * H, B = p->B, NCH = p->nch;
+  const int budget = max_dyn_smem() - static_bytes - 1024;
+  if (budget <= 0) return false;
+  const bool cm = p->layout == MOE_LAYOUT_CHANNEL_MAJOR;
+  const int x_bytes = (int)align_up((size_t)B * H * 2, 128);
+  const int u_bytes = p->pre_norm ? x_bytes : 0;
+  const int lg_bytes = (p->mode == MODE_LAYERS) ? (int)align_up((size_t)B * p->E * 4, 128) : 0;
+  // keys: router top-k keys [B*E] and channel-sparse candidates [k*I]
+  size_t nkeys = (p->mode == MODE_LAYERS) ? (size_t)B * p->E : 0;
+  if (cm) nkeys = std::max(nkeys, (size_t)p->k * p->I);
+  const int keys_bytes = (int)align_up(std::max<size_t>(nkeys, 1) * 4, 128);
+  const int kept_bytes = cm ? (int)align_up((size_t)std::max(p->keep, 1) * 4, 128) : 0;
+  int stage;
+  if (cm || p->wtype == MOE_W_BF16) stage = NCH * 3 * rowb;
+  else stage = NCH * (3 * (H / 2) + 2 * (H / 32)) + rowb;
+  stage = std::max(stage, p->rows_per_job * rowb);
+  if (p->I_sh > 0) stage = std::max(stage, NCH * 3 * rowb);
+  stage = (int)align_up(stage, 128);
+  const int fixed = x_bytes + u_bytes + lg_bytes + keys_bytes + kept_bytes;
+  const int nst = std::min(8, (budget - fixed - 256) / stage);
+  if (nst < 2) return false;
+  p->stage_bytes = stage;
+  p->nstages = nst;
+  int off = nst * stage;
+  p->off_x = off; off += x_bytes;
+  p->off_u = off; off += u_bytes;
+  p->off_lg = off; off += lg_bytes;
+  p->off_keys = off; off += keys_bytes;
+  p->off_kept = off; off += kept_bytes;
+  p->off_bar = off; off += (int)align_up((size_t)3 * nst * 8, 128);  // full, empty, dots-ready
+  p->smem_bytes = off;
+  return true;
+}
+
+template <int MODE, int BMAX, int WT, int LAYOUT, int NCH, int HV>
+cudaError_t launch_decode_h(const DecodeParams& p0, int grid, cudaStream_t s) {
+  auto kern = decode_kernel<MODE, BMAX, WT, LAYOUT, NCH, HV>;
+  cudaFuncAttributes fa;
+  cudaError_t err = cudaFuncGetAttributes(&fa, kern);
+  if (err != cudaSuccess) return err;
+  DecodeParams p = p0;
+  if (!plan_smem(&p, (int)fa.sharedSizeBytes)) return cudaErrorInvalidConfiguration;
+  err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem_bytes);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(kCtaThreads);
   cfg.dynamicSmemBytes = p.smem_bytes;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -176,6 +146,29 @@ cudaError_t launch_decode_t(const DecodeParams& p, int grid, cudaStream_t s) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, p);
+}
+
+// Full-row dot loops are specialised for H = 2048 (HV = H/256 = 8 vectors per
+// lane); other hidden sizes use the guarded generic loop.
+template <int MODE, int BMAX, int WT, int LAYOUT, int NCH>
+cudaError_t launch_decode_n(const DecodeParams& p, int grid, cudaStream_t s) {
+  if (p.H == 2048) return launch_decode_h<MODE, BMAX, WT, LAYOUT, NCH, 8>(p, grid, s);
+  return launch_decode_h<MODE, BMAX, WT, LAYOUT, NCH, 0>(p, grid, s);
+}
+
+template <int MODE, int BMAX, int WT, int LAYOUT>
+cudaError_t launch_decode_m(const DecodeParams& p, int grid, cudaStream_t s) {
+  if constexpr (BMAX == 1 && WT == MOE_W_BF16 && LAYOUT == MOE_LAYOUT_PLANAR) {
+    if (p.nch == 8) return launch_decode_n<MODE, BMAX, WT, LAYOUT, 8>(p, grid, s);
+  }
+  if (p.nch != 4) return cudaErrorInvalidValue;
+  return launch_decode_n<MODE, BMAX, WT, LAYOUT, 4>(p, grid, s);
+}
+
+template <int BMAX, int WT, int LAYOUT>
+cudaError_t launch_decode_t(const DecodeParams& p, int grid, cudaStream_t s) {
+  if (p.mode == MODE_LAYERS) return launch_decode_m<MODE_LAYERS, BMAX, WT, LAYOUT>(p, grid, s);
+  return launch_decode_m<MODE_EXPERTS, BMAX, WT, LAYOUT>(p, grid, s);
 }
 
 moe_status launch_decode(const DecodeParams& p, int bmax, cudaStream_t s) {
@@ -192,6 +185,7 @@ moe_status launch_decode(const DecodeParams& p, int bmax, cudaStream_t s) {
     err = (bmax == 1) ? launch_decode_t<1, MOE_W_INT4_G64, MOE_LAYOUT_PLANAR>(p, grid, s)
                       : launch_decode_t<kMaxB, MOE_W_INT4_G64, MOE_LAYOUT_PLANAR>(p, grid, s);
   }
+  if (err == cudaErrorInvalidConfiguration) return MOE_ERR_UNSUPPORTED;
   return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -209,7 +203,7 @@ void fill_layer(LayerW* lw, const moe_layer_desc* d) {
   lw->scores = nullptr;
 }
 
-void fill_common(DecodeParams* p, const moe_layer_desc* d, int B, const Plan& pl, void* ws) {
+void fill_common(DecodeParams* p, const moe_layer_desc* d, int B, void* ws) {
   std::memset(p, 0, sizeof(*p));
   p->B = B;
   p->H = d->H;
@@ -219,19 +213,9 @@ void fill_common(DecodeParams* p, const moe_layer_desc* d, int B, const Plan& pl
   p->I_sh = d->I_shared;
   p->wtype = d->wtype;
   p->layout = d->layout;
-  p->nch = pl.nch;
-  p->nch_sh = pl.nch_sh;
-  p->rows_per_job = pl.rows_per_job;
-  p->nstages = pl.nstages;
-  p->stage_bytes = pl.stage_bytes;
-  p->off_x = pl.off_x;
-  p->off_lg = pl.off_lg;
-  p->off_dots = pl.off_dots;
-  p->off_hs = pl.off_hs;
-  p->off_keys = pl.off_keys;
-  p->off_kept = pl.off_kept;
-  p->off_bar = pl.off_bar;
-  p->smem_bytes = pl.smem_bytes;
+  p->nch = pick_nch(d, B);
+  p->nch_sh = p->nch;
+  p->rows_per_job = 2 * p->nch;
   const WsLayout w = ws_layout(B, d->H, d->E);
   uint8_t* base = static_cast<uint8_t*>(ws);
   p->ctl = reinterpret_cast<WsControl*>(base);
@@ -323,10 +307,8 @@ moe_status moe_expert_forward(const moe_layer_desc* d, const void* x, int32_t B,
   if (B > kMaxB || d->H > 2048) return MOE_ERR_UNSUPPORTED;
   moe_status st = check_weights(d, false);
   if (st != MOE_OK) return st;
-  Plan pl;
-  if (!make_plan(d, B, MODE_EXPERTS, 0, &pl)) return MOE_ERR_UNSUPPORTED;
   DecodeParams p;
-  fill_common(&p, d, B, pl, ws);
+  fill_common(&p, d, B, ws);
   p.L = 1;
   p.mode = MODE_EXPERTS;
   p.I_sh = 0;
@@ -335,12 +317,13 @@ moe_status moe_expert_forward(const moe_layer_desc* d, const void* x, int32_t B,
   p.ids_in = ids;
   p.w_in = w;
   fill_layer(&p.layer[0], d);
-  return launch_decode(p, pl.bmax, (cudaStream_t)stream);
+  return launch_decode(p, B <= 1 ? 1 : kMaxB, (cudaStream_t)stream);
 }
 
-moe_status moe_stack_forward(const moe_layer_desc* layers, int32_t L, const void* x, int32_t B, void* x_out,
-                             void* x_hist_opt, float* y_hist_opt, int32_t* ids_hist_opt, float* w_hist_opt,
-                             void* ws, size_t ws_bytes, moe_stream_t stream) {
+moe_status moe_stack_forward(const moe_layer_desc* layers, int32_t L, const void* x, int32_t B, uint32_t flags,
+                             void* x_out, void* x_hist_opt, float* y_hist_opt, int32_t* ids_hist_opt,
+                             float* w_hist_opt, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  if (flags & ~(uint32_t)MOE_STACK_PRE_RMSNORM) return MOE_ERR_INVALID;
   if (layers == nullptr || L < 1 || L > kMaxLayers || !x || !ws) return MOE_ERR_INVALID;
   const moe_layer_desc* d = &layers[0];
   if (!valid_shape(d) || B < 1 || B > 256) return MOE_ERR_INVALID;
@@ -356,12 +339,12 @@ moe_status moe_stack_forward(const moe_layer_desc* layers, int32_t L, const void
     moe_status st = check_weights(&layers[l], true);
     if (st != MOE_OK) return st;
   }
-  Plan pl;
-  if (!make_plan(d, B, MODE_LAYERS, 0, &pl)) return MOE_ERR_UNSUPPORTED;
+  const bool pre_norm = (flags & MOE_STACK_PRE_RMSNORM) != 0;
   DecodeParams p;
-  fill_common(&p, d, B, pl, ws);
+  fill_common(&p, d, B, ws);
   p.L = L;
   p.mode = MODE_LAYERS;
+  p.pre_norm = pre_norm ? 1 : 0;
   p.x_in = static_cast<const uint16_t*>(x);
   p.x_out = static_cast<uint16_t*>(x_out);
   p.x_hist = static_cast<uint16_t*>(x_hist_opt);
@@ -369,7 +352,7 @@ moe_status moe_stack_forward(const moe_layer_desc* layers, int32_t L, const void
   p.ids_out = ids_hist_opt;
   p.w_out = w_hist_opt;
   for (int l = 0; l < L; ++l) fill_layer(&p.layer[l], &layers[l]);
-  return launch_decode(p, pl.bmax, (cudaStream_t)stream);
+  return launch_decode(p, B <= 1 ? 1 : kMaxB, (cudaStream_t)stream);
 }
 
 moe_status moe_layer_forward(const moe_layer_desc* d, const void* x, int32_t B, float* y, void* x_next_opt,
@@ -385,10 +368,8 @@ moe_status moe_layer_forward(const moe_layer_desc* d, const void* x, int32_t B, 
   if (ws_bytes < moe_workspace_bytes(d, B)) return MOE_ERR_INVALID;
   moe_status st = check_weights(d, true);
   if (st != MOE_OK) return st;
-  Plan pl;
-  if (!make_plan(d, B, MODE_LAYERS, 0, &pl)) return MOE_ERR_UNSUPPORTED;
   DecodeParams p;
-  fill_common(&p, d, B, pl, ws);
+  fill_common(&p, d, B, ws);
   p.L = 1;
   p.mode = MODE_LAYERS;
   p.x_in = static_cast<const uint16_t*>(x);
@@ -397,7 +378,7 @@ moe_status moe_layer_forward(const moe_layer_desc* d, const void* x, int32_t B, 
   p.ids_out = ids_out_opt;
   p.w_out = w_out_opt;
   fill_layer(&p.layer[0], d);
-  return launch_decode(p, pl.bmax, (cudaStream_t)stream);
+  return launch_decode(p, B <= 1 ? 1 : kMaxB, (cudaStream_t)stream);
 }
 
 moe_status moe_channel_topk_forward(const moe_layer_desc* d, const void* x, int32_t B, const int32_t* ids,
@@ -412,12 +393,10 @@ moe_status moe_channel_topk_forward(const moe_layer_desc* d, const void* x, int3
   if ((long long)d->k * d->I > kMaxCand || d->H > 2048) return MOE_ERR_UNSUPPORTED;
   if (!aligned16(x) || !aligned16(y) || !aligned16(ws) || !aligned16(d->gate)) return MOE_ERR_INVALID;
   if (ws_bytes < moe_workspace_bytes(d, 1)) return MOE_ERR_INVALID;
-  Plan pl;
-  if (!make_plan(d, 1, MODE_EXPERTS, keep, &pl)) return MOE_ERR_UNSUPPORTED;
   // tokens run one after another through the same workspace
   for (int b = 0; b < B; ++b) {
     DecodeParams p;
-    fill_common(&p, d, 1, pl, ws);
+    fill_common(&p, d, 1, ws);
     p.L = 1;
     p.mode = MODE_EXPERTS;
     p.I_sh = 0;

@@ -60,13 +60,14 @@ struct DecodeParams {
   int wtype;    // MOE_W_BF16 / MOE_W_INT4_G64
   int layout;   // MOE_LAYOUT_PLANAR / MOE_LAYOUT_CHANNEL_MAJOR
   int keep;     // channel-sparse keep count
+  int pre_norm; // stack: RMS-normalise each layer's input (unit weight, eps 1e-6)
   int nch;      // channels per job (routed); shared jobs use nch_sh
   int nch_sh;
   int rows_per_job;  // router rows per job
   int nstages;
   int stage_bytes;
   // shared-memory carve-up (byte offsets from the dynamic smem base)
-  int off_x, off_lg, off_dots, off_hs, off_route, off_keys, off_kept, off_bar, smem_bytes;
+  int off_x, off_u, off_lg, off_keys, off_kept, off_bar, smem_bytes;
   // io
   const uint16_t* x_in;   // [B, H]
   uint16_t* x_out;        // [B, H] final x (or null)
@@ -96,7 +97,6 @@ struct RouteSmem {
   int rank_base[kMaxE / 32];
   int ids[kMaxB][kMaxK];
   float w[kMaxB][kMaxK];
-  float wmap_unit[kMaxK];    // channel-sparse (B = 1): weight per unit
   uint32_t hist[256];
   int scan[kThreads];
   int sel_prefix, sel_rank;
@@ -114,12 +114,14 @@ struct Job {
 };
 
 // Walks one CTA's job sequence: for each layer, its router rows, then its
-// shared channels, then its routed channels (known only after top-k).
+// shared channels, then its routed channels (known only after top-k). All
+// counters are 32-bit; the only divisions happen once per layer.
 struct JobCursor {
   int layer;
   int type;
-  long long t;    // cursor inside the current type's range
-  long long t1;   // end of the range
+  int t;    // cursor inside the current type's range
+  int t1;   // end of the range (-1: routed range not known yet)
+  int u, c; // routed planar: t = u * I + c
 
   __device__ void begin_layer(const DecodeParams& p, int l) {
     layer = l;
@@ -127,38 +129,36 @@ struct JobCursor {
     set_range(p);
   }
   __device__ void set_range(const DecodeParams& p) {
-    const long long G = gridDim.x, c = blockIdx.x;
-    for (;;) {
-      if (type == JOB_ROUTER) {
-        if (p.mode == MODE_LAYERS && p.layer[layer].router != nullptr) {
-          t = c * p.E / G; t1 = (c + 1) * p.E / G;
-          if (t < t1) return;
-        }
-        type = JOB_SHARED;
+    const long long G = gridDim.x, cb = blockIdx.x;
+    if (type == JOB_ROUTER) {
+      if (p.mode == MODE_LAYERS && layer < p.L && p.layer[layer].router != nullptr) {
+        t = (int)(cb * p.E / G); t1 = (int)((cb + 1) * p.E / G);
+        if (t < t1) return;
       }
-      if (type == JOB_SHARED) {
-        if (p.mode == MODE_LAYERS && p.I_sh > 0) {
-          t = c * p.I_sh / G; t1 = (c + 1) * p.I_sh / G;
-          if (t < t1) return;
-        }
-        type = JOB_ROUTED;
-        t = -1; t1 = -1;  // set once the routing is known
-        return;
-      }
-      return;
+      type = JOB_SHARED;
     }
+    if (type == JOB_SHARED) {
+      if (p.mode == MODE_LAYERS && p.I_sh > 0) {
+        t = (int)(cb * p.I_sh / G); t1 = (int)((cb + 1) * p.I_sh / G);
+        if (t < t1) return;
+      }
+      type = JOB_ROUTED;
+    }
+    t = -1; t1 = -1;  // routed: set once the routing is known
   }
   // Routed range of this CTA once the number of routed channels R is known.
-  __device__ void set_routed(long long R) {
-    const long long G = gridDim.x, c = blockIdx.x;
-    t = c * R / G; t1 = (c + 1) * R / G;
+  __device__ void set_routed(int R, int I) {
+    const long long G = gridDim.x, cb = blockIdx.x;
+    t = (int)(cb * R / G); t1 = (int)((cb + 1) * R / G);
+    u = t / I; c = t - u * I;
   }
-  __device__ bool routed_known() const { return !(type == JOB_ROUTED && t1 < 0); }
 };
 
 __device__ __forceinline__ long long llmin(long long a, long long b) { return a < b ? a : b; }
 
-__device__ __forceinline__ float silu_f(float z) { return z / (1.0f + expf(-z)); }
+// SiLU with the fast exponential and division intrinsics (relative error a
+// few ulp; __fdividef returns 0 when 1 + e^-z overflows past 2^126, the limit).
+__device__ __forceinline__ float silu_f(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
 
 // dot of 8 bf16 weights with 8 bf16 activations
 __device__ __forceinline__ float dot8_bf16(const uint4& wv, const uint4& xv) {
@@ -171,6 +171,50 @@ __device__ __forceinline__ float dot8_bf16(const uint4& wv, const uint4& xv) {
   a = fmaf(bf16_lo(wv.w), bf16_lo(xv.w), a);
   a = fmaf(bf16_hi(wv.w), bf16_hi(xv.w), a);
   return a;
+}
+
+// ---- tensor-core dot products of bf16 rows with one token (batch 1) ----
+//
+// A row segment of 256 bf16 weights w[0..256) is one 16x16 A tile of
+// mma.m16n8k16 with A[i][k] = w[8i + k] (k < 8) and w[128 + 8i + k - 8]
+// (k >= 8): one ldmatrix.x4 reads it as a contiguous 512-byte block (lane L
+// points at byte 16L), so the read is free of bank conflicts. B holds x in the
+// matching positions: B0[k][j] pairs with A row j (j < 8) and B1[k][j] with A
+// row 8 + j. The dot product of the segment is the sum of the diagonal
+// D0[i][i] + D1[8+j][j]; summed over segments the diagonals accumulate the
+// full row. Products of bf16 are exact in fp32; accumulation is fp32.
+__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t& a0, uint32_t& a1, uint32_t& a2,
+                                            uint32_t& a3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(a0), "=r"(a1), "=r"(a2), "=r"(a3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// B fragments of x for one 256-element segment (4 words per lane):
+// lane (g = lane/4, t = lane%4) needs bf16 pairs at 8g + 2t + {0, 128}
+// (B0) and 64 + 8g + 2t + {0, 128} (B1).
+__device__ __forceinline__ void x_frag(const uint16_t* xseg, int lane, uint32_t (&b)[4]) {
+  const uint32_t* w = reinterpret_cast<const uint32_t*>(xseg);
+  const int o = (8 * (lane >> 2) + 2 * (lane & 3)) >> 1;
+  b[0] = w[o];
+  b[1] = w[o + 64];
+  b[2] = w[o + 32];
+  b[3] = w[o + 96];
+}
+
+// Sum the diagonals of D0 and D1 held by this lane (lanes 4g + g/2).
+__device__ __forceinline__ float diag_part(const float (&d0)[4], const float (&d1)[4], int lane) {
+  const int g = lane >> 2, t = lane & 3;
+  if (t != (g >> 1)) return 0.f;
+  return (g & 1) ? (d0[1] + d1[3]) : (d0[0] + d1[2]);
 }
 
 // int4: two's-complement nibble j of word w (elements 8m..8m+7 of a row live

@@ -1,13 +1,55 @@
 // Body of the persistent decode kernel (see decode.cuh for the design).
+//
+// Roles inside a CTA (288 threads):
+//   warps 0-7  consumers: dot products, SwiGLU, down projection, top-k,
+//              grid barriers, epilogue; synchronise with named barrier 1;
+//   warp 8     producer: walks the same job sequence and issues the bulk
+//              copies of each job into a free stage of the ring (full/empty
+//              mbarriers per stage), running ahead of the consumers.
 #pragma once
 
 #include "decode.cuh"
 
 namespace moedec {
 
+constexpr int kConsumers = kThreads;          // 256 consumer threads
+constexpr int kCtaThreads = kThreads + 32;    // + one producer warp
+
+__device__ __forceinline__ void cbar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+__device__ __forceinline__ int cbar_or(int pred) {
+  int r;
+  asm volatile(
+      "{ .reg .pred p, q; setp.ne.s32 p, %1, 0; bar.red.or.pred q, 1, 256, p; selp.s32 %0, 1, 0, q; }"
+      : "=r"(r)
+      : "r"(pred)
+      : "memory");
+  return r;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void red_release_gpu(unsigned long long* p, unsigned long long v) {
+  asm volatile("red.release.gpu.global.add.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ unsigned long long ld_relaxed_gpu(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ int ld_acquire_cta(const int* p) {
+  int v;
+  asm volatile("ld.acquire.cta.shared::cta.s32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_cta(int* p, int v) {
+  asm volatile("st.release.cta.shared::cta.s32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+
 // ---------------------------------------------------------------- block helpers
 
-// Exclusive prefix sum over the CTA; `total` receives the sum. All threads call.
+// Exclusive prefix sum over the 256 consumer threads; `total` gets the sum.
 __device__ __forceinline__ int block_excl_scan(int v, int* scratch, int* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int inc = v;
@@ -17,7 +59,7 @@ __device__ __forceinline__ int block_excl_scan(int v, int* scratch, int* total) 
     if (lane >= o) inc += t;
   }
   if (lane == 31) scratch[warp] = inc;
-  __syncthreads();
+  cbar();
   if (warp == 0) {
     int t = lane < kWarps ? scratch[lane] : 0;
     int ti = t;
@@ -29,23 +71,57 @@ __device__ __forceinline__ int block_excl_scan(int v, int* scratch, int* total) 
     if (lane < kWarps) scratch[lane] = ti - t;
     if (lane == kWarps - 1) scratch[kWarps] = ti;
   }
-  __syncthreads();
+  cbar();
   int r = inc - v + scratch[warp];
   *total = scratch[kWarps];
-  __syncthreads();
+  cbar();
   return r;
+}
+
+// Transpose-style reduction of NV per-lane values across a warp. Afterwards
+// the warp's sums are written to out[0..NV) (smem).
+template <int NV>
+__device__ __forceinline__ void warp_reduce_multi(float (&v)[NV], float* out) {
+  static_assert((NV & (NV - 1)) == 0, "NV must be a power of two");
+  const int lane = threadIdx.x & 31;
+  int base = 0;
+  // halving steps (offsets 16, 8, ...) while more than one value remains
+  constexpr int S = (NV >= 32) ? 5 : (NV >= 16 ? 4 : (NV >= 8 ? 3 : (NV >= 4 ? 2 : (NV >= 2 ? 1 : 0))));
+#pragma unroll
+  for (int s = 0; s < S; ++s) {
+    const int off = 16 >> s;
+    const int C = NV >> s;
+    const bool up = (lane & off) != 0;
+#pragma unroll
+    for (int i = 0; i < C / 2; ++i) {
+      const float send = up ? v[i] : v[i + C / 2];
+      const float keep = up ? v[i + C / 2] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+    if (up) base += C / 2;
+  }
+  // remaining offsets: plain butterfly sums of the values each lane keeps
+  constexpr int CF = NV >> S;
+#pragma unroll
+  for (int s = S; s < 5; ++s) {
+    const int off = 16 >> s;
+#pragma unroll
+    for (int i = 0; i < CF; ++i) v[i] += __shfl_xor_sync(0xffffffffu, v[i], off);
+  }
+  if ((lane & ((1 << (5 - S)) - 1)) == 0) {
+#pragma unroll
+    for (int i = 0; i < CF; ++i) out[base + i] = v[i];
+  }
 }
 
 // ---------------------------------------------------------------- top-k
 
-// One warp selects the k largest of lg[0, E) (ties -> lowest index) in
-// descending order, the renormalised softmax weights over them, and the gap
-// between the k-th and (k+1)-th logit. E <= 1024, k <= 32.
-__device__ __forceinline__ void warp_topk(const float* lg, int E, int k, int* ids, float* w,
-                                          float* margin_out) {
+// One warp: the kk largest keys among keys[0, n) (n <= 1024), ties to the
+// lowest position; positions in descending key order -> out_pos[0, kk).
+__device__ __forceinline__ void warp_select(const uint32_t* keys, int n, int kk, int* out_pos) {
   const int lane = threadIdx.x & 31;
-  const int per = (E + 31) >> 5;
-  const int lo = lane * per, hi = min(E, lo + per);
+  const int per = (n + 31) >> 5;
+  const int lo = min(n, lane * per), hi = min(n, lo + per);
   uint32_t taken = 0, bk = 0;
   int bi = -1;
   auto rescan = [&]() {
@@ -53,696 +129,977 @@ __device__ __forceinline__ void warp_topk(const float* lg, int E, int k, int* id
     bi = -1;
     for (int i = lo; i < hi; ++i) {
       if ((taken >> (i - lo)) & 1u) continue;
-      const uint32_t kk = float_key(lg[i]);
-      if (bi < 0 || kk > bk) { bk = kk; bi = i; }
+      const uint32_t kv = keys[i];
+      if (bi < 0 || kv > bk) { bk = kv; bi = i; }
     }
   };
   rescan();
-  float l0 = 0.f, lk = 0.f, mine = 0.f, margin = INFINITY;
-  const int rounds = (k < E) ? k + 1 : k;
-  for (int r = 0; r < rounds; ++r) {
+  for (int r = 0; r < kk; ++r) {
     const uint32_t m = __reduce_max_sync(0xffffffffu, bi >= 0 ? bk : 0u);
     const uint32_t ball = __ballot_sync(0xffffffffu, bi >= 0 && bk == m);
     const int win = __ffs(ball) - 1;
-    const int idx = __shfl_sync(0xffffffffu, bi, win);
-    const float val = key_float(m);
-    if (r < k) {
-      if (lane == 0) ids[r] = idx;
-      if (lane == r) mine = val;
-      if (r == 0) l0 = val;
-      if (r == k - 1) lk = val;
-    } else {
-      margin = lk - val;
-    }
+    const int pos = __shfl_sync(0xffffffffu, bi, win);
+    if (lane == 0) out_pos[r] = pos;
     if (lane == win) {
-      taken |= 1u << (idx - lo);
+      taken |= 1u << (pos - lo);
       rescan();
     }
   }
-  const float e = (lane < k) ? expf(mine - l0) : 0.f;
+}
+
+// Renormalised softmax weights over the chosen logits l[0..k) (l[0] largest).
+__device__ __forceinline__ void warp_weights(const float* l, int k, float* w) {
+  const int lane = threadIdx.x & 31;
+  const float e = (lane < k) ? expf(l[lane] - l[0]) : 0.f;
   const float s = warp_sum(e);
   if (lane < k) w[lane] = e / s;
-  if (lane == 0 && margin_out != nullptr) *margin_out = margin;
-}
-
-// ---------------------------------------------------------------- job compute
-
-// Gate/up dot products of `n` channels of bf16 rows for the tokens in `mask`.
-// Row (ch, mat) starts at stage + ch*ch_stride + mat*mat_stride (mat 0 = gate,
-// 1 = up). dots[(2*ch + mat)*BMAX + b].
-template <int BMAX>
-__device__ __forceinline__ void dots_bf16(const uint8_t* stage, int n, int ch_stride, int mat_stride,
-                                          const uint4* xs4, int H8, uint32_t mask, float* dots) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int pidx = warp; pidx < 2 * n; pidx += kWarps) {
-    const int ch = pidx >> 1, mat = pidx & 1;
-    const uint4* row = reinterpret_cast<const uint4*>(stage + ch * ch_stride + mat * mat_stride);
-    float part[BMAX];
-#pragma unroll
-    for (int b = 0; b < BMAX; ++b) part[b] = 0.f;
-    for (int v = lane; v < H8; v += 32) {
-      const uint4 wv = row[v];
-#pragma unroll
-      for (int b = 0; b < BMAX; ++b)
-        if ((mask >> b) & 1u) part[b] += dot8_bf16(wv, xs4[b * H8 + v]);
-    }
-#pragma unroll
-    for (int b = 0; b < BMAX; ++b)
-      if ((mask >> b) & 1u) {
-        const float s = warp_sum(part[b]);
-        if (lane == 0) dots[pidx * BMAX + b] = s;
-      }
-  }
-}
-
-// int4 gate/up rows: codes [n][H/2] at gc / uc, scales [n][H/64] bf16 at gs / us.
-template <int BMAX>
-__device__ __forceinline__ void dots_int4(const uint8_t* stage, int n, int H, int nch, const uint4* xs4,
-                                          uint32_t mask, float* dots) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int H8 = H >> 3, rowc = H >> 1, rows = H >> 5;  // code bytes / scale bytes per row
-  const int gc = 0, uc = nch * rowc, gs = 3 * nch * rowc, us = gs + nch * rows;
-  for (int pidx = warp; pidx < 2 * n; pidx += kWarps) {
-    const int ch = pidx >> 1, mat = pidx & 1;
-    const uint4* codes = reinterpret_cast<const uint4*>(stage + (mat ? uc : gc) + ch * rowc);
-    const uint16_t* sc = reinterpret_cast<const uint16_t*>(stage + (mat ? us : gs) + ch * rows);
-    float part[BMAX];
-#pragma unroll
-    for (int b = 0; b < BMAX; ++b) part[b] = 0.f;
-    for (int v = lane; v < (H >> 5); v += 32) {  // 16-byte code vector = 32 elements
-      const uint4 cv = codes[v];
-      const float s = bf16_to_f(sc[v >> 1]);
-      float q[4][8];
-      int4x8_to_f(cv.x, q[0]);
-      int4x8_to_f(cv.y, q[1]);
-      int4x8_to_f(cv.z, q[2]);
-      int4x8_to_f(cv.w, q[3]);
-#pragma unroll
-      for (int b = 0; b < BMAX; ++b)
-        if ((mask >> b) & 1u) {
-          float a = 0.f;
-#pragma unroll
-          for (int m = 0; m < 4; ++m) {
-            float xf[8];
-            unpack8(xs4[b * H8 + 4 * v + m], xf);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) a = fmaf(q[m][j], xf[j], a);
-          }
-          part[b] = fmaf(s, a, part[b]);
-        }
-    }
-#pragma unroll
-    for (int b = 0; b < BMAX; ++b)
-      if ((mask >> b) & 1u) {
-        const float s = warp_sum(part[b]);
-        if (lane == 0) dots[pidx * BMAX + b] = s;
-      }
-  }
-}
-
-// h[ch][b] = w_b * silu(g) * u for tokens in mask, 0 otherwise.
-template <int BMAX>
-__device__ __forceinline__ void swiglu_h(int n, uint32_t mask, const float* wts, const float* dots, float* hs) {
-  for (int t = threadIdx.x; t < n * BMAX; t += kThreads) {
-    const int ch = t / BMAX, b = t % BMAX;
-    float h = 0.f;
-    if ((mask >> b) & 1u) {
-      const float g = dots[(2 * ch) * BMAX + b], u = dots[(2 * ch + 1) * BMAX + b];
-      h = wts[b] * silu_f(g) * u;
-    }
-    hs[ch * BMAX + b] = h;
-  }
-}
-
-// acc[b][0..8) += sum_ch h[ch][b] * D^T[ch][8v .. 8v+8) for bf16 down rows.
-template <int BMAX>
-__device__ __forceinline__ void down_bf16(const uint8_t* stage, int n, int ch_stride, int down_off, int H8,
-                                          uint32_t mask, const float* hs, float (&acc)[BMAX][8]) {
-  const int v = threadIdx.x;
-  if (v >= H8) return;
-  for (int ch = 0; ch < n; ++ch) {
-    const uint4 dv = reinterpret_cast<const uint4*>(stage + down_off + ch * ch_stride)[v];
-    float d[8];
-    unpack8(dv, d);
-#pragma unroll
-    for (int b = 0; b < BMAX; ++b)
-      if ((mask >> b) & 1u) {
-        const float h = hs[ch * BMAX + b];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc[b][i] = fmaf(h, d[i], acc[b][i]);
-      }
-  }
-}
-
-// int4 down rows: codes [n][H/2] at dc, one scale row [H] bf16 at ds (the job
-// lies inside one 64-channel group, so the scale factors out of the job).
-template <int BMAX>
-__device__ __forceinline__ void down_int4(const uint8_t* stage, int n, int H, int nch, uint32_t mask,
-                                          const float* hs, float (&acc)[BMAX][8]) {
-  const int v = threadIdx.x, H8 = H >> 3, rowc = H >> 1;
-  if (v >= H8) return;
-  const int dc = 2 * nch * rowc, ds = 3 * nch * rowc + 2 * nch * (H >> 5);
-  float s[8];
-  unpack8(reinterpret_cast<const uint4*>(stage + ds)[v], s);
-  float inner[BMAX][8];
-#pragma unroll
-  for (int b = 0; b < BMAX; ++b)
-#pragma unroll
-    for (int i = 0; i < 8; ++i) inner[b][i] = 0.f;
-  for (int ch = 0; ch < n; ++ch) {
-    const uint32_t wv = reinterpret_cast<const uint32_t*>(stage + dc + ch * rowc)[v];
-    float q[8];
-    int4x8_to_f(wv, q);
-#pragma unroll
-    for (int b = 0; b < BMAX; ++b)
-      if ((mask >> b) & 1u) {
-        const float h = hs[ch * BMAX + b];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) inner[b][i] = fmaf(h, q[i], inner[b][i]);
-      }
-  }
-#pragma unroll
-  for (int b = 0; b < BMAX; ++b)
-    if ((mask >> b) & 1u)
-#pragma unroll
-      for (int i = 0; i < 8; ++i) acc[b][i] = fmaf(s[i], inner[b][i], acc[b][i]);
 }
 
 // ---------------------------------------------------------------- the kernel
 
-template <int BMAX, int WT, int LAYOUT>
-__global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_constant__ DecodeParams p) {
+template <int MODE, int BMAX, int WT, int LAYOUT, int NCH, int HV>
+__global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_constant__ DecodeParams p) {
+  constexpr int NR = 2 * NCH;        // dot rows per job (gate+up rows; router rows)
+  constexpr int NV = NR * BMAX;      // values reduced per job
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ RouteSmem rs;
-  __shared__ int route_ready_layer_s;
-  __shared__ int bad_s, okw_s;
-  __shared__ unsigned long long target_s;
+  __shared__ int route_ready_s, abort_s, bad_s, okw_s;
+  __shared__ long long jp_s, jc_s;
+  __shared__ float dotbuf[16][NV];
+  __shared__ float hbuf[kWarps][NCH * BMAX];
+  __shared__ uint32_t cand_key[kWarps * kMaxK];
+  __shared__ int cand_idx[kWarps * kMaxK];
+  __shared__ int sel_pos[kWarps][kMaxK];
+  __shared__ float sel_l[kWarps][kMaxK];
 
   const int tid = threadIdx.x;
-  const int warp = tid >> 5;
+  const int warp = tid >> 5, lane = tid & 31;
   const int G = gridDim.x, cta = blockIdx.x;
   const int B = p.B, H = p.H, H8 = H >> 3, E = p.E, I = p.I, k = p.k;
-  const int rowb = 2 * H;  // bf16 row bytes
+  const int rowb = 2 * H;
   uint8_t* ring = smem;
-  uint16_t* xs = reinterpret_cast<uint16_t*>(smem + p.off_x);
+  uint16_t* xs = reinterpret_cast<uint16_t*>(smem + p.off_x);  // residual stream x
   const uint4* xs4 = reinterpret_cast<const uint4*>(xs);
+  // MoE input u: RMS-normalised x with the pre-norm, else x itself
+  uint16_t* us = (MODE == MODE_LAYERS && p.pre_norm) ? reinterpret_cast<uint16_t*>(smem + p.off_u) : xs;
+  const uint4* us4 = reinterpret_cast<const uint4*>(us);
   float* lg = reinterpret_cast<float*>(smem + p.off_lg);
-  float* dots = reinterpret_cast<float*>(smem + p.off_dots);
-  float* hs = reinterpret_cast<float*>(smem + p.off_hs);
   uint32_t* keys = reinterpret_cast<uint32_t*>(smem + p.off_keys);
   int* kept = reinterpret_cast<int*>(smem + p.off_kept);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.off_bar);
+  uint64_t* empty = full + p.nstages;
+  uint64_t* hready = empty + p.nstages;
   WsControl* ctl = p.ctl;
 
   if (tid == 0) {
-    for (int s = 0; s < p.nstages; ++s) mbar_init(&full[s], 1);
+    for (int s = 0; s < p.nstages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kWarps);
+      mbar_init(&hready[s], kWarps);
+    }
     fence_mbar_init();
-    route_ready_layer_s = -1;
+    route_ready_s = -1;
+    abort_s = 0;
+    jp_s = 0;
+    jc_s = 0;
   }
-  // x_0 -> shared memory (and x_hist[0])
-  for (int i = tid; i < B * H8; i += kThreads) {
-    const uint4 v = reinterpret_cast<const uint4*>(p.x_in)[i];
-    reinterpret_cast<uint4*>(xs)[i] = v;
-  }
+  for (int i = tid; i < B * H8; i += kCtaThreads)
+    reinterpret_cast<uint4*>(xs)[i] = reinterpret_cast<const uint4*>(p.x_in)[i];
   if (p.x_hist != nullptr) {
     const long long n = (long long)B * H8;
-    for (long long i = cta * n / G + tid; i < (cta + 1) * n / G; i += kThreads)
+    for (long long i = cta * n / G + tid; i < (cta + 1) * n / G; i += kCtaThreads)
       reinterpret_cast<uint4*>(p.x_hist)[i] = reinterpret_cast<const uint4*>(p.x_in)[i];
   }
   __syncthreads();
 
-  // ------------------------------------------------------------ producer (thread 0)
-  JobCursor pcur;
-  long long jp = 0;  // jobs issued
-  long long jc = 0;  // jobs consumed
-  uint64_t pol = 0;
-  if (tid == 0) {
-    pol = policy_evict_first();
-    pcur.begin_layer(p, 0);
-  }
-
+  // Job sequence, shared by producer and consumers.
   auto next_job = [&](JobCursor& cur, Job& j, int ready_layer) -> bool {
     for (;;) {
       if (cur.layer >= p.L) { j.type = JOB_END; return true; }
       if (cur.type == JOB_ROUTER) {
-        const int n = (int)llmin(p.rows_per_job, cur.t1 - cur.t);
-        j = Job{JOB_ROUTER, cur.layer, 0, (int)cur.t, n};
+        const int n = min(p.rows_per_job, cur.t1 - cur.t);
+        j = Job{JOB_ROUTER, cur.layer, 0, cur.t, n};
         cur.t += n;
         if (cur.t >= cur.t1) { cur.type = JOB_SHARED; cur.set_range(p); }
         return true;
       }
       if (cur.type == JOB_SHARED) {
-        const int c = (int)cur.t;
-        const int n = (int)llmin(p.nch_sh - c % p.nch_sh, cur.t1 - cur.t);
-        j = Job{JOB_SHARED, cur.layer, 0, c, n};
+        const int n = min(NCH, cur.t1 - cur.t);
+        j = Job{JOB_SHARED, cur.layer, 0, cur.t, n};
         cur.t += n;
         if (cur.t >= cur.t1) { cur.type = JOB_ROUTED; cur.t = -1; cur.t1 = -1; }
         return true;
       }
-      // routed
       if (cur.t1 < 0) {
-        if (ready_layer != cur.layer) return false;
-        cur.set_routed(LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR ? (long long)rs.ncand : (long long)rs.U * I);
+        if (ready_layer < cur.layer) return false;
+        cur.set_routed(LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR ? rs.ncand : rs.U * I, I);
       }
       if (cur.t >= cur.t1) { cur.begin_layer(p, cur.layer + 1); continue; }
       if (LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR) {
-        const int pos = (int)cur.t;
+        const int pos = cur.t;
         const int j0 = kept[pos];
         int n = 1;
-        while (n < p.nch && cur.t + n < cur.t1 && kept[pos + n] == j0 + n && (j0 + n) % I != 0) ++n;
+        while (n < NCH && cur.t + n < cur.t1 && kept[pos + n] == j0 + n && (j0 + n) % I != 0) ++n;
         j = Job{JOB_ROUTED, cur.layer, pos, j0, n};
         cur.t += n;
       } else {
-        const int u = (int)(cur.t / I), c = (int)(cur.t % I);
-        const int n = (int)llmin(min(p.nch - c % p.nch, I - c), cur.t1 - cur.t);
-        j = Job{JOB_ROUTED, cur.layer, u, c, n};
+        int n;
+        if (WT == MOE_W_INT4_G64) {
+          // int4 jobs stay inside one 64-channel scale group: cut at multiples of NCH
+          n = min(min(NCH - (cur.c & (NCH - 1)), I - cur.c), cur.t1 - cur.t);
+        } else {
+          // bf16 jobs may run on into the next expert (two segments at most)
+          n = min(min(NCH, cur.t1 - cur.t), 2 * I - cur.c);
+        }
+        j = Job{JOB_ROUTED, cur.layer, cur.u, cur.c, n};
         cur.t += n;
+        cur.c += n;
+        while (cur.c >= I) { cur.c -= I; ++cur.u; }
       }
       return true;
     }
   };
 
-  auto issue = [&](const Job& j, int slot) {
-    uint64_t* bar = &full[slot];
-    uint8_t* dst = ring + (size_t)slot * p.stage_bytes;
-    const LayerW& Lw = p.layer[j.layer];
-    if (j.type == JOB_ROUTER) {
-      const uint32_t bytes = (uint32_t)j.n * rowb;
-      mbar_expect_tx(bar, bytes);
-      bulk_g2s(dst, Lw.router + (size_t)j.c0 * rowb, bytes, bar, pol);
-    } else if (j.type == JOB_SHARED) {
-      const uint32_t bytes = (uint32_t)j.n * rowb;
-      mbar_expect_tx(bar, 3 * bytes);
-      const size_t off = (size_t)j.c0 * rowb;
-      bulk_g2s(dst, Lw.sh_gate + off, bytes, bar, pol);
-      bulk_g2s(dst + p.nch_sh * rowb, Lw.sh_up + off, bytes, bar, pol);
-      bulk_g2s(dst + 2 * p.nch_sh * rowb, Lw.sh_down + off, bytes, bar, pol);
-    } else if (LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR) {
-      const uint32_t bytes = (uint32_t)j.n * 3 * rowb;
-      mbar_expect_tx(bar, bytes);
-      bulk_g2s(dst, Lw.gate + (size_t)j.c0 * 3 * rowb, bytes, bar, pol);
-    } else if (WT == MOE_W_BF16) {
-      const int e = rs.unit_e[j.u];
-      const uint32_t bytes = (uint32_t)j.n * rowb;
-      const size_t off = ((size_t)e * I + j.c0) * rowb;
-      mbar_expect_tx(bar, 3 * bytes);
-      bulk_g2s(dst, Lw.gate + off, bytes, bar, pol);
-      bulk_g2s(dst + p.nch * rowb, Lw.up + off, bytes, bar, pol);
-      bulk_g2s(dst + 2 * p.nch * rowb, Lw.down + off, bytes, bar, pol);
-    } else {  // int4 planar
-      const int e = rs.unit_e[j.u];
-      const int rowc = H >> 1, rows = H >> 5;
-      const uint32_t cb = (uint32_t)j.n * rowc, sb = (uint32_t)j.n * rows;
-      const size_t offc = ((size_t)e * I + j.c0) * rowc, offs = ((size_t)e * I + j.c0) * rows;
-      const size_t offd = ((size_t)e * (I >> 6) + (j.c0 >> 6)) * rowb;
-      mbar_expect_tx(bar, 3 * cb + 2 * sb + rowb);
-      bulk_g2s(dst, Lw.gate + offc, cb, bar, pol);
-      bulk_g2s(dst + p.nch * rowc, Lw.up + offc, cb, bar, pol);
-      bulk_g2s(dst + 2 * p.nch * rowc, Lw.down + offc, cb, bar, pol);
-      bulk_g2s(dst + 3 * p.nch * rowc, Lw.gate_s + offs, sb, bar, pol);
-      bulk_g2s(dst + 3 * p.nch * rowc + p.nch * rows, Lw.up_s + offs, sb, bar, pol);
-      bulk_g2s(dst + 3 * p.nch * rowc + 2 * p.nch * rows, Lw.down_s + offd, rowb, bar, pol);
-    }
-  };
-
-  // Thread 0: issue every job that is known and has a free stage.
-  auto produce = [&]() {
-    if (tid != 0) return;
-    const int ready = route_ready_layer_s;
-    while (jp < jc + p.nstages) {
-      JobCursor save = pcur;
-      Job j;
-      if (!next_job(pcur, j, ready)) { pcur = save; break; }
-      if (j.type == JOB_END) { pcur = save; break; }
-      issue(j, (int)(jp % p.nstages));
-      ++jp;
-    }
-  };
-
-  // ------------------------------------------------------------ consumer
-  JobCursor ccur;
-  ccur.begin_layer(p, 0);
-  float acc[BMAX][8];
-#pragma unroll
-  for (int b = 0; b < BMAX; ++b)
-#pragma unroll
-    for (int i = 0; i < 8; ++i) acc[b][i] = 0.f;
-
-  const float ones[kMaxB] = {1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f};
-  const uint32_t all_tokens = (B >= 32) ? 0xffffffffu : ((1u << B) - 1u);
-
-  // Error path: before leaving, wait (bounded) for every copy this CTA has in
-  // flight so no bulk copy lands in shared memory after the CTA exits.
-  auto drain = [&]() {
-    if (tid == 0)
-      for (long long q = jc; q < jp; ++q) mbar_wait(&full[q % p.nstages], (uint32_t)((q / p.nstages) & 1));
-    __syncthreads();
-  };
-
-  // Consume one job: wait for its stage, compute, release the stage.
-  // Returns false on a timeout (status already recorded).
-  auto consume = [&](const Job& j) -> bool {
-    const int slot = (int)(jc % p.nstages);
-    const uint32_t parity = (uint32_t)((jc / p.nstages) & 1);
-    const uint8_t* st = ring + (size_t)slot * p.stage_bytes;
-    const bool ok = mbar_wait(&full[slot], parity);
-    if (j.type == JOB_ROUTER) {
-      if (ok) {
-        for (int r = warp; r < j.n; r += kWarps) {
-          const uint4* row = reinterpret_cast<const uint4*>(st + r * rowb);
-          float part[BMAX];
-#pragma unroll
-          for (int b = 0; b < BMAX; ++b) part[b] = 0.f;
-          for (int v = (tid & 31); v < H8; v += 32) {
-            const uint4 wv = row[v];
-#pragma unroll
-            for (int b = 0; b < BMAX; ++b)
-              if (b < B) part[b] += dot8_bf16(wv, xs4[b * H8 + v]);
+  // ================================================================ producer
+  if (warp == kWarps) {
+    if (lane == 0) {
+      const uint64_t pol = policy_evict_first();
+      JobCursor pc;
+      pc.begin_layer(p, 0);
+      long long jp = 0;
+      int pslot = 0;
+      uint32_t pph = 0;
+      for (;;) {
+        Job j;
+        JobCursor save = pc;
+        if (!next_job(pc, j, ld_acquire_cta(&route_ready_s))) {
+          // routed jobs of this layer: wait until the consumers publish routing
+          pc = save;
+          const long long t0 = clock64();
+          while (ld_acquire_cta(&route_ready_s) < pc.layer) {
+            if (ld_acquire_cta(&abort_s) || clock64() - t0 > kWaitBudgetCycles) goto producer_done;
+            __nanosleep(64);
           }
+          continue;
+        }
+        if (j.type == JOB_END) break;
+        const int slot = pslot;
+        if (jp >= p.nstages) {
+          const uint32_t par = pph ^ 1u;
+          const long long t0 = clock64();
+          while (!mbar_try_wait_sleep(&empty[slot], par, 20000)) {
+            if (ld_acquire_cta(&abort_s) || clock64() - t0 > kWaitBudgetCycles) goto producer_done;
+          }
+        }
+        uint64_t* bar = &full[slot];
+        uint8_t* dst = ring + (size_t)slot * p.stage_bytes;
+        const LayerW& Lw = p.layer[j.layer];
+        if (j.type == JOB_ROUTER) {
+          const uint32_t bytes = (uint32_t)j.n * rowb;
+          mbar_expect_tx(bar, bytes);
+          bulk_g2s(dst, Lw.router + (size_t)j.c0 * rowb, bytes, bar, pol);
+        } else if (j.type == JOB_SHARED) {
+          const uint32_t bytes = (uint32_t)j.n * rowb;
+          const size_t off = (size_t)j.c0 * rowb;
+          mbar_expect_tx(bar, 3 * bytes);
+          bulk_g2s(dst, Lw.sh_gate + off, bytes, bar, pol);
+          bulk_g2s(dst + NCH * rowb, Lw.sh_up + off, bytes, bar, pol);
+          bulk_g2s(dst + 2 * NCH * rowb, Lw.sh_down + off, bytes, bar, pol);
+        } else if (LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR) {
+          const uint32_t bytes = (uint32_t)j.n * 3 * rowb;
+          mbar_expect_tx(bar, bytes);
+          bulk_g2s(dst, Lw.gate + (size_t)j.c0 * 3 * rowb, bytes, bar, pol);
+        } else if (WT == MOE_W_BF16) {
+          const int n1 = min(j.n, I - j.c0);
+          mbar_expect_tx(bar, 3u * (uint32_t)j.n * rowb);
+          for (int sg = 0; sg < 2; ++sg) {
+            const int ns = sg ? j.n - n1 : n1;
+            if (ns <= 0) break;
+            const int e = rs.unit_e[j.u + sg];
+            const uint32_t bytes = (uint32_t)ns * rowb;
+            const size_t off = ((size_t)e * I + (sg ? 0 : j.c0)) * rowb;
+            uint8_t* d0 = dst + (sg ? n1 : 0) * rowb;
+            bulk_g2s(d0, Lw.gate + off, bytes, bar, pol);
+            bulk_g2s(d0 + NCH * rowb, Lw.up + off, bytes, bar, pol);
+            bulk_g2s(d0 + 2 * NCH * rowb, Lw.down + off, bytes, bar, pol);
+          }
+        } else {
+          const int e = rs.unit_e[j.u];
+          const int rowc = H >> 1, rows = H >> 5;
+          const uint32_t cb = (uint32_t)j.n * rowc, sb = (uint32_t)j.n * rows;
+          const size_t offc = ((size_t)e * I + j.c0) * rowc, offs = ((size_t)e * I + j.c0) * rows;
+          const size_t offd = ((size_t)e * (I >> 6) + (j.c0 >> 6)) * rowb;
+          mbar_expect_tx(bar, 3 * cb + 2 * sb + rowb);
+          bulk_g2s(dst, Lw.gate + offc, cb, bar, pol);
+          bulk_g2s(dst + NCH * rowc, Lw.up + offc, cb, bar, pol);
+          bulk_g2s(dst + 2 * NCH * rowc, Lw.down + offc, cb, bar, pol);
+          bulk_g2s(dst + 3 * NCH * rowc, Lw.gate_s + offs, sb, bar, pol);
+          bulk_g2s(dst + 3 * NCH * rowc + NCH * rows, Lw.up_s + offs, sb, bar, pol);
+          bulk_g2s(dst + 3 * NCH * rowc + 2 * NCH * rows, Lw.down_s + offd, rowb, bar, pol);
+        }
+        ++jp;
+        if (++pslot == p.nstages) { pslot = 0; pph ^= 1u; }
+        *(volatile long long*)&jp_s = jp;
+      }
+    producer_done:;
+    }
+    __syncwarp();
+  } else {
+    // ============================================================== consumers
+    JobCursor ccur;
+    ccur.begin_layer(p, 0);
+    int cslot = 0;          // stage of the next job
+    uint32_t cph = 0;       // its phase parity
+    long long jc = 0;       // jobs consumed
+    unsigned long long bar_base = 0, nbar = 0;
+    if (tid == 0) bar_base = (ld_relaxed_gpu(&ctl->bar) / (unsigned long long)G) * (unsigned long long)G;
+
+    float acc[BMAX][8];
 #pragma unroll
-          for (int b = 0; b < BMAX; ++b)
-            if (b < B) {
-              const float s = warp_sum(part[b]);
-              if ((tid & 31) == 0) p.logits[b * E + j.c0 + r] = s;
+    for (int b = 0; b < BMAX; ++b)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[b][i] = 0.f;
+    const int H8c = H8;
+    const bool has_v = tid < H8;
+    const uint32_t all_tokens = (1u << B) - 1u;
+    // tensor-core dots (B = 1, H = 2048): x fragments for the 8 segments
+    constexpr bool kMmaDots = (BMAX == 1 && HV == 8);
+    uint32_t xf_frag[kMmaDots ? 8 : 1][4];
+    auto load_xfrag = [&]() {
+      if constexpr (kMmaDots) {
+#pragma unroll
+        for (int t = 0; t < 8; ++t) x_frag(us + 256 * t, lane, xf_frag[t]);
+      }
+    };
+
+    auto arrive_grid = [&]() -> unsigned long long {  // thread 0 only
+      red_release_gpu(&ctl->bar, 1ull);
+      ++nbar;
+      return bar_base + nbar * (unsigned long long)G;
+    };
+    auto wait_grid = [&](unsigned long long target) -> bool {  // thread 0 only
+      if (ld_acquire_gpu(&ctl->bar) >= target) return true;
+      const long long t0 = clock64();
+      while (ld_acquire_gpu(&ctl->bar) < target)
+        if (clock64() - t0 > kWaitBudgetCycles) return false;
+      return true;
+    };
+    auto grid_sync = [&]() -> bool {
+      cbar();
+      if (tid == 0) okw_s = wait_grid(arrive_grid()) ? 1 : 0;
+      cbar();
+      return okw_s != 0;
+    };
+    // bounded mbarrier wait that gives up at once after an abort
+    auto wait_mb = [&](uint64_t* bar, uint32_t parity) -> bool {
+      if (mbar_try_wait_sleep(bar, parity, 20000)) return true;
+      const long long t0 = clock64();
+      while (!mbar_try_wait_sleep(bar, parity, 20000)) {
+        if (*(volatile int*)&abort_s || clock64() - t0 > kWaitBudgetCycles) return false;
+      }
+      return true;
+    };
+
+    // Dot products of RPW rows (one warp's share of a job) with token b's x,
+    // summed over the warp. Lane takes vectors v = i*32 + lane of H; HV =
+    // H/256 vectors per lane when H is a multiple of 256 (no guards, x loaded
+    // once for all rows), else a guarded generic loop. int4 rows carry one
+    // bf16 scale per 64 elements (sc[r][v >> 3]).
+    auto rows_dot = [&](const uint8_t* const* rowp, const uint16_t* const* scp, int nrows, int b, bool int4row,
+                        float* out) {
+      constexpr int RPW = NCH * 2 / kWarps > 0 ? NCH * 2 / kWarps : 1;
+      float s8[RPW][8];
+#pragma unroll
+      for (int r = 0; r < RPW; ++r)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) s8[r][e] = 0.f;
+      const uint4* xb = us4 + b * H8c;
+      if constexpr (kMmaDots) {
+        if (!int4row) {
+          float d0[RPW][4], d1[RPW][4];
+#pragma unroll
+          for (int r = 0; r < RPW; ++r)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) { d0[r][i] = 0.f; d1[r][i] = 0.f; }
+#pragma unroll
+          for (int t = 0; t < 8; ++t)
+#pragma unroll
+            for (int r = 0; r < RPW; ++r)
+              if (r < nrows) {
+                uint32_t a0, a1, a2, a3;
+                ldmatrix_x4(smem_u32(rowp[r]) + 512 * t + 16 * lane, a0, a1, a2, a3);
+                mma_bf16_16816(d0[r], a0, a1, a2, a3, xf_frag[t][0], xf_frag[t][1]);
+                mma_bf16_16816(d1[r], a0, a1, a2, a3, xf_frag[t][2], xf_frag[t][3]);
+              }
+#pragma unroll
+          for (int r = 0; r < RPW; ++r) out[r] = warp_sum(diag_part(d0[r], d1[r], lane));
+          return;
+        }
+      }
+      if (HV > 0) {
+#pragma unroll
+        for (int i = 0; i < (HV > 0 ? HV : 1); ++i) {
+          const int v = i * 32 + lane;
+          float xf[8];
+          unpack8(xb[v], xf);
+#pragma unroll
+          for (int r = 0; r < RPW; ++r)
+            if (r < nrows) {
+              float wf[8];
+              if (!int4row) {
+                unpack8(reinterpret_cast<const uint4*>(rowp[r])[v], wf);
+              } else {
+                int4x8_to_f(reinterpret_cast<const uint32_t*>(rowp[r])[v], wf);
+                const float sv = bf16_to_f(scp[r][v >> 3]);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) wf[e] *= sv;
+              }
+#pragma unroll
+              for (int e = 0; e < 8; ++e) s8[r][e] = fmaf(wf[e], xf[e], s8[r][e]);
+            }
+        }
+      } else {
+        for (int v = lane; v < H8c; v += 32) {
+          float xf[8];
+          unpack8(xb[v], xf);
+#pragma unroll
+          for (int r = 0; r < RPW; ++r)
+            if (r < nrows) {
+              float wf[8];
+              if (!int4row) unpack8(reinterpret_cast<const uint4*>(rowp[r])[v], wf);
+              else {
+                int4x8_to_f(reinterpret_cast<const uint32_t*>(rowp[r])[v], wf);
+                const float sv = bf16_to_f(scp[r][v >> 3]);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) wf[e] *= sv;
+              }
+#pragma unroll
+              for (int e = 0; e < 8; ++e) s8[r][e] = fmaf(wf[e], xf[e], s8[r][e]);
             }
         }
       }
-      if (__syncthreads_or(!ok)) { set_status(ctl, kStatusTimeout); return false; }
-    } else {
-      uint32_t mask;
-      const float* wts;
-      int nstride;
-      if (j.type == JOB_SHARED) {
-        mask = all_tokens;
-        wts = ones;
-        nstride = p.nch_sh;
-      } else if (LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR) {
-        mask = 1u;
+#pragma unroll
+      for (int r = 0; r < RPW; ++r) {
+        const float t = ((s8[r][0] + s8[r][1]) + (s8[r][2] + s8[r][3])) + ((s8[r][4] + s8[r][5]) + (s8[r][6] + s8[r][7]));
+        out[r] = warp_sum(t);
+      }
+    };
+
+    // ---- one job, per warp: its dot rows, then (after all warps' dots) the
+    // SwiGLU activations and this thread's H-slice of the down projection
+    auto consume = [&](const Job& j) -> bool {
+      constexpr int RPW = NCH * 2 / kWarps > 0 ? NCH * 2 / kWarps : 1;
+      const int slot = cslot;
+      const uint32_t ph = cph;
+      const uint8_t* st = ring + (size_t)slot * p.stage_bytes;
+      bool ok = wait_mb(&full[slot], ph);
+      // token masks and router weights of the (at most two) segments
+      uint32_t mask0, mask1 = 0u;
+      const float* wts0 = nullptr;
+      const float* wts1 = nullptr;
+      int n1 = j.n;
+      if (j.type == JOB_ROUTER || j.type == JOB_SHARED) mask0 = all_tokens;
+      else if (LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR) {
+        mask0 = 1u;
         const int e = j.c0 / I;
         int u = 0;
         while (u < rs.U - 1 && rs.unit_e[u] != e) ++u;
-        wts = &rs.wmap_unit[u];
-        nstride = 0;
+        wts0 = &rs.unit_w[u][0];
       } else {
-        mask = rs.unit_mask[j.u];
-        wts = rs.unit_w[j.u];
-        nstride = p.nch;
-      }
-      const bool shared_or_bf16 = (j.type == JOB_SHARED) || (WT == MOE_W_BF16);
-      if (ok) {
-        if (LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR && j.type != JOB_SHARED)
-          dots_bf16<BMAX>(st, j.n, 3 * rowb, rowb, xs4, H8, mask, dots);
-        else if (shared_or_bf16)
-          dots_bf16<BMAX>(st, j.n, rowb, nstride * rowb, xs4, H8, mask, dots);
-        else
-          dots_int4<BMAX>(st, j.n, H, p.nch, xs4, mask, dots);
-      }
-      if (__syncthreads_or(!ok)) { set_status(ctl, kStatusTimeout); return false; }
-      swiglu_h<BMAX>(j.n, mask, wts, dots, hs);
-      __syncthreads();
-      if (LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR && j.type != JOB_SHARED)
-        down_bf16<BMAX>(st, j.n, 3 * rowb, 2 * rowb, H8, mask, hs, acc);
-      else if (shared_or_bf16)
-        down_bf16<BMAX>(st, j.n, rowb, 2 * nstride * rowb, H8, mask, hs, acc);
-      else
-        down_int4<BMAX>(st, j.n, H, p.nch, mask, hs, acc);
-      __syncthreads();
-    }
-    ++jc;
-    produce();
-    return true;
-  };
-
-  // Build the routed units (touched experts, ascending) from rs.ids / rs.w.
-  // Returns false if ids were out of range or repeated within a token.
-  auto build_units = [&]() -> bool {
-    const int nw = (E + 31) >> 5;
-    if (tid == 0) bad_s = 0;
-    for (int i = tid; i < nw; i += kThreads) rs.bitmap[i] = 0u;
-    __syncthreads();
-    for (int t = tid; t < B * k; t += kThreads) {
-      const int e = rs.ids[t / k][t % k];
-      if (e < 0 || e >= E) bad_s = 1;
-      else atomicOr(&rs.bitmap[e >> 5], 1u << (e & 31));
-    }
-    __syncthreads();
-    if (warp == 0) {
-      const int lane = tid & 31;
-      const int c = lane < nw ? __popc(rs.bitmap[lane]) : 0;
-      int inc = c;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int t = __shfl_up_sync(0xffffffffu, inc, o);
-        if (lane >= o) inc += t;
-      }
-      if (lane < nw) rs.rank_base[lane] = inc - c;
-      if (lane == 31) rs.U = inc;
-    }
-    __syncthreads();
-    for (int u = tid; u < rs.U; u += kThreads) {
-      rs.unit_mask[u] = 0u;
-#pragma unroll
-      for (int b = 0; b < kMaxB; ++b) rs.unit_w[u][b] = 0.f;
-    }
-    for (int e = tid; e < E; e += kThreads)
-      if ((rs.bitmap[e >> 5] >> (e & 31)) & 1u)
-        rs.unit_e[rs.rank_base[e >> 5] + __popc(rs.bitmap[e >> 5] & ((1u << (e & 31)) - 1u))] = e;
-    __syncthreads();
-    for (int t = tid; t < B * k; t += kThreads) {
-      const int b = t / k, e = rs.ids[b][t % k];
-      if (e < 0 || e >= E) continue;
-      const int u = rs.rank_base[e >> 5] + __popc(rs.bitmap[e >> 5] & ((1u << (e & 31)) - 1u));
-      const uint32_t old = atomicOr(&rs.unit_mask[u], 1u << b);
-      if (old & (1u << b)) bad_s = 1;
-      else rs.unit_w[u][b] = rs.w[b][t % k];
-    }
-    __syncthreads();
-    return bad_s == 0;
-  };
-
-  // Channel-sparse (B = 1): keep the p.keep best candidates of the routed
-  // units' channels by score; fills kept[] ascending and rs.ncand.
-  auto select_channels = [&](int l) {
-    const int N = rs.U * I;
-    const float* sc = p.layer[l].scores;  // token 0's [E, I] block
-    for (int q = tid; q < N; q += kThreads) {
-      const int u = q / I, c = q - u * I;
-      keys[q] = float_key(__ldg(sc + (size_t)rs.unit_e[u] * I + c));
-    }
-    if (tid < rs.U) {
-      // weight of each unit for token 0
-      rs.wmap_unit[tid] = rs.unit_w[tid][0];
-    }
-    __syncthreads();
-    const int keep = p.keep;
-    uint32_t T = 0;
-    int rank = 0;
-    if (keep > 0 && keep < N) {
-      uint32_t prefix = 0, pmask = 0;
-      rank = keep;
-      for (int shift = 24; shift >= 0; shift -= 8) {
-        rs.hist[tid] = 0u;
-        __syncthreads();
-        for (int q = tid; q < N; q += kThreads) {
-          const uint32_t kk = keys[q];
-          if ((kk & pmask) == prefix) atomicAdd(&rs.hist[(kk >> shift) & 255u], 1u);
+        mask0 = rs.unit_mask[j.u];
+        wts0 = rs.unit_w[j.u];
+        if (WT == MOE_W_BF16) {
+          n1 = min(j.n, I - j.c0);
+          if (n1 < j.n) { mask1 = rs.unit_mask[j.u + 1]; wts1 = rs.unit_w[j.u + 1]; }
         }
-        __syncthreads();
-        if (warp == 0) {
-          const int lane = tid & 31;
-          uint32_t c8[8], loc = 0;
+      }
+      const uint32_t mask_any = mask0 | mask1;
+      int ch_stride, mat_stride, down_off;
+      if (j.type == JOB_ROUTER) { ch_stride = rowb; mat_stride = 0; down_off = 0; }
+      else if (j.type == JOB_SHARED || (LAYOUT == MOE_LAYOUT_PLANAR && WT == MOE_W_BF16)) {
+        ch_stride = rowb; mat_stride = NCH * rowb; down_off = 2 * NCH * rowb;
+      } else if (LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR) {
+        ch_stride = 3 * rowb; mat_stride = rowb; down_off = 2 * rowb;
+      } else {
+        ch_stride = H >> 1; mat_stride = NCH * (H >> 1); down_off = 2 * NCH * (H >> 1);
+      }
+      const bool int4_rows = (WT == MOE_W_INT4_G64) && (j.type == JOB_ROUTED);
+      const int ndot = (j.type == JOB_ROUTER) ? j.n : 2 * j.n;
+      float* db = dotbuf[slot];
+      // 1. this warp's dot rows: rows warp + 8*i
+      if (ok) {
+        const uint8_t* rowp[RPW];
+        const uint16_t* scp[RPW];
+        int nr = 0;
 #pragma unroll
-          for (int i = 0; i < 8; ++i) { c8[i] = rs.hist[255 - 8 * lane - i]; loc += c8[i]; }
-          uint32_t inc = loc;
+        for (int i = 0; i < RPW; ++i) {
+          const int r = warp + kWarps * i;
+          const int ch = (j.type == JOB_ROUTER) ? r : (r >> 1);
+          const int mat = (j.type == JOB_ROUTER) ? 0 : (r & 1);
+          rowp[i] = st + ch * ch_stride + mat * mat_stride;
+          scp[i] = int4_rows ? reinterpret_cast<const uint16_t*>(st + 3 * NCH * (H >> 1) + (mat * NCH + ch) * (H >> 5))
+                             : nullptr;
+          if (r < ndot) nr = i + 1;
+        }
+        if (nr > 0) {
 #pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t t = __shfl_up_sync(0xffffffffu, inc, o);
-            if (lane >= o) inc += t;
+          for (int b = 0; b < BMAX; ++b)
+            if ((mask_any >> b) & 1u) {
+              float t[RPW];
+              rows_dot(rowp, scp, nr, b, int4_rows, t);
+              if (lane == 0)
+#pragma unroll
+                for (int i = 0; i < RPW; ++i)
+                  if (i < nr) {
+                    const int r = warp + kWarps * i;
+                    if (j.type == JOB_ROUTER) p.logits[b * E + j.c0 + r] = t[i];
+                    else db[r * BMAX + b] = t[i];
+                  }
+            }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&hready[slot]);
+      // 2. SwiGLU activations and the down projection, once every warp's dots are in
+      if (j.type != JOB_ROUTER) {
+        ok = ok && wait_mb(&hready[slot], ph);
+        if (ok) {
+          for (int idx = lane; idx < NCH * BMAX; idx += 32) {
+            const int ch = idx / BMAX, b = idx % BMAX;
+            const uint32_t m = ch < n1 ? mask0 : mask1;
+            const float* wt = ch < n1 ? wts0 : wts1;
+            float h = 0.f;
+            if (ch < j.n && ((m >> b) & 1u)) {
+              const float g = db[(2 * ch) * BMAX + b], u = db[(2 * ch + 1) * BMAX + b];
+              h = (wt ? wt[b] : 1.f) * silu_f(g) * u;
+            }
+            hbuf[warp][idx] = h;
           }
-          const uint32_t exc = inc - loc;
-          const bool hit = exc < (uint32_t)rank && (uint32_t)rank <= inc;
-          if (hit) {
-            uint32_t cum = exc;
+          __syncwarp();
+          if (has_v) {
+            if (!int4_rows) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              if (cum + c8[i] >= (uint32_t)rank) {
-                rs.sel_rank = rank - (int)cum;
-                rs.sel_prefix = (int)(prefix | ((uint32_t)(255 - 8 * lane - i) << shift));
-                break;
-              }
-              cum += c8[i];
+              for (int ch = 0; ch < NCH; ++ch)
+                if (ch < j.n) {
+                  float d[8];
+                  unpack8(reinterpret_cast<const uint4*>(st + down_off + ch * ch_stride)[tid], d);
+                  const uint32_t m = ch < n1 ? mask0 : mask1;
+#pragma unroll
+                  for (int b = 0; b < BMAX; ++b)
+                    if ((m >> b) & 1u) {
+                      const float h = hbuf[warp][ch * BMAX + b];
+#pragma unroll
+                      for (int i = 0; i < 8; ++i) acc[b][i] = fmaf(h, d[i], acc[b][i]);
+                    }
+                }
+            } else {
+              const int rows = H >> 5;
+              float s[8];
+              unpack8(reinterpret_cast<const uint4*>(st + 3 * NCH * (H >> 1) + 2 * NCH * rows)[tid], s);
+              float inner[BMAX][8];
+#pragma unroll
+              for (int b = 0; b < BMAX; ++b)
+#pragma unroll
+                for (int i = 0; i < 8; ++i) inner[b][i] = 0.f;
+#pragma unroll
+              for (int ch = 0; ch < NCH; ++ch)
+                if (ch < j.n) {
+                  float q[8];
+                  int4x8_to_f(reinterpret_cast<const uint32_t*>(st + down_off + ch * ch_stride)[tid], q);
+#pragma unroll
+                  for (int b = 0; b < BMAX; ++b)
+                    if ((mask0 >> b) & 1u) {
+                      const float h = hbuf[warp][ch * BMAX + b];
+#pragma unroll
+                      for (int i = 0; i < 8; ++i) inner[b][i] = fmaf(h, q[i], inner[b][i]);
+                    }
+                }
+#pragma unroll
+              for (int b = 0; b < BMAX; ++b)
+                if ((mask0 >> b) & 1u)
+#pragma unroll
+                  for (int i = 0; i < 8; ++i) acc[b][i] = fmaf(s[i], inner[b][i], acc[b][i]);
             }
           }
         }
-        __syncthreads();
-        prefix = (uint32_t)rs.sel_prefix;
-        rank = rs.sel_rank;
-        pmask |= 255u << shift;
       }
-      T = prefix;
-    }
-    // ordered compaction: kept iff key > T, or key == T among the first `rank`
-    const int chunk = (N + kThreads - 1) / kThreads;
-    const int lo = min(N, tid * chunk), hi = min(N, lo + chunk);
-    auto is_kept_all = [&](int) { return keep >= N; };
-    int eq = 0;
-    if (keep > 0 && keep < N)
-      for (int q = lo; q < hi; ++q) eq += (keys[q] == T);
-    int tot;
-    const int eq_before = block_excl_scan(eq, rs.scan, &tot);
-    int cnt = 0;
-    {
-      int e_seen = eq_before;
-      for (int q = lo; q < hi; ++q) {
-        bool kp;
-        if (keep <= 0) kp = false;
-        else if (is_kept_all(q)) kp = true;
-        else {
-          const uint32_t kk = keys[q];
-          kp = kk > T || (kk == T && e_seen < rank);
-          e_seen += (kk == T);
-        }
-        cnt += kp;
-      }
-    }
-    const int pos0 = block_excl_scan(cnt, rs.scan, &tot);
-    {
-      int e_seen = eq_before, pos = pos0;
-      for (int q = lo; q < hi; ++q) {
-        bool kp;
-        if (keep <= 0) kp = false;
-        else if (is_kept_all(q)) kp = true;
-        else {
-          const uint32_t kk = keys[q];
-          kp = kk > T || (kk == T && e_seen < rank);
-          e_seen += (kk == T);
-        }
-        if (kp && pos < keep) {
-          const int u = q / I;
-          kept[pos++] = rs.unit_e[u] * I + (q - u * I);
-        }
-      }
-    }
-    if (tid == 0) { rs.ncand = min(tot, keep); rs.sectors = 0ull; }
-    __syncthreads();
-    // sectors the kernel reads: union of the kept channels' 32-byte sectors
-    const unsigned long long base = (unsigned long long)(uintptr_t)p.layer[l].gate;
-    const unsigned long long cb = 3ull * rowb;
-    unsigned long long sec = 0;
-    for (int i = tid; i < rs.ncand; i += kThreads) {
-      const unsigned long long s0 = (base + (unsigned long long)kept[i] * cb) >> 5;
-      const unsigned long long s1 = (base + (unsigned long long)(kept[i] + 1) * cb - 1) >> 5;
-      sec += s1 - s0 + 1;
-      if (i > 0 && ((base + (unsigned long long)(kept[i - 1] + 1) * cb - 1) >> 5) == s0) sec -= 1;
-    }
-    if (sec) atomicAdd(&rs.sectors, sec);
-    __syncthreads();
-  };
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[slot]);
+      if (++cslot == p.nstages) { cslot = 0; cph ^= 1u; }
+      ++jc;
+      if (!ok) *(volatile int*)&abort_s = 1;
+      return ok;
+    };
 
-  // ------------------------------------------------------------ main loop
-  produce();  // prefetch layer 0's router rows and shared channels
-
-  for (int l = 0; l < p.L; ++l) {
-    float* yacc = p.yacc + (size_t)(l & 1) * B * H;
-    // 1. zero this CTA's slice of the accumulator used by this layer
-    {
-      const long long n4 = (long long)B * H / 4;
-      for (long long i = cta * n4 / G + tid; i < (cta + 1) * n4 / G; i += kThreads)
-        reinterpret_cast<float4*>(yacc)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    Job j;
-    if (p.mode == MODE_LAYERS) {
-      // 2. router rows of this CTA -> logits in the workspace
-      while (ccur.layer == l && ccur.type == JOB_ROUTER) {
-        next_job(ccur, j, -1);
-        if (!consume(j)) { drain(); return; }
-      }
-      // 3. split grid barrier: arrive now, run the shared expert, then wait
-      __syncthreads();
-      if (tid == 0) {
-        __threadfence();
-        const unsigned long long n = (unsigned long long)G;
-        const unsigned long long ticket = atom_add_release_gpu(&ctl->bar, 1ull);
-        target_s = (ticket / n + 1ull) * n;
-      }
-      while (ccur.layer == l && ccur.type == JOB_SHARED) {
-        next_job(ccur, j, -1);
-        if (!consume(j)) { drain(); return; }
-      }
-      {
-        __syncthreads();
-        if (tid == 0) {
-          int ok = 1;
-          if (ld_acquire_gpu(&ctl->bar) < target_s) {
-            const long long t0 = clock64();
-            while (ld_acquire_gpu(&ctl->bar) < target_s)
-              if (clock64() - t0 > kWaitBudgetCycles) { ok = 0; set_status(ctl, kStatusTimeout); break; }
-          }
-          __threadfence();
-          okw_s = ok;
-        }
-        __syncthreads();
-        if (!okw_s) { drain(); return; }
-      }
-      // 4. logits -> shared memory, top-k per token (one warp per token)
-      for (int i = tid; i < B * E; i += kThreads) lg[i] = __ldcg(p.logits + i);
-      __syncthreads();
-      if (warp < B) warp_topk(lg + warp * E, E, k, rs.ids[warp], rs.w[warp], nullptr);
-      __syncthreads();
-      if (cta == 0 && p.ids_out != nullptr)
-        for (int t = tid; t < B * k; t += kThreads) {
-          p.ids_out[(size_t)l * B * k + t] = rs.ids[t / k][t % k];
-          p.w_out[(size_t)l * B * k + t] = rs.w[t / k][t % k];
-        }
-    } else {
-      // experts only: routing supplied by the caller
-      for (int t = tid; t < B * k; t += kThreads) {
-        rs.ids[t / k][t % k] = p.ids_in[t];
-        rs.w[t / k][t % k] = p.w_in[t];
-      }
-      if (!grid_barrier(ctl)) { drain(); return; }  // accumulator zeroed everywhere
-    }
-    // 5. routed units (+ channel selection), then stream the routed channels
-    if (!build_units() && cta == 0 && tid == 0) set_status(ctl, kStatusBadIds);
-    if (LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR) {
-      select_channels(l);
-      if (cta == 0) {
-        if (p.kept_out != nullptr)
-          for (int i = tid; i < rs.ncand; i += kThreads) p.kept_out[(size_t)l * p.keep + i] = kept[i];
-        if (tid == 0 && p.sectors_out != nullptr) p.sectors_out[l] = rs.sectors;
-      }
-    }
-    if (tid == 0) route_ready_layer_s = l;
-    __syncthreads();
-    produce();
-    for (;;) {
-      const JobCursor save = ccur;
-      if (!next_job(ccur, j, l) || j.type == JOB_END || j.layer != l) { ccur = save; break; }
-      if (!consume(j)) { drain(); return; }
-    }
-    ccur.begin_layer(p, l + 1);
-    // 6. partial sums -> L2 accumulator; grid barrier
-    if (tid < H8) {
+    // ---- pre-norm: us[b] = bf16(x[b] / sqrt(mean(x[b]^2) + eps)), unit weight
+    auto normalize_x = [&]() {
+      float ss[BMAX];
+#pragma unroll
+      for (int b = 0; b < BMAX; ++b) ss[b] = 0.f;
+      float xv[BMAX][8];
 #pragma unroll
       for (int b = 0; b < BMAX; ++b)
-        if (b < B) {
-          float* dst = yacc + (size_t)b * H + 8 * tid;
-          red_add_v4(dst, acc[b][0], acc[b][1], acc[b][2], acc[b][3]);
-          red_add_v4(dst + 4, acc[b][4], acc[b][5], acc[b][6], acc[b][7]);
+        if (b < B && has_v) {
+          unpack8(xs4[b * H8c + tid], xv[b]);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) acc[b][i] = 0.f;
+          for (int i = 0; i < 8; ++i) ss[b] = fmaf(xv[b][i], xv[b][i], ss[b]);
         }
-    }
-    if (!grid_barrier(ctl)) { drain(); return; }
-    // 7. epilogue: y, residual, outputs (each CTA writes its slice)
-    {
+#pragma unroll
+      for (int b = 0; b < BMAX; ++b) {
+        const float t = warp_sum(ss[b]);
+        if (lane == 0) hbuf[warp][b] = t;
+      }
+      cbar();
+#pragma unroll
+      for (int b = 0; b < BMAX; ++b)
+        if (b < B && has_v) {
+          float t = 0.f;
+#pragma unroll
+          for (int w = 0; w < kWarps; ++w) t += hbuf[w][b];
+          const float sc = rsqrtf(t / (float)H + 1e-6f);
+          uint4 o;
+          o.x = uint32_t(f_to_bf16(xv[b][0] * sc)) | (uint32_t(f_to_bf16(xv[b][1] * sc)) << 16);
+          o.y = uint32_t(f_to_bf16(xv[b][2] * sc)) | (uint32_t(f_to_bf16(xv[b][3] * sc)) << 16);
+          o.z = uint32_t(f_to_bf16(xv[b][4] * sc)) | (uint32_t(f_to_bf16(xv[b][5] * sc)) << 16);
+          o.w = uint32_t(f_to_bf16(xv[b][6] * sc)) | (uint32_t(f_to_bf16(xv[b][7] * sc)) << 16);
+          reinterpret_cast<uint4*>(us)[b * H8c + tid] = o;
+        }
+      cbar();
+    };
+    if constexpr (MODE == MODE_LAYERS)
+      if (p.pre_norm) normalize_x();
+    load_xfrag();
+
+    // ---- routed units from rs.ids / rs.w (ascending expert ids)
+    auto build_units = [&]() -> bool {
+      if (tid == 0) bad_s = 0;
+      if constexpr (BMAX == 1) {
+        cbar();
+        if (warp == 0) {
+          const int e = lane < k ? rs.ids[0][lane] : 0x7fffffff;
+          const float wl = lane < k ? rs.w[0][lane] : 0.f;
+          int rank = 0, dup = 0;
+          for (int i = 0; i < k; ++i) {
+            const int o = __shfl_sync(0xffffffffu, e, i);
+            rank += (o < e) || (o == e && i < lane);
+            dup |= (o == e && i != lane);
+          }
+          if (lane < k) {
+            const bool valid = e >= 0 && e < E && !dup;
+            rs.unit_e[rank] = valid ? e : 0;
+            rs.unit_mask[rank] = valid ? 1u : 0u;
+            rs.unit_w[rank][0] = valid ? wl : 0.f;
+            if (!valid) bad_s = 1;
+          }
+          if (lane == 0) rs.U = k;
+        }
+        cbar();
+        return bad_s == 0;
+      } else {
+      const int nw = (E + 31) >> 5;
+      for (int i = tid; i < nw; i += kConsumers) rs.bitmap[i] = 0u;
+      cbar();
+      for (int t = tid; t < B * k; t += kConsumers) {
+        const int e = rs.ids[t / k][t % k];
+        if (e < 0 || e >= E) bad_s = 1;
+        else atomicOr(&rs.bitmap[e >> 5], 1u << (e & 31));
+      }
+      cbar();
+      if (warp == 0) {
+        const int c = lane < nw ? __popc(rs.bitmap[lane]) : 0;
+        int inc = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int t = __shfl_up_sync(0xffffffffu, inc, o);
+          if (lane >= o) inc += t;
+        }
+        if (lane < nw) rs.rank_base[lane] = inc - c;
+        if (lane == 31) rs.U = inc;
+      }
+      cbar();
+      for (int u = tid; u < rs.U; u += kConsumers) {
+        rs.unit_mask[u] = 0u;
+#pragma unroll
+        for (int b = 0; b < kMaxB; ++b) rs.unit_w[u][b] = 0.f;
+      }
+      for (int e = tid; e < E; e += kConsumers)
+        if ((rs.bitmap[e >> 5] >> (e & 31)) & 1u)
+          rs.unit_e[rs.rank_base[e >> 5] + __popc(rs.bitmap[e >> 5] & ((1u << (e & 31)) - 1u))] = e;
+      cbar();
+      for (int t = tid; t < B * k; t += kConsumers) {
+        const int b = t / k, e = rs.ids[b][t % k];
+        if (e < 0 || e >= E) continue;
+        const int u = rs.rank_base[e >> 5] + __popc(rs.bitmap[e >> 5] & ((1u << (e & 31)) - 1u));
+        const uint32_t old = atomicOr(&rs.unit_mask[u], 1u << b);
+        if (old & (1u << b)) bad_s = 1;
+        else rs.unit_w[u][b] = rs.w[b][t % k];
+      }
+      cbar();
+      return bad_s == 0;
+      }
+    };
+
+    // ---- top-k of every token from lg[B][E]
+    // B = 1, k <= 8: every warp's largest key is >= T = the smallest of the
+    // warp maxima, so at least 8 keys reach T and the k-th largest key is >= T.
+    // Only keys >= T are ranked (each against the other candidates); ties go to
+    // the lower index. The routed units (ascending expert id) are built in the
+    // same pass.
+    auto route_b1_small_k = [&]() {
+      uint32_t kq[4];
+      uint32_t kmax = 0u;
+      bool has = false;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int idx = tid + kConsumers * q;
+        kq[q] = 0u;
+        if (idx < E) { kq[q] = float_key(lg[idx]); kmax = max(kmax, kq[q]); has = true; }
+      }
+      const uint32_t wm = __reduce_max_sync(0xffffffffu, kmax);
+      const bool whas = __any_sync(0xffffffffu, has);
+      if (lane == 0) { sel_pos[0][warp] = whas ? 1 : 0; cand_key[warp] = wm; }
+      cbar();
+      uint32_t T = 0xffffffffu;
+      int nw = 0;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w)
+        if (sel_pos[0][w]) { T = min(T, cand_key[w]); ++nw; }
+      if (nw < k) T = 0u;  // too few warps hold keys: rank them all
+      // candidates: count per warp, then place
+      int mine = 0;
+      uint32_t ball[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int idx = tid + kConsumers * q;
+        ball[q] = __ballot_sync(0xffffffffu, idx < E && kq[q] >= T);
+        mine += __popc(ball[q]);
+      }
+      cbar();  // everyone has read cand_key[] / sel_pos[0][]
+      if (lane == 0) sel_pos[1][warp] = mine;
+      cbar();
+      int base = 0, C = 0;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        const int c = sel_pos[1][w];
+        if (w < warp) base += c;
+        C += c;
+      }
+      int* cidx = reinterpret_cast<int*>(lg);  // logits are in kq[] now
+      {
+        int off = base;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          if ((ball[q] >> lane) & 1u) {
+            const int pos = off + __popc(ball[q] & ((1u << lane) - 1u));
+            keys[pos] = kq[q];
+            cidx[pos] = tid + kConsumers * q;
+          }
+          off += __popc(ball[q]);
+        }
+      }
+      cbar();
+      if (C <= 32) {
+        // one warp ranks the candidates with shuffles and finishes the routing
+        if (warp == 0) {
+          const bool valid = lane < C;
+          const uint32_t kc = valid ? keys[lane] : 0u;
+          const int ic = valid ? cidx[lane] : 0x7fffffff;
+          int rank = 0;
+#pragma unroll 8
+          for (int o = 0; o < 32; ++o) {
+            const uint32_t ko = __shfl_sync(0xffffffffu, kc, o);
+            const int io = __shfl_sync(0xffffffffu, ic, o);
+            rank += (ko > kc) || (ko == kc && io < ic);
+          }
+          const bool sel = valid && rank < k;
+          const uint32_t top = __reduce_max_sync(0xffffffffu, valid ? kc : 0u);
+          const float e = sel ? __expf(key_float(kc) - key_float(top)) : 0.f;
+          const float ssum = warp_sum(e);
+          const float wl = e / ssum;
+          int urank = 0;
+#pragma unroll 8
+          for (int o = 0; o < 32; ++o) {
+            const int io = __shfl_sync(0xffffffffu, ic, o);
+            const bool so = __shfl_sync(0xffffffffu, sel, o);
+            urank += so && io < ic;
+          }
+          if (sel) {
+            rs.ids[0][rank] = ic;
+            rs.w[0][rank] = wl;
+            rs.unit_e[urank] = ic;
+            rs.unit_mask[urank] = 1u;
+            rs.unit_w[urank][0] = wl;
+          }
+          if (lane == 0) rs.U = k;
+        }
+        cbar();
+        return;
+      }
+      for (int c = tid; c < C; c += kConsumers) {
+        const uint32_t kc = keys[c];
+        const int ic = cidx[c];
+        int rank = 0;
+        for (int o = 0; o < C; ++o) {
+          const uint32_t ko = keys[o];
+          rank += (ko > kc) || (ko == kc && cidx[o] < ic);
+        }
+        if (rank < k) { sel_pos[2][rank] = ic; cand_key[kWarps + rank] = kc; }
+      }
+      cbar();
+      if (warp == 0) {
+        const int e = lane < k ? sel_pos[2][lane] : 0x7fffffff;
+        if (lane < k) sel_l[0][lane] = key_float(cand_key[kWarps + lane]);
+        __syncwarp();
+        warp_weights(sel_l[0], k, rs.w[0]);
+        __syncwarp();
+        if (lane < k) rs.ids[0][lane] = e;
+        // units: ascending expert id
+        int urank = 0;
+        for (int i = 0; i < k; ++i) urank += __shfl_sync(0xffffffffu, e, i) < e;
+        if (lane < k) {
+          rs.unit_e[urank] = e;
+          rs.unit_mask[urank] = 1u;
+          rs.unit_w[urank][0] = rs.w[0][lane];
+        }
+        if (lane == 0) rs.U = k;
+      }
+      cbar();
+    };
+
+    auto route = [&]() {
+      if constexpr (BMAX == 1) {
+        // two levels: each warp takes the best k of its 1/8 of the experts,
+        // warp 0 picks the best k of those candidates
+        const int per8 = (E + kWarps - 1) / kWarps;
+        const int lo = min(E, warp * per8), n = min(E, lo + per8) - lo;
+        const int kk = min(k, n);
+        for (int i = tid; i < E; i += kConsumers) keys[i] = float_key(lg[i]);
+        cbar();
+        if (kk > 0) warp_select(keys + lo, n, kk, sel_pos[warp]);
+        __syncwarp();
+        for (int i = lane; i < k; i += 32) {
+          cand_key[warp * k + i] = (i < kk) ? keys[lo + sel_pos[warp][i]] : 0u;
+          cand_idx[warp * k + i] = (i < kk) ? lo + sel_pos[warp][i] : -1;
+        }
+        cbar();
+        if (warp == 0) {
+          warp_select(cand_key, kWarps * k, k, sel_pos[0]);
+          __syncwarp();
+          if (lane < k) {
+            const int q = sel_pos[0][lane];
+            rs.ids[0][lane] = cand_idx[q];
+            sel_l[0][lane] = key_float(cand_key[q]);
+          }
+          __syncwarp();
+          warp_weights(sel_l[0], k, rs.w[0]);
+        }
+        cbar();
+      } else {
+        // one warp per token
+        for (int i = tid; i < B * E; i += kConsumers) keys[i] = float_key(lg[i]);
+        cbar();
+        if (warp < B) {
+          warp_select(keys + warp * E, E, k, sel_pos[warp]);
+          __syncwarp();
+          if (lane < k) {
+            rs.ids[warp][lane] = sel_pos[warp][lane];
+            sel_l[warp][lane] = lg[warp * E + sel_pos[warp][lane]];
+          }
+          __syncwarp();
+          warp_weights(sel_l[warp], k, rs.w[warp]);
+        }
+        cbar();
+      }
+    };
+
+    // ---- channel-sparse selection (B = 1): kept[] ascending, rs.ncand
+    auto select_channels = [&](int l) {
+      const int N = rs.U * I;
+      const float* sc = p.layer[l].scores;
+      for (int q = tid; q < N; q += kConsumers) {
+        const int u = q / I, c = q - u * I;
+        keys[q] = float_key(__ldg(sc + (size_t)rs.unit_e[u] * I + c));
+      }
+      cbar();
+      const int keep = p.keep;
+      uint32_t T = 0;
+      int rank = 0;
+      if (keep > 0 && keep < N) {
+        uint32_t prefix = 0, pmask = 0;
+        rank = keep;
+        for (int shift = 24; shift >= 0; shift -= 8) {
+          rs.hist[tid] = 0u;
+          cbar();
+          for (int q = tid; q < N; q += kConsumers) {
+            const uint32_t kk = keys[q];
+            if ((kk & pmask) == prefix) atomicAdd(&rs.hist[(kk >> shift) & 255u], 1u);
+          }
+          cbar();
+          if (warp == 0) {
+            uint32_t c8[8], loc = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) { c8[i] = rs.hist[255 - 8 * lane - i]; loc += c8[i]; }
+            uint32_t inc = loc;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+              const uint32_t t = __shfl_up_sync(0xffffffffu, inc, o);
+              if (lane >= o) inc += t;
+            }
+            const uint32_t exc = inc - loc;
+            if (exc < (uint32_t)rank && (uint32_t)rank <= inc) {
+              uint32_t cum = exc;
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                if (cum + c8[i] >= (uint32_t)rank) {
+                  rs.sel_rank = rank - (int)cum;
+                  rs.sel_prefix = (int)(prefix | ((uint32_t)(255 - 8 * lane - i) << shift));
+                  break;
+                }
+                cum += c8[i];
+              }
+            }
+          }
+          cbar();
+          prefix = (uint32_t)rs.sel_prefix;
+          rank = rs.sel_rank;
+          pmask |= 255u << shift;
+        }
+        T = prefix;
+      }
+      const int chunk = (N + kConsumers - 1) / kConsumers;
+      const int lo = min(N, tid * chunk), hi = min(N, lo + chunk);
+      const bool all = keep >= N;
+      int eq = 0;
+      if (keep > 0 && !all)
+        for (int q = lo; q < hi; ++q) eq += (keys[q] == T);
+      int tot;
+      const int eq_before = block_excl_scan(eq, rs.scan, &tot);
+      auto kept_at = [&](int q, int& e_seen) -> bool {
+        if (keep <= 0) return false;
+        if (all) return true;
+        const uint32_t kk = keys[q];
+        const bool kp = kk > T || (kk == T && e_seen < rank);
+        e_seen += (kk == T);
+        return kp;
+      };
+      int cnt = 0;
+      {
+        int e_seen = eq_before;
+        for (int q = lo; q < hi; ++q) cnt += kept_at(q, e_seen);
+      }
+      const int pos0 = block_excl_scan(cnt, rs.scan, &tot);
+      {
+        int e_seen = eq_before, pos = pos0;
+        for (int q = lo; q < hi; ++q)
+          if (kept_at(q, e_seen) && pos < keep) {
+            const int u = q / I;
+            kept[pos++] = rs.unit_e[u] * I + (q - u * I);
+          }
+      }
+      if (tid == 0) { rs.ncand = min(tot, keep); rs.sectors = 0ull; }
+      cbar();
+      const unsigned long long base = (unsigned long long)(uintptr_t)p.layer[l].gate;
+      const unsigned long long cb = 3ull * rowb;
+      unsigned long long sec = 0;
+      for (int i = tid; i < rs.ncand; i += kConsumers) {
+        const unsigned long long s0 = (base + (unsigned long long)kept[i] * cb) >> 5;
+        const unsigned long long s1 = (base + (unsigned long long)(kept[i] + 1) * cb - 1) >> 5;
+        sec += s1 - s0 + 1;
+        if (i > 0 && ((base + (unsigned long long)(kept[i - 1] + 1) * cb - 1) >> 5) == s0) sec -= 1;
+      }
+      if (sec) atomicAdd(&rs.sectors, sec);
+      cbar();
+    };
+
+    bool failed = false;
+    Job j;
+    for (int l = 0; l < p.L && !failed; ++l) {
+      float* yacc = p.yacc + (size_t)(l & 1) * B * H;
+      {
+        const long long n4 = (long long)B * H / 4;
+        for (long long i = cta * n4 / G + tid; i < (cta + 1) * n4 / G; i += kConsumers)
+          reinterpret_cast<float4*>(yacc)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      // phase 0: router rows, 1: shared expert, 2: routed experts
+      int phase = (MODE == MODE_LAYERS) ? 0 : 1;
+      int ready = l - 1;
+      unsigned long long target = 0;
+      for (;;) {
+        const JobCursor save = ccur;
+        const bool got = next_job(ccur, j, ready);
+        const bool in_layer = got && j.type != JOB_END && j.layer == l;
+        if (in_layer && j.type == phase) {
+          if (!consume(j)) { failed = true; break; }
+          continue;
+        }
+        ccur = save;
+        if (phase == 0) {
+          // router logits written: arrive at the grid barrier, keep working
+          cbar();
+          if (tid == 0) target = arrive_grid();
+          phase = 1;
+          continue;
+        }
+        if (phase == 1) {
+          if constexpr (MODE == MODE_LAYERS) {
+            if (tid == 0) okw_s = wait_grid(target) ? 1 : 0;
+            cbar();
+            if (!okw_s) { failed = true; if (tid == 0) set_status(ctl, kStatusTimeout); break; }
+            for (int i = tid; i < B * E; i += kConsumers) lg[i] = __ldcg(p.logits + i);
+            cbar();
+            if (BMAX == 1 && k <= kWarps) route_b1_small_k();
+            else route();
+            if (cta == 0 && p.ids_out != nullptr)
+              for (int t = tid; t < B * k; t += kConsumers) {
+                p.ids_out[(size_t)l * B * k + t] = rs.ids[t / k][t % k];
+                p.w_out[(size_t)l * B * k + t] = rs.w[t / k][t % k];
+              }
+          } else {
+            for (int t = tid; t < B * k; t += kConsumers) {
+              rs.ids[t / k][t % k] = p.ids_in[t];
+              rs.w[t / k][t % k] = p.w_in[t];
+            }
+            if (!grid_sync()) { failed = true; if (tid == 0) set_status(ctl, kStatusTimeout); break; }
+          }
+          const bool units_done = MODE == MODE_LAYERS && BMAX == 1 && k <= kWarps;
+          if (!units_done && !build_units() && cta == 0 && tid == 0) set_status(ctl, kStatusBadIds);
+          if constexpr (LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR) {
+            select_channels(l);
+            if (cta == 0) {
+              if (p.kept_out != nullptr)
+                for (int i = tid; i < rs.ncand; i += kConsumers) p.kept_out[(size_t)l * p.keep + i] = kept[i];
+              if (tid == 0 && p.sectors_out != nullptr) p.sectors_out[l] = rs.sectors;
+            }
+          }
+          if (tid == 0) st_release_cta(&route_ready_s, l);
+          ready = l;
+          phase = 2;
+          continue;
+        }
+        break;
+      }
+      if (cbar_or(failed)) { failed = true; break; }
+      ccur.begin_layer(p, l + 1);
+      // partial sums -> L2 accumulator
+      if (has_v) {
+#pragma unroll
+        for (int b = 0; b < BMAX; ++b)
+          if (b < B) {
+            float* dst = yacc + (size_t)b * H + 8 * tid;
+            red_add_v4(dst, acc[b][0], acc[b][1], acc[b][2], acc[b][3]);
+            red_add_v4(dst + 4, acc[b][4], acc[b][5], acc[b][6], acc[b][7]);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[b][i] = 0.f;
+          }
+      }
+      if (!grid_sync()) { failed = true; if (tid == 0) set_status(ctl, kStatusTimeout); break; }
+      // epilogue: y, residual, outputs (each CTA writes its slice)
       const long long n4 = (long long)B * H / 4;
       const long long s0 = cta * n4 / G, s1 = (cta + 1) * n4 / G;
       float* yh = p.y_hist ? p.y_hist + (size_t)l * B * H : nullptr;
       float* yo = (l == p.L - 1) ? p.y_out : nullptr;
-      if (p.mode == MODE_LAYERS) {
-        // every CTA needs the whole next x
-        for (long long i = tid; i < n4; i += kThreads) {
+      if constexpr (MODE == MODE_LAYERS) {
+        for (long long i = tid; i < n4; i += kConsumers) {
           const float4 y4 = __ldcg(reinterpret_cast<const float4*>(yacc) + i);
           uint2 xv = reinterpret_cast<uint2*>(xs)[i];
           const float x0 = bf16_lo(xv.x) + y4.x, x1 = bf16_hi(xv.x) + y4.y;
@@ -757,15 +1114,28 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             if (l == p.L - 1 && p.x_out) reinterpret_cast<uint2*>(p.x_out)[i] = xv;
           }
         }
+        cbar();
+        if (p.pre_norm) normalize_x();
+        load_xfrag();
       } else {
-        for (long long i = s0 + tid; i < s1; i += kThreads) {
+        for (long long i = s0 + tid; i < s1; i += kConsumers) {
           const float4 y4 = __ldcg(reinterpret_cast<const float4*>(yacc) + i);
           if (yo) reinterpret_cast<float4*>(yo)[i] = y4;
           if (yh) reinterpret_cast<float4*>(yh)[i] = y4;
         }
       }
-      __syncthreads();
     }
+    if (failed && tid == 0) {
+      jc_s = jc;
+      st_release_cta(&abort_s, 1);
+    }
+  }
+  __syncthreads();
+  // on an error path, wait (bounded) for the copies still in flight so that
+  // none lands in shared memory after the CTA has exited
+  if (tid == 0 && abort_s) {
+    const long long issued = jp_s;
+    for (long long q = jc_s; q < issued; ++q) mbar_wait(&full[q % p.nstages], (uint32_t)((q / p.nstages) & 1));
   }
 }
 

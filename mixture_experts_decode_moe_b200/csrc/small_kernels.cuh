@@ -42,23 +42,29 @@ __global__ void __launch_bounds__(kThreads) router_logits_kernel(const uint16_t*
 __global__ void __launch_bounds__(kThreads) topk_kernel(const float* __restrict__ logits, int B, int E, int k,
                                                         int32_t* ids, float* w, float* margin) {
   extern __shared__ __align__(16) uint8_t sm[];
-  float* lg = reinterpret_cast<float*>(sm);
-  __shared__ int ids_s[kWarps][kMaxK];
+  uint32_t* keys = reinterpret_cast<uint32_t*>(sm);
+  __shared__ int pos_s[kWarps][kMaxK + 1];
+  __shared__ float l_s[kWarps][kMaxK + 1];
   __shared__ float w_s[kWarps][kMaxK];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.x * kWarps + warp;
   if (b >= B) return;
-  float* l = lg + warp * E;
-  for (int i = lane; i < E; i += 32) l[i] = logits[(size_t)b * E + i];
+  uint32_t* kw = keys + warp * E;
+  const float* lb = logits + (size_t)b * E;
+  for (int i = lane; i < E; i += 32) kw[i] = float_key(lb[i]);
   __syncwarp();
-  float mg;
-  warp_topk(l, E, k, ids_s[warp], w_s[warp], &mg);
+  const int kk = (k < E) ? k + 1 : k;
+  warp_select(kw, E, kk, pos_s[warp]);
+  __syncwarp();
+  for (int i = lane; i < kk; i += 32) l_s[warp][i] = key_float(kw[pos_s[warp][i]]);
+  __syncwarp();
+  warp_weights(l_s[warp], k, w_s[warp]);
   __syncwarp();
   for (int i = lane; i < k; i += 32) {
-    ids[(size_t)b * k + i] = ids_s[warp][i];
+    ids[(size_t)b * k + i] = pos_s[warp][i];
     w[(size_t)b * k + i] = w_s[warp][i];
   }
-  if (lane == 0 && margin != nullptr) margin[b] = mg;
+  if (lane == 0 && margin != nullptr) margin[b] = (k < E) ? l_s[warp][k - 1] - l_s[warp][k] : INFINITY;
 }
 
 // Stable counting sort of the (token, slot) pairs by expert, one CTA.

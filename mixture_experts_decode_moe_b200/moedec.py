@@ -27,6 +27,7 @@ MOE_OK, MOE_ERR_INVALID, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_TIMEOUT = ra
 MOE_W_BF16, MOE_W_INT4_G64 = 0, 1
 MOE_EXPERT_SWIGLU, MOE_EXPERT_LINEAR = 0, 1
 MOE_LAYOUT_PLANAR, MOE_LAYOUT_CHANNEL_MAJOR = 0, 1
+MOE_STACK_PRE_RMSNORM = 1
 
 EXPORTS = [
     "moe_abi_version", "moe_status_string", "moe_workspace_bytes", "moe_workspace_init",
@@ -60,7 +61,7 @@ _lib.moe_get_status.argtypes = [_P, _P]
 _lib.moe_route_topk.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _S, _P]
 _lib.moe_expert_forward.argtypes = [ctypes.POINTER(LayerDesc), _P, _I, _P, _P, _P, _P, _S, _P]
 _lib.moe_layer_forward.argtypes = [ctypes.POINTER(LayerDesc), _P, _I, _P, _P, _P, _P, _P, _S, _P]
-_lib.moe_stack_forward.argtypes = [ctypes.POINTER(LayerDesc), _I, _P, _I, _P, _P, _P, _P, _P, _P, _S, _P]
+_lib.moe_stack_forward.argtypes = [ctypes.POINTER(LayerDesc), _I, _P, _I, ctypes.c_uint32, _P, _P, _P, _P, _P, _P, _S, _P]
 _lib.moe_channel_topk_forward.argtypes = [ctypes.POINTER(LayerDesc), _P, _I, _P, _P, _P, _I, _P, _P, _P,
                                           _P, _S, _P]
 _lib.moe_touched_experts.argtypes = [_P, _I, _I, _I, _P, _P, _P, _P, _P]
@@ -152,9 +153,9 @@ def moe_layer_forward(desc, x, y, ws, x_next=None, ids_out=None, w_out=None, str
 
 
 def moe_stack_forward(descs, x, x_out, ws, x_hist=None, y_hist=None, ids_hist=None, w_hist=None,
-                      stream=None):
+                      flags=0, stream=None):
     arr = (LayerDesc * len(descs))(*descs)
-    _check(_lib.moe_stack_forward(arr, len(descs), _ptr(x), x.shape[0], _ptr(x_out), _ptr(x_hist),
+    _check(_lib.moe_stack_forward(arr, len(descs), _ptr(x), x.shape[0], flags, _ptr(x_out), _ptr(x_hist),
                                   _ptr(y_hist), _ptr(ids_hist), _ptr(w_hist), _ptr(ws), ws.numel(),
                                   _stream(stream)), "moe_stack_forward")
 

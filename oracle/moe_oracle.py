@@ -32,7 +32,10 @@ Readings where the pages are silent (each is listed in the design doc):
   * the top-k decision is taken on the logits rounded to fp32, the
     precision the GPU path decides in; weights use the fp64 logits.
   * the shared expert is added with weight 1 (no gate is described).
-  * the stack residual is x_next = bf16_rne(x + y), no norm, no attention.
+  * the stack residual is x_next = bf16_rne(x + y), no attention; with the
+    pre-norm option each layer's MoE input is u = bf16_rne(x / rms(x)),
+    rms(x) = sqrt(mean(x^2) + 1e-6), unit norm weight (without it a stack of
+    N(0, 0.02) SwiGLU layers grows without bound: see rmsnorm_bf16).
   * int4: two's-complement nibbles, element 2i in the low nibble, symmetric
     (zero point 0), value = q * s with one bf16 scale per 64 consecutive
     input elements.
@@ -255,6 +258,34 @@ def dense_mixture(x, router, experts: ExpertFn, E: int) -> np.ndarray:
     for e in range(E):
         y += p[e] * swiglu_expert(x, *experts(e))
     return y
+
+
+RMS_EPS = 1e-6
+
+
+def rmsnorm_bf16(x: np.ndarray, eps: float = RMS_EPS) -> np.ndarray:
+    """Pre-norm MoE input u = bf16_rne(x / sqrt(mean(x^2) + eps)), unit weight.
+
+    The pages give only the depth of the decode stack ([MoE-intro], 40
+    blocks), not the block internals. Transformer blocks normalise the hidden
+    state before the feed-forward layer; without it, a residual stack of
+    random N(0, 0.02) SwiGLU experts at hidden 2048 grows roughly
+    quadratically per layer and overflows fp32 after about 25 layers.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    return bf16_round(x / np.sqrt(np.mean(x * x) + eps))
+
+
+def stack_layer(x: np.ndarray, router: np.ndarray, experts: ExpertFn, k: int,
+                shared: tuple | None = None, pre_norm: bool = True):
+    """One layer of the attention-free decode stack.
+
+    u = rmsnorm_bf16(x) (or x without the pre-norm); y = MoE(u);
+    x_next = bf16_rne(x + y). Returns (x_next, y, ids, w, logits, margin).
+    """
+    u = rmsnorm_bf16(x) if pre_norm else np.asarray(x, dtype=np.float64)
+    y, ids, w, logits, margin = moe_layer(u, router, experts, k, shared)
+    return residual_bf16(x, y), y, ids, w, logits, margin
 
 
 def residual_bf16(x: np.ndarray, y: np.ndarray) -> np.ndarray:

@@ -75,8 +75,10 @@ def test_invalid_arguments_rejected_before_launch(M):
     d = desc(M)
     assert lib.moe_layer_forward(ctypes.byref(d), dummy, 1, dummy, None, None, None, dummy, 1 << 20,
                                  None) == 1  # no weights
-    assert lib.moe_stack_forward(ctypes.byref(d), 0, dummy, 1, dummy, None, None, None, None, dummy,
+    assert lib.moe_stack_forward(ctypes.byref(d), 0, dummy, 1, 0, dummy, None, None, None, None, dummy,
                                  1 << 20, None) == 1
+    assert lib.moe_stack_forward(ctypes.byref(d), 1, dummy, 1, 2, dummy, None, None, None, None, dummy,
+                                 1 << 20, None) == 1  # unknown flag
     assert lib.moe_workspace_init(None, 0, None) == 1
     assert lib.moe_get_status(None, None) == 1
     cm = desc(M, E=128, I=768, layout=1)

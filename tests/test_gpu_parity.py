@@ -212,7 +212,8 @@ def test_layer_forward_shapes(M, S, H, E, I, k, I_sh, B):
             assert rel_err(f64(y[b]), dense) <= REL_TOL
 
 
-def test_stack_small_teacher_forced(M, S):
+@pytest.mark.parametrize("pre_norm", [True, False])
+def test_stack_small_teacher_forced(M, S, pre_norm):
     H, E, I, k, I_sh, Lc, B = 512, 32, 192, 4, 128, 5, 2
     layers = [S.swiglu_layer_bf16(H, E, I, I_sh, seed=900 + l, device=DEV, router_scale=0.5) for l in range(Lc)]
     descs = [planar_desc(M, Ld, H, E, I, k) for Ld in layers]
@@ -223,7 +224,8 @@ def test_stack_small_teacher_forced(M, S):
     yh = torch.empty((Lc, B, H), dtype=torch.float32, device=DEV)
     ih = torch.empty((Lc, B, k), dtype=torch.int32, device=DEV)
     wh = torch.empty((Lc, B, k), dtype=torch.float32, device=DEV)
-    M.moe_stack_forward(descs, x, xo, ws, x_hist=xh, y_hist=yh, ids_hist=ih, w_hist=wh)
+    M.moe_stack_forward(descs, x, xo, ws, x_hist=xh, y_hist=yh, ids_hist=ih, w_hist=wh,
+                        flags=M.MOE_STACK_PRE_RMSNORM if pre_norm else 0)
     torch.cuda.synchronize()
     assert torch.equal(xh[0], x) and torch.equal(xh[Lc], xo)
     log = []
@@ -231,11 +233,11 @@ def test_stack_small_teacher_forced(M, S):
         HL = HostLayer(layers[l])
         for b in range(B):
             xl = f64(xh[l, b])
-            yo, io, wo, lo, _ = O.moe_layer(xl, HL.R, HL.expert, k, shared=HL.shared)
+            xn, yo, io, wo, lo, _ = O.stack_layer(xl, HL.R, HL.expert, k, shared=HL.shared, pre_norm=pre_norm)
             if check_ids(ih[l, b].tolist(), io, lo, log, f"l{l}b{b}"):
                 continue
             assert rel_err(f64(yh[l, b]), yo) <= REL_TOL
-            assert rel_err(f64(xh[l + 1, b]), O.residual_bf16(xl, yo)) <= REL_TOL
+            assert rel_err(f64(xh[l + 1, b]), xn) <= REL_TOL
             assert np.allclose(f64(wh[l, b]), wo, rtol=1e-5)
 
 

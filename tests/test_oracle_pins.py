@@ -473,3 +473,33 @@ def test_layer_bytes_closed_forms():
     assert O.swiglu_expert_bytes(2048, 512, "int4") == 1_671_168
     assert O.layer_bytes_b1(2048, 256, 512, 8, I_shared=512, wtype="int4") == 20_709_376
     assert O.layer_bytes_b1(512, 16, 256, 2) == 1_589_248
+
+
+# ---------------------------------------------------------------- stack pre-norm
+
+
+def test_rmsnorm_closed_forms():
+    # constant vector c: mean(x^2) = c^2, so u = c / sqrt(c^2 + eps) ~ sign(c)
+    x = np.full(64, 3.0)
+    u = O.rmsnorm_bf16(x)
+    assert np.all(u == O.bf16_round(np.array([3.0 / math.sqrt(9.0 + O.RMS_EPS)]))[0])
+    # scale invariance (up to eps): rms(a x) normalises to the same u
+    r = rng(17)
+    x = r.normal(0, 1, 256)
+    assert np.array_equal(O.rmsnorm_bf16(x), O.rmsnorm_bf16(1024.0 * x))
+    # unit rms output (before bf16 rounding: within bf16 precision)
+    assert abs(np.sqrt(np.mean(O.rmsnorm_bf16(x) ** 2)) - 1.0) < 1e-2
+
+
+def test_stack_layer_residual_uses_unnormalised_x():
+    r = rng(18)
+    H, E, I, k = 32, 4, 8, 2
+    R, ex = make_layer(r, H, E, I)
+    x = O.bf16_round(r.normal(0, 5, H))
+    xn, y, ids, w, _, _ = O.stack_layer(x, R, lambda e: ex[e], k)
+    u = O.rmsnorm_bf16(x)
+    y2, ids2, *_ = O.moe_layer(u, R, lambda e: ex[e], k)
+    assert np.allclose(y, y2) and ids.tolist() == ids2.tolist()
+    assert np.array_equal(xn, O.residual_bf16(x, y))
+    xn0, y0, *_ = O.stack_layer(x, R, lambda e: ex[e], k, pre_norm=False)
+    assert np.allclose(y0, O.moe_layer(x, R, lambda e: ex[e], k)[0])
