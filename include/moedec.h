@@ -200,6 +200,39 @@ moe_status moe_touched_experts(const int32_t* ids, int32_t B, int32_t k, int32_t
                                int32_t* count, uint32_t* bitmap_opt, int32_t* offsets_opt,
                                int32_t* pairs_opt, moe_stream_t stream);
 
+/* ---- No-allocation variant (the pages have no counterpart; it is a service
+ * for callers that cannot allocate device memory) ----------------------------
+ *
+ * Some callers cannot call cudaMalloc (or any allocating routine) at the
+ * point where they run a layer: code that records into a stream while the
+ * runtime forbids allocation calls, plug-in hosts whose device memory is all
+ * owned by the host's own pool, or real-time loops that must never block on
+ * the allocator. moe_layer_forward_static() computes exactly what
+ * moe_layer_forward() computes, but its scratch space is a fixed array inside
+ * the library (MOE_STATIC_SCRATCH_BYTES per device, held by every GPU that
+ * loads the library until the process exits) instead of a workspace the
+ * caller passes. The caller still passes inputs and outputs.
+ *
+ *  - The scratch needed is moe_workspace_bytes(desc, B); a shape that needs
+ *    more than MOE_STATIC_SCRATCH_BYTES is rejected with MOE_ERR_UNSUPPORTED
+ *    before anything is launched.
+ *  - The first call on a device looks up the array's device address (once per
+ *    device, with that device current). Make that first call outside any
+ *    stream capture.
+ *  - All calls on a device share the one array and it keeps the previous
+ *    call's contents; each call first clears the part that must start at zero
+ *    (the status word and barrier counter). Calls whose executions overlap on
+ *    the GPU (concurrent streams, or host threads on one device) race on the
+ *    array: serialise them.
+ *  - status_out_opt (device int32, or NULL) receives the call's device status
+ *    (the value moe_get_status() would report) after the kernel, stream-ordered.
+ *  - Nothing is allocated or freed: no cudaMalloc/cudaFree, no library routine
+ *    that allocates. */
+#define MOE_STATIC_SCRATCH_BYTES (144u * 1024u)
+moe_status moe_layer_forward_static(const moe_layer_desc* desc, const void* x, int32_t B, float* y,
+                                    void* x_next_opt, int32_t* ids_out_opt, float* w_out_opt,
+                                    int32_t* status_out_opt, moe_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -6,6 +6,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "small_kernels.cuh"
 
@@ -416,3 +417,54 @@ moe_status moe_channel_topk_forward(const moe_layer_desc* d, const void* x, int3
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- no-allocation variant
+//
+// A library-owned scratch array stands in for the caller's workspace. In host
+// code the symbol below is only a handle: its device address is looked up with
+// cudaGetSymbolAddress (per device, with that device current) and that
+// address is what the kernel receives.
+namespace {
+
+static __device__ __align__(256) unsigned char g_static_scratch[MOE_STATIC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_mu;
+void* g_static_addr[kMaxDevices] = {};
+
+moe_status static_scratch_address(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (g_static_addr[dev] == nullptr) {
+    void* addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_static_scratch) != cudaSuccess || addr == nullptr) return MOE_ERR_CUDA;
+    g_static_addr[dev] = addr;
+  }
+  *out = g_static_addr[dev];
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" moe_status moe_layer_forward_static(const moe_layer_desc* desc, const void* x, int32_t B, float* y,
+                                                void* x_next_opt, int32_t* ids_out_opt, float* w_out_opt,
+                                                int32_t* status_out_opt, moe_stream_t stream) {
+  const size_t need = moe_workspace_bytes(desc, B);
+  if (need == 0) return MOE_ERR_INVALID;
+  if (need > MOE_STATIC_SCRATCH_BYTES) return MOE_ERR_UNSUPPORTED;  // beyond the fixed scratch size
+  void* scratch = nullptr;
+  moe_status st = static_scratch_address(&scratch);
+  if (st != MOE_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  // the previous call's status word and barrier counter must not leak into this one
+  if (cudaMemsetAsync(scratch, 0, sizeof(WsControl), s) != cudaSuccess) return MOE_ERR_CUDA;
+  st = moe_layer_forward(desc, x, B, y, x_next_opt, ids_out_opt, w_out_opt, scratch, MOE_STATIC_SCRATCH_BYTES,
+                         stream);
+  if (st != MOE_OK) return st;
+  if (status_out_opt != nullptr &&
+      cudaMemcpyAsync(status_out_opt, scratch, sizeof(int32_t), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}

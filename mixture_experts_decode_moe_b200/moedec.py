@@ -28,11 +28,13 @@ MOE_W_BF16, MOE_W_INT4_G64 = 0, 1
 MOE_EXPERT_SWIGLU, MOE_EXPERT_LINEAR = 0, 1
 MOE_LAYOUT_PLANAR, MOE_LAYOUT_CHANNEL_MAJOR = 0, 1
 MOE_STACK_PRE_RMSNORM = 1
+MOE_STATIC_SCRATCH_BYTES = 144 * 1024
 
 EXPORTS = [
     "moe_abi_version", "moe_status_string", "moe_workspace_bytes", "moe_workspace_init",
     "moe_get_status", "moe_route_topk", "moe_expert_forward", "moe_layer_forward",
     "moe_stack_forward", "moe_channel_topk_forward", "moe_touched_experts",
+    "moe_layer_forward_static",
 ]
 
 
@@ -65,6 +67,7 @@ _lib.moe_stack_forward.argtypes = [ctypes.POINTER(LayerDesc), _I, _P, _I, ctypes
 _lib.moe_channel_topk_forward.argtypes = [ctypes.POINTER(LayerDesc), _P, _I, _P, _P, _P, _I, _P, _P, _P,
                                           _P, _S, _P]
 _lib.moe_touched_experts.argtypes = [_P, _I, _I, _I, _P, _P, _P, _P, _P]
+_lib.moe_layer_forward_static.argtypes = [ctypes.POINTER(LayerDesc), _P, _I, _P, _P, _P, _P, _P, _P]
 for _f in EXPORTS[3:]:
     getattr(_lib, _f).restype = ctypes.c_int
 
@@ -170,3 +173,12 @@ def moe_touched_experts(ids, E, count, bitmap=None, offsets=None, pairs=None, st
     B, k = ids.shape
     _check(_lib.moe_touched_experts(_ptr(ids), B, k, E, _ptr(count), _ptr(bitmap), _ptr(offsets),
                                     _ptr(pairs), _stream(stream)), "moe_touched_experts")
+
+
+def moe_layer_forward_static(desc, x, y, x_next=None, ids_out=None, w_out=None, status_out=None, stream=None):
+    """moe_layer_forward without a caller workspace: the library's fixed scratch
+    array is used instead (see include/moedec.h for who needs this and the
+    rules on sharing it)."""
+    _check(_lib.moe_layer_forward_static(ctypes.byref(desc), _ptr(x), x.shape[0], _ptr(y), _ptr(x_next),
+                                         _ptr(ids_out), _ptr(w_out), _ptr(status_out), _stream(stream)),
+           "moe_layer_forward_static")
