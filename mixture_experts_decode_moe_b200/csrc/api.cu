@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "small_kernels.cuh"
+#include "linear.cuh"
 
 using namespace moedec;
 
@@ -31,6 +32,24 @@ inline WsLayout ws_layout(int B, int H, int E) {
   off = align_up(off + (size_t)B * E * sizeof(float));
   w.yacc = off;
   off = align_up(off + 2 * (size_t)B * H * sizeof(float));
+  w.total = off;
+  return w;
+}
+
+// LINEAR experts: control block, the plan, and the packed token rows of the
+// tensor-core units (at most B*k + 32*min(E, B*k) rows of H bf16).
+struct LinWsLayout {
+  size_t plan, xp, total;
+  int xp_rows_max;
+};
+inline LinWsLayout lin_ws_layout(int B, int H, int E, int k) {
+  LinWsLayout w;
+  size_t off = sizeof(WsControl);
+  w.plan = off;
+  off = align_up(off + sizeof(LinPlan));
+  w.xp = off;
+  w.xp_rows_max = B * k + kTcRowsPerLoad * std::min(E, B * k);
+  off = align_up(off + (size_t)w.xp_rows_max * H * 2);
   w.total = off;
   return w;
 }
@@ -224,6 +243,76 @@ void fill_common(DecodeParams* p, const moe_layer_desc* d, int B, void* ws) {
   p->yacc = reinterpret_cast<float*>(base + w.yacc);
 }
 
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor map over a row-major [rows][cols] array: box 64 x box_rows,
+// 128-byte swizzle (the K-major tcgen05 operand layout).
+bool encode_bf16_2d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_tiled_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)kTcBlockK, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+moe_status linear_forward(const moe_layer_desc* d, const void* x, int B, const int32_t* ids, const float* w, float* y,
+                          void* ws, cudaStream_t s) {
+  const int H = d->H;
+  const int sms = sm_count();
+  if (sms <= 0) return MOE_ERR_CUDA;
+  const LinWsLayout wl = lin_ws_layout(B, H, d->E, d->k);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  LinTcParams tp;
+  std::memset(&tp, 0, sizeof(tp));
+  LinParams& lp = tp.lp;
+  lp.B = B;
+  lp.H = H;
+  lp.E = d->E;
+  lp.k = d->k;
+  lp.x = static_cast<const uint16_t*>(x);
+  lp.W = static_cast<const uint16_t*>(d->gate);
+  lp.ids = ids;
+  lp.w = w;
+  lp.y = y;
+  lp.plan = reinterpret_cast<LinPlan*>(base + wl.plan);
+  lp.xp = reinterpret_cast<uint16_t*>(base + wl.xp);
+  lp.xp_rows_max = wl.xp_rows_max;
+  lp.num_sms = sms;
+  lp.ctl = reinterpret_cast<WsControl*>(base);
+  if (!encode_bf16_2d(&tp.tmap_w, d->gate, (uint64_t)H, (uint64_t)d->E * H, kTcBlockM)) return MOE_ERR_CUDA;
+  if (!encode_bf16_2d(&tp.tmap_x, lp.xp, (uint64_t)H, (uint64_t)wl.xp_rows_max, kTcRowsPerLoad)) return MOE_ERR_CUDA;
+  if (cudaMemsetAsync(y, 0, (size_t)B * H * sizeof(float), s) != cudaSuccess) return MOE_ERR_CUDA;
+  linear_plan_kernel<<<1, kThreads, 0, s>>>(lp);
+  linear_gather_kernel<<<sms * 4, kThreads, 0, s>>>(lp);
+  const int gemv_smem = (kTcMin - 1) * H * 2;
+  if (cudaFuncSetAttribute(linear_gemv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, gemv_smem) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  linear_gemv_kernel<<<sms * 2, kThreads, gemv_smem, s>>>(lp);
+  if (cudaFuncSetAttribute(linear_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmem) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  linear_tc_kernel<<<sms, kThreads, kTcSmem, s>>>(tp);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
 bool same_shape(const moe_layer_desc* a, const moe_layer_desc* b) {
   return a->H == b->H && a->E == b->E && a->I == b->I && a->k == b->k && a->kind == b->kind &&
          a->wtype == b->wtype && a->layout == b->layout && a->I_shared == b->I_shared;
@@ -248,6 +337,7 @@ const char* moe_status_string(moe_status s) {
 
 size_t moe_workspace_bytes(const moe_layer_desc* d, int32_t B) {
   if (!valid_shape(d) || B < 1 || B > 256) return 0;
+  if (d->kind == MOE_EXPERT_LINEAR) return std::max(ws_layout(B, d->H, d->E).total, lin_ws_layout(B, d->H, d->E, d->k).total);
   return ws_layout(B, d->H, d->E).total;
 }
 
@@ -304,6 +394,12 @@ moe_status moe_expert_forward(const moe_layer_desc* d, const void* x, int32_t B,
   if (!valid_shape(d) || !x || !ids || !w || !y || !ws) return MOE_ERR_INVALID;
   if (!aligned16(x) || !aligned16(y) || !aligned16(ws) || B < 1 || B > 256) return MOE_ERR_INVALID;
   if (ws_bytes < moe_workspace_bytes(d, B)) return MOE_ERR_INVALID;
+  if (d->kind == MOE_EXPERT_LINEAR) {
+    if (d->wtype != MOE_W_BF16 || d->layout != MOE_LAYOUT_PLANAR) return MOE_ERR_UNSUPPORTED;
+    if (d->H % 256 != 0 || d->gate == nullptr || !aligned16(d->gate) || !aligned16(w) || !aligned16(ids))
+      return MOE_ERR_INVALID;
+    return linear_forward(d, x, B, ids, w, y, ws, (cudaStream_t)stream);
+  }
   if (d->kind != MOE_EXPERT_SWIGLU || d->layout != MOE_LAYOUT_PLANAR) return MOE_ERR_UNSUPPORTED;
   if (B > kMaxB || d->H > 2048) return MOE_ERR_UNSUPPORTED;
   moe_status st = check_weights(d, false);
