@@ -189,6 +189,21 @@ moe_status moe_channel_topk_forward(const moe_layer_desc* desc, const void* x, i
                                     unsigned long long* sectors,
                                     void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* Channel-sparse decode stack (one token): per layer l, u_l = x_l (or its RMS
+ * normalisation with MOE_STACK_PRE_RMSNORM), the router picks k experts of u_l
+ * as in moe_route_topk, then only the `keep` best channels of those experts by
+ * scores[l, e, c] are read and applied as in moe_channel_topk_forward;
+ * x_{l+1} = bf16_rne(x_l + y_l). layers[L]: CHANNEL_MAJOR bf16 SWIGLU with a
+ * router, same shape. x [1, H] bf16; scores [L, E, I] fp32; x_out [1, H];
+ * optional x_hist [L+1, H], y_hist [L, H], ids_hist / w_hist [L, k],
+ * kept_hist [L, keep] (ascending); sectors [L] = 32-byte sectors of routed
+ * weights read per layer. 1 <= L <= 64, 0 <= keep <= k*I. */
+moe_status moe_channel_stack_forward(const moe_layer_desc* layers, int32_t L, const void* x, uint32_t flags,
+                                     const float* scores, int32_t keep, void* x_out, void* x_hist_opt,
+                                     float* y_hist_opt, int32_t* ids_hist_opt, float* w_hist_opt,
+                                     int32_t* kept_hist_opt, unsigned long long* sectors,
+                                     void* ws, size_t ws_bytes, moe_stream_t stream);
+
 /* Touched experts of a batch: the union of the B tokens' expert sets.
  *   ids [B, k] int32 (distinct per token, < E); count [1] int32 = |union|;
  *   bitmap_opt [ceil(E/32)] uint32, bit e set iff expert e is touched;

@@ -452,6 +452,50 @@ moe_status moe_stack_forward(const moe_layer_desc* layers, int32_t L, const void
   return launch_decode(p, B <= 1 ? 1 : kMaxB, (cudaStream_t)stream);
 }
 
+moe_status moe_channel_stack_forward(const moe_layer_desc* layers, int32_t L, const void* x, uint32_t flags,
+                                     const float* scores, int32_t keep, void* x_out, void* x_hist_opt,
+                                     float* y_hist_opt, int32_t* ids_hist_opt, float* w_hist_opt,
+                                     int32_t* kept_hist_opt, unsigned long long* sectors, void* ws,
+                                     size_t ws_bytes, moe_stream_t stream) {
+  if (layers == nullptr || L < 1 || L > kMaxLayers || !x || !scores || !sectors || !ws) return MOE_ERR_INVALID;
+  if (flags & ~(uint32_t)MOE_STACK_PRE_RMSNORM) return MOE_ERR_INVALID;
+  const moe_layer_desc* d = &layers[0];
+  if (!valid_shape(d)) return MOE_ERR_INVALID;
+  if (d->kind != MOE_EXPERT_SWIGLU || d->layout != MOE_LAYOUT_CHANNEL_MAJOR || d->wtype != MOE_W_BF16)
+    return MOE_ERR_INVALID;
+  if (keep < 0 || keep > d->k * d->I) return MOE_ERR_INVALID;
+  if ((long long)d->k * d->I > kMaxCand || d->H > 2048) return MOE_ERR_UNSUPPORTED;
+  if ((ids_hist_opt == nullptr) != (w_hist_opt == nullptr)) return MOE_ERR_INVALID;
+  if (!aligned16(x) || !aligned16(ws) || !aligned16(scores) || (x_out && !aligned16(x_out)) ||
+      (x_hist_opt && !aligned16(x_hist_opt)) || (y_hist_opt && !aligned16(y_hist_opt)))
+    return MOE_ERR_INVALID;
+  if (ws_bytes < moe_workspace_bytes(d, 1)) return MOE_ERR_INVALID;
+  for (int l = 0; l < L; ++l) {
+    if (!same_shape(&layers[l], d)) return MOE_ERR_INVALID;
+    moe_status st = check_weights(&layers[l], true);
+    if (st != MOE_OK) return st;
+  }
+  DecodeParams p;
+  fill_common(&p, d, 1, ws);
+  p.L = L;
+  p.mode = MODE_LAYERS;
+  p.pre_norm = (flags & MOE_STACK_PRE_RMSNORM) ? 1 : 0;
+  p.keep = keep;
+  p.x_in = static_cast<const uint16_t*>(x);
+  p.x_out = static_cast<uint16_t*>(x_out);
+  p.x_hist = static_cast<uint16_t*>(x_hist_opt);
+  p.y_hist = y_hist_opt;
+  p.ids_out = ids_hist_opt;
+  p.w_out = w_hist_opt;
+  p.kept_out = kept_hist_opt;
+  p.sectors_out = sectors;
+  for (int l = 0; l < L; ++l) {
+    fill_layer(&p.layer[l], &layers[l]);
+    p.layer[l].scores = scores + (size_t)l * d->E * d->I;
+  }
+  return launch_decode(p, 1, (cudaStream_t)stream);
+}
+
 moe_status moe_layer_forward(const moe_layer_desc* d, const void* x, int32_t B, float* y, void* x_next_opt,
                              int32_t* ids_out_opt, float* w_out_opt, void* ws, size_t ws_bytes,
                              moe_stream_t stream) {

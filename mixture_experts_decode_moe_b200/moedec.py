@@ -34,7 +34,7 @@ EXPORTS = [
     "moe_abi_version", "moe_status_string", "moe_workspace_bytes", "moe_workspace_init",
     "moe_get_status", "moe_route_topk", "moe_expert_forward", "moe_layer_forward",
     "moe_stack_forward", "moe_channel_topk_forward", "moe_touched_experts",
-    "moe_layer_forward_static",
+    "moe_layer_forward_static", "moe_channel_stack_forward",
 ]
 
 
@@ -67,6 +67,8 @@ _lib.moe_stack_forward.argtypes = [ctypes.POINTER(LayerDesc), _I, _P, _I, ctypes
 _lib.moe_channel_topk_forward.argtypes = [ctypes.POINTER(LayerDesc), _P, _I, _P, _P, _P, _I, _P, _P, _P,
                                           _P, _S, _P]
 _lib.moe_touched_experts.argtypes = [_P, _I, _I, _I, _P, _P, _P, _P, _P]
+_lib.moe_channel_stack_forward.argtypes = [ctypes.POINTER(LayerDesc), _I, _P, ctypes.c_uint32, _P, _I, _P, _P, _P,
+                                           _P, _P, _P, _P, _P, _S, _P]
 _lib.moe_layer_forward_static.argtypes = [ctypes.POINTER(LayerDesc), _P, _I, _P, _P, _P, _P, _P, _P]
 for _f in EXPORTS[3:]:
     getattr(_lib, _f).restype = ctypes.c_int
@@ -167,6 +169,15 @@ def moe_channel_topk_forward(desc, x, ids, w, scores, keep, y, sectors, ws, kept
     _check(_lib.moe_channel_topk_forward(ctypes.byref(desc), _ptr(x), x.shape[0], _ptr(ids), _ptr(w),
                                          _ptr(scores), keep, _ptr(y), _ptr(kept), _ptr(sectors), _ptr(ws),
                                          ws.numel(), _stream(stream)), "moe_channel_topk_forward")
+
+
+def moe_channel_stack_forward(descs, x, scores, keep, x_out, sectors, ws, x_hist=None, y_hist=None, ids_hist=None,
+                              w_hist=None, kept_hist=None, flags=0, stream=None):
+    arr = (LayerDesc * len(descs))(*descs)
+    _check(_lib.moe_channel_stack_forward(arr, len(descs), _ptr(x), flags, _ptr(scores), keep, _ptr(x_out),
+                                          _ptr(x_hist), _ptr(y_hist), _ptr(ids_hist), _ptr(w_hist),
+                                          _ptr(kept_hist), _ptr(sectors), _ptr(ws), ws.numel(), _stream(stream)),
+           "moe_channel_stack_forward")
 
 
 def moe_touched_experts(ids, E, count, bitmap=None, offsets=None, pairs=None, stream=None):

@@ -403,6 +403,19 @@ def channel_sparse_forward(x: np.ndarray, channel: Callable[[int, int], np.ndarr
     return y
 
 
+def channel_stack_layer(x: np.ndarray, router: np.ndarray, channel: Callable[[int, int], np.ndarray],
+                        scores: np.ndarray, k: int, keep: int, I: int, pre_norm: bool = True):
+    """One layer of the channel-sparse decode stack: u = rmsnorm_bf16(x) (or
+    x), routing of u, the `keep` best channels of the routed experts by the
+    given scores [E, I], y from the kept channels only, x_next = bf16(x + y).
+    Returns (x_next, y, ids, w, logits, kept)."""
+    u = rmsnorm_bf16(x) if pre_norm else np.asarray(x, dtype=np.float64)
+    ids, w, logits, _ = route_topk(u, router, k)
+    kept = channel_topk_select(scores, ids, keep)
+    y = channel_sparse_forward(u, channel, ids, w, kept, I)
+    return residual_bf16(x, y), y, ids, w, logits, kept
+
+
 def sectors_touched(ranges: Iterable[tuple]) -> int:
     """Distinct 32-byte sectors covering the half-open byte ranges [lo, hi).
 

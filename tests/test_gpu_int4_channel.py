@@ -226,3 +226,38 @@ def test_channel_topk_edge_cases(M, S, keep_mode):
             planar = O.moe_experts_given(f64(x[b]), lambda e: (host[e][:, 0], host[e][:, 1], host[e][:, 2]),
                                          ids[b].tolist(), f64(wt[b]))
             assert rel_err(f64(y[b]), planar) <= REL_TOL
+
+
+@pytest.mark.parametrize("pre_norm", [True, False])
+def test_channel_stack_small_teacher_forced(M, S, pre_norm):
+    H, E, I, k, Lc, keep = 512, 16, 64, 4, 3, 37
+    layers = [S.channel_major_layer(H, E, I, seed=600 + l, device=DEV, router_scale=0.5) for l in range(Lc)]
+    descs = [M.make_desc(H, E, I, k, layout=M.MOE_LAYOUT_CHANNEL_MAJOR, router=Ld["router"], gate=Ld["cm"])
+             for Ld in layers]
+    scale = S.channel_scale(E, I, seed=610, device=DEV)
+    scores = torch.cat([S.channel_scores(1, E, I, scale, seed=620 + l, device=DEV) for l in range(Lc)])
+    x = S.tokens(1, H, seed=630, device=DEV)
+    ws = M.alloc_workspace(descs[0], 1)
+    xo = torch.empty((1, H), dtype=torch.bfloat16, device=DEV)
+    xh = torch.empty((Lc + 1, H), dtype=torch.bfloat16, device=DEV)
+    yh = torch.empty((Lc, H), dtype=torch.float32, device=DEV)
+    ih = torch.empty((Lc, k), dtype=torch.int32, device=DEV)
+    wh = torch.empty((Lc, k), dtype=torch.float32, device=DEV)
+    kh = torch.empty((Lc, keep), dtype=torch.int32, device=DEV)
+    sec = torch.empty((Lc,), dtype=torch.int64, device=DEV)
+    M.moe_channel_stack_forward(descs, x, scores, keep, xo, sec, ws, x_hist=xh, y_hist=yh, ids_hist=ih,
+                                w_hist=wh, kept_hist=kh, flags=M.MOE_STACK_PRE_RMSNORM if pre_norm else 0)
+    torch.cuda.synchronize()
+    assert M.moe_get_status(ws) == M.MOE_OK
+    log = []
+    for l in range(Lc):
+        host = f64(layers[l]["cm"])
+        xl = f64(xh[l])
+        xn, yo, io, wo, lo, kept = O.channel_stack_layer(xl, f64(layers[l]["router"]), lambda e, c: host[e][c],
+                                                         scores[l].cpu().numpy(), k, keep, I, pre_norm=pre_norm)
+        if check_ids(ih[l].tolist(), io, lo, log, f"l{l}"):
+            continue
+        assert kh[l].cpu().numpy().tolist() == kept.tolist()
+        assert int(sec[l]) == O.sectors_touched(O.channel_major_ranges(kept, H, base=layers[l]["cm"].data_ptr()))
+        assert rel_err(f64(yh[l]), yo) <= REL_TOL
+        assert rel_err(f64(xh[l + 1]), xn) <= REL_TOL
