@@ -45,12 +45,6 @@ def peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def algorithmic_layer_bytes(H, E, I, k, I_sh):
-    """Bytes one batch-1 token must read in one layer: router [E,H] + k routed
-    SwiGLU experts (3*I*H) + the shared expert (3*I_sh*H), all bf16."""
-    return 2 * (E * H + k * 3 * I * H + 3 * I_sh * H)
-
-
 # ---------------------------------------------------------------- distributed plumbing
 
 
@@ -143,21 +137,206 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
-# ---------------------------------------------------------------- model setup
+# ---------------------------------------------------------------- workloads
+#
+# Each workload sets up its synthetic inputs on the device and provides:
+#   step(i)      one step on device-resident inputs (the timed unit)
+#   e2e_step(i)  the same through host (pinned) buffers: input H2D, output D2H
+#   nbytes(i)    algorithmic bytes the step must read (router, routed experts
+#                or kept channels, shared expert; exact routing of that step)
+# plus tokens per step, launches per step and a config description.
 
 
-def build_stack(torch, M, S, device):
-    w = S.WORKLOADS[WORKLOAD]
-    H, E, I, k, I_sh, nl = w["H"], w["E"], w["I"], w["k"], w["I_shared"], w["layers"]
-    layers, descs = [], []
-    for l in range(nl):
-        Ld = S.swiglu_layer_bf16(H, E, I, I_sh, seed=S.weight_seed(w["cfg"], l), device=device,
-                                 router_scale=w["router_scale"])
-        layers.append(Ld)
-        descs.append(M.make_desc(H, E, I, k, router=Ld["router"], gate=Ld["gate"], up=Ld["up"],
-                                 down_t=Ld["down_t"], sh_gate=Ld["sh_gate"], sh_up=Ld["sh_up"],
-                                 sh_down_t=Ld["sh_down_t"]))
-    return w, layers, descs
+def a3b_config(name, w, B, layers=None):
+    return {"workload": name + ("" if B == 1 else f"_b{B}"), "layers": layers or w["layers"], "hidden": w["H"],
+            "experts": w["E"], "top_k": w["k"], "expert_intermediate": w["I"], "shared_intermediate": w["I_shared"],
+            "batch": B, "pre_norm": "rms", "l2": "inputs larger than L2 (weights of 40 layers, tens of GB)"}
+
+
+class A3BStack:
+    """40-layer A3B-shaped SwiGLU stack (bf16 or int4 experts), batch B, pre-norm."""
+
+    def __init__(self, torch, M, S, device, rank, wtype="bf16", B=1, steps=0, layers=0):
+        self.torch, self.M, self.S, self.dev = torch, M, S, device
+        self.name = "a3b_bf16" if wtype == "bf16" else "a3b_int4"
+        w = S.WORKLOADS[self.name]
+        self.w = w
+        H, E, I, k, I_sh, nl = w["H"], w["E"], w["I"], w["k"], w["I_shared"], layers or w["layers"]
+        self.H, self.E, self.I, self.k, self.I_sh, self.nl, self.B = H, E, I, k, I_sh, nl, B
+        gen = S.swiglu_layer_bf16 if wtype == "bf16" else S.swiglu_layer_int4
+        self.layers = [gen(H, E, I, I_sh, seed=S.weight_seed(w["cfg"], l), device=device,
+                           router_scale=w["router_scale"]) for l in range(nl)]
+        kw = {} if wtype == "bf16" else {"wtype": M.MOE_W_INT4_G64}
+        self.descs = []
+        for L in self.layers:
+            extra = {} if wtype == "bf16" else {"gate_s": L["gate_s"], "up_s": L["up_s"], "down_s": L["down_s"]}
+            self.descs.append(M.make_desc(H, E, I, k, router=L["router"], gate=L["gate"], up=L["up"],
+                                          down_t=L["down_t"], sh_gate=L["sh_gate"], sh_up=L["sh_up"],
+                                          sh_down_t=L["sh_down_t"], **kw, **extra))
+        self.ntok = 256
+        self.xs = S.tokens(self.ntok * B, H, seed=S.act_seed(w["cfg"]) + 97 * rank, device=device)
+        self.ws = M.alloc_workspace(self.descs[0], B, device)
+        self.x_out = torch.empty((B, H), dtype=torch.bfloat16, device=device)
+        self.ids_hist = torch.zeros((max(steps, 1), nl, B, k), dtype=torch.int32, device=device)
+        self.w_hist = torch.zeros((max(steps, 1), nl, B, k), dtype=torch.float32, device=device)
+        self.expert_bytes = 3 * I * H * 2 if wtype == "bf16" else 3 * I * H // 2 + 3 * I * (H // 64) * 2
+        self.tokens_per_step = B
+        self.launches_per_step = 1
+        self.kernel = f"decode_kernel<layers,B{B},{wtype},planar>"
+        self.record = 0
+
+    def _x(self, i):
+        j = i % self.ntok
+        return self.xs[j * self.B:(j + 1) * self.B]
+
+    def step(self, i, stream):
+        r = self.record
+        kw = {"ids_hist": self.ids_hist[r], "w_hist": self.w_hist[r]} if r < self.ids_hist.shape[0] else {}
+        self.M.moe_stack_forward(self.descs, self._x(i), self.x_out, self.ws, flags=self.M.MOE_STACK_PRE_RMSNORM,
+                                 stream=stream, **kw)
+
+    def host_buffers(self):
+        t = self.torch
+        self.x_host = self.xs.cpu().pin_memory()
+        self.out_host = t.empty((self.B, self.H), dtype=t.bfloat16).pin_memory()
+        self.x_dev = t.empty((self.B, self.H), dtype=t.bfloat16, device=self.dev)
+        return self.B * self.H * 2, self.B * self.H * 2
+
+    def e2e_step(self, i, stream):
+        j = i % self.ntok
+        self.x_dev.copy_(self.x_host[j * self.B:(j + 1) * self.B], non_blocking=True)
+        self.M.moe_stack_forward(self.descs, self.x_dev, self.x_out, self.ws, flags=self.M.MOE_STACK_PRE_RMSNORM,
+                                 stream=stream)
+        self.out_host.copy_(self.x_out, non_blocking=True)
+
+    def nbytes(self, r):
+        """Bytes of timed step r: per layer router + touched experts + shared."""
+        ids = self.ids_hist[r].cpu()
+        total = 0
+        for l in range(self.nl):
+            touched = len(set(ids[l].reshape(-1).tolist()))
+            total += 2 * self.E * self.H + touched * self.expert_bytes + 3 * self.I_sh * self.H * 2
+        return total
+
+    def config(self):
+        return a3b_config(self.name, self.w, self.B, self.nl)
+
+
+class ChannelStack:
+    """48-layer channel-major stack, batch 1, channel top-k keep over given scores."""
+
+    def __init__(self, torch, M, S, device, rank, frac=0.13, steps=0):
+        self.torch, self.M, self.S, self.dev = torch, M, S, device
+        w = S.WORKLOADS["channel_topk"]
+        H, E, I, k, nl = w["H"], w["E"], w["I"], w["k"], w["layers"]
+        self.H, self.E, self.I, self.k, self.nl = H, E, I, k, nl
+        self.keep = S.keep_count(frac, k, I)
+        self.frac = frac
+        self.layers = [S.channel_major_layer(H, E, I, seed=S.weight_seed(5, l), device=device) for l in range(nl)]
+        self.descs = [M.make_desc(H, E, I, k, layout=M.MOE_LAYOUT_CHANNEL_MAJOR, router=L["router"], gate=L["cm"])
+                      for L in self.layers]
+        scale = [S.channel_scale(E, I, seed=S.weight_seed(5, l) + 7, device=device) for l in range(nl)]
+        self.nsc = 16  # distinct per-token score sets
+        self.scores = torch.stack([torch.cat([S.channel_scores(1, E, I, scale[l], seed=S.act_seed(5, l) + 1000 * t,
+                                                               device=device) for l in range(nl)])
+                                   for t in range(self.nsc)])
+        self.xs = S.tokens(256, H, seed=S.act_seed(5) + 97 * rank, device=device)
+        self.ws = M.alloc_workspace(self.descs[0], 1, device)
+        self.x_out = torch.empty((1, H), dtype=torch.bfloat16, device=device)
+        self.sectors = torch.empty((nl,), dtype=torch.int64, device=device)
+        self.tokens_per_step = 1
+        self.launches_per_step = 1
+        self.kernel = "decode_kernel<layers,B1,bf16,channel-major>"
+
+    def step(self, i, stream):
+        self.M.moe_channel_stack_forward(self.descs, self.xs[i % 256:][:1], self.scores[i % self.nsc], self.keep,
+                                         self.x_out, self.sectors, self.ws, flags=self.M.MOE_STACK_PRE_RMSNORM,
+                                         stream=stream)
+
+    def host_buffers(self):
+        t = self.torch
+        self.x_host = self.xs.cpu().pin_memory()
+        self.out_host = t.empty((1, self.H), dtype=t.bfloat16).pin_memory()
+        self.x_dev = t.empty((1, self.H), dtype=t.bfloat16, device=self.dev)
+        return self.H * 2, self.H * 2
+
+    def e2e_step(self, i, stream):
+        self.x_dev.copy_(self.x_host[i % 256:][:1], non_blocking=True)
+        self.M.moe_channel_stack_forward(self.descs, self.x_dev, self.scores[i % self.nsc], self.keep, self.x_out,
+                                         self.sectors, self.ws, flags=self.M.MOE_STACK_PRE_RMSNORM, stream=stream)
+        self.out_host.copy_(self.x_out, non_blocking=True)
+
+    def nbytes(self, r):
+        # router + kept channels (gate row, up row, down column) + the 8 score rows read
+        return self.nl * (2 * self.E * self.H + self.keep * 3 * self.H * 2 + self.k * self.I * 4)
+
+    def config(self):
+        return {"workload": f"channel_topk_{int(round(100 * self.frac))}pct", "layers": self.nl, "hidden": self.H,
+                "experts": self.E, "top_k": self.k, "channels": self.I, "keep": self.keep, "batch": 1,
+                "pre_norm": "rms", "l2": "inputs larger than L2 (58 GB of channel-major weights)"}
+
+
+class BatchSweep:
+    """64 experts of one 8192 x 8192 bf16 matrix, top-3 uniform ids, batch B."""
+
+    def __init__(self, torch, M, S, device, rank, B=256, steps=0):
+        self.torch, self.M, self.S, self.dev = torch, M, S, device
+        w = S.WORKLOADS["batch_sweep"]
+        H, E, k = w["H"], w["E"], w["k"]
+        self.H, self.E, self.k, self.B = H, E, k, B
+        self.W = S.linear_experts(E, H, seed=S.weight_seed(3, 0), device=device)
+        self.desc = M.make_desc(H, E, H, k, kind=M.MOE_EXPERT_LINEAR, gate=self.W)
+        self.nsets = 16
+        self.xs = [S.tokens(B, H, seed=S.act_seed(3) + 31 * t + 97 * rank, device=device) for t in range(self.nsets)]
+        self.ids = [S.uniform_ids(B, E, k, seed=S.act_seed(3) + 1000 + 31 * t + 97 * rank, device=device)
+                    for t in range(self.nsets)]
+        self.wts = torch.ones((B, k), device=device)
+        self.ws = M.alloc_workspace(self.desc, B, device)
+        self.y = torch.empty((B, H), dtype=torch.float32, device=device)
+        self.touched = [len(set(i.reshape(-1).tolist())) for i in self.ids]
+        self.tokens_per_step = B
+        self.launches_per_step = 4  # plan, gather, GEMV engine, tensor-core engine (+ a memset)
+        self.kernel = "linear plan+gather+gemv+tcgen05"
+
+    def step(self, i, stream):
+        t = i % self.nsets
+        self.M.moe_expert_forward(self.desc, self.xs[t], self.ids[t], self.wts, self.y, self.ws, stream=stream)
+
+    def host_buffers(self):
+        t = self.torch
+        self.x_host = [x.cpu().pin_memory() for x in self.xs]
+        self.id_host = [i.cpu().pin_memory() for i in self.ids]
+        self.y_host = t.empty((self.B, self.H), dtype=t.float32).pin_memory()
+        self.x_dev = t.empty((self.B, self.H), dtype=t.bfloat16, device=self.dev)
+        self.id_dev = t.empty((self.B, self.k), dtype=t.int32, device=self.dev)
+        return self.B * self.H * 2 + self.B * self.k * 4, self.B * self.H * 4
+
+    def e2e_step(self, i, stream):
+        t = i % self.nsets
+        self.x_dev.copy_(self.x_host[t], non_blocking=True)
+        self.id_dev.copy_(self.id_host[t], non_blocking=True)
+        self.M.moe_expert_forward(self.desc, self.x_dev, self.id_dev, self.wts, self.y, self.ws, stream=stream)
+        self.y_host.copy_(self.y, non_blocking=True)
+
+    def nbytes(self, r):
+        return self.touched[r % self.nsets] * self.H * self.H * 2
+
+    def config(self):
+        return {"workload": f"batch_sweep_b{self.B}", "experts": self.E, "top_k": self.k, "hidden": self.H,
+                "batch": self.B, "expected_touched": self.E * (1 - (1 - self.k / self.E) ** self.B),
+                "l2": "inputs larger than L2 (8.6 GB of expert matrices)"}
+
+
+def make_workload(name, torch, M, S, device, rank, args):
+    if name == "a3b_bf16":
+        return A3BStack(torch, M, S, device, rank, "bf16", args.batch or 1, steps=args.steps, layers=args.layers)
+    if name == "a3b_int4":
+        return A3BStack(torch, M, S, device, rank, "int4", args.batch or 1, steps=args.steps, layers=args.layers)
+    if name == "channel_topk":
+        return ChannelStack(torch, M, S, device, rank, args.keep_frac, steps=args.steps)
+    if name == "batch_sweep":
+        return BatchSweep(torch, M, S, device, rank, args.batch or 256, steps=args.steps)
+    raise SystemExit(f"unknown workload {name}")
 
 
 # ---------------------------------------------------------------- CPU oracle timing
@@ -166,8 +345,8 @@ def build_stack(torch, M, S, device):
 def oracle_rate(layers, w, xs, budget_s=12.0, max_layers=None, start_token=0):
     """Time the fp64 oracle (as it stands) layer by layer on whole tokens.
 
-    Token t goes through layers 0..L-1 (residual between layers); per layer the
-    oracle copies the router, the shared expert and only the routed experts'
+    Token t goes through layers 0..L-1 (RMS pre-norm, MoE, residual: the same
+    stack the device runs); per layer the oracle copies the router, the shared expert and only the routed experts'
     weights to the host, converts them to fp64 and computes. Stops after the
     budget (at least one layer). Returns (tok/s, layers done, seconds)."""
     from oracle import moe_oracle as O
@@ -185,8 +364,7 @@ def oracle_rate(layers, w, xs, budget_s=12.0, max_layers=None, start_token=0):
         R = f64(Ld["router"])
         shared = (f64(Ld["sh_gate"]), f64(Ld["sh_up"]), f64(Ld["sh_down_t"]))
         experts = lambda e, Ld=Ld: (f64(Ld["gate"][e]), f64(Ld["up"][e]), f64(Ld["down_t"][e]))
-        y, *_ = O.moe_layer(x, R, experts, k, shared=shared)
-        x = O.residual_bf16(x, y)
+        x, *_ = O.stack_layer(x, R, experts, k, shared=shared, pre_norm=True)
         done += 1
         if done % nl == 0:
             tok += 1
@@ -214,6 +392,10 @@ def run_reference(args):
     ws_n, rank, local = dist_env()
     if rank != 0:
         return 0
+    if args.workload != WORKLOAD or (args.batch or 1) != 1:
+        print(json.dumps({"impl": "reference", "unavailable": "the oracle arm is timed on the default workload "
+                          f"({WORKLOAD}, batch 1) only"}), flush=True)
+        return 0
     import torch
     from mixture_experts_decode_moe_b200 import synth as S
     w = S.WORKLOADS[WORKLOAD]
@@ -238,8 +420,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sec, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "layers": nl, "hidden": H, "experts": E, "top_k": k,
-                   "expert_intermediate": I, "shared_intermediate": I_sh, "batch": 1},
+        "config": dict(a3b_config(WORKLOAD, w, 1), parallelism="single"),
         "cpu_baseline": {"value": value, "unit": "tok/s", "cores": cores, "kind": "oracle",
                          "sample": f"per step >= {per_step:.2f} s of whole layers ({n_layers} layer passes "
                                    f"timed in all), scaled to tokens through {nl} layers; routed-expert "
@@ -248,6 +429,21 @@ def run_reference(args):
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def nvtx_push(torch, name):
+    """Mark a region for profiler filtering (a no-op where NVTX is unavailable)."""
+    try:
+        torch.cuda.nvtx.range_push(name)
+    except Exception:
+        pass
+
+
+def nvtx_pop(torch):
+    try:
+        torch.cuda.nvtx.range_pop()
+    except Exception:
+        pass
 
 
 def run_ours(args):
@@ -261,73 +457,64 @@ def run_ours(args):
     from mixture_experts_decode_moe_b200 import moedec as M
     from mixture_experts_decode_moe_b200 import synth as S
 
-    w, layers, descs = build_stack(torch, M, S, device)
-    H, E, I, k, I_sh, nl = w["H"], w["E"], w["I"], w["k"], w["I_shared"], w["layers"]
-    B = 1
-    xs = S.tokens(w["tokens"], H, seed=S.act_seed(w["cfg"]) + 97 * rank, device=device)
-    ws = M.alloc_workspace(descs[0], B, device)
-    x_out = torch.empty((B, H), dtype=torch.bfloat16, device=device)
+    wl = make_workload(args.workload, torch, M, S, device, rank, args)
     stream = torch.cuda.current_stream(device)
     torch.cuda.synchronize()
-
-    def step(i):
-        M.moe_stack_forward(descs, xs[i % w["tokens"]:][:B], x_out, ws, flags=M.MOE_STACK_PRE_RMSNORM,
-                            stream=stream)
-
+    wl.record = 10 ** 9  # no routing record during warm-up
     for i in range(args.warmup):
-        step(i)
+        wl.step(i, stream)
     torch.cuda.synchronize()
-    st = M.moe_get_status(ws, stream)
+    st = M.moe_get_status(wl.ws, stream)
     if st != M.MOE_OK:
         raise SystemExit(f"device status after warm-up: {M.moe_status_string(st)}")
 
-    # ---- device-timed region: inputs resident in HBM
+    # ---- device-timed region: inputs resident in HBM (larger than L2)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     barrier(ws_n)
     torch.cuda.synchronize()
+    nvtx_push(torch, "timed")
     with ClockSampler(local) as clk:
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
         t0.record(stream)
         for i in range(args.steps):
+            wl.record = i
             ev[i][0].record(stream)
-            step(args.warmup + i)
+            wl.step(args.warmup + i, stream)
             ev[i][1].record(stream)
         t1.record(stream)
         torch.cuda.synchronize()
+    nvtx_pop(torch)
     barrier(ws_n)
+    wl.record = 10 ** 9
     total_ms = max_over_ranks(t0.elapsed_time(t1), ws_n, device)
     launch_ms = [a.elapsed_time(b) for a, b in ev]
-    kern_ms = statistics.mean(launch_ms)
     clocks = clk.summary()
-    if M.moe_get_status(ws, stream) != M.MOE_OK:
+    if M.moe_get_status(wl.ws, stream) != M.MOE_OK:
         raise SystemExit("device status error in timed region")
+    step_bytes = [wl.nbytes(i) for i in range(args.steps)]
 
     # ---- end to end through the C ABI with host buffers (pinned), copies timed
-    x_host = xs.cpu().pin_memory()
-    out_host = torch.empty((B, H), dtype=torch.bfloat16).pin_memory()
-    x_dev = torch.empty((B, H), dtype=torch.bfloat16, device=device)
+    h2d, d2h = wl.host_buffers()
     barrier(ws_n)
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
+    nvtx_push(torch, "e2e")
     e0.record(stream)
     for i in range(args.steps):
-        j = (args.warmup + i) % w["tokens"]
-        x_dev.copy_(x_host[j:j + B], non_blocking=True)
-        M.moe_stack_forward(descs, x_dev, x_out, ws, flags=M.MOE_STACK_PRE_RMSNORM, stream=stream)
-        out_host.copy_(x_out, non_blocking=True)
+        wl.e2e_step(args.warmup + i, stream)
     e1.record(stream)
     torch.cuda.synchronize()
+    nvtx_pop(torch)
     barrier(ws_n)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), ws_n, device)
 
-    layer_bytes = algorithmic_layer_bytes(H, E, I, k, I_sh)
-    launch_bytes = layer_bytes * nl * B
     hbm, hbm_kind = peaks()
-    achieved = launch_bytes / (kern_ms * 1e-3) / 1e9
+    # achieved = algorithmic bytes of each launch / its device time, averaged
+    achieved = statistics.mean(b / (ms * 1e-3) / 1e9 for b, ms in zip(step_bytes, launch_ms))
     traffic = None
-    tfile = os.path.join(ROOT, "profiles", "decode_kernel_a3b_bf16_traffic.json")
+    tfile = os.path.join(ROOT, "profiles", f"traffic_{wl.config()['workload']}.json")
     if os.path.exists(tfile):
         try:
             with open(tfile) as f:
@@ -337,30 +524,30 @@ def run_ours(args):
         except Exception:
             traffic = None
 
-    tokens_total = args.steps * B * ws_n
+    tokens_total = args.steps * wl.tokens_per_step * ws_n
     value = tokens_total / (total_ms * 1e-3)
+    cfg = wl.config()
+    cfg["parallelism"] = f"replicas{ws_n}" if ws_n > 1 else "single"
     line = {
         "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": ws_n, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "layers": nl, "hidden": H, "experts": E, "top_k": k,
-                   "expert_intermediate": I, "shared_intermediate": I_sh, "batch": B,
-                   "parallelism": f"replicas{ws_n}" if ws_n > 1 else "single",
-                   "l2": "inputs larger than L2: 64.7 GB of weights, each token reads 2.31 GB"},
+        "config": cfg,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm, "traffic": traffic, "peak_kind": hbm_kind,
-                     "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
-                     "kernel": "decode_kernel<1,bf16,planar>", "algorithmic_bytes_per_launch": launch_bytes},
-        "e2e": {"value": tokens_total / (e2e_ms * 1e-3), "unit": "tok/s", "h2d_bytes_per_step": B * H * 2,
-                "d2h_bytes_per_step": B * H * 2},
-        "gpu_launches": args.steps,
+                     "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS, "kernel": wl.kernel,
+                     "algorithmic_bytes_per_launch": statistics.mean(step_bytes)},
+        "e2e": {"value": tokens_total / (e2e_ms * 1e-3), "unit": "tok/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps * wl.launches_per_step,
         "clocks": clocks,
     }
-    if rank == 0 and ws_n == 1 and not args.no_cpu_baseline:
-        tps, done, dt = oracle_rate(layers, w, xs, budget_s=args.cpu_budget)
+    if args.workload == "a3b_bf16" and rank == 0 and ws_n == 1 and not args.no_cpu_baseline:
+        tps, done, dt = oracle_rate(wl.layers, wl.w, wl.xs, budget_s=args.cpu_budget)
         line["cpu_baseline"] = {"value": tps, "unit": "tok/s", "cores": blas_threads(), "kind": "oracle",
                                 "sample": f"{done} layer passes of the stack in {dt:.1f} s, scaled to tokens "
-                                          f"through {nl} layers (fp64; routed-expert slices copied from the device)"}
+                                          f"through {wl.nl} layers (fp64; routed-expert slices copied from the "
+                                          "device; RMS pre-norm as on the device)"}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if ws_n > 1:
@@ -387,6 +574,11 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default=WORKLOAD, choices=["a3b_bf16", "a3b_int4", "channel_topk", "batch_sweep"])
+    ap.add_argument("--batch", type=int, default=0, help="batch (a3b_int4: 1 or 8; batch_sweep: 1..256)")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="fewer stack layers (profiling captures only; the metric is quoted on the full stack)")
+    ap.add_argument("--keep-frac", type=float, default=0.13, help="channel_topk budget (0.13 or 0.18)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 warm-up steps
     if args.impl == "reference":

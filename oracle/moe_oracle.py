@@ -25,7 +25,7 @@ Pages cited (titles as printed):
                blog), §2 "핵심 개념" (active ratio, touched-expert formula,
                memory table, "둘째 식 — 배치의 함정"), §3 [A] and [B].
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
   * phi is SiLU (the layer is a SwiGLU MLP; [Reader] only writes phi).
   * routing = softmax over all E logits, top-k by logit (descending, ties to
     the lowest expert index), weights renormalised over the chosen k.
@@ -295,7 +295,7 @@ def residual_bf16(x: np.ndarray, y: np.ndarray) -> np.ndarray:
 
 def linear_experts(x: np.ndarray, weight: Callable[[int], np.ndarray],
                    ids: Sequence[int], w: Sequence[float]) -> np.ndarray:
-    """Expert = one matrix ([Beam] §3: 'expert = one 8192x8192 bf16 matrix').
+    """Experts that are one square bf16 matrix each ([Beam] §3 [A]/[B]).
 
     y = sum_i w_i W_{ids_i} x with W_e [H_out, H_in].
     """
