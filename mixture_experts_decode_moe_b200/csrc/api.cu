@@ -102,15 +102,22 @@ moe_status check_weights(const moe_layer_desc* d, bool need_router) {
   return MOE_OK;
 }
 
-// Channels per job (template NCH): 8 for bf16 planar batch-1 decoding (96 KB
-// jobs, two stages), 4 otherwise.
+// Batch-1 bf16 rows of 2048: the kernel's warp-owned-channel path.
+inline bool fast_path(const moe_layer_desc* d, int B) {
+  return B == 1 && d->wtype == MOE_W_BF16 && d->H == 2048;
+}
+
+// Channels per job (template NCH). The warp-owned-channel path takes jobs of
+// 4 channels (48 KB stages, one warp per channel, two warp groups); other
+// bf16 planar batch-1 shapes take 8 (96 KB jobs), everything else 4.
 inline int pick_nch(const moe_layer_desc* d, int B) {
+  if (fast_path(d, B)) return 4;
   return (B == 1 && d->wtype == MOE_W_BF16 && d->layout == MOE_LAYOUT_PLANAR) ? 8 : 4;
 }
 
 // Shared-memory carve-up of the persistent decode kernel: as many ring stages
 // as fit next to the fixed tiles, given the kernel's static shared memory.
-bool plan_smem(DecodeParams* p, int static_bytes) {
+bool plan_smem(DecodeParams* p, int static_bytes, bool fast) {
   const int H = p->H, rowb = 2 * H, B = p->B, NCH = p->nch;
   const int budget = max_dyn_smem() - static_bytes - 1024;
   if (budget <= 0) return false;
@@ -120,16 +127,18 @@ bool plan_smem(DecodeParams* p, int static_bytes) {
   const int lg_bytes = (p->mode == MODE_LAYERS) ? (int)align_up((size_t)B * p->E * 4, 128) : 0;
   // keys: router top-k keys [B*E] and channel-sparse candidates [k*I]
   size_t nkeys = (p->mode == MODE_LAYERS) ? (size_t)B * p->E : 0;
-  if (cm) nkeys = std::max(nkeys, (size_t)p->k * p->I);
+  if (cm) nkeys = std::max(nkeys, (size_t)p->k * p->I + (size_t)p->k * p->I / 32 + 1);  // padded q + q / 32
   const int keys_bytes = (int)align_up(std::max<size_t>(nkeys, 1) * 4, 128);
   const int kept_bytes = cm ? (int)align_up((size_t)std::max(p->keep, 1) * 4, 128) : 0;
+  const int ysum_bytes = fast ? (int)align_up((size_t)H * 4, 128) : 0;
+  const int xf_bytes = fast ? H * 2 : 0;  // x fragments, [segment][lane] x 16 B
   int stage;
   if (cm || p->wtype == MOE_W_BF16) stage = NCH * 3 * rowb;
   else stage = NCH * (3 * (H / 2) + 2 * (H / 32)) + rowb;
   stage = std::max(stage, p->rows_per_job * rowb);
   if (p->I_sh > 0) stage = std::max(stage, NCH * 3 * rowb);
   stage = (int)align_up(stage, 128);
-  const int fixed = x_bytes + u_bytes + lg_bytes + keys_bytes + kept_bytes;
+  const int fixed = x_bytes + u_bytes + lg_bytes + keys_bytes + kept_bytes + ysum_bytes + xf_bytes;
   const int nst = std::min(8, (budget - fixed - 256) / stage);
   if (nst < 2) return false;
   p->stage_bytes = stage;
@@ -140,6 +149,8 @@ bool plan_smem(DecodeParams* p, int static_bytes) {
   p->off_lg = off; off += lg_bytes;
   p->off_keys = off; off += keys_bytes;
   p->off_kept = off; off += kept_bytes;
+  p->off_ysum = off; off += ysum_bytes;
+  p->off_xf = off; off += xf_bytes;
   p->off_bar = off; off += (int)align_up((size_t)3 * nst * 8, 128);  // full, empty, dots-ready
   p->smem_bytes = off;
   return true;
@@ -152,7 +163,8 @@ cudaError_t launch_decode_h(const DecodeParams& p0, int grid, cudaStream_t s) {
   cudaError_t err = cudaFuncGetAttributes(&fa, kern);
   if (err != cudaSuccess) return err;
   DecodeParams p = p0;
-  if (!plan_smem(&p, (int)fa.sharedSizeBytes)) return cudaErrorInvalidConfiguration;
+  constexpr bool kFast = (BMAX == 1 && WT == MOE_W_BF16 && HV == 8);
+  if (!plan_smem(&p, (int)fa.sharedSizeBytes, kFast)) return cudaErrorInvalidConfiguration;
   err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem_bytes);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
@@ -178,7 +190,7 @@ cudaError_t launch_decode_n(const DecodeParams& p, int grid, cudaStream_t s) {
 
 template <int MODE, int BMAX, int WT, int LAYOUT>
 cudaError_t launch_decode_m(const DecodeParams& p, int grid, cudaStream_t s) {
-  if constexpr (BMAX == 1 && WT == MOE_W_BF16 && LAYOUT == MOE_LAYOUT_PLANAR) {
+  if constexpr (BMAX == 1 && WT == MOE_W_BF16) {
     if (p.nch == 8) return launch_decode_n<MODE, BMAX, WT, LAYOUT, 8>(p, grid, s);
   }
   if (p.nch != 4) return cudaErrorInvalidValue;

@@ -67,7 +67,7 @@ struct DecodeParams {
   int nstages;
   int stage_bytes;
   // shared-memory carve-up (byte offsets from the dynamic smem base)
-  int off_x, off_u, off_lg, off_keys, off_kept, off_bar, smem_bytes;
+  int off_x, off_u, off_lg, off_keys, off_kept, off_ysum, off_xf, off_bar, smem_bytes;
   // io
   const uint16_t* x_in;   // [B, H]
   uint16_t* x_out;        // [B, H] final x (or null)
@@ -86,17 +86,18 @@ struct DecodeParams {
   LayerW layer[kMaxLayers];
 };
 
-// Per-CTA routing state in shared memory.
+// Per-CTA routing state in shared memory, sized for at most BMAX tokens.
+template <int BMAX>
 struct RouteSmem {
   int U;                     // routed units (touched experts, ascending)
   int ncand;                 // channel-sparse: number of kept channels
-  int unit_e[kMaxB * kMaxK];
-  uint32_t unit_mask[kMaxB * kMaxK];
-  float unit_w[kMaxB * kMaxK][kMaxB];
+  int unit_e[BMAX * kMaxK];
+  uint32_t unit_mask[BMAX * kMaxK];
+  float unit_w[BMAX * kMaxK][BMAX];
   uint32_t bitmap[kMaxE / 32];
   int rank_base[kMaxE / 32];
-  int ids[kMaxB][kMaxK];
-  float w[kMaxB][kMaxK];
+  int ids[BMAX][kMaxK];
+  float w[BMAX][kMaxK];
   uint32_t hist[256];
   int scan[kThreads];
   int sel_prefix, sel_rank;

@@ -155,14 +155,39 @@ __device__ __forceinline__ void warp_weights(const float* l, int k, float* w) {
   if (lane < k) w[lane] = e / s;
 }
 
+// Cross-warp sum of per-warp output accumulators (64 per lane, element
+// 256 c + 8 lane + e in acc[8 c + e]) into ysum (element 256 c + 8 lane + e
+// at 256 c + 32 e + lane): at step st warp W adds its chunk (W + st) % 8, so
+// no two warps touch a chunk at once; one barrier per step. W is a template
+// argument so that every register index is a constant.
+template <int W>
+__device__ __forceinline__ void ysum_steps(float (&acc)[64], float* ysum, int lane) {
+#pragma unroll
+  for (int st = 0; st < 8; ++st) {
+    const int c = (W + st) & 7;
+    float* yc = ysum + 256 * c + lane;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      yc[32 * e] = st == 0 ? acc[8 * c + e] : yc[32 * e] + acc[8 * c + e];
+      acc[8 * c + e] = 0.f;
+    }
+    cbar();
+  }
+}
+
 // ---------------------------------------------------------------- the kernel
 
 template <int MODE, int BMAX, int WT, int LAYOUT, int NCH, int HV>
 __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_constant__ DecodeParams p) {
   constexpr int NR = 2 * NCH;        // dot rows per job (gate+up rows; router rows)
   constexpr int NV = NR * BMAX;      // values reduced per job
+  // Batch-1 bf16 rows of 2048 elements: every warp owns whole channels (see
+  // consume_fast); job q goes to warp group q % kGroups of NCH warps.
+  constexpr bool kFast = (BMAX == 1 && WT == MOE_W_BF16 && HV == 8);
+  static_assert(!kFast || (NCH == 2 || NCH == 4 || NCH == 8), "warp groups of 2, 4 or 8 warps");
+  constexpr int kGroups = kFast ? kWarps / NCH : 1;
   extern __shared__ __align__(1024) uint8_t smem[];
-  __shared__ RouteSmem rs;
+  __shared__ RouteSmem<BMAX> rs;
   __shared__ int route_ready_s, abort_s, bad_s, okw_s;
   __shared__ long long jp_s, jc_s;
   __shared__ float dotbuf[16][NV];
@@ -194,7 +219,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
   if (tid == 0) {
     for (int s = 0; s < p.nstages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kWarps);
+      mbar_init(&empty[s], kFast ? NCH : kWarps);
       mbar_init(&hready[s], kWarps);
     }
     fence_mbar_init();
@@ -205,6 +230,8 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
   }
   for (int i = tid; i < B * H8; i += kCtaThreads)
     reinterpret_cast<uint4*>(xs)[i] = reinterpret_cast<const uint4*>(p.x_in)[i];
+  if constexpr (kFast)
+    for (int i = tid; i < H; i += kCtaThreads) reinterpret_cast<float*>(smem + p.off_ysum)[i] = 0.f;
   if (p.x_hist != nullptr) {
     const long long n = (long long)B * H8;
     for (long long i = cta * n / G + tid; i < (cta + 1) * n / G; i += kCtaThreads)
@@ -239,7 +266,9 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
         const int pos = cur.t;
         const int j0 = kept[pos];
         int n = 1;
-        while (n < NCH && cur.t + n < cur.t1 && kept[pos + n] == j0 + n && (j0 + n) % I != 0) ++n;
+        if (kFast) n = min(NCH, cur.t1 - cur.t);  // any kept channels, one per warp
+        else
+          while (n < NCH && cur.t + n < cur.t1 && kept[pos + n] == j0 + n && (j0 + n) % I != 0) ++n;
         j = Job{JOB_ROUTED, cur.layer, pos, j0, n};
         cur.t += n;
       } else {
@@ -306,9 +335,16 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
           bulk_g2s(dst + NCH * rowb, Lw.sh_up + off, bytes, bar, pol);
           bulk_g2s(dst + 2 * NCH * rowb, Lw.sh_down + off, bytes, bar, pol);
         } else if (LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR) {
-          const uint32_t bytes = (uint32_t)j.n * 3 * rowb;
-          mbar_expect_tx(bar, bytes);
-          bulk_g2s(dst, Lw.gate + (size_t)j.c0 * 3 * rowb, bytes, bar, pol);
+          // one copy per run of consecutive kept channels (12 KB per channel)
+          const uint32_t cb = 3u * (uint32_t)rowb;
+          mbar_expect_tx(bar, (uint32_t)j.n * cb);
+          for (int i = 0; i < j.n;) {
+            const int c0 = kept[j.u + i];
+            int r = 1;
+            while (i + r < j.n && kept[j.u + i + r] == c0 + r) ++r;
+            bulk_g2s(dst + (size_t)i * cb, Lw.gate + (size_t)c0 * cb, (uint32_t)r * cb, bar, pol);
+            i += r;
+          }
         } else if (WT == MOE_W_BF16) {
           const int n1 = min(j.n, I - j.c0);
           mbar_expect_tx(bar, 3u * (uint32_t)j.n * rowb);
@@ -364,9 +400,16 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
     const uint32_t all_tokens = (1u << B) - 1u;
     // tensor-core dots (B = 1, H = 2048): x fragments for the 8 segments
     constexpr bool kMmaDots = (BMAX == 1 && HV == 8);
-    uint32_t xf_frag[kMmaDots ? 8 : 1][4];
+    // fast path: the fragments live in shared memory, [segment][lane] x 16 B
+    uint32_t xf_frag[(kMmaDots && !kFast) ? 8 : 1][4];
+    uint4* xfs = reinterpret_cast<uint4*>(smem + p.off_xf);
     auto load_xfrag = [&]() {
-      if constexpr (kMmaDots) {
+      if constexpr (kFast) {
+        uint32_t f[4];
+        x_frag(us + 256 * warp, lane, f);
+        xfs[tid] = make_uint4(f[0], f[1], f[2], f[3]);
+        cbar();
+      } else if constexpr (kMmaDots) {
 #pragma unroll
         for (int t = 0; t < 8; ++t) x_frag(us + 256 * t, lane, xf_frag[t]);
       }
@@ -631,6 +674,100 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
       return ok;
     };
 
+    // ---- batch-1 bf16 fast path: a warp owns whole channels. Each job of the
+    // sequence goes to one warp group (NCH warps; job q to group q % kGroups);
+    // warp wi of the group takes channel wi of the job: its gate and up dots,
+    // h = w_e SiLU(g) u, and its down row, accumulated in 64 registers per
+    // lane (elements 256 i + 8 lane + e). Warps never wait for one another
+    // inside a job; the stage is released once the group's NCH warps arrive.
+    // Router jobs give warp wi the rows wi and wi + NCH.
+    float accf[kFast ? 64 : 1];
+#pragma unroll
+    for (int i = 0; i < (kFast ? 64 : 1); ++i) accf[i] = 0.f;
+    const int my_group = kFast ? warp / NCH : 0;
+    const int wi = kFast ? warp % NCH : 0;
+    // dots of one or two bf16 rows of 2048 elements with us (tensor-core
+    // diagonals, 8 segments of 256); every lane receives both sums
+    auto dot2 = [&](const uint8_t* r0, const uint8_t* r1, bool two, float& o0, float& o1) {
+      float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
+      float b0[4] = {0.f, 0.f, 0.f, 0.f}, b1[4] = {0.f, 0.f, 0.f, 0.f};
+      if constexpr (kFast) {
+        const uint32_t s0 = smem_u32(r0) + 16 * lane, s1 = smem_u32(r1) + 16 * lane;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          const uint4 xf = xfs[32 * t + lane];
+          uint32_t q0, q1, q2, q3;
+          ldmatrix_x4(s0 + 512 * t, q0, q1, q2, q3);
+          mma_bf16_16816(a0, q0, q1, q2, q3, xf.x, xf.y);
+          mma_bf16_16816(a1, q0, q1, q2, q3, xf.z, xf.w);
+          if (two) {
+            ldmatrix_x4(s1 + 512 * t, q0, q1, q2, q3);
+            mma_bf16_16816(b0, q0, q1, q2, q3, xf.x, xf.y);
+            mma_bf16_16816(b1, q0, q1, q2, q3, xf.z, xf.w);
+          }
+        }
+      }
+      o0 = warp_sum(diag_part(a0, a1, lane));
+      o1 = two ? warp_sum(diag_part(b0, b1, lane)) : 0.f;
+    };
+    auto consume_fast = [&](const Job& j) -> bool {
+      const int slot = cslot;
+      const uint32_t ph = cph;
+      bool ok = true;
+      if ((int)(jc % kGroups) == my_group) {
+        ok = wait_mb(&full[slot], ph);
+        if (ok) {
+          const uint8_t* st = ring + (size_t)slot * p.stage_bytes;
+          if (j.type == JOB_ROUTER) {
+            const int r0 = wi, r1 = wi + NCH;
+            if (r0 < j.n) {
+              float o0, o1;
+              dot2(st + r0 * rowb, st + r1 * rowb, r1 < j.n, o0, o1);
+              if (lane == 0) {
+                p.logits[j.c0 + r0] = o0;
+                if (r1 < j.n) p.logits[j.c0 + r1] = o1;
+              }
+            }
+          } else if (wi < j.n) {
+            const uint8_t *g, *u, *d;
+            float wt;
+            if (LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR && j.type == JOB_ROUTED) {
+              g = st + (size_t)wi * 3 * rowb;
+              u = g + rowb;
+              d = g + 2 * rowb;
+              const int e = kept[j.u + wi] / I;
+              int q = 0;
+              while (q < rs.U - 1 && rs.unit_e[q] != e) ++q;
+              wt = rs.unit_w[q][0];
+            } else {
+              g = st + wi * rowb;
+              u = g + NCH * rowb;
+              d = g + 2 * NCH * rowb;
+              if (j.type == JOB_SHARED) wt = 1.f;
+              else wt = rs.unit_w[j.u + (wi < I - j.c0 ? 0 : 1)][0];
+            }
+            float gv, uv;
+            dot2(g, u, true, gv, uv);
+            const float h = wt * silu_f(gv) * uv;
+            const uint4* d4 = reinterpret_cast<const uint4*>(d);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              float dv[8];
+              unpack8(d4[32 * i + lane], dv);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) accf[8 * i + e] = fmaf(h, dv[e], accf[8 * i + e]);
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[slot]);
+      }
+      if (++cslot == p.nstages) { cslot = 0; cph ^= 1u; }
+      ++jc;
+      if (!ok) *(volatile int*)&abort_s = 1;
+      return ok;
+    };
+
     // ---- pre-norm: us[b] = bf16(x[b] / sqrt(mean(x[b]^2) + eps)), unit weight
     auto normalize_x = [&]() {
       float ss[BMAX];
@@ -720,7 +857,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
       for (int u = tid; u < rs.U; u += kConsumers) {
         rs.unit_mask[u] = 0u;
 #pragma unroll
-        for (int b = 0; b < kMaxB; ++b) rs.unit_w[u][b] = 0.f;
+        for (int b = 0; b < BMAX; ++b) rs.unit_w[u][b] = 0.f;
       }
       for (int e = tid; e < E; e += kConsumers)
         if ((rs.bitmap[e >> 5] >> (e & 31)) & 1u)
@@ -742,22 +879,31 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
     // ---- top-k of every token from lg[B][E]
     // B = 1, k <= 8: every warp's largest key is >= T = the smallest of the
     // warp maxima, so at least 8 keys reach T and the k-th largest key is >= T.
-    // Only keys >= T are ranked (each against the other candidates); ties go to
-    // the lower index. The routed units (ascending expert id) are built in the
-    // same pass.
-    auto route_b1_small_k = [&]() {
+    // Only keys >= T are ranked: with at most 32 candidates every thread
+    // compares 4 candidate pairs and adds to a shared rank counter; ties go
+    // to the lower index. The routed units (ascending expert id) are built in
+    // the same pass. Logits come from lg[] or straight from the workspace.
+    auto route_b1_small_k = [&](bool from_ws) {
       uint32_t kq[4];
       uint32_t kmax = 0u;
       bool has = false;
+      // expert i sits in warp i % 8 (lane (i / 8) % 32, slot i / 256): every
+      // warp holds keys as soon as E >= 8
+      auto key_idx = [&](int q) { return kConsumers * q + kWarps * lane + warp; };
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const int idx = tid + kConsumers * q;
+        const int idx = key_idx(q);
         kq[q] = 0u;
-        if (idx < E) { kq[q] = float_key(lg[idx]); kmax = max(kmax, kq[q]); has = true; }
+        if (idx < E) {
+          kq[q] = float_key(from_ws ? __ldcg(p.logits + idx) : lg[idx]);
+          kmax = max(kmax, kq[q]);
+          has = true;
+        }
       }
       const uint32_t wm = __reduce_max_sync(0xffffffffu, kmax);
       const bool whas = __any_sync(0xffffffffu, has);
       if (lane == 0) { sel_pos[0][warp] = whas ? 1 : 0; cand_key[warp] = wm; }
+      if (warp == 0) sel_pos[1][lane] = 0;  // rank counters
       cbar();
       uint32_t T = 0xffffffffu;
       int nw = 0;
@@ -770,21 +916,20 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
       uint32_t ball[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const int idx = tid + kConsumers * q;
+        const int idx = key_idx(q);
         ball[q] = __ballot_sync(0xffffffffu, idx < E && kq[q] >= T);
         mine += __popc(ball[q]);
       }
-      cbar();  // everyone has read cand_key[] / sel_pos[0][]
-      if (lane == 0) sel_pos[1][warp] = mine;
+      if (lane == 0) sel_pos[2][warp] = mine;
       cbar();
       int base = 0, C = 0;
 #pragma unroll
       for (int w = 0; w < kWarps; ++w) {
-        const int c = sel_pos[1][w];
+        const int c = sel_pos[2][w];
         if (w < warp) base += c;
         C += c;
       }
-      int* cidx = reinterpret_cast<int*>(lg);  // logits are in kq[] now
+      int* cidx = reinterpret_cast<int*>(lg);
       {
         int off = base;
 #pragma unroll
@@ -792,40 +937,47 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
           if ((ball[q] >> lane) & 1u) {
             const int pos = off + __popc(ball[q] & ((1u << lane) - 1u));
             keys[pos] = kq[q];
-            cidx[pos] = tid + kConsumers * q;
+            cidx[pos] = key_idx(q);
           }
           off += __popc(ball[q]);
         }
       }
       cbar();
       if (C <= 32) {
-        // one warp ranks the candidates with shuffles and finishes the routing
+        {
+          const int i = tid & 31, j0 = (tid >> 5) * 4;
+          int cnt = 0;
+          if (i < C) {
+            const uint32_t ki = keys[i];
+            const int ii = cidx[i];
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+              const int jx = j0 + jj;
+              if (jx < C) {
+                const uint32_t kj = keys[jx];
+                cnt += (kj > ki) || (kj == ki && cidx[jx] < ii);
+              }
+            }
+          }
+          if (cnt) atomicAdd(&sel_pos[1][i], cnt);
+        }
+        cbar();
         if (warp == 0) {
-          const bool valid = lane < C;
-          const uint32_t kc = valid ? keys[lane] : 0u;
-          const int ic = valid ? cidx[lane] : 0x7fffffff;
-          int rank = 0;
-#pragma unroll 8
-          for (int o = 0; o < 32; ++o) {
-            const uint32_t ko = __shfl_sync(0xffffffffu, kc, o);
-            const int io = __shfl_sync(0xffffffffu, ic, o);
-            rank += (ko > kc) || (ko == kc && io < ic);
+          if (lane < C) {
+            const int r = sel_pos[1][lane];
+            if (r < k) { cand_key[kWarps + r] = keys[lane]; cand_idx[r] = cidx[lane]; }
           }
-          const bool sel = valid && rank < k;
-          const uint32_t top = __reduce_max_sync(0xffffffffu, valid ? kc : 0u);
-          const float e = sel ? __expf(key_float(kc) - key_float(top)) : 0.f;
-          const float ssum = warp_sum(e);
-          const float wl = e / ssum;
+          __syncwarp();
+          const bool sel = lane < k;
+          const uint32_t kc = sel ? cand_key[kWarps + lane] : 0u;
+          const int ic = sel ? cand_idx[lane] : 0x7fffffff;
+          const float e = sel ? __expf(key_float(kc) - key_float(cand_key[kWarps])) : 0.f;
+          const float wl = e / warp_sum(e);
           int urank = 0;
-#pragma unroll 8
-          for (int o = 0; o < 32; ++o) {
-            const int io = __shfl_sync(0xffffffffu, ic, o);
-            const bool so = __shfl_sync(0xffffffffu, sel, o);
-            urank += so && io < ic;
-          }
+          for (int m = 0; m < k; ++m) urank += cand_idx[m] < ic;
           if (sel) {
-            rs.ids[0][rank] = ic;
-            rs.w[0][rank] = wl;
+            rs.ids[0][lane] = ic;
+            rs.w[0][lane] = wl;
             rs.unit_e[urank] = ic;
             rs.unit_mask[urank] = 1u;
             rs.unit_w[urank][0] = wl;
@@ -913,101 +1065,139 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
     };
 
     // ---- channel-sparse selection (B = 1): kept[] ascending, rs.ncand
+    // Candidate q = u * I + c (routed unit u in ascending expert order,
+    // channel c). The keep-th largest key T is found bit by bit below the
+    // common prefix of all keys (count of keys >= T | bit, one warp reduction
+    // and one barrier per bit, keys held in registers); the kept set is every
+    // key > T plus the first r keys == T in index order (r = keep - #{> T}).
+    // The ascending list comes from contiguous per-thread chunks and one
+    // prefix scan. Keys sit in shared memory at q + q / 32 (conflict-free for
+    // both the row and the chunk walks).
     auto select_channels = [&](int l) {
+      constexpr int KR = kMaxCand / kConsumers;  // key rows per thread
       const int N = rs.U * I;
+      const int rows = (N + kConsumers - 1) / kConsumers;
       const float* sc = p.layer[l].scores;
-      for (int q = tid; q < N; q += kConsumers) {
-        const int u = q / I, c = q - u * I;
-        keys[q] = float_key(__ldg(sc + (size_t)rs.unit_e[u] * I + c));
-      }
-      cbar();
-      const int keep = p.keep;
-      uint32_t T = 0;
-      int rank = 0;
-      if (keep > 0 && keep < N) {
-        uint32_t prefix = 0, pmask = 0;
-        rank = keep;
-        for (int shift = 24; shift >= 0; shift -= 8) {
-          rs.hist[tid] = 0u;
-          cbar();
-          for (int q = tid; q < N; q += kConsumers) {
-            const uint32_t kk = keys[q];
-            if ((kk & pmask) == prefix) atomicAdd(&rs.hist[(kk >> shift) & 255u], 1u);
+      const float invI = 1.0f / (float)I;
+      auto pad = [](int q) { return q + (q >> 5); };
+      // 1. keys: row-major q = i * 256 + tid, all loads in flight at once
+      uint32_t kr[KR];
+      {
+        float kv[KR];
+#pragma unroll
+        for (int i = 0; i < KR; ++i) {
+          const int q = i * kConsumers + tid;
+          kv[i] = 0.f;
+          if (i < rows && q < N) {
+            const int u = __float2int_rz(((float)q + 0.5f) * invI);
+            kv[i] = __ldg(sc + (size_t)rs.unit_e[u] * I + (q - u * I));
           }
-          cbar();
-          if (warp == 0) {
-            uint32_t c8[8], loc = 0;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) { c8[i] = rs.hist[255 - 8 * lane - i]; loc += c8[i]; }
-            uint32_t inc = loc;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-              const uint32_t t = __shfl_up_sync(0xffffffffu, inc, o);
-              if (lane >= o) inc += t;
-            }
-            const uint32_t exc = inc - loc;
-            if (exc < (uint32_t)rank && (uint32_t)rank <= inc) {
-              uint32_t cum = exc;
-#pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                if (cum + c8[i] >= (uint32_t)rank) {
-                  rs.sel_rank = rank - (int)cum;
-                  rs.sel_prefix = (int)(prefix | ((uint32_t)(255 - 8 * lane - i) << shift));
-                  break;
-                }
-                cum += c8[i];
-              }
-            }
-          }
-          cbar();
-          prefix = (uint32_t)rs.sel_prefix;
-          rank = rs.sel_rank;
-          pmask |= 255u << shift;
         }
-        T = prefix;
-      }
-      const int chunk = (N + kConsumers - 1) / kConsumers;
-      const int lo = min(N, tid * chunk), hi = min(N, lo + chunk);
-      const bool all = keep >= N;
-      int eq = 0;
-      if (keep > 0 && !all)
-        for (int q = lo; q < hi; ++q) eq += (keys[q] == T);
-      int tot;
-      const int eq_before = block_excl_scan(eq, rs.scan, &tot);
-      auto kept_at = [&](int q, int& e_seen) -> bool {
-        if (keep <= 0) return false;
-        if (all) return true;
-        const uint32_t kk = keys[q];
-        const bool kp = kk > T || (kk == T && e_seen < rank);
-        e_seen += (kk == T);
-        return kp;
-      };
-      int cnt = 0;
-      {
-        int e_seen = eq_before;
-        for (int q = lo; q < hi; ++q) cnt += kept_at(q, e_seen);
-      }
-      const int pos0 = block_excl_scan(cnt, rs.scan, &tot);
-      {
-        int e_seen = eq_before, pos = pos0;
-        for (int q = lo; q < hi; ++q)
-          if (kept_at(q, e_seen) && pos < keep) {
-            const int u = q / I;
-            kept[pos++] = rs.unit_e[u] * I + (q - u * I);
+#pragma unroll
+        for (int i = 0; i < KR; ++i) {
+          const int q = i * kConsumers + tid;
+          kr[i] = 0u;
+          if (i < rows && q < N) {
+            kr[i] = float_key(kv[i]);
+            keys[pad(q)] = kr[i];
           }
+        }
       }
-      if (tid == 0) { rs.ncand = min(tot, keep); rs.sectors = 0ull; }
+      const int keep = p.keep;
+      const bool all = keep >= N;
+      uint32_t T = 0u;
+      int r = 0;
+      int* cnt_s = rs.scan;  // [2][8] per-warp counts, double-buffered
+      int par = 0;
+      // (absent keys are 0 and every threshold tried is >= 1)
+      auto count_ge = [&](uint32_t c) -> int {
+        int n = 0;
+#pragma unroll
+        for (int i0 = 0; i0 < KR; i0 += 8)
+          if (i0 < rows) {
+#pragma unroll
+            for (int i = i0; i < i0 + 8; ++i) n += kr[i] >= c ? 1 : 0;
+          }
+        n = (int)__reduce_add_sync(0xffffffffu, (uint32_t)n);
+        if (lane == 0) cnt_s[8 * par + warp] = n;
+        cbar();
+        int t = 0;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) t += cnt_s[8 * par + w];
+        par ^= 1;
+        return t;
+      };
+      if (keep > 0 && !all) {
+        // 2. common prefix of all keys (from the smallest and largest key)
+        uint32_t kmax = 0u, kmin = 0xffffffffu;
+#pragma unroll
+        for (int i = 0; i < KR; ++i)
+          if (i < rows && i * kConsumers + tid < N) { kmax = max(kmax, kr[i]); kmin = min(kmin, max(kr[i], 1u)); }
+        kmax = __reduce_max_sync(0xffffffffu, kmax);
+        kmin = __reduce_min_sync(0xffffffffu, kmin);
+        if (lane == 0) { cand_key[warp] = kmax; cand_key[kWarps + warp] = kmin; }
+        cbar();
+        kmax = 0u;
+        kmin = 0xffffffffu;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) { kmax = max(kmax, cand_key[w]); kmin = min(kmin, cand_key[kWarps + w]); }
+        const uint32_t diff = kmax ^ kmin;
+        const int top = diff ? 31 - __clz(diff) : -1;
+        T = top >= 0 ? kmax & ~(0xffffffffu >> (31 - top)) : kmax;  // the prefix, zeros below
+        // 3. largest T with #{key >= T} >= keep: the keep-th largest key
+        for (int bit = top; bit >= 0; --bit) {
+          const uint32_t c = T | (1u << bit);
+          if (count_ge(c) >= keep) T = c;
+        }
+        r = keep - (T == 0xffffffffu ? 0 : count_ge(T + 1u));
+      }
+      cbar();  // keys[] complete
+      // 4. ordered compaction over contiguous chunks: thread t takes
+      // q in [t * chunk, (t + 1) * chunk)
+      if (keep > 0) {
+        const int chunk = rows;  // ceil(N / 256)
+        const int q0 = min(N, tid * chunk), q1 = min(N, q0 + chunk);
+        int ng = 0, ne = 0;
+        for (int q = q0; q < q1; ++q) {
+          const uint32_t kk = keys[pad(q)];
+          ng += (all || kk > T) ? 1 : 0;
+          ne += (!all && kk == T) ? 1 : 0;
+        }
+        int tot;
+        const int pre = block_excl_scan(ng | (ne << 16), rs.scan + 16, &tot);
+        int pg = pre & 0xffff, pe = pre >> 16;
+        int u = __float2int_rz(((float)q0 + 0.5f) * invI), c = q0 - u * I;
+        for (int q = q0; q < q1; ++q) {
+          const uint32_t kk = keys[pad(q)];
+          const bool gt = all || kk > T;
+          const bool eq = !all && kk == T;
+          if (gt || (eq && pe < r)) kept[pg + min(pe, r)] = rs.unit_e[u] * I + c;
+          pg += gt ? 1 : 0;
+          pe += eq ? 1 : 0;
+          if (++c == I) { c = 0; ++u; }
+        }
+      }
+      if (tid == 0) rs.ncand = keep > 0 ? min(N, keep) : 0;
       cbar();
+      // sectors: each kept channel's byte range, less a sector shared with
+      // the previous kept channel; per-warp sums, then one add per warp
       const unsigned long long base = (unsigned long long)(uintptr_t)p.layer[l].gate;
       const unsigned long long cb = 3ull * rowb;
-      unsigned long long sec = 0;
+      uint32_t sec = 0;
       for (int i = tid; i < rs.ncand; i += kConsumers) {
         const unsigned long long s0 = (base + (unsigned long long)kept[i] * cb) >> 5;
         const unsigned long long s1 = (base + (unsigned long long)(kept[i] + 1) * cb - 1) >> 5;
-        sec += s1 - s0 + 1;
+        sec += (uint32_t)(s1 - s0 + 1);
         if (i > 0 && ((base + (unsigned long long)(kept[i - 1] + 1) * cb - 1) >> 5) == s0) sec -= 1;
       }
-      if (sec) atomicAdd(&rs.sectors, sec);
+      sec = __reduce_add_sync(0xffffffffu, sec);
+      if (lane == 0) rs.scan[warp] = (int)sec;
+      cbar();
+      if (tid == 0) {
+        unsigned long long t = 0;
+        for (int w = 0; w < kWarps; ++w) t += (uint32_t)rs.scan[w];
+        rs.sectors = t;
+      }
       cbar();
     };
 
@@ -1024,64 +1214,112 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
       int phase = (MODE == MODE_LAYERS) ? 0 : 1;
       int ready = l - 1;
       unsigned long long target = 0;
+      const bool route_early = kFast && MODE == MODE_LAYERS;
+      // routing of layer l: logits (after the router barrier) or the given
+      // ids -> routed units (and kept channels), published to the producer
+      auto do_route = [&]() -> bool {
+        constexpr bool kWarpRoute = MODE == MODE_LAYERS && BMAX == 1;
+        bool units_done = false;
+        if constexpr (MODE == MODE_LAYERS) {
+          if (kWarpRoute && k <= kWarps) {
+            if (tid == 0) okw_s = wait_grid(target) ? 1 : 0;
+            cbar();
+            if (!okw_s) { if (tid == 0) set_status(ctl, kStatusTimeout); return false; }
+            route_b1_small_k(true);
+            units_done = true;
+          } else {
+            if (tid == 0) okw_s = wait_grid(target) ? 1 : 0;
+            cbar();
+            if (!okw_s) { if (tid == 0) set_status(ctl, kStatusTimeout); return false; }
+            for (int i = tid; i < B * E; i += kConsumers) lg[i] = __ldcg(p.logits + i);
+            cbar();
+            if (BMAX == 1 && k <= kWarps) { route_b1_small_k(false); units_done = true; }
+            else route();
+          }
+          if (cta == 0 && p.ids_out != nullptr)
+            for (int t = tid; t < B * k; t += kConsumers) {
+              p.ids_out[(size_t)l * B * k + t] = rs.ids[t / k][t % k];
+              p.w_out[(size_t)l * B * k + t] = rs.w[t / k][t % k];
+            }
+        } else {
+          for (int t = tid; t < B * k; t += kConsumers) {
+            rs.ids[t / k][t % k] = p.ids_in[t];
+            rs.w[t / k][t % k] = p.w_in[t];
+          }
+          if (!grid_sync()) { if (tid == 0) set_status(ctl, kStatusTimeout); return false; }
+        }
+        if (!units_done && !build_units() && cta == 0 && tid == 0) set_status(ctl, kStatusBadIds);
+        if constexpr (LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR) {
+          select_channels(l);
+          if (cta == 0) {
+            if (p.kept_out != nullptr)
+              for (int i = tid; i < rs.ncand; i += kConsumers) p.kept_out[(size_t)l * p.keep + i] = kept[i];
+            if (tid == 0 && p.sectors_out != nullptr) p.sectors_out[l] = rs.sectors;
+          }
+        }
+        if (tid == 0) st_release_cta(&route_ready_s, l);
+        ready = l;
+        return true;
+      };
       for (;;) {
         const JobCursor save = ccur;
         const bool got = next_job(ccur, j, ready);
         const bool in_layer = got && j.type != JOB_END && j.layer == l;
         if (in_layer && j.type == phase) {
-          if (!consume(j)) { failed = true; break; }
+          bool okj;
+          if constexpr (kFast) okj = consume_fast(j);
+          else okj = consume(j);
+          if (!okj) { failed = true; break; }
           continue;
         }
         ccur = save;
         if (phase == 0) {
-          // router logits written: arrive at the grid barrier, keep working
+          // router logits written: arrive at the grid barrier; on the fast
+          // path route at once (the shared expert's compute then overlaps the
+          // routed copies' latency), else do the shared expert first
           cbar();
           if (tid == 0) target = arrive_grid();
+          if (route_early && !do_route()) { failed = true; break; }
           phase = 1;
           continue;
         }
         if (phase == 1) {
-          if constexpr (MODE == MODE_LAYERS) {
-            if (tid == 0) okw_s = wait_grid(target) ? 1 : 0;
-            cbar();
-            if (!okw_s) { failed = true; if (tid == 0) set_status(ctl, kStatusTimeout); break; }
-            for (int i = tid; i < B * E; i += kConsumers) lg[i] = __ldcg(p.logits + i);
-            cbar();
-            if (BMAX == 1 && k <= kWarps) route_b1_small_k();
-            else route();
-            if (cta == 0 && p.ids_out != nullptr)
-              for (int t = tid; t < B * k; t += kConsumers) {
-                p.ids_out[(size_t)l * B * k + t] = rs.ids[t / k][t % k];
-                p.w_out[(size_t)l * B * k + t] = rs.w[t / k][t % k];
-              }
-          } else {
-            for (int t = tid; t < B * k; t += kConsumers) {
-              rs.ids[t / k][t % k] = p.ids_in[t];
-              rs.w[t / k][t % k] = p.w_in[t];
-            }
-            if (!grid_sync()) { failed = true; if (tid == 0) set_status(ctl, kStatusTimeout); break; }
-          }
-          const bool units_done = MODE == MODE_LAYERS && BMAX == 1 && k <= kWarps;
-          if (!units_done && !build_units() && cta == 0 && tid == 0) set_status(ctl, kStatusBadIds);
-          if constexpr (LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR) {
-            select_channels(l);
-            if (cta == 0) {
-              if (p.kept_out != nullptr)
-                for (int i = tid; i < rs.ncand; i += kConsumers) p.kept_out[(size_t)l * p.keep + i] = kept[i];
-              if (tid == 0 && p.sectors_out != nullptr) p.sectors_out[l] = rs.sectors;
-            }
-          }
-          if (tid == 0) st_release_cta(&route_ready_s, l);
-          ready = l;
+          if (!(route_early || do_route())) { failed = true; break; }
           phase = 2;
           continue;
         }
+
         break;
       }
       if (cbar_or(failed)) { failed = true; break; }
       ccur.begin_layer(p, l + 1);
       // partial sums -> L2 accumulator
-      if (has_v) {
+      if constexpr (kFast) {
+        // warps -> shared sum in 8 steps: at step s warp w adds its chunk
+        // (w + s) % 8 (elements 256 c + 8 lane + e, stored at 256 c + 32 e +
+        // lane), so no two warps touch a chunk at once; then thread t adds
+        // elements 8t..8t+7 to the L2 accumulator
+        float* ysum = reinterpret_cast<float*>(smem + p.off_ysum);
+        switch (warp) {
+          case 0: ysum_steps<0>(accf, ysum, lane); break;
+          case 1: ysum_steps<1>(accf, ysum, lane); break;
+          case 2: ysum_steps<2>(accf, ysum, lane); break;
+          case 3: ysum_steps<3>(accf, ysum, lane); break;
+          case 4: ysum_steps<4>(accf, ysum, lane); break;
+          case 5: ysum_steps<5>(accf, ysum, lane); break;
+          case 6: ysum_steps<6>(accf, ysum, lane); break;
+          default: ysum_steps<7>(accf, ysum, lane); break;
+        }
+        float v[8];
+        {
+          const float* yt = ysum + 256 * (tid >> 5) + (tid & 31);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) v[e] = yt[32 * e];
+        }
+        float* dst = yacc + 8 * tid;
+        red_add_v4(dst, v[0], v[1], v[2], v[3]);
+        red_add_v4(dst + 4, v[4], v[5], v[6], v[7]);
+      } else if (has_v) {
 #pragma unroll
         for (int b = 0; b < BMAX; ++b)
           if (b < B) {
