@@ -13,7 +13,8 @@
 namespace moedec {
 
 constexpr int kConsumers = kThreads;          // 256 consumer threads
-constexpr int kCtaThreads = kThreads + 32;    // + one producer warp
+constexpr int kProducers = 2;                // producer warps (alternate jobs)
+constexpr int kCtaThreads = kThreads + 32 * kProducers;
 
 __device__ __forceinline__ void cbar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 __device__ __forceinline__ int cbar_or(int pred) {
@@ -188,8 +189,8 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
   constexpr int kGroups = kFast ? kWarps / NCH : 1;
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ RouteSmem<BMAX> rs;
-  __shared__ int route_ready_s, abort_s, bad_s, okw_s;
-  __shared__ long long jp_s, jc_s;
+  __shared__ int route_ready_s, prod_layer_s[kProducers], abort_s, bad_s, okw_s;
+  __shared__ long long jp_s[kProducers], jc_s;
   __shared__ float dotbuf[16][NV];
   __shared__ float hbuf[kWarps][NCH * BMAX];
   __shared__ uint32_t cand_key[kWarps * kMaxK];
@@ -223,9 +224,12 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
       mbar_init(&hready[s], kWarps);
     }
     fence_mbar_init();
-    route_ready_s = -1;
+    route_ready_s = -1;  // last layer whose routing the consumers published
+    for (int q = 0; q < kProducers; ++q) {
+      prod_layer_s[q] = -1;  // last layer whose routed jobs producer q issued
+      jp_s[q] = 0;           // jobs producer q has passed (its own ones issued)
+    }
     abort_s = 0;
-    jp_s = 0;
     jc_s = 0;
   }
   for (int i = tid; i < B * H8; i += kCtaThreads)
@@ -290,95 +294,129 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
   };
 
   // ================================================================ producer
-  if (warp == kWarps) {
-    if (lane == 0) {
-      const uint64_t pol = policy_evict_first();
-      JobCursor pc;
-      pc.begin_layer(p, 0);
-      long long jp = 0;
-      int pslot = 0;
-      uint32_t pph = 0;
-      for (;;) {
-        Job j;
-        JobCursor save = pc;
-        if (!next_job(pc, j, ld_acquire_cta(&route_ready_s))) {
-          // routed jobs of this layer: wait until the consumers publish routing
-          pc = save;
-          const long long t0 = clock64();
-          while (ld_acquire_cta(&route_ready_s) < pc.layer) {
-            if (ld_acquire_cta(&abort_s) || clock64() - t0 > kWaitBudgetCycles) goto producer_done;
-            __nanosleep(64);
-          }
-          continue;
+  // The whole warp walks the job sequence (uniform control flow: every lane
+  // computes the same job); lane 0 arms the stage's barrier with the job's
+  // byte count and issues its copies. Routed jobs of layer l wait until the
+  // consumers publish routing for layer l.
+  if (warp >= kWarps) {
+    // producer pi issues the jobs q with q % kProducers == pi; both walk the
+    // whole sequence so that slots and phases stay in step
+    const int pi = warp - kWarps;
+    const uint64_t pol = policy_evict_first();
+    JobCursor pc;
+    pc.begin_layer(p, 0);
+    long long jp = 0;
+    int pslot = 0;
+    uint32_t pph = 0;
+    int ready = -1;  // routing of layers <= ready is known
+    int pub = -1;    // last value published to prod_layer_s
+    for (;;) {
+      Job j;
+      const bool got = next_job(pc, j, ready);
+      {
+        // once the cursor reaches layer cl, the routing of cl - 1 is no
+        // longer read here: let the consumers overwrite it
+        const int cl = !got ? pc.layer : (j.type == JOB_END ? p.L : j.layer);
+        if (cl - 1 > pub) {
+          pub = cl - 1;
+          if (lane == 0) st_release_cta(&prod_layer_s[pi], pub);
         }
-        if (j.type == JOB_END) break;
-        const int slot = pslot;
-        if (jp >= p.nstages) {
-          const uint32_t par = pph ^ 1u;
-          const long long t0 = clock64();
-          while (!mbar_try_wait_sleep(&empty[slot], par, 20000)) {
-            if (ld_acquire_cta(&abort_s) || clock64() - t0 > kWaitBudgetCycles) goto producer_done;
-          }
+      }
+      if (!got) {
+        // the cursor stopped at the routed jobs of pc.layer: spin (no sleep,
+        // so the first copies follow the routing at once) until the
+        // consumers publish a routed layer >= pc.layer. The published value
+        // only grows, so a producer that falls behind a CTA without work in
+        // some layers still reads it correctly.
+        const long long t0 = clock64();
+        int rl;
+        while ((rl = ld_acquire_cta(&route_ready_s)) < pc.layer) {
+          if (*(volatile int*)&abort_s || clock64() - t0 > kWaitBudgetCycles) goto producer_done;
         }
+        ready = pc.layer;
+        (void)rl;
+        continue;
+      }
+      if (j.type == JOB_END) break;
+      const int slot = pslot;
+      if ((int)(jp % kProducers) != pi) {
+        ++jp;
+        if (++pslot == p.nstages) { pslot = 0; pph ^= 1u; }
+        continue;
+      }
+      if (jp >= p.nstages) {
+        const uint32_t par = pph ^ 1u;
+        const long long t0 = clock64();
+        while (!mbar_try_wait_sleep(&empty[slot], par, 20000)) {
+          if (*(volatile int*)&abort_s || clock64() - t0 > kWaitBudgetCycles) goto producer_done;
+        }
+      }
+      {
         uint64_t* bar = &full[slot];
         uint8_t* dst = ring + (size_t)slot * p.stage_bytes;
         const LayerW& Lw = p.layer[j.layer];
-        if (j.type == JOB_ROUTER) {
-          const uint32_t bytes = (uint32_t)j.n * rowb;
-          mbar_expect_tx(bar, bytes);
-          bulk_g2s(dst, Lw.router + (size_t)j.c0 * rowb, bytes, bar, pol);
-        } else if (j.type == JOB_SHARED) {
-          const uint32_t bytes = (uint32_t)j.n * rowb;
-          const size_t off = (size_t)j.c0 * rowb;
-          mbar_expect_tx(bar, 3 * bytes);
-          bulk_g2s(dst, Lw.sh_gate + off, bytes, bar, pol);
-          bulk_g2s(dst + NCH * rowb, Lw.sh_up + off, bytes, bar, pol);
-          bulk_g2s(dst + 2 * NCH * rowb, Lw.sh_down + off, bytes, bar, pol);
-        } else if (LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR) {
-          // one copy per run of consecutive kept channels (12 KB per channel)
-          const uint32_t cb = 3u * (uint32_t)rowb;
-          mbar_expect_tx(bar, (uint32_t)j.n * cb);
-          for (int i = 0; i < j.n;) {
-            const int c0 = kept[j.u + i];
-            int r = 1;
-            while (i + r < j.n && kept[j.u + i + r] == c0 + r) ++r;
-            bulk_g2s(dst + (size_t)i * cb, Lw.gate + (size_t)c0 * cb, (uint32_t)r * cb, bar, pol);
-            i += r;
+        // lane 0 issues the job's copies one after another (one thread
+        // issuing is faster than several issuing at once)
+        if (lane == 0) {
+          if (j.type == JOB_ROUTER) {
+            const uint32_t bytes = (uint32_t)j.n * rowb;
+            mbar_expect_tx(bar, bytes);
+            bulk_g2s(dst, Lw.router + (size_t)j.c0 * rowb, bytes, bar, pol);
+          } else if (j.type == JOB_SHARED) {
+            const uint32_t bytes = (uint32_t)j.n * rowb;
+            const size_t off = (size_t)j.c0 * rowb;
+            mbar_expect_tx(bar, 3 * bytes);
+            bulk_g2s(dst, Lw.sh_gate + off, bytes, bar, pol);
+            bulk_g2s(dst + NCH * rowb, Lw.sh_up + off, bytes, bar, pol);
+            bulk_g2s(dst + 2 * NCH * rowb, Lw.sh_down + off, bytes, bar, pol);
+          } else if (LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR) {
+            // one copy per run of consecutive kept channels (12 KB each)
+            const uint32_t cb = 3u * (uint32_t)rowb;
+            mbar_expect_tx(bar, (uint32_t)j.n * cb);
+            for (int i = 0; i < j.n;) {
+              const int c0 = kept[j.u + i];
+              int r = 1;
+              while (i + r < j.n && kept[j.u + i + r] == c0 + r) ++r;
+              bulk_g2s(dst + (size_t)i * cb, Lw.gate + (size_t)c0 * cb, (uint32_t)r * cb, bar, pol);
+              i += r;
+            }
+          } else if (WT == MOE_W_BF16) {
+            // a job may run on into the next expert: two segments at most
+            const int n1 = min(j.n, I - j.c0);
+            mbar_expect_tx(bar, 3u * (uint32_t)j.n * rowb);
+            for (int sg = 0; sg < 2; ++sg) {
+              const int ns = sg ? j.n - n1 : n1;
+              if (ns <= 0) break;
+              const int e = rs.unit_e[j.u + sg];
+              const uint32_t bytes = (uint32_t)ns * rowb;
+              const size_t off = ((size_t)e * I + (sg ? 0 : j.c0)) * rowb;
+              uint8_t* d0 = dst + (sg ? n1 : 0) * rowb;
+              bulk_g2s(d0, Lw.gate + off, bytes, bar, pol);
+              bulk_g2s(d0 + NCH * rowb, Lw.up + off, bytes, bar, pol);
+              bulk_g2s(d0 + 2 * NCH * rowb, Lw.down + off, bytes, bar, pol);
+            }
+          } else {
+            const int e = rs.unit_e[j.u];
+            const int rowc = H >> 1, rows = H >> 5;
+            const uint32_t cb = (uint32_t)j.n * rowc, sb = (uint32_t)j.n * rows;
+            const size_t offc = ((size_t)e * I + j.c0) * rowc, offs = ((size_t)e * I + j.c0) * rows;
+            const size_t offd = ((size_t)e * (I >> 6) + (j.c0 >> 6)) * rowb;
+            mbar_expect_tx(bar, 3 * cb + 2 * sb + rowb);
+            bulk_g2s(dst, Lw.gate + offc, cb, bar, pol);
+            bulk_g2s(dst + NCH * rowc, Lw.up + offc, cb, bar, pol);
+            bulk_g2s(dst + 2 * NCH * rowc, Lw.down + offc, cb, bar, pol);
+            bulk_g2s(dst + 3 * NCH * rowc, Lw.gate_s + offs, sb, bar, pol);
+            bulk_g2s(dst + 3 * NCH * rowc + NCH * rows, Lw.up_s + offs, sb, bar, pol);
+            bulk_g2s(dst + 3 * NCH * rowc + 2 * NCH * rows, Lw.down_s + offd, rowb, bar, pol);
           }
-        } else if (WT == MOE_W_BF16) {
-          const int n1 = min(j.n, I - j.c0);
-          mbar_expect_tx(bar, 3u * (uint32_t)j.n * rowb);
-          for (int sg = 0; sg < 2; ++sg) {
-            const int ns = sg ? j.n - n1 : n1;
-            if (ns <= 0) break;
-            const int e = rs.unit_e[j.u + sg];
-            const uint32_t bytes = (uint32_t)ns * rowb;
-            const size_t off = ((size_t)e * I + (sg ? 0 : j.c0)) * rowb;
-            uint8_t* d0 = dst + (sg ? n1 : 0) * rowb;
-            bulk_g2s(d0, Lw.gate + off, bytes, bar, pol);
-            bulk_g2s(d0 + NCH * rowb, Lw.up + off, bytes, bar, pol);
-            bulk_g2s(d0 + 2 * NCH * rowb, Lw.down + off, bytes, bar, pol);
-          }
-        } else {
-          const int e = rs.unit_e[j.u];
-          const int rowc = H >> 1, rows = H >> 5;
-          const uint32_t cb = (uint32_t)j.n * rowc, sb = (uint32_t)j.n * rows;
-          const size_t offc = ((size_t)e * I + j.c0) * rowc, offs = ((size_t)e * I + j.c0) * rows;
-          const size_t offd = ((size_t)e * (I >> 6) + (j.c0 >> 6)) * rowb;
-          mbar_expect_tx(bar, 3 * cb + 2 * sb + rowb);
-          bulk_g2s(dst, Lw.gate + offc, cb, bar, pol);
-          bulk_g2s(dst + NCH * rowc, Lw.up + offc, cb, bar, pol);
-          bulk_g2s(dst + 2 * NCH * rowc, Lw.down + offc, cb, bar, pol);
-          bulk_g2s(dst + 3 * NCH * rowc, Lw.gate_s + offs, sb, bar, pol);
-          bulk_g2s(dst + 3 * NCH * rowc + NCH * rows, Lw.up_s + offs, sb, bar, pol);
-          bulk_g2s(dst + 3 * NCH * rowc + 2 * NCH * rows, Lw.down_s + offd, rowb, bar, pol);
         }
-        ++jp;
-        if (++pslot == p.nstages) { pslot = 0; pph ^= 1u; }
-        *(volatile long long*)&jp_s = jp;
+        __syncwarp();
       }
-    producer_done:;
+      ++jp;
+      if (++pslot == p.nstages) { pslot = 0; pph ^= 1u; }
+      if (lane == 0) *(volatile long long*)&jp_s[pi] = jp;
     }
+  producer_done:;
     __syncwarp();
   } else {
     // ============================================================== consumers
@@ -1220,6 +1258,14 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
       auto do_route = [&]() -> bool {
         constexpr bool kWarpRoute = MODE == MODE_LAYERS && BMAX == 1;
         bool units_done = false;
+        // the producer must be done with the previous layer's routing
+        // before it is overwritten (it always is, unless this CTA had no
+        // work at all in some layers)
+        if (tid == 0 && l > 0) {
+          const long long t0 = clock64();
+          while (min(ld_acquire_cta(&prod_layer_s[0]), ld_acquire_cta(&prod_layer_s[1])) < l - 1)
+            if (clock64() - t0 > kWaitBudgetCycles) { set_status(ctl, kStatusTimeout); break; }
+        }
         if constexpr (MODE == MODE_LAYERS) {
           if (kWarpRoute && k <= kWarps) {
             if (tid == 0) okw_s = wait_grid(target) ? 1 : 0;
@@ -1372,8 +1418,10 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
   // on an error path, wait (bounded) for the copies still in flight so that
   // none lands in shared memory after the CTA has exited
   if (tid == 0 && abort_s) {
-    const long long issued = jp_s;
-    for (long long q = jc_s; q < issued; ++q) mbar_wait(&full[q % p.nstages], (uint32_t)((q / p.nstages) & 1));
+    // job q was issued iff producer q % kProducers got past it
+    const long long issued = max(jp_s[0], jp_s[1]);
+    for (long long q = jc_s; q < issued; ++q)
+      if (q < jp_s[q % kProducers]) mbar_wait(&full[q % p.nstages], (uint32_t)((q / p.nstages) & 1));
   }
 }
 
