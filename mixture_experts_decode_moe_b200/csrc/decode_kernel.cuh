@@ -323,18 +323,18 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
         }
       }
       if (!got) {
-        // the cursor stopped at the routed jobs of pc.layer: spin (no sleep,
-        // so the first copies follow the routing at once) until the
-        // consumers publish a routed layer >= pc.layer. The published value
-        // only grows, so a producer that falls behind a CTA without work in
-        // some layers still reads it correctly.
+        // the cursor stopped at the routed jobs of pc.layer: poll (plain
+        // loads and short sleeps, which leave the shared-memory pipe to the
+        // consumers routing meanwhile) until the consumers publish a routed
+        // layer >= pc.layer, then one acquire load orders the reads of the
+        // routing after it. The published value only grows.
         const long long t0 = clock64();
-        int rl;
-        while ((rl = ld_acquire_cta(&route_ready_s)) < pc.layer) {
+        while (*(volatile int*)&route_ready_s < pc.layer) {
           if (*(volatile int*)&abort_s || clock64() - t0 > kWaitBudgetCycles) goto producer_done;
+          __nanosleep(20);
         }
+        (void)ld_acquire_cta(&route_ready_s);
         ready = pc.layer;
-        (void)rl;
         continue;
       }
       if (j.type == JOB_END) break;
@@ -441,12 +441,41 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
     // fast path: the fragments live in shared memory, [segment][lane] x 16 B
     uint32_t xf_frag[(kMmaDots && !kFast) ? 8 : 1][4];
     uint4* xfs = reinterpret_cast<uint4*>(smem + p.off_xf);
+    // fast path: thread t owns elements 8t..8t+7 of x (4 bf16 words). With
+    // the pre-norm their u = bf16(x * rsqrt(mean(x^2) + eps)), else u = x;
+    // word m of thread t (segment s = t / 32) is word o + 32 k' of that
+    // segment's fragment table with o = 4 (t % 8) + m and k' = (t / 8) % 4,
+    // i.e. component {0, 2, 1, 3}[k'] of lane 4 (t % 8) + m: each thread
+    // writes its own words, no pass through a u buffer.
+    auto fast_frags = [&](const float* xv, bool norm) {
+      float sc = 1.f;
+      if (norm) {
+        float ss = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) ss = fmaf(xv[i], xv[i], ss);
+        ss = warp_sum(ss);
+        if (lane == 0) hbuf[warp][0] = ss;
+        cbar();
+        float t = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) t += hbuf[w][0];
+        sc = rsqrtf(t / (float)H + 1e-6f);
+      }
+      uint32_t* xw = reinterpret_cast<uint32_t*>(xfs);
+      const int seg = tid >> 5, kk = (tid >> 3) & 3;
+      const int comp = (kk == 1) ? 2 : (kk == 2 ? 1 : kk);
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const uint32_t w = uint32_t(f_to_bf16(xv[2 * m] * sc)) | (uint32_t(f_to_bf16(xv[2 * m + 1] * sc)) << 16);
+        xw[(seg * 32 + 4 * (tid & 7) + m) * 4 + comp] = w;
+      }
+      cbar();
+    };
     auto load_xfrag = [&]() {
       if constexpr (kFast) {
-        uint32_t f[4];
-        x_frag(us + 256 * warp, lane, f);
-        xfs[tid] = make_uint4(f[0], f[1], f[2], f[3]);
-        cbar();
+        float xv[8];
+        unpack8(xs4[tid], xv);
+        fast_frags(xv, MODE == MODE_LAYERS && p.pre_norm);
       } else if constexpr (kMmaDots) {
 #pragma unroll
         for (int t = 0; t < 8; ++t) x_frag(us + 256 * t, lane, xf_frag[t]);
@@ -748,25 +777,51 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
       o0 = warp_sum(diag_part(a0, a1, lane));
       o1 = two ? warp_sum(diag_part(b0, b1, lane)) : 0.f;
     };
+    // named barrier of this warp's group (ids 2.., NCH warps)
+    auto group_bar = [&]() {
+      asm volatile("bar.sync %0, %1;" ::"r"(2 + my_group), "r"(NCH * 32) : "memory");
+    };
     auto consume_fast = [&](const Job& j) -> bool {
       const int slot = cslot;
       const uint32_t ph = cph;
       bool ok = true;
       if ((int)(jc % kGroups) == my_group) {
         ok = wait_mb(&full[slot], ph);
-        if (ok) {
-          const uint8_t* st = ring + (size_t)slot * p.stage_bytes;
-          if (j.type == JOB_ROUTER) {
-            const int r0 = wi, r1 = wi + NCH;
-            if (r0 < j.n) {
-              float o0, o1;
-              dot2(st + r0 * rowb, st + r1 * rowb, r1 < j.n, o0, o1);
-              if (lane == 0) {
-                p.logits[j.c0 + r0] = o0;
-                if (r1 < j.n) p.logits[j.c0 + r1] = o1;
+        if (j.type == JOB_ROUTER) {
+          // rows split over K: warp wi of the group takes segments
+          // [wi * SPW, (wi + 1) * SPW) of every row; partials meet in
+          // dotbuf (double-buffered by job) after a group barrier that every
+          // warp of the group reaches, and warp 0 of the group writes
+          constexpr int SPW = 8 / NCH;
+          float* part = dotbuf[warp + kWarps * (int)((jc / kGroups) & 1)];
+          if (ok) {
+            const uint8_t* st = ring + (size_t)slot * p.stage_bytes;
+            const uint32_t sbase = smem_u32(st) + 16 * lane;
+            for (int r = 0; r < j.n; ++r) {
+              float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+              for (int q = 0; q < SPW; ++q) {
+                const int t = wi * SPW + q;
+                const uint4 xf = xfs[32 * t + lane];
+                uint32_t q0, q1, q2, q3;
+                ldmatrix_x4(sbase + r * rowb + 512 * t, q0, q1, q2, q3);
+                mma_bf16_16816(a0, q0, q1, q2, q3, xf.x, xf.y);
+                mma_bf16_16816(a1, q0, q1, q2, q3, xf.z, xf.w);
               }
+              const float pv = warp_sum(diag_part(a0, a1, lane));
+              if (lane == 0) part[r] = pv;
             }
-          } else if (wi < j.n) {
+          }
+          group_bar();
+          if (ok && wi == 0 && lane < j.n) {
+            float t = 0.f;
+#pragma unroll
+            for (int w = 0; w < NCH; ++w) t += dotbuf[my_group * NCH + w + kWarps * (int)((jc / kGroups) & 1)][lane];
+            p.logits[j.c0 + lane] = t;
+          }
+        } else if (ok) {
+          const uint8_t* st = ring + (size_t)slot * p.stage_bytes;
+          if (wi < j.n) {
             const uint8_t *g, *u, *d;
             float wt;
             if (LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR && j.type == JOB_ROUTED) {
@@ -841,7 +896,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
         }
       cbar();
     };
-    if constexpr (MODE == MODE_LAYERS)
+    if constexpr (MODE == MODE_LAYERS && !kFast)
       if (p.pre_norm) normalize_x();
     load_xfrag();
 
@@ -1263,8 +1318,12 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
         // work at all in some layers)
         if (tid == 0 && l > 0) {
           const long long t0 = clock64();
-          while (min(ld_acquire_cta(&prod_layer_s[0]), ld_acquire_cta(&prod_layer_s[1])) < l - 1)
+          while (min(*(volatile int*)&prod_layer_s[0], *(volatile int*)&prod_layer_s[1]) < l - 1) {
             if (clock64() - t0 > kWaitBudgetCycles) { set_status(ctl, kStatusTimeout); break; }
+            __nanosleep(20);
+          }
+          (void)ld_acquire_cta(&prod_layer_s[0]);
+          (void)ld_acquire_cta(&prod_layer_s[1]);
         }
         if constexpr (MODE == MODE_LAYERS) {
           if (kWarpRoute && k <= kWarps) {
@@ -1382,7 +1441,37 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
       const long long s0 = cta * n4 / G, s1 = (cta + 1) * n4 / G;
       float* yh = p.y_hist ? p.y_hist + (size_t)l * B * H : nullptr;
       float* yo = (l == p.L - 1) ? p.y_out : nullptr;
-      if constexpr (MODE == MODE_LAYERS) {
+      if constexpr (MODE == MODE_LAYERS && kFast) {
+        // thread t: elements 8t..8t+7 (float4 slots 2t, 2t+1)
+        const float4 ya = __ldcg(reinterpret_cast<const float4*>(yacc) + 2 * tid);
+        const float4 yb = __ldcg(reinterpret_cast<const float4*>(yacc) + 2 * tid + 1);
+        float xv[8];
+        unpack8(xs4[tid], xv);
+        const float yv[8] = {ya.x, ya.y, ya.z, ya.w, yb.x, yb.y, yb.z, yb.w};
+        uint4 xn;
+        uint32_t* xnw = reinterpret_cast<uint32_t*>(&xn);
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const uint16_t lo = f_to_bf16(xv[2 * m] + yv[2 * m]), hi = f_to_bf16(xv[2 * m + 1] + yv[2 * m + 1]);
+          xnw[m] = uint32_t(lo) | (uint32_t(hi) << 16);
+          xv[2 * m] = bf16_to_f(lo);
+          xv[2 * m + 1] = bf16_to_f(hi);
+        }
+        reinterpret_cast<uint4*>(xs)[tid] = xn;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const long long i = 2 * tid + h;
+          if (i >= s0 && i < s1) {
+            const float4 y4 = h ? yb : ya;
+            const uint2 x2 = make_uint2(xnw[2 * h], xnw[2 * h + 1]);
+            if (yh) reinterpret_cast<float4*>(yh)[i] = y4;
+            if (yo) reinterpret_cast<float4*>(yo)[i] = y4;
+            if (p.x_hist) reinterpret_cast<uint2*>(p.x_hist + (size_t)(l + 1) * B * H)[i] = x2;
+            if (l == p.L - 1 && p.x_out) reinterpret_cast<uint2*>(p.x_out)[i] = x2;
+          }
+        }
+        fast_frags(xv, p.pre_norm != 0);
+      } else if constexpr (MODE == MODE_LAYERS) {
         for (long long i = tid; i < n4; i += kConsumers) {
           const float4 y4 = __ldcg(reinterpret_cast<const float4*>(yacc) + i);
           uint2 xv = reinterpret_cast<uint2*>(xs)[i];
