@@ -243,7 +243,7 @@ moe_status moe_touched_experts(const int32_t* ids, int32_t B, int32_t k, int32_t
  *    (the value moe_get_status() would report) after the kernel, stream-ordered.
  *  - Nothing is allocated or freed: no cudaMalloc/cudaFree, no library routine
  *    that allocates. */
-#define MOE_STATIC_SCRATCH_BYTES (144u * 1024u)
+#define MOE_STATIC_SCRATCH_BYTES (256u * 1024u)
 moe_status moe_layer_forward_static(const moe_layer_desc* desc, const void* x, int32_t B, float* y,
                                     void* x_next_opt, int32_t* ids_out_opt, float* w_out_opt,
                                     int32_t* status_out_opt, moe_stream_t stream);

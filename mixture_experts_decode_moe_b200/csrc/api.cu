@@ -28,10 +28,10 @@ struct WsLayout {
 inline WsLayout ws_layout(int B, int H, int E) {
   WsLayout w;
   size_t off = sizeof(WsControl);
-  w.logits = off;
-  off = align_up(off + (size_t)B * E * sizeof(float));
-  w.yacc = off;
-  off = align_up(off + 2 * (size_t)B * H * sizeof(float));
+  w.logits = off;  // 8 bytes per logit: {value, tag} on the batch-1 path
+  off = align_up(off + (size_t)B * E * sizeof(unsigned long long));
+  w.yacc = off;     // three layer accumulators in rotation
+  off = align_up(off + 3 * (size_t)B * H * sizeof(float));
   w.total = off;
   return w;
 }
@@ -108,10 +108,11 @@ inline bool fast_path(const moe_layer_desc* d, int B) {
 }
 
 // Channels per job (template NCH). The warp-owned-channel path takes jobs of
-// 4 channels (48 KB stages, one warp per channel, two warp groups); other
-// bf16 planar batch-1 shapes take 8 (96 KB jobs), everything else 4.
+// 8 channels for planar experts (96 KB stages, one warp per channel) and 4
+// for channel-major ones (48 KB stages, two warp groups, room for the
+// selection buffers); other bf16 planar batch-1 shapes take 8, the rest 4.
 inline int pick_nch(const moe_layer_desc* d, int B) {
-  if (fast_path(d, B)) return 4;
+  if (fast_path(d, B)) return d->layout == MOE_LAYOUT_PLANAR ? 8 : 4;
   return (B == 1 && d->wtype == MOE_W_BF16 && d->layout == MOE_LAYOUT_PLANAR) ? 8 : 4;
 }
 
@@ -610,8 +611,11 @@ extern "C" moe_status moe_layer_forward_static(const moe_layer_desc* desc, const
   moe_status st = static_scratch_address(&scratch);
   if (st != MOE_OK) return st;
   cudaStream_t s = (cudaStream_t)stream;
-  // the previous call's status word and barrier counter must not leak into this one
-  if (cudaMemsetAsync(scratch, 0, sizeof(WsControl), s) != cudaSuccess) return MOE_ERR_CUDA;
+  // the previous call's status word and barrier counter must not leak into
+  // this one; the counter restarts, so the tagged logit words of the previous
+  // call (which carry the same tags) are cleared as well
+  const WsLayout wl = ws_layout(B, desc->H, desc->E);
+  if (cudaMemsetAsync(scratch, 0, wl.yacc, s) != cudaSuccess) return MOE_ERR_CUDA;
   st = moe_layer_forward(desc, x, B, y, x_next_opt, ids_out_opt, w_out_opt, scratch, MOE_STATIC_SCRATCH_BYTES,
                          stream);
   if (st != MOE_OK) return st;

@@ -39,6 +39,9 @@ __device__ __forceinline__ unsigned long long ld_relaxed_gpu(const unsigned long
   asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
   return v;
 }
+__device__ __forceinline__ void st_relaxed_gpu_u64(unsigned long long* p, unsigned long long v) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
 __device__ __forceinline__ int ld_acquire_cta(const int* p) {
   int v;
   asm volatile("ld.acquire.cta.shared::cta.s32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
@@ -190,6 +193,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ RouteSmem<BMAX> rs;
   __shared__ int route_ready_s, prod_layer_s[kProducers], abort_s, bad_s, okw_s;
+  __shared__ uint32_t ltag_s;  // logit tag of layer 0 in this launch (fast path)
   __shared__ long long jp_s[kProducers], jc_s;
   __shared__ float dotbuf[16][NV];
   __shared__ float hbuf[kWarps][NCH * BMAX];
@@ -426,7 +430,15 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
     uint32_t cph = 0;       // its phase parity
     long long jc = 0;       // jobs consumed
     unsigned long long bar_base = 0, nbar = 0;
-    if (tid == 0) bar_base = (ld_relaxed_gpu(&ctl->bar) / (unsigned long long)G) * (unsigned long long)G;
+    if (tid == 0) {
+      bar_base = (ld_relaxed_gpu(&ctl->bar) / (unsigned long long)G) * (unsigned long long)G;
+      // every launch passes at least one grid barrier, so bar_base / G differs
+      // between launches on a workspace and the tags (launch * 64 + layer,
+      // top bit set so that a cleared word never matches) do not repeat; a
+      // slot is rewritten only after the grid barrier that follows every
+      // reader's routing, so a reader never meets a later layer's tag
+      ltag_s = 0x80000000u | ((uint32_t)(bar_base / (unsigned long long)G) * (uint32_t)kMaxLayers);
+    }
 
     float acc[BMAX][8];
 #pragma unroll
@@ -817,7 +829,14 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
             float t = 0.f;
 #pragma unroll
             for (int w = 0; w < NCH; ++w) t += dotbuf[my_group * NCH + w + kWarps * (int)((jc / kGroups) & 1)][lane];
-            p.logits[j.c0 + lane] = t;
+            if (k <= kWarps) {
+              // {value, tag}: readers poll the word itself, no router barrier
+              const unsigned long long tag = (unsigned long long)(0x80000000u | (ltag_s + (uint32_t)j.layer));
+              st_relaxed_gpu_u64(reinterpret_cast<unsigned long long*>(p.logits) + j.c0 + lane,
+                                 (tag << 32) | __float_as_uint(t));
+            } else {
+              p.logits[j.c0 + lane] = t;  // read after the router barrier
+            }
           }
         } else if (ok) {
           const uint8_t* st = ring + (size_t)slot * p.stage_bytes;
@@ -976,7 +995,10 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
     // compares 4 candidate pairs and adds to a shared rank counter; ties go
     // to the lower index. The routed units (ascending expert id) are built in
     // the same pass. Logits come from lg[] or straight from the workspace.
-    auto route_b1_small_k = [&](bool from_ws) {
+    // src: 0 = lg[] (shared), 1 = workspace floats (after the router
+    // barrier), 2 = workspace {value, tag} words of layer `lay`, polled until
+    // the tag matches (bounded; a timeout clears okw_s, which the caller set)
+    auto route_b1_small_k = [&](int src, int lay) -> bool {
       uint32_t kq[4];
       uint32_t kmax = 0u;
       bool has = false;
@@ -988,7 +1010,23 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
         const int idx = key_idx(q);
         kq[q] = 0u;
         if (idx < E) {
-          kq[q] = float_key(from_ws ? __ldcg(p.logits + idx) : lg[idx]);
+          float v;
+          if (src == 2) {
+            const unsigned long long* w = reinterpret_cast<const unsigned long long*>(p.logits) + idx;
+            const uint32_t want = 0x80000000u | (ltag_s + (uint32_t)lay);
+            unsigned long long t = ld_relaxed_gpu(w);
+            if ((uint32_t)(t >> 32) != want) {
+              const long long t0 = clock64();
+              do {
+                t = ld_relaxed_gpu(w);
+              } while ((uint32_t)(t >> 32) != want && clock64() - t0 < kWaitBudgetCycles);
+              if ((uint32_t)(t >> 32) != want) okw_s = 0;
+            }
+            v = __uint_as_float((uint32_t)t);
+          } else {
+            v = src == 1 ? __ldcg(p.logits + idx) : lg[idx];
+          }
+          kq[q] = float_key(v);
           kmax = max(kmax, kq[q]);
           has = true;
         }
@@ -998,6 +1036,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
       if (lane == 0) { sel_pos[0][warp] = whas ? 1 : 0; cand_key[warp] = wm; }
       if (warp == 0) sel_pos[1][lane] = 0;  // rank counters
       cbar();
+      if (!okw_s) return false;
       uint32_t T = 0xffffffffu;
       int nw = 0;
 #pragma unroll
@@ -1078,7 +1117,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
           if (lane == 0) rs.U = k;
         }
         cbar();
-        return;
+        return true;
       }
       for (int c = tid; c < C; c += kConsumers) {
         const uint32_t kc = keys[c];
@@ -1109,6 +1148,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
         if (lane == 0) rs.U = k;
       }
       cbar();
+      return true;
     };
 
     auto route = [&]() {
@@ -1296,12 +1336,27 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
 
     bool failed = false;
     Job j;
+    // layer 0's accumulator: zeroed here, ordered before any CTA adds into it
+    // by the router barrier, by the ids barrier (given ids), or on the fast
+    // path (no router barrier) by one grid barrier now
+    {
+      const long long n4 = (long long)B * H / 4;
+      for (long long i = cta * n4 / G + tid; i < (cta + 1) * n4 / G; i += kConsumers)
+        reinterpret_cast<float4*>(p.yacc)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if constexpr (kFast && MODE == MODE_LAYERS)
+        if (k <= kWarps && !grid_sync()) { failed = true; if (tid == 0) set_status(ctl, kStatusTimeout); }
+    }
     for (int l = 0; l < p.L && !failed; ++l) {
-      float* yacc = p.yacc + (size_t)(l & 1) * B * H;
+      // accumulators rotate over three buffers: layer l adds into l % 3 and
+      // zeroes its slice of (l + 1) % 3, last read in layer l - 2's epilogue
+      // (finished everywhere before the barrier that ended layer l - 1) and
+      // next written after the barrier that ends layer l
+      float* yacc = p.yacc + (size_t)(l % 3) * B * H;
       {
+        float* ynext = p.yacc + (size_t)((l + 1) % 3) * B * H;
         const long long n4 = (long long)B * H / 4;
         for (long long i = cta * n4 / G + tid; i < (cta + 1) * n4 / G; i += kConsumers)
-          reinterpret_cast<float4*>(yacc)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+          reinterpret_cast<float4*>(ynext)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
       }
       // phase 0: router rows, 1: shared expert, 2: routed experts
       int phase = (MODE == MODE_LAYERS) ? 0 : 1;
@@ -1326,11 +1381,16 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
           (void)ld_acquire_cta(&prod_layer_s[1]);
         }
         if constexpr (MODE == MODE_LAYERS) {
-          if (kWarpRoute && k <= kWarps) {
+          if (kFast && k <= kWarps) {
+            // logits straight from their tagged words (okw_s = 1 was set
+            // before the phase barrier)
+            if (!route_b1_small_k(2, l)) { if (tid == 0) set_status(ctl, kStatusTimeout); return false; }
+            units_done = true;
+          } else if (kWarpRoute && k <= kWarps) {
             if (tid == 0) okw_s = wait_grid(target) ? 1 : 0;
             cbar();
             if (!okw_s) { if (tid == 0) set_status(ctl, kStatusTimeout); return false; }
-            route_b1_small_k(true);
+            route_b1_small_k(1, l);
             units_done = true;
           } else {
             if (tid == 0) okw_s = wait_grid(target) ? 1 : 0;
@@ -1338,7 +1398,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
             if (!okw_s) { if (tid == 0) set_status(ctl, kStatusTimeout); return false; }
             for (int i = tid; i < B * E; i += kConsumers) lg[i] = __ldcg(p.logits + i);
             cbar();
-            if (BMAX == 1 && k <= kWarps) { route_b1_small_k(false); units_done = true; }
+            if (BMAX == 1 && k <= kWarps) { route_b1_small_k(0, l); units_done = true; }
             else route();
           }
           if (cta == 0 && p.ids_out != nullptr)
@@ -1382,8 +1442,9 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
           // router logits written: arrive at the grid barrier; on the fast
           // path route at once (the shared expert's compute then overlaps the
           // routed copies' latency), else do the shared expert first
+          if (tid == 0) okw_s = 1;
           cbar();
-          if (tid == 0) target = arrive_grid();
+          if (!(kFast && MODE == MODE_LAYERS && k <= kWarps) && tid == 0) target = arrive_grid();
           if (route_early && !do_route()) { failed = true; break; }
           phase = 1;
           continue;

@@ -28,7 +28,7 @@ MOE_W_BF16, MOE_W_INT4_G64 = 0, 1
 MOE_EXPERT_SWIGLU, MOE_EXPERT_LINEAR = 0, 1
 MOE_LAYOUT_PLANAR, MOE_LAYOUT_CHANNEL_MAJOR = 0, 1
 MOE_STACK_PRE_RMSNORM = 1
-MOE_STATIC_SCRATCH_BYTES = 144 * 1024
+MOE_STATIC_SCRATCH_BYTES = 256 * 1024
 
 EXPORTS = [
     "moe_abi_version", "moe_status_string", "moe_workspace_bytes", "moe_workspace_init",

@@ -188,6 +188,8 @@ def test_expert_forward_bad_ids_sets_status(M, S, tiny):
     (1024, 37, 200, 3, 96, 3),  # E not a multiple of 32, ragged I, shared expert
     (2048, 64, 128, 8, 64, 8),  # a3b hidden, max batch
     (512, 16, 256, 16, 0, 2),   # k = E: dense softmax mixture
+    (2048, 8, 64, 8, 0, 1),     # batch-1 fast path, one expert per warp's keys, k = E
+    (2048, 24, 128, 12, 64, 1), # batch-1 fast path with k > 8 (router barrier, two-level top-k)
 ])
 def test_layer_forward_shapes(M, S, H, E, I, k, I_sh, B):
     L = S.swiglu_layer_bf16(H, E, I, I_sh, seed=123, device=DEV)
