@@ -104,7 +104,7 @@ moe_status check_weights(const moe_layer_desc* d, bool need_router) {
 
 // Batch-1 bf16 rows of 2048: the kernel's warp-owned-channel path.
 inline bool fast_path(const moe_layer_desc* d, int B) {
-  return B == 1 && d->wtype == MOE_W_BF16 && d->H == 2048;
+  return B == 1 && d->H == 2048 && (d->wtype == MOE_W_BF16 || d->layout == MOE_LAYOUT_PLANAR);
 }
 
 // Channels per job (template NCH). The warp-owned-channel path takes jobs of
@@ -112,7 +112,7 @@ inline bool fast_path(const moe_layer_desc* d, int B) {
 // for channel-major ones (48 KB stages, two warp groups, room for the
 // selection buffers); other bf16 planar batch-1 shapes take 8, the rest 4.
 inline int pick_nch(const moe_layer_desc* d, int B) {
-  if (fast_path(d, B)) return d->layout == MOE_LAYOUT_PLANAR ? 8 : 4;
+  if (fast_path(d, B)) return (d->layout == MOE_LAYOUT_PLANAR && d->wtype == MOE_W_BF16) ? 8 : 4;
   return (B == 1 && d->wtype == MOE_W_BF16 && d->layout == MOE_LAYOUT_PLANAR) ? 8 : 4;
 }
 
@@ -164,7 +164,7 @@ cudaError_t launch_decode_h(const DecodeParams& p0, int grid, cudaStream_t s) {
   cudaError_t err = cudaFuncGetAttributes(&fa, kern);
   if (err != cudaSuccess) return err;
   DecodeParams p = p0;
-  constexpr bool kFast = (BMAX == 1 && WT == MOE_W_BF16 && HV == 8);
+  constexpr bool kFast = (BMAX == 1 && HV == 8 && (WT == MOE_W_BF16 || LAYOUT == MOE_LAYOUT_PLANAR));
   if (!plan_smem(&p, (int)fa.sharedSizeBytes, kFast)) return cudaErrorInvalidConfiguration;
   err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem_bytes);
   if (err != cudaSuccess) return err;

@@ -187,7 +187,9 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
   constexpr int NV = NR * BMAX;      // values reduced per job
   // Batch-1 bf16 rows of 2048 elements: every warp owns whole channels (see
   // consume_fast); job q goes to warp group q % kGroups of NCH warps.
-  constexpr bool kFast = (BMAX == 1 && WT == MOE_W_BF16 && HV == 8);
+  // (int4 experts too, planar: their router and shared rows are bf16)
+  constexpr bool kFast = (BMAX == 1 && HV == 8 && (WT == MOE_W_BF16 || LAYOUT == MOE_LAYOUT_PLANAR));
+  constexpr bool kFastI4 = kFast && WT == MOE_W_INT4_G64;
   static_assert(!kFast || (NCH == 2 || NCH == 4 || NCH == 8), "warp groups of 2, 4 or 8 warps");
   constexpr int kGroups = kFast ? kWarps / NCH : 1;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -476,11 +478,15 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
       uint32_t* xw = reinterpret_cast<uint32_t*>(xfs);
       const int seg = tid >> 5, kk = (tid >> 3) & 3;
       const int comp = (kk == 1) ? 2 : (kk == 2 ? 1 : kk);
+      uint4 uw;
+      uint32_t* uwp = reinterpret_cast<uint32_t*>(&uw);
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
         const uint32_t w = uint32_t(f_to_bf16(xv[2 * m] * sc)) | (uint32_t(f_to_bf16(xv[2 * m + 1] * sc)) << 16);
         xw[(seg * 32 + 4 * (tid & 7) + m) * 4 + comp] = w;
+        uwp[m] = w;
       }
+      if constexpr (kFastI4) reinterpret_cast<uint4*>(us)[tid] = uw;  // u for the int4 rows' FMA dots
       cbar();
     };
     auto load_xfrag = [&]() {
@@ -840,7 +846,49 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
           }
         } else if (ok) {
           const uint8_t* st = ring + (size_t)slot * p.stage_bytes;
-          if (wi < j.n) {
+          if (kFastI4 && j.type == JOB_ROUTED) {
+            if (wi < j.n) {
+              // int4 channel: codes of its gate/up rows (H/2 bytes each) and
+              // their bf16 scales (one per 64 inputs); lane v-vectors of 8
+              // inputs, v = 32 i + lane, scale index v / 8. The down row's
+              // codes are scaled per output by the job's scale row.
+              const int rowc = H >> 1, rws = H >> 5;
+              const uint32_t* gc = reinterpret_cast<const uint32_t*>(st + wi * rowc);
+              const uint32_t* uc = reinterpret_cast<const uint32_t*>(st + NCH * rowc + wi * rowc);
+              const uint32_t* dc = reinterpret_cast<const uint32_t*>(st + 2 * NCH * rowc + wi * rowc);
+              const uint16_t* gs = reinterpret_cast<const uint16_t*>(st + 3 * NCH * rowc + wi * rws);
+              const uint16_t* ust = reinterpret_cast<const uint16_t*>(st + 3 * NCH * rowc + NCH * rws + wi * rws);
+              const uint4* ds = reinterpret_cast<const uint4*>(st + 3 * NCH * rowc + 2 * NCH * rws);
+              float ga = 0.f, ua = 0.f;
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const int v = 32 * i + lane;
+                float xf[8], qg[8], qu[8];
+                unpack8(us4[v], xf);
+                int4x8_to_f(gc[v], qg);
+                int4x8_to_f(uc[v], qu);
+                float pg = 0.f, pu = 0.f;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                  pg = fmaf(qg[e], xf[e], pg);
+                  pu = fmaf(qu[e], xf[e], pu);
+                }
+                ga = fmaf(bf16_to_f(gs[v >> 3]), pg, ga);
+                ua = fmaf(bf16_to_f(ust[v >> 3]), pu, ua);
+              }
+              const float gv = warp_sum(ga), uv = warp_sum(ua);
+              const float h = rs.unit_w[j.u][0] * silu_f(gv) * uv;
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const int v = 32 * i + lane;
+                float q[8], sv[8];
+                int4x8_to_f(dc[v], q);
+                unpack8(ds[v], sv);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) accf[8 * i + e] = fmaf(h * sv[e], q[e], accf[8 * i + e]);
+              }
+            }
+          } else if (wi < j.n) {
             const uint8_t *g, *u, *d;
             float wt;
             if (LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR && j.type == JOB_ROUTED) {
