@@ -279,10 +279,10 @@ class ChannelStack:
 class BatchSweep:
     """64 experts of one 8192 x 8192 bf16 matrix, top-3 uniform ids, batch B."""
 
-    def __init__(self, torch, M, S, device, rank, B=256, steps=0):
+    def __init__(self, torch, M, S, device, rank, B=256, steps=0, experts=0):
         self.torch, self.M, self.S, self.dev = torch, M, S, device
         w = S.WORKLOADS["batch_sweep"]
-        H, E, k = w["H"], w["E"], w["k"]
+        H, E, k = w["H"], experts or w["E"], w["k"]
         self.H, self.E, self.k, self.B = H, E, k, B
         self.W = S.linear_experts(E, H, seed=S.weight_seed(3, 0), device=device)
         self.desc = M.make_desc(H, E, H, k, kind=M.MOE_EXPERT_LINEAR, gate=self.W)
@@ -335,7 +335,7 @@ def make_workload(name, torch, M, S, device, rank, args):
     if name == "channel_topk":
         return ChannelStack(torch, M, S, device, rank, args.keep_frac, steps=args.steps)
     if name == "batch_sweep":
-        return BatchSweep(torch, M, S, device, rank, args.batch or 256, steps=args.steps)
+        return BatchSweep(torch, M, S, device, rank, args.batch or 256, steps=args.steps, experts=args.experts)
     raise SystemExit(f"unknown workload {name}")
 
 
@@ -578,6 +578,8 @@ def main():
     ap.add_argument("--batch", type=int, default=0, help="batch (a3b_int4: 1 or 8; batch_sweep: 1..256)")
     ap.add_argument("--layers", type=int, default=0,
                     help="fewer stack layers (profiling captures only; the metric is quoted on the full stack)")
+    ap.add_argument("--experts", type=int, default=0,
+                    help="fewer batch-sweep experts (profiling captures only; the sweep is quoted on 64)")
     ap.add_argument("--keep-frac", type=float, default=0.13, help="channel_topk budget (0.13 or 0.18)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 warm-up steps
