@@ -86,12 +86,12 @@ typedef enum { MOE_LAYOUT_PLANAR = 0, MOE_LAYOUT_CHANNEL_MAJOR = 1 } moe_layout;
 typedef struct {
   int32_t H;      /* hidden size; multiple of 64 (of 512 for int4)           */
   int32_t E;      /* routed experts, 1..1024                                   */
-  int32_t I;      /* expert intermediate size (channels); multiple of 64 for int4 */
+  int32_t I;      /* expert intermediate size (channels), 1..65536; multiple of 64 for int4 */
   int32_t k;      /* experts per token, 1..min(E, 32)                          */
   int32_t kind;   /* moe_ekind                                                 */
   int32_t wtype;  /* moe_wtype                                                 */
   int32_t layout; /* moe_layout                                                */
-  int32_t I_shared; /* shared-expert intermediate size, 0 = no shared expert  */
+  int32_t I_shared; /* shared-expert intermediate size, 0..65536, 0 = none   */
   const void* router;          /* [E, H] bf16; may be NULL when ids are given */
   const void* gate;            /* see Layouts above                           */
   const void* up;

@@ -78,6 +78,7 @@ bool valid_shape(const moe_layer_desc* d) {
   if (d->layout != MOE_LAYOUT_PLANAR && d->layout != MOE_LAYOUT_CHANNEL_MAJOR) return false;
   if (d->wtype == MOE_W_INT4_G64 && (d->H % 512 != 0 || d->I % 64 != 0)) return false;
   if (d->I_shared < 0) return false;
+  if (d->I > 65536 || d->I_shared > 65536) return false;  // keeps per-CTA range products in 32 bits
   return true;
 }
 

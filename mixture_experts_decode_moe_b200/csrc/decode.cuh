@@ -130,17 +130,18 @@ struct JobCursor {
     set_range(p);
   }
   __device__ void set_range(const DecodeParams& p) {
-    const long long G = gridDim.x, cb = blockIdx.x;
+    // 32-bit products: E <= 1024 and I_sh, routed channels < 2^21, grid < 2^11
+    const unsigned G = gridDim.x, cb = blockIdx.x;
     if (type == JOB_ROUTER) {
       if (p.mode == MODE_LAYERS && layer < p.L && p.layer[layer].router != nullptr) {
-        t = (int)(cb * p.E / G); t1 = (int)((cb + 1) * p.E / G);
+        t = (int)(cb * (unsigned)p.E / G); t1 = (int)((cb + 1) * (unsigned)p.E / G);
         if (t < t1) return;
       }
       type = JOB_SHARED;
     }
     if (type == JOB_SHARED) {
       if (p.mode == MODE_LAYERS && p.I_sh > 0) {
-        t = (int)(cb * p.I_sh / G); t1 = (int)((cb + 1) * p.I_sh / G);
+        t = (int)(cb * (unsigned)p.I_sh / G); t1 = (int)((cb + 1) * (unsigned)p.I_sh / G);
         if (t < t1) return;
       }
       type = JOB_ROUTED;
@@ -149,8 +150,8 @@ struct JobCursor {
   }
   // Routed range of this CTA once the number of routed channels R is known.
   __device__ void set_routed(int R, int I) {
-    const long long G = gridDim.x, cb = blockIdx.x;
-    t = (int)(cb * R / G); t1 = (int)((cb + 1) * R / G);
+    const unsigned G = gridDim.x, cb = blockIdx.x;
+    t = (int)(cb * (unsigned)R / G); t1 = (int)((cb + 1) * (unsigned)R / G);
     u = t / I; c = t - u * I;
   }
 };

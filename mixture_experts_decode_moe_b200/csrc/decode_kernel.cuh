@@ -244,7 +244,8 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
     for (int i = tid; i < H; i += kCtaThreads) reinterpret_cast<float*>(smem + p.off_ysum)[i] = 0.f;
   if (p.x_hist != nullptr) {
     const long long n = (long long)B * H8;
-    for (long long i = cta * n / G + tid; i < (cta + 1) * n / G; i += kCtaThreads)
+    for (long long i = (unsigned)cta * (unsigned)n / (unsigned)G + tid; i < (unsigned)(cta + 1) * (unsigned)n / (unsigned)G;
+         i += kCtaThreads)
       reinterpret_cast<uint4*>(p.x_hist)[i] = reinterpret_cast<const uint4*>(p.x_in)[i];
   }
   __syncthreads();
@@ -1384,12 +1385,16 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
 
     bool failed = false;
     Job j;
+    // this CTA's slice [ys0, ys1) of the B*H/4 float4 slots of an accumulator
+    // (outputs, zeroing); B*H/4 <= 2^14, so 32-bit products suffice
+    const int n4s = B * H / 4;
+    const int ys0 = (int)((unsigned)cta * (unsigned)n4s / (unsigned)G);
+    const int ys1 = (int)((unsigned)(cta + 1) * (unsigned)n4s / (unsigned)G);
     // layer 0's accumulator: zeroed here, ordered before any CTA adds into it
     // by the router barrier, by the ids barrier (given ids), or on the fast
     // path (no router barrier) by one grid barrier now
     {
-      const long long n4 = (long long)B * H / 4;
-      for (long long i = cta * n4 / G + tid; i < (cta + 1) * n4 / G; i += kConsumers)
+      for (int i = ys0 + tid; i < ys1; i += kConsumers)
         reinterpret_cast<float4*>(p.yacc)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
       if constexpr (kFast && MODE == MODE_LAYERS)
         if (k <= kWarps && !grid_sync()) { failed = true; if (tid == 0) set_status(ctl, kStatusTimeout); }
@@ -1402,8 +1407,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
       float* yacc = p.yacc + (size_t)(l % 3) * B * H;
       {
         float* ynext = p.yacc + (size_t)((l + 1) % 3) * B * H;
-        const long long n4 = (long long)B * H / 4;
-        for (long long i = cta * n4 / G + tid; i < (cta + 1) * n4 / G; i += kConsumers)
+        for (int i = ys0 + tid; i < ys1; i += kConsumers)
           reinterpret_cast<float4*>(ynext)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
       }
       // phase 0: router rows, 1: shared expert, 2: routed experts
@@ -1546,8 +1550,8 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
       }
       if (!grid_sync()) { failed = true; if (tid == 0) set_status(ctl, kStatusTimeout); break; }
       // epilogue: y, residual, outputs (each CTA writes its slice)
-      const long long n4 = (long long)B * H / 4;
-      const long long s0 = cta * n4 / G, s1 = (cta + 1) * n4 / G;
+      const long long n4 = n4s;
+      const long long s0 = ys0, s1 = ys1;
       float* yh = p.y_hist ? p.y_hist + (size_t)l * B * H : nullptr;
       float* yo = (l == p.L - 1) ? p.y_out : nullptr;
       if constexpr (MODE == MODE_LAYERS && kFast) {
