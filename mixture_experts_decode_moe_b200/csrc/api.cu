@@ -109,11 +109,11 @@ inline bool fast_path(const moe_layer_desc* d, int B) {
 }
 
 // Channels per job (template NCH). The warp-owned-channel path takes jobs of
-// 8 channels for planar experts (96 KB stages, one warp per channel) and 4
-// for channel-major ones (48 KB stages, two warp groups, room for the
-// selection buffers); other bf16 planar batch-1 shapes take 8, the rest 4.
+// 4 channels (48 KB stages for bf16: four stages in flight, two warp groups
+// of four warps, one channel per warp); other bf16 planar batch-1 shapes
+// take 8, the rest 4.
 inline int pick_nch(const moe_layer_desc* d, int B) {
-  if (fast_path(d, B)) return (d->layout == MOE_LAYOUT_PLANAR && d->wtype == MOE_W_BF16) ? 8 : 4;
+  if (fast_path(d, B)) return 4;
   return (B == 1 && d->wtype == MOE_W_BF16 && d->layout == MOE_LAYOUT_PLANAR) ? 8 : 4;
 }
 
@@ -186,7 +186,11 @@ cudaError_t launch_decode_h(const DecodeParams& p0, int grid, cudaStream_t s) {
 // lane); other hidden sizes use the guarded generic loop.
 template <int MODE, int BMAX, int WT, int LAYOUT, int NCH>
 cudaError_t launch_decode_n(const DecodeParams& p, int grid, cudaStream_t s) {
-  if (p.H == 2048) return launch_decode_h<MODE, BMAX, WT, LAYOUT, NCH, 8>(p, grid, s);
+  if (p.H == 2048) {
+    // batch-1 H = 2048 kernels are the pipelined fast path: 4 channels per job
+    if constexpr (BMAX == 1 && NCH != 4) return cudaErrorInvalidValue;
+    else return launch_decode_h<MODE, BMAX, WT, LAYOUT, NCH, 8>(p, grid, s);
+  }
   return launch_decode_h<MODE, BMAX, WT, LAYOUT, NCH, 0>(p, grid, s);
 }
 

@@ -28,7 +28,11 @@ struct alignas(16) WsControl {
   uint32_t status;          // 0 = ok, else a moe_status
   uint32_t pad0;
   unsigned long long bar;   // grid-barrier arrival counter (monotonic)
-  unsigned long long pad[30];
+  unsigned long long pad[14];
+  // batch-1 decode: routed jobs handed out per layer (layer l uses
+  // pool[l % 3]), in a cache line of their own
+  uint32_t pool[4];
+  uint32_t pad2[28];
 };
 static_assert(sizeof(WsControl) == 256, "control block is 256 bytes");
 

@@ -148,6 +148,10 @@ struct JobCursor {
     }
     t = -1; t1 = -1;  // routed: set once the routing is known
   }
+  // Routed range given directly (batch 1: the same every layer).
+  __device__ void set_routed_fixed(const int4& r) {
+    t = r.x; t1 = r.y; u = r.z; c = r.w;
+  }
   // Routed range of this CTA once the number of routed channels R is known.
   __device__ void set_routed(int R, int I) {
     const unsigned G = gridDim.x, cb = blockIdx.x;

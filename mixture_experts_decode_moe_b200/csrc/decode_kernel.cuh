@@ -192,11 +192,17 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
   constexpr bool kFastI4 = kFast && WT == MOE_W_INT4_G64;
   static_assert(!kFast || (NCH == 2 || NCH == 4 || NCH == 8), "warp groups of 2, 4 or 8 warps");
   constexpr int kGroups = kFast ? kWarps / NCH : 1;
+  // fast path: warp group g and producer g form pipeline g with the ring
+  // stages s, s % kPipes == g, and count their jobs independently
+  constexpr int kPipes = kFast ? kGroups : 1;
+  static_assert(!kFast || kPipes == kProducers, "one producer per warp group on the fast path");
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ RouteSmem<BMAX> rs;
   __shared__ int route_ready_s, prod_layer_s[kProducers], abort_s, bad_s, okw_s;
   __shared__ uint32_t ltag_s;  // logit tag of layer 0 in this launch (fast path)
-  __shared__ long long jp_s[kProducers], jc_s;
+  __shared__ long long jp_s[kProducers], jc_s, jcg_s[kProducers];
+  __shared__ Job jdesc[8];     // fast path: the job held by each stage
+  __shared__ int rcnt_s[2 * kProducers];  // fast path: router-partial counters
   __shared__ float dotbuf[16][NV];
   __shared__ float hbuf[kWarps][NCH * BMAX];
   __shared__ uint32_t cand_key[kWarps * kMaxK];
@@ -237,6 +243,8 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
     }
     abort_s = 0;
     jc_s = 0;
+    for (int q = 0; q < kProducers; ++q) jcg_s[q] = 0;
+    for (int q = 0; q < 2 * kProducers; ++q) rcnt_s[q] = 0;
   }
   for (int i = tid; i < B * H8; i += kCtaThreads)
     reinterpret_cast<uint4*>(xs)[i] = reinterpret_cast<const uint4*>(p.x_in)[i];
@@ -250,6 +258,17 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
   }
   __syncthreads();
 
+  // At batch 1 the routed channel count is the same every layer (k * I, or
+  // the kept count), so this CTA's routed range {t0, t1, unit, channel} is
+  // computed once here instead of on the critical path after each routing.
+  int4 rfix = make_int4(0, 0, 0, 0);
+  if constexpr (BMAX == 1) {
+    const int N1 = k * I;
+    const int R1 = (LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR) ? (p.keep > 0 ? min(N1, p.keep) : 0) : N1;
+    const int t0 = (int)((unsigned)cta * (unsigned)R1 / (unsigned)G);
+    const int t1 = (int)((unsigned)(cta + 1) * (unsigned)R1 / (unsigned)G);
+    rfix = make_int4(t0, t1, t0 / I, t0 - (t0 / I) * I);
+  }
   // Job sequence, shared by producer and consumers.
   auto next_job = [&](JobCursor& cur, Job& j, int ready_layer) -> bool {
     for (;;) {
@@ -270,7 +289,8 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
       }
       if (cur.t1 < 0) {
         if (ready_layer < cur.layer) return false;
-        cur.set_routed(LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR ? rs.ncand : rs.U * I, I);
+        if constexpr (BMAX == 1) cur.set_routed_fixed(rfix);
+        else cur.set_routed(LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR ? rs.ncand : rs.U * I, I);
       }
       if (cur.t >= cur.t1) { cur.begin_layer(p, cur.layer + 1); continue; }
       if (LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR) {
@@ -306,6 +326,173 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
   // byte count and issues its copies. Routed jobs of layer l wait until the
   // consumers publish routing for layer l.
   if (warp >= kWarps) {
+    if constexpr (kFast) {
+    // ---- pipeline producer pi: per layer, its share of the static jobs
+    // (router rows, shared channels: static job s belongs to pipe s % 2),
+    // then routed jobs taken from the layer's pool (an atomic counter, the
+    // next one grabbed while the current one is issued), then an end marker.
+    const int pi = warp - kWarps;
+    const uint64_t pol = policy_evict_first();
+    const int nps = (p.nstages - pi + kPipes - 1) / kPipes;
+    int pm = 0;
+    uint32_t pph = 0;
+    long long lq = 0;
+    const unsigned Gu = (unsigned)G, cu = (unsigned)cta;
+    const int rr0 = (MODE == MODE_LAYERS) ? (int)(cu * (unsigned)E / Gu) : 0;
+    const int rr1 = (MODE == MODE_LAYERS) ? (int)((cu + 1) * (unsigned)E / Gu) : 0;
+    const int sr0 = (MODE == MODE_LAYERS) ? (int)(cu * (unsigned)p.I_sh / Gu) : 0;
+    const int sr1 = (MODE == MODE_LAYERS) ? (int)((cu + 1) * (unsigned)p.I_sh / Gu) : 0;
+    const int R1 = (LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR) ? (p.keep > 0 ? min(k * I, p.keep) : 0) : k * I;
+    const int nj = (R1 + NCH - 1) / NCH;
+    int held = -1;  // a pool index grabbed ahead for the coming layer
+    // wait for this pipe's next stage to be free, then describe the job
+    auto take_stage = [&](const Job& jb) -> int {
+      const int slot = pi + kPipes * pm;
+      if (lq >= nps) {
+        const long long t0 = clock64();
+        while (!mbar_try_wait_sleep(&empty[slot], pph ^ 1u, 20000)) {
+          if (*(volatile int*)&abort_s || clock64() - t0 > kWaitBudgetCycles) return -1;
+        }
+      }
+      if (lane == 0) jdesc[slot] = jb;
+      return slot;
+    };
+    auto next_stage = [&]() {
+      ++lq;
+      if (++pm == nps) { pm = 0; pph ^= 1u; }
+      if (lane == 0) *(volatile long long*)&jp_s[pi] = lq;
+    };
+    for (int l = 0; l < p.L; ++l) {
+      const LayerW& Lw = p.layer[l];
+      int sidx = 0;
+      for (int r = rr0; r < rr1; r += p.rows_per_job, ++sidx) {
+        if (sidx % kPipes != pi) continue;
+        const Job jb{JOB_ROUTER, l, 0, r, min(p.rows_per_job, rr1 - r)};
+        const int slot = take_stage(jb);
+        if (slot < 0) goto producer_done;
+        if (lane == 0) {
+          const uint32_t bytes = (uint32_t)jb.n * rowb;
+          mbar_expect_tx(&full[slot], bytes);
+          bulk_g2s(ring + (size_t)slot * p.stage_bytes, Lw.router + (size_t)r * rowb, bytes, &full[slot], pol);
+        }
+        __syncwarp();
+        next_stage();
+      }
+      for (int c = sr0; c < sr1; c += NCH, ++sidx) {
+        if (sidx % kPipes != pi) continue;
+        const Job jb{JOB_SHARED, l, 0, c, min(NCH, sr1 - c)};
+        const int slot = take_stage(jb);
+        if (slot < 0) goto producer_done;
+        if (lane == 0) {
+          uint8_t* dst = ring + (size_t)slot * p.stage_bytes;
+          const uint32_t bytes = (uint32_t)jb.n * rowb;
+          const size_t off = (size_t)c * rowb;
+          mbar_expect_tx(&full[slot], 3 * bytes);
+          bulk_g2s(dst, Lw.sh_gate + off, bytes, &full[slot], pol);
+          bulk_g2s(dst + NCH * rowb, Lw.sh_up + off, bytes, &full[slot], pol);
+          bulk_g2s(dst + 2 * NCH * rowb, Lw.sh_down + off, bytes, &full[slot], pol);
+        }
+        __syncwarp();
+        next_stage();
+      }
+      {
+        // routing of layer l (plain polls with short sleeps, then one acquire)
+        const long long t0 = clock64();
+        while (*(volatile int*)&route_ready_s < l) {
+          if (*(volatile int*)&abort_s || clock64() - t0 > kWaitBudgetCycles) goto producer_done;
+          __nanosleep(20);
+        }
+        (void)ld_acquire_cta(&route_ready_s);
+      }
+      // pool grabs: lane 0 alone touches the counter, the warp shares the
+      // value (every lane must walk the same jobs); at most nj + 8 grabs
+      for (int it = 0;; ++it) {
+        if (it > nj + 8) goto producer_done;
+        int idx = held;
+        held = -1;
+        if (idx < 0) {
+          unsigned v = 0;
+          if (lane == 0) v = atomicAdd(&ctl->pool[l % 3], 1u);
+          idx = (int)__shfl_sync(0xffffffffu, v, 0);
+        }
+        if (idx >= nj) {
+          const Job jb{JOB_END, l, 0, 0, 0};
+          const int slot = take_stage(jb);
+          if (slot < 0) goto producer_done;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&full[slot]);
+          next_stage();
+          break;
+        }
+        unsigned nxt = 0;
+        if (lane == 0) nxt = atomicAdd(&ctl->pool[l % 3], 1u);  // in flight while the copies issue
+        const int ch0 = idx * NCH, n = min(NCH, R1 - ch0);
+        Job jb;
+        if constexpr (LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR) {
+          jb = Job{JOB_ROUTED, l, ch0, 0, n};
+        } else {
+          const int u = ch0 / I;
+          jb = Job{JOB_ROUTED, l, u, ch0 - u * I, n};
+        }
+        const int slot = take_stage(jb);
+        if (slot < 0) goto producer_done;
+        if (lane == 0) {
+          uint64_t* bar = &full[slot];
+          uint8_t* dst = ring + (size_t)slot * p.stage_bytes;
+          if constexpr (LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR) {
+            const uint32_t cb = 3u * (uint32_t)rowb;
+            mbar_expect_tx(bar, (uint32_t)n * cb);
+            for (int i = 0; i < n;) {
+              const int c0 = kept[ch0 + i];
+              int r = 1;
+              while (i + r < n && kept[ch0 + i + r] == c0 + r) ++r;
+              bulk_g2s(dst + (size_t)i * cb, Lw.gate + (size_t)c0 * cb, (uint32_t)r * cb, bar, pol);
+              i += r;
+            }
+          } else if constexpr (WT == MOE_W_BF16) {
+            const int n1 = min(n, I - jb.c0);
+            mbar_expect_tx(bar, 3u * (uint32_t)n * rowb);
+            for (int sg = 0; sg < 2; ++sg) {
+              const int ns = sg ? n - n1 : n1;
+              if (ns <= 0) break;
+              const int e = rs.unit_e[jb.u + sg];
+              const uint32_t bytes = (uint32_t)ns * rowb;
+              const size_t off = ((size_t)e * I + (sg ? 0 : jb.c0)) * rowb;
+              uint8_t* d0 = dst + (sg ? n1 : 0) * rowb;
+              bulk_g2s(d0, Lw.gate + off, bytes, bar, pol);
+              bulk_g2s(d0 + NCH * rowb, Lw.up + off, bytes, bar, pol);
+              bulk_g2s(d0 + 2 * NCH * rowb, Lw.down + off, bytes, bar, pol);
+            }
+          } else {
+            const int e = rs.unit_e[jb.u];
+            const int rowc = H >> 1, rws = H >> 5;
+            const uint32_t cbt = (uint32_t)n * rowc, sb = (uint32_t)n * rws;
+            const size_t offc = ((size_t)e * I + jb.c0) * rowc, offs = ((size_t)e * I + jb.c0) * rws;
+            const size_t offd = ((size_t)e * (I >> 6) + (jb.c0 >> 6)) * rowb;
+            mbar_expect_tx(bar, 3 * cbt + 2 * sb + rowb);
+            bulk_g2s(dst, Lw.gate + offc, cbt, bar, pol);
+            bulk_g2s(dst + NCH * rowc, Lw.up + offc, cbt, bar, pol);
+            bulk_g2s(dst + 2 * NCH * rowc, Lw.down + offc, cbt, bar, pol);
+            bulk_g2s(dst + 3 * NCH * rowc, Lw.gate_s + offs, sb, bar, pol);
+            bulk_g2s(dst + 3 * NCH * rowc + NCH * rws, Lw.up_s + offs, sb, bar, pol);
+            bulk_g2s(dst + 3 * NCH * rowc + 2 * NCH * rws, Lw.down_s + offd, rowb, bar, pol);
+          }
+        }
+        __syncwarp();
+        next_stage();
+        held = (int)__shfl_sync(0xffffffffu, nxt, 0);
+      }
+      // done with layer l's routing: the consumers may overwrite it; grab
+      // ahead for the next layer (its counter was cleared two layers ago)
+      if (lane == 0) st_release_cta(&prod_layer_s[pi], l);
+      {
+        unsigned v = 0;
+        if (lane == 0 && l + 1 < p.L) v = atomicAdd(&ctl->pool[(l + 1) % 3], 1u);
+        v = __shfl_sync(0xffffffffu, v, 0);
+        held = (l + 1 < p.L) ? (int)v : -1;
+      }
+    }
+    } else {
     // producer pi issues the jobs q with q % kProducers == pi; both walk the
     // whole sequence so that slots and phases stay in step
     const int pi = warp - kWarps;
@@ -423,6 +610,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
       if (++pslot == p.nstages) { pslot = 0; pph ^= 1u; }
       if (lane == 0) *(volatile long long*)&jp_s[pi] = jp;
     }
+    }  // producer model
   producer_done:;
     __syncwarp();
   } else {
@@ -800,52 +988,53 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
     auto group_bar = [&]() {
       asm volatile("bar.sync %0, %1;" ::"r"(2 + my_group), "r"(NCH * 32) : "memory");
     };
-    auto consume_fast = [&](const Job& j) -> bool {
-      const int slot = cslot;
-      const uint32_t ph = cph;
-      bool ok = true;
-      if ((int)(jc % kGroups) == my_group) {
-        ok = wait_mb(&full[slot], ph);
+    // run one job that has landed in `slot` (fast path)
+    auto run_job = [&](const Job& j, int slot, int buf) {
+      {
         if (j.type == JOB_ROUTER) {
           // rows split over K: warp wi of the group takes segments
-          // [wi * SPW, (wi + 1) * SPW) of every row; partials meet in
-          // dotbuf (double-buffered by job) after a group barrier that every
-          // warp of the group reaches, and warp 0 of the group writes
+          // [wi * SPW, (wi + 1) * SPW) of every row; the last warp of the
+          // group to finish (a shared counter, double-buffered by job) sums
+          // the partials and writes the logits, so no warp waits for another
           constexpr int SPW = 8 / NCH;
-          float* part = dotbuf[warp + kWarps * (int)((jc / kGroups) & 1)];
-          if (ok) {
-            const uint8_t* st = ring + (size_t)slot * p.stage_bytes;
-            const uint32_t sbase = smem_u32(st) + 16 * lane;
-            for (int r = 0; r < j.n; ++r) {
-              float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
+          float* part = dotbuf[warp + kWarps * buf];
+          const uint8_t* st = ring + (size_t)slot * p.stage_bytes;
+          const uint32_t sbase = smem_u32(st) + 16 * lane;
+          for (int r = 0; r < j.n; ++r) {
+            float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-              for (int q = 0; q < SPW; ++q) {
-                const int t = wi * SPW + q;
-                const uint4 xf = xfs[32 * t + lane];
-                uint32_t q0, q1, q2, q3;
-                ldmatrix_x4(sbase + r * rowb + 512 * t, q0, q1, q2, q3);
-                mma_bf16_16816(a0, q0, q1, q2, q3, xf.x, xf.y);
-                mma_bf16_16816(a1, q0, q1, q2, q3, xf.z, xf.w);
+            for (int q = 0; q < SPW; ++q) {
+              const int t = wi * SPW + q;
+              const uint4 xf = xfs[32 * t + lane];
+              uint32_t q0, q1, q2, q3;
+              ldmatrix_x4(sbase + r * rowb + 512 * t, q0, q1, q2, q3);
+              mma_bf16_16816(a0, q0, q1, q2, q3, xf.x, xf.y);
+              mma_bf16_16816(a1, q0, q1, q2, q3, xf.z, xf.w);
+            }
+            const float pv = warp_sum(diag_part(a0, a1, lane));
+            if (lane == 0) part[r] = pv;
+          }
+          if (lane == 0) {
+            __threadfence_block();
+            int* cnt = &rcnt_s[2 * my_group + buf];
+            if (atomicAdd(cnt, 1) == NCH - 1) {
+              __threadfence_block();
+              for (int r = 0; r < j.n; ++r) {
+                float t = 0.f;
+                for (int w = 0; w < NCH; ++w) t += dotbuf[my_group * NCH + w + kWarps * buf][r];
+                if (k <= kWarps) {
+                  // {value, tag}: readers poll the word itself, no router barrier
+                  const unsigned long long tag = (unsigned long long)(0x80000000u | (ltag_s + (uint32_t)j.layer));
+                  st_relaxed_gpu_u64(reinterpret_cast<unsigned long long*>(p.logits) + j.c0 + r,
+                                     (tag << 32) | __float_as_uint(t));
+                } else {
+                  p.logits[j.c0 + r] = t;  // read after the router barrier
+                }
               }
-              const float pv = warp_sum(diag_part(a0, a1, lane));
-              if (lane == 0) part[r] = pv;
+              *cnt = 0;
             }
           }
-          group_bar();
-          if (ok && wi == 0 && lane < j.n) {
-            float t = 0.f;
-#pragma unroll
-            for (int w = 0; w < NCH; ++w) t += dotbuf[my_group * NCH + w + kWarps * (int)((jc / kGroups) & 1)][lane];
-            if (k <= kWarps) {
-              // {value, tag}: readers poll the word itself, no router barrier
-              const unsigned long long tag = (unsigned long long)(0x80000000u | (ltag_s + (uint32_t)j.layer));
-              st_relaxed_gpu_u64(reinterpret_cast<unsigned long long*>(p.logits) + j.c0 + lane,
-                                 (tag << 32) | __float_as_uint(t));
-            } else {
-              p.logits[j.c0 + lane] = t;  // read after the router barrier
-            }
-          }
-        } else if (ok) {
+        } else {
           const uint8_t* st = ring + (size_t)slot * p.stage_bytes;
           if (kFastI4 && j.type == JOB_ROUTED) {
             if (wi < j.n) {
@@ -920,13 +1109,31 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
             }
           }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[slot]);
       }
-      if (++cslot == p.nstages) { cslot = 0; cph ^= 1u; }
-      ++jc;
+    };
+    // fast path: take this group's next job from its pipeline, run it and
+    // release the stage; returns the job type (JOB_END closes the routed
+    // phase) or -1 when the wait failed
+    const int cnps = kFast ? (p.nstages - my_group + kPipes - 1) / kPipes : 1;
+    int cpm = 0;
+    uint32_t cpph = 0;
+    long long lc = 0;
+    auto consume_pipe = [&]() -> int {
+      const int slot = my_group + kPipes * cpm;
+      const bool ok = wait_mb(&full[slot], cpph);
+      int ty = -1;
+      if (ok) {
+        const Job j = jdesc[slot];
+        ty = j.type;
+        if (ty != JOB_END) run_job(j, slot, (int)(lc & 1));
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[slot]);
+      ++lc;
+      if (++cpm == cnps) { cpm = 0; cpph ^= 1u; }
+      if (lane == 0 && wi == 0) *(volatile long long*)&jcg_s[my_group] = lc;
       if (!ok) *(volatile int*)&abort_s = 1;
-      return ok;
+      return ty;
     };
 
     // ---- pre-norm: us[b] = bf16(x[b] / sqrt(mean(x[b]^2) + eps)), unit weight
@@ -1385,6 +1592,19 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
 
     bool failed = false;
     Job j;
+    // fast path: this group's static jobs per layer (router rows in jobs of
+    // rows_per_job, shared channels in jobs of NCH; static job s belongs to
+    // pipe s % kPipes)
+    int own_router = 0, own_shared = 0;
+    const int nj_pool = ((LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR) ? (p.keep > 0 ? min(k * I, p.keep) : 0) : k * I) / NCH + 1;
+    if constexpr (kFast && MODE == MODE_LAYERS) {
+      const unsigned Gu = (unsigned)G, cu = (unsigned)cta;
+      const int nr = (int)((cu + 1) * (unsigned)E / Gu) - (int)(cu * (unsigned)E / Gu);
+      const int ns = (int)((cu + 1) * (unsigned)p.I_sh / Gu) - (int)(cu * (unsigned)p.I_sh / Gu);
+      const int nrj = (nr + p.rows_per_job - 1) / p.rows_per_job, nsj = (ns + NCH - 1) / NCH;
+      for (int sx = 0; sx < nrj + nsj; ++sx)
+        if (sx % kPipes == my_group) { if (sx < nrj) ++own_router; else ++own_shared; }
+    }
     // this CTA's slice [ys0, ys1) of the B*H/4 float4 slots of an accumulator
     // (outputs, zeroing); B*H/4 <= 2^14, so 32-bit products suffice
     const int n4s = B * H / 4;
@@ -1396,6 +1616,8 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
     {
       for (int i = ys0 + tid; i < ys1; i += kConsumers)
         reinterpret_cast<float4*>(p.yacc)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      // routed-job pools of layers 0 and 1 (layer l clears the pool of l + 2)
+      if (kFast && cta == 0 && tid == 0) { ctl->pool[0] = 0u; ctl->pool[1] = 0u; }
       if constexpr (kFast && MODE == MODE_LAYERS)
         if (k <= kWarps && !grid_sync()) { failed = true; if (tid == 0) set_status(ctl, kStatusTimeout); }
     }
@@ -1409,6 +1631,10 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
         float* ynext = p.yacc + (size_t)((l + 1) % 3) * B * H;
         for (int i = ys0 + tid; i < ys1; i += kConsumers)
           reinterpret_cast<float4*>(ynext)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        // the pool of layer l + 2: its last users (layer l - 1's producers)
+        // finished before the barrier that ended layer l - 1, its next users
+        // start after the barrier that ends layer l
+        if (kFast && cta == 0 && tid == 0) ctl->pool[(l + 2) % 3] = 0u;
       }
       // phase 0: router rows, 1: shared expert, 2: routed experts
       int phase = (MODE == MODE_LAYERS) ? 0 : 1;
@@ -1478,15 +1704,29 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
         ready = l;
         return true;
       };
+      if constexpr (kFast) {
+        // pipeline g: this group's router jobs, routing (whole CTA), its
+        // shared jobs, then routed jobs until the end marker
+        bool fl = false;
+        for (int i = 0; i < own_router; ++i) fl = fl || consume_pipe() != JOB_ROUTER;
+        if (tid == 0) okw_s = 1;
+        if (cbar_or(fl)) { failed = true; break; }
+        if (!(MODE == MODE_LAYERS && k <= kWarps) && MODE == MODE_LAYERS && tid == 0) target = arrive_grid();
+        if (!do_route()) { failed = true; break; }
+        for (int i = 0; i < own_shared && !fl; ++i) fl = consume_pipe() != JOB_SHARED;
+        for (int it = 0; !fl; ++it) {
+          const int ty = consume_pipe();
+          if (ty == JOB_END) break;
+          fl = ty != JOB_ROUTED || it > nj_pool + 8;  // a pipe gets at most all jobs
+        }
+        failed = fl;
+      } else {
       for (;;) {
         const JobCursor save = ccur;
         const bool got = next_job(ccur, j, ready);
         const bool in_layer = got && j.type != JOB_END && j.layer == l;
         if (in_layer && j.type == phase) {
-          bool okj;
-          if constexpr (kFast) okj = consume_fast(j);
-          else okj = consume(j);
-          if (!okj) { failed = true; break; }
+          if (!consume(j)) { failed = true; break; }
           continue;
         }
         ccur = save;
@@ -1508,6 +1748,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
         }
 
         break;
+      }
       }
       if (cbar_or(failed)) { failed = true; break; }
       ccur.begin_layer(p, l + 1);
@@ -1620,10 +1861,19 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
   // on an error path, wait (bounded) for the copies still in flight so that
   // none lands in shared memory after the CTA has exited
   if (tid == 0 && abort_s) {
-    // job q was issued iff producer q % kProducers got past it
-    const long long issued = max(jp_s[0], jp_s[1]);
-    for (long long q = jc_s; q < issued; ++q)
-      if (q < jp_s[q % kProducers]) mbar_wait(&full[q % p.nstages], (uint32_t)((q / p.nstages) & 1));
+    if constexpr (kFast) {
+      // pipeline g: jobs [consumed, issued) of its stages
+      for (int g = 0; g < kPipes; ++g) {
+        const int n = (p.nstages - g + kPipes - 1) / kPipes;
+        for (long long q = jcg_s[g]; q < jp_s[g]; ++q)
+          mbar_wait(&full[g + kPipes * (int)(q % n)], (uint32_t)((q / n) & 1));
+      }
+    } else {
+      // job q was issued iff producer q % kProducers got past it
+      const long long issued = max(jp_s[0], jp_s[1]);
+      for (long long q = jc_s; q < issued; ++q)
+        if (q < jp_s[q % kProducers]) mbar_wait(&full[q % p.nstages], (uint32_t)((q / p.nstages) & 1));
+    }
   }
 }
 
