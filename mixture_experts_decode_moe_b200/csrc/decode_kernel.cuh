@@ -1261,27 +1261,37 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
       // expert i sits in warp i % 8 (lane (i / 8) % 32, slot i / 256): every
       // warp holds keys as soon as E >= 8
       auto key_idx = [&](int q) { return kConsumers * q + kWarps * lane + warp; };
+      if (src == 2) {
+        // tagged words polled in order (a warp's 32 words are 256 contiguous
+        // bytes, two L2 lines per poll), values to lg[]
+        const unsigned long long* wb = reinterpret_cast<const unsigned long long*>(p.logits);
+        const uint32_t want = 0x80000000u | (ltag_s + (uint32_t)lay);
+        unsigned long long t[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (kConsumers * q + tid < E) t[q] = ld_relaxed_gpu(wb + kConsumers * q + tid);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int i = kConsumers * q + tid;
+          if (i < E) {
+            if ((uint32_t)(t[q] >> 32) != want) {
+              const long long t0 = clock64();
+              do {
+                t[q] = ld_relaxed_gpu(wb + i);
+              } while ((uint32_t)(t[q] >> 32) != want && clock64() - t0 < kWaitBudgetCycles);
+              if ((uint32_t)(t[q] >> 32) != want) okw_s = 0;
+            }
+            lg[i] = __uint_as_float((uint32_t)t[q]);
+          }
+        }
+        cbar();
+      }
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const int idx = key_idx(q);
         kq[q] = 0u;
         if (idx < E) {
-          float v;
-          if (src == 2) {
-            const unsigned long long* w = reinterpret_cast<const unsigned long long*>(p.logits) + idx;
-            const uint32_t want = 0x80000000u | (ltag_s + (uint32_t)lay);
-            unsigned long long t = ld_relaxed_gpu(w);
-            if ((uint32_t)(t >> 32) != want) {
-              const long long t0 = clock64();
-              do {
-                t = ld_relaxed_gpu(w);
-              } while ((uint32_t)(t >> 32) != want && clock64() - t0 < kWaitBudgetCycles);
-              if ((uint32_t)(t >> 32) != want) okw_s = 0;
-            }
-            v = __uint_as_float((uint32_t)t);
-          } else {
-            v = src == 1 ? __ldcg(p.logits + idx) : lg[idx];
-          }
+          const float v = src == 1 ? __ldcg(p.logits + idx) : lg[idx];
           kq[q] = float_key(v);
           kmax = max(kmax, kq[q]);
           has = true;
