@@ -39,6 +39,11 @@ __device__ __forceinline__ unsigned long long ld_relaxed_gpu(const unsigned long
   asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
   return v;
 }
+// two 8-byte words with one 16-byte load (each word read whole)
+__device__ __forceinline__ void ld_relaxed_gpu_v2(const unsigned long long* p, unsigned long long& a,
+                                                  unsigned long long& b) {
+  asm volatile("ld.relaxed.gpu.global.v2.u64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "l"(p) : "memory");
+}
 __device__ __forceinline__ void st_relaxed_gpu_u64(unsigned long long* p, unsigned long long v) {
   asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
@@ -1244,6 +1249,102 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
       }
     };
 
+    // ---- B = 1, k <= 8, E <= 256, tagged logit words of layer `lay`: one
+    // warp routes alone, with no CTA barrier, while the other warps go on
+    // with their jobs. Lane l polls words 64q + 2l and 64q + 2l + 1 (q < 4;
+    // the warp's four 16-byte loads cover the 2 KB once) until all carry the
+    // layer's tag, then the k largest are taken by k rounds of a warp-wide
+    // argmax (ties: the lower expert index), followed by the softmax over the
+    // k and the units in ascending expert id. Returns false on a poll timeout.
+    // A logit whose key is 0 (a NaN with every bit set) is never selected.
+    auto route_warp = [&](int lay) -> bool {
+      const unsigned long long* wb = reinterpret_cast<const unsigned long long*>(p.logits);
+      const uint32_t want = 0x80000000u | (ltag_s + (uint32_t)lay);
+      uint32_t key[8];
+      bool done[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        done[q] = 64 * q + 2 * lane >= E;
+        key[2 * q] = 0u;
+        key[2 * q + 1] = 0u;
+      }
+      const long long t0 = clock64();
+      for (;;) {
+        unsigned long long a[4], b[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (!done[q]) ld_relaxed_gpu_v2(wb + 64 * q + 2 * lane, a[q], b[q]);
+        bool all = true;
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (!done[q]) {
+            const int i = 64 * q + 2 * lane;
+            const bool has_b = i + 1 < E;
+            if ((uint32_t)(a[q] >> 32) == want && (!has_b || (uint32_t)(b[q] >> 32) == want)) {
+              done[q] = true;
+              key[2 * q] = float_key(__uint_as_float((uint32_t)a[q]));
+              key[2 * q + 1] = has_b ? float_key(__uint_as_float((uint32_t)b[q])) : 0u;
+            } else {
+              all = false;
+            }
+          }
+        if (__all_sync(0xffffffffu, all)) break;
+        if (__any_sync(0xffffffffu, clock64() - t0 > kWaitBudgetCycles)) return false;  // warp-uniform
+      }
+      // slot s of lane l holds expert 64 (s / 2) + 2 l + s % 2: slots in
+      // ascending index order, so a strict > keeps the lowest index of a tie
+      auto slot_idx = [&](int s) { return 64 * (s >> 1) + 2 * lane + (s & 1); };
+      uint32_t bk = key[0];
+      int bs = 0;
+#pragma unroll
+      for (int s = 1; s < 8; ++s)
+        if (key[s] > bk) { bk = key[s]; bs = s; }
+      for (int r = 0; r < k; ++r) {
+        const uint32_t M = __reduce_max_sync(0xffffffffu, bk);
+        const uint32_t tie = __ballot_sync(0xffffffffu, bk == M);
+        int wl = __ffs(tie) - 1;
+        if (tie & (tie - 1)) {
+          // several lanes hold M: the lowest expert index wins
+          const uint32_t mi = __reduce_min_sync(0xffffffffu, bk == M ? (uint32_t)slot_idx(bs) : 0xffffffffu);
+          wl = __ffs(__ballot_sync(0xffffffffu, bk == M && (uint32_t)slot_idx(bs) == mi)) - 1;
+        }
+        if (lane == wl) {
+          cand_key[kWarps + r] = M;
+          cand_idx[r] = slot_idx(bs);
+#pragma unroll
+          for (int s = 0; s < 8; ++s)
+            if (s == bs) key[s] = 0u;
+          bk = key[0];
+          bs = 0;
+#pragma unroll
+          for (int s = 1; s < 8; ++s)
+            if (key[s] > bk) { bk = key[s]; bs = s; }
+        }
+      }
+      __syncwarp();
+      const bool sel = lane < k;
+      const uint32_t kc = sel ? cand_key[kWarps + lane] : 0u;
+      const int ic = sel ? cand_idx[lane] : 0x7fffffff;
+      const float e = sel ? __expf(key_float(kc) - key_float(cand_key[kWarps])) : 0.f;
+      const float wl = e / warp_sum(e);
+      int urank = 0;
+      for (int m = 0; m < k; ++m) urank += cand_idx[m] < ic;
+      if (sel) {
+        rs.ids[0][lane] = ic;
+        rs.w[0][lane] = wl;
+        rs.unit_e[urank] = ic;
+        rs.unit_mask[urank] = 1u;
+        rs.unit_w[urank][0] = wl;
+        if (cta == 0 && p.ids_out != nullptr) {
+          p.ids_out[(size_t)lay * k + lane] = ic;
+          p.w_out[(size_t)lay * k + lane] = wl;
+        }
+      }
+      if (lane == 0) rs.U = k;
+      __syncwarp();
+      return true;
+    };
+
     // ---- top-k of every token from lg[B][E]
     // B = 1, k <= 8: every warp's largest key is >= T = the smallest of the
     // warp maxima, so at least 8 keys reach T and the k-th largest key is >= T.
@@ -1668,8 +1769,21 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
           (void)ld_acquire_cta(&prod_layer_s[0]);
           (void)ld_acquire_cta(&prod_layer_s[1]);
         }
+        bool ids_done = false;
         if constexpr (MODE == MODE_LAYERS) {
-          if (kFast && k <= kWarps) {
+          if (kFast && LAYOUT == MOE_LAYOUT_PLANAR && k <= kWarps && E <= 256) {
+            // warp 0 routes; the other warps need nothing from it and go on
+            if constexpr (kFast && LAYOUT == MOE_LAYOUT_PLANAR) {
+              if (warp != 0) return true;
+              if (!route_warp(l)) {
+                // the others learn of it through the abort flag
+                if (lane == 0) { set_status(ctl, kStatusTimeout); st_release_cta(&abort_s, 1); }
+                return false;
+              }
+            }
+            units_done = true;
+            ids_done = true;
+          } else if (kFast && k <= kWarps) {
             // logits straight from their tagged words (okw_s = 1 was set
             // before the phase barrier)
             if (!route_b1_small_k(2, l)) { if (tid == 0) set_status(ctl, kStatusTimeout); return false; }
@@ -1689,7 +1803,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
             if (BMAX == 1 && k <= kWarps) { route_b1_small_k(0, l); units_done = true; }
             else route();
           }
-          if (cta == 0 && p.ids_out != nullptr)
+          if (cta == 0 && p.ids_out != nullptr && !ids_done)
             for (int t = tid; t < B * k; t += kConsumers) {
               p.ids_out[(size_t)l * B * k + t] = rs.ids[t / k][t % k];
               p.w_out[(size_t)l * B * k + t] = rs.w[t / k][t % k];
@@ -1722,7 +1836,14 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
         if (tid == 0) okw_s = 1;
         if (cbar_or(fl)) { failed = true; break; }
         if (!(MODE == MODE_LAYERS && k <= kWarps) && MODE == MODE_LAYERS && tid == 0) target = arrive_grid();
-        if (!do_route()) { failed = true; break; }
+        // planar: a failed routing (warp 0 alone) skips this warp's jobs and
+        // every warp meets the others at the barrier after the routed phase;
+        // channel-major: all threads agree on it
+        if constexpr (LAYOUT == MOE_LAYOUT_PLANAR) {
+          fl = !do_route();
+        } else {
+          if (!do_route()) { failed = true; break; }
+        }
         for (int i = 0; i < own_shared && !fl; ++i) fl = consume_pipe() != JOB_SHARED;
         for (int it = 0; !fl; ++it) {
           const int ty = consume_pipe();
