@@ -438,6 +438,118 @@ def channel_major_ranges(kept: Iterable[int], H: int, base: int = 0, elem_bytes:
 
 
 # ----------------------------------------------------------------------------
+# Weight-only channel screen. [Reader] "가중치만으로 만든 reader":
+#   step 1 ("삼원 스케치로 선별한다"): the gate row g_j and up row v_j are
+#   rotated in blocks of 128 coordinates by a random Hadamard transform R
+#   (orthogonal, so g^T x = (R g)^T (R x)); each rotated block is stored as
+#   ternary codes in {-1, 0, 1}, one fp16 scale and rho_b, the block's mean
+#   squared quantisation error. At decode time x is rotated once and the
+#   sketch gives g_hat ~ g^T x and v_hat ~ v^T x.
+#   step 2 ("출력 단위 점수로 상위 k개를 정확히 계산한다", eq. 1): the score
+#   of channel j is s_j = w_j ||d_j|| |phi(g_hat_j) v_hat_j|, with w_j the
+#   router weight of its expert and ||d_j|| the norm of its down column,
+#   computed once at load; one top-k runs across all routed experts.
+# Readings where the page is silent:
+#   * R = H_128 diag(s) / sqrt(128) per block: H_128 the Sylvester Hadamard
+#     matrix, s a given vector of H random signs (an input). Both sides work
+#     with the unnormalised u = H_128 (s * v); (R g)^T (R x) = u_g^T u_x / 128.
+#   * the ternary code of a block is the ternary-weight-network rule (Li and
+#     Liu, 2016): threshold delta = 0.7 * mean|u|, code = sign(u) where
+#     |u| > delta, else 0; scale = mean of |u| over the nonzero codes, stored
+#     as fp16 (rounded through fp32, both round-to-nearest-even).
+#   * rho_b = mean over the block of ((u - scale * code) / sqrt(128))^2, the
+#     error in the orthonormal rotation's units, with the stored scale.
+# For bf16 rows whose block values span less than 2^38 in magnitude, u, the
+# sum of |u| and the code decisions are exact in fp64, so any exact
+# implementation (matrix product or butterfly) gives the same codes.
+# ----------------------------------------------------------------------------
+
+READER_BLOCK = 128
+TWN_THRESHOLD = 0.7
+
+
+def sylvester_hadamard(n: int) -> np.ndarray:
+    """H_1 = [1]; H_2m = [[H_m, H_m], [H_m, -H_m]] (entries +-1, unnormalised)."""
+    h = np.ones((1, 1))
+    while h.shape[0] < n:
+        h = np.block([[h, h], [h, -h]])
+    if h.shape[0] != n:
+        raise ValueError("n must be a power of two")
+    return h
+
+
+def reader_rotate(v: np.ndarray, signs: np.ndarray) -> np.ndarray:
+    """u = H_128 (s * v) on each block of 128 coordinates (unnormalised)."""
+    v = np.asarray(v, dtype=np.float64)
+    hm = sylvester_hadamard(READER_BLOCK)
+    blocks = (np.asarray(signs, dtype=np.float64) * v).reshape(-1, READER_BLOCK)
+    return (blocks @ hm.T).reshape(-1)
+
+
+def fp16_through_fp32(a: float) -> float:
+    """fp64 -> fp32 -> fp16, each round-to-nearest-even; returned as fp64."""
+    return float(np.float16(np.float32(a)))
+
+
+def ternary_block(u: np.ndarray):
+    """One rotated block -> (codes int8 [128], fp16 scale, rho)."""
+    u = np.asarray(u, dtype=np.float64)
+    a = np.abs(u)
+    delta = TWN_THRESHOLD * (a.sum() / READER_BLOCK)
+    nz = a > delta
+    codes = np.where(nz, np.sign(u), 0.0).astype(np.int8)
+    n = int(nz.sum())
+    scale = fp16_through_fp32(a[nz].sum() / n) if n else 0.0
+    rho = float(np.mean(((u - scale * codes) / math.sqrt(READER_BLOCK)) ** 2))
+    return codes, scale, rho
+
+
+def reader_sketch_row(v: np.ndarray, signs: np.ndarray):
+    """Sketch of one row: codes int8 [H], scales [H/128], rho [H/128]."""
+    u = reader_rotate(v, signs)
+    parts = [ternary_block(b) for b in u.reshape(-1, READER_BLOCK)]
+    codes = np.concatenate([p[0] for p in parts])
+    return codes, np.array([p[1] for p in parts]), np.array([p[2] for p in parts])
+
+
+def reader_estimate(x: np.ndarray, codes: np.ndarray, scales: np.ndarray, signs: np.ndarray) -> float:
+    """Sketch estimate of v^T x: sum over blocks of scale_b codes_b . u_x,b / 128."""
+    ux = reader_rotate(x, signs).reshape(-1, READER_BLOCK)
+    c = np.asarray(codes, dtype=np.float64).reshape(-1, READER_BLOCK)
+    return float(np.sum(np.asarray(scales, dtype=np.float64) * np.sum(c * ux, axis=1)) / READER_BLOCK)
+
+
+def reader_estimate_bound(x: np.ndarray, codes: np.ndarray, scales: np.ndarray) -> float:
+    """sum_b scale_b * (number of nonzero codes in b) * sum_{i in b} |x_i| / 128:
+    a bound on every |partial sum| of the estimate (each |u_x,i| <= sum_b |x|)."""
+    xa = np.abs(np.asarray(x, dtype=np.float64)).reshape(-1, READER_BLOCK).sum(axis=1)
+    nzc = (np.asarray(codes).reshape(-1, READER_BLOCK) != 0).sum(axis=1)
+    return float(np.sum(np.abs(np.asarray(scales, dtype=np.float64)) * nzc * xa) / READER_BLOCK)
+
+
+def reader_score(w_e: float, dnorm: float, g_hat: float, v_hat: float) -> float:
+    """Eq. 1: s = w_e ||d|| |phi(g_hat) v_hat|, phi = SiLU."""
+    return float(w_e * dnorm * abs(silu(np.float64(g_hat)) * v_hat))
+
+
+def reader_screen(x: np.ndarray, ids: Sequence[int], w: Sequence[float], sketch, I: int, signs: np.ndarray):
+    """Scores [len(ids), I] and estimates [len(ids), I, 2] of the routed
+    experts' channels. sketch(e, c) -> (codes_g, scales_g, codes_v, scales_v,
+    dnorm)."""
+    k = len(ids)
+    scores = np.zeros((k, I))
+    est = np.zeros((k, I, 2))
+    for t, e in enumerate(ids):
+        for c in range(I):
+            cg, sg, cv, sv, dn = sketch(int(e), c)
+            gh = reader_estimate(x, cg, sg, signs)
+            vh = reader_estimate(x, cv, sv, signs)
+            est[t, c] = (gh, vh)
+            scores[t, c] = reader_score(float(w[t]), dn, gh, vh)
+    return scores, est
+
+
+# ----------------------------------------------------------------------------
 # Bytes-per-token accounting and decode ceiling.
 # [MoE-arith] "Two Numbers Instead of One" / moe_promise.py: ceiling =
 # achieved bandwidth / bytes per token. [Beam] §2 memory table: resident =

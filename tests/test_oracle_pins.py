@@ -503,3 +503,119 @@ def test_stack_layer_residual_uses_unnormalised_x():
     assert np.array_equal(xn, O.residual_bf16(x, y))
     xn0, y0, *_ = O.stack_layer(x, R, lambda e: ex[e], k, pre_norm=False)
     assert np.allclose(y0, O.moe_layer(x, R, lambda e: ex[e], k)[0])
+
+
+# ---------------------------------------------------------------- reader screen
+# [Reader] "가중치만으로 만든 reader", step 1 (rotated ternary sketch) and
+# step 2 (eq. 1 scores).
+
+
+def test_hadamard_matches_popcount_definition_and_is_orthogonal():
+    # Sylvester's recursion against the closed form H[i][j] = (-1)^popcount(i & j),
+    # and H H^T = n I (so R = H diag(s) / sqrt(n) is orthogonal).
+    for n in (1, 2, 8, 128):
+        h = O.sylvester_hadamard(n)
+        i = np.arange(n)
+        closed = np.array([[(-1.0) ** bin(a & b).count("1") for b in i] for a in i])
+        assert np.array_equal(h, closed)
+        assert np.array_equal(h @ h.T, n * np.eye(n))
+
+
+def test_rotation_preserves_dot_products():
+    # The page's reason for the rotation: g^T x = (R g)^T (R x). With the
+    # unnormalised u = H (s * v) that is u_g . u_x / 128.
+    r = rng(41)
+    H = 512
+    s = r.choice([-1.0, 1.0], H)
+    g, x = O.bf16_round(r.normal(0, 0.02, H)), O.bf16_round(r.normal(0, 1, H))
+    lhs = float(O.reader_rotate(g, s) @ O.reader_rotate(x, s)) / 128
+    assert abs(lhs - float(g @ x)) <= 1e-12 * float(np.abs(g) @ np.abs(x)) * 128
+    # a basis vector e_h maps to s_h times column h % 128 of H_128 in its block
+    e = np.zeros(H)
+    e[300] = 1.0
+    u = O.reader_rotate(e, s).reshape(-1, 128)
+    col = O.sylvester_hadamard(128)[:, 300 % 128] * s[300]
+    assert np.array_equal(u[300 // 128], col)
+    assert not np.any(np.delete(u, 300 // 128, axis=0))
+
+
+def test_ternary_block_hand_example():
+    # mean|u| = 21/128, delta = 0.7 * 21/128 ~ 0.115: codes (+1, -1, +1), the
+    # scale the mean |u| of those three = 7, rho = (3^2 + 3^2 + 6^2) / 128 / 128.
+    u = np.zeros(128)
+    u[:3] = (10.0, -10.0, 1.0)
+    codes, scale, rho = O.ternary_block(u)
+    assert codes[:3].tolist() == [1, -1, 1] and not np.any(codes[3:])
+    assert scale == 7.0
+    assert abs(rho - (9 + 9 + 36) / 128 / 128) <= 1e-15  # 1/sqrt(128) is not exact in fp64
+    # every |u| equal to the mean: delta = 0.7 * mean < |u| keeps them all;
+    # a single value carrying the whole mass is the only code kept
+    c2, s2, _ = O.ternary_block(np.full(128, -2.0))
+    assert np.all(c2 == -1) and s2 == 2.0
+    u3 = np.zeros(128)
+    u3[5] = 100.0
+    c3, s3, _ = O.ternary_block(u3)
+    assert c3[5] == 1 and s3 == 100.0 and np.count_nonzero(c3) == 1
+
+
+def test_ternary_block_exact_for_ternary_input_and_zero_block():
+    # u = a * c with c ternary: delta = 0.7 a nnz/128 < a, so the codes are c,
+    # the scale a (exact in fp16 for a = 0.375), rho = 0. All-zero block: no codes.
+    r = rng(42)
+    c = r.choice([-1, 0, 1], 128).astype(np.int8)
+    codes, scale, rho = O.ternary_block(0.375 * c)
+    assert np.array_equal(codes, c) and scale == 0.375 and rho == 0.0
+    codes, scale, rho = O.ternary_block(np.zeros(128))
+    assert not np.any(codes) and scale == 0.0 and rho == 0.0
+
+
+def test_fp16_scale_rounding_matches_library():
+    # fp64 -> fp32 -> fp16 round-to-nearest-even against torch's conversions.
+    torch = pytest.importorskip("torch")
+    r = rng(43)
+    for a in r.uniform(1e-4, 30.0, 200):
+        want = torch.tensor(a, dtype=torch.float64).to(torch.float32).to(torch.float16).item()
+        assert O.fp16_through_fp32(a) == want
+
+
+def test_estimate_is_exact_when_the_row_is_its_own_sketch():
+    # A row built from ternary codes and fp16 scales by the inverse rotation
+    # (H^-1 = H / 128, diag(s)^-1 = diag(s)) has that sketch exactly, and the
+    # estimate then equals the true dot product.
+    r = rng(44)
+    H = 256
+    s = r.choice([-1.0, 1.0], H)
+    c = r.choice([-1, 0, 1], H).astype(np.int8)
+    scales = np.array([0.5, 0.25])
+    u = (c.reshape(-1, 128) * scales[:, None]).reshape(-1)
+    hm = O.sylvester_hadamard(128)
+    row = s * ((u.reshape(-1, 128) @ hm) / 128).reshape(-1)
+    codes, sc, rho = O.reader_sketch_row(row, s)
+    assert np.array_equal(codes, c) and np.array_equal(sc, scales) and np.all(rho == 0)
+    x = O.bf16_round(r.normal(0, 1, H))
+    assert abs(O.reader_estimate(x, codes, sc, s) - float(row @ x)) <= 1e-12 * float(np.abs(row) @ np.abs(x)) * 64
+
+
+def test_estimate_error_bounded_by_rho():
+    # Cauchy-Schwarz per block: |g^T x - g_hat| <= sum_b sqrt(128 rho_b) ||R x_b||
+    # (the error vector of block b has squared norm 128 rho_b in the
+    # orthonormal rotation's units).
+    r = rng(45)
+    H = 512
+    s = r.choice([-1.0, 1.0], H)
+    g = O.bf16_round(r.normal(0, 0.02, H))
+    x = O.bf16_round(r.normal(0, 1, H))
+    codes, sc, rho = O.reader_sketch_row(g, s)
+    ux = O.reader_rotate(x, s).reshape(-1, 128) / math.sqrt(128)
+    bound = float(np.sum(np.sqrt(128 * rho) * np.linalg.norm(ux, axis=1)))
+    err = abs(float(g @ x) - O.reader_estimate(x, codes, sc, s))
+    assert err <= bound * (1 + 1e-9)
+    assert 0 < err  # a real approximation
+
+
+def test_eq1_score_hand_values():
+    # s = w ||d|| |phi(g) v| with phi = SiLU: 0.5 * 2 * |silu(1) * (-3)| = 3 / (1 + e^-1)
+    assert abs(O.reader_score(0.5, 2.0, 1.0, -3.0) - 3.0 / (1.0 + math.exp(-1.0))) < 1e-15
+    # the sign of v_hat and of phi(g_hat) do not matter; a zero estimate scores 0
+    assert O.reader_score(0.5, 2.0, -1.0, 3.0) == O.reader_score(0.5, 2.0, -1.0, -3.0)
+    assert O.reader_score(0.5, 2.0, 0.0, 5.0) == 0.0
