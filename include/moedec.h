@@ -248,6 +248,47 @@ moe_status moe_layer_forward_static(const moe_layer_desc* desc, const void* x, i
                                     void* x_next_opt, int32_t* ids_out_opt, float* w_out_opt,
                                     int32_t* status_out_opt, moe_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * Weight-only channel screen ([Reader] "가중치만으로 만든 reader", step 1:
+ * the gate and up rows of every channel are rotated in blocks of 128
+ * coordinates by a random Hadamard transform and stored as ternary codes with
+ * one fp16 scale and one squared error rho per block; step 2, eq. 1: a
+ * channel's score is w_e ||d_j|| |SiLU(g_hat_j) v_hat_j| from the sketch
+ * estimates g_hat ~ g_j.x and v_hat ~ v_j.x). The scores feed
+ * moe_channel_topk_forward's `scores` input.
+ *
+ * Rotation: R = H_128 diag(s) / sqrt(128) per block, H_128 the Sylvester
+ * Hadamard matrix, s = signs[H] (+1 or -1 as int8, chosen by the caller at
+ * random once per model and shared by the builder and the screen).
+ * Ternary rule per rotated block u (unnormalised, u = H_128 (s * v)):
+ * delta = 0.7 * mean|u|, code = sign(u) where |u| > delta else 0, scale =
+ * mean |u| over the coded coordinates rounded to fp16 (through fp32),
+ * rho = mean((u - scale * code)^2) / 128. Decisions are taken in fp64.
+ *
+ * Layout (j = e*I + c, row r = 0 gate / 1 up):
+ *   codes  [E*I][2][H/16] uint32: coordinate h of a row in word h/16, bit
+ *          2(h%16) = nonzero, bit 2(h%16)+1 = negative (2 bits per code);
+ *   scales [E*I][2][H/128] uint16 (fp16 bit patterns);
+ *   rho    [E*I][2][H/128] fp32;
+ *   dnorm  [E*I] fp32 = ||down column of channel j||.
+ * All device pointers, owned by the caller; codes/scales/dnorm 4-byte
+ * aligned. desc: CHANNEL_MAJOR bf16 SWIGLU with gate = [E][I][3][H];
+ * H % 128 == 0 and H <= 2048, else MOE_ERR_UNSUPPORTED. */
+
+/* Builds the sketch of every channel of one layer (once per model load). */
+moe_status moe_reader_build(const moe_layer_desc* desc, const int8_t* signs, uint32_t* codes,
+                            uint16_t* scales, float* rho, float* dnorm, moe_stream_t stream);
+
+/* Screen of B tokens (1 <= B <= 256): for each token b and each of its
+ * routed experts e = ids[b, slot] (w[b, slot] its router weight), writes
+ * scores[b, e, c] for c < I; rows of experts token b did not route to, and
+ * of ids outside [0, E), are not written. est_opt [B, k, I, 2] fp32 receives {g_hat, v_hat} (or NULL).
+ * x [B, H] bf16 is the expert input (the normalised x under pre-norm). */
+moe_status moe_reader_screen(const moe_layer_desc* desc, const void* x, int32_t B, const int32_t* ids,
+                             const float* w, const int8_t* signs, const uint32_t* codes,
+                             const uint16_t* scales, const float* dnorm, float* scores, float* est_opt,
+                             moe_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -10,6 +10,7 @@
 
 #include "small_kernels.cuh"
 #include "linear.cuh"
+#include "reader.cuh"
 
 using namespace moedec;
 
@@ -404,6 +405,47 @@ moe_status moe_touched_experts(const int32_t* ids, int32_t B, int32_t k, int32_t
   if (B < 1 || B > 256 || k < 1 || k > kMaxK || E < 1 || E > kMaxE || k > E) return MOE_ERR_INVALID;
   touched_kernel<<<1, kThreads, 0, (cudaStream_t)stream>>>(ids, B, k, E, count, bitmap_opt, offsets_opt,
                                                            pairs_opt);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+static bool reader_shape_ok(const moe_layer_desc* d) {
+  return d->kind == MOE_EXPERT_SWIGLU && d->layout == MOE_LAYOUT_CHANNEL_MAJOR && d->wtype == MOE_W_BF16;
+}
+
+moe_status moe_reader_build(const moe_layer_desc* d, const int8_t* signs, uint32_t* codes, uint16_t* scales,
+                            float* rho, float* dnorm, moe_stream_t stream) {
+  if (!valid_shape(d) || !reader_shape_ok(d) || !d->gate || !signs || !codes || !scales || !rho || !dnorm)
+    return MOE_ERR_INVALID;
+  if (d->H % kRdBlock != 0 || d->H > 2048) return MOE_ERR_UNSUPPORTED;
+  if (!aligned16(d->gate) || ((uintptr_t)codes & 3u) || ((uintptr_t)rho & 3u) || ((uintptr_t)dnorm & 3u) ||
+      ((uintptr_t)scales & 1u))
+    return MOE_ERR_INVALID;
+  const long long nch = (long long)d->E * d->I;
+  if (nch > 0x7fffffffLL) return MOE_ERR_UNSUPPORTED;
+  reader_build_kernel<<<(unsigned)nch, kRdBlock, 0, (cudaStream_t)stream>>>(
+      static_cast<const uint16_t*>(d->gate), signs, d->H, codes, scales, rho, dnorm);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status moe_reader_screen(const moe_layer_desc* d, const void* x, int32_t B, const int32_t* ids,
+                             const float* w, const int8_t* signs, const uint32_t* codes, const uint16_t* scales,
+                             const float* dnorm, float* scores, float* est_opt, moe_stream_t stream) {
+  if (!valid_shape(d) || !reader_shape_ok(d) || !x || !ids || !w || !signs || !codes || !scales || !dnorm ||
+      !scores)
+    return MOE_ERR_INVALID;
+  if (B < 1 || B > 256) return MOE_ERR_INVALID;
+  if (d->H % kRdBlock != 0 || d->H > 2048) return MOE_ERR_UNSUPPORTED;
+  if (((uintptr_t)x & 1u) || ((uintptr_t)codes & 3u) || ((uintptr_t)dnorm & 3u) || ((uintptr_t)scales & 1u) ||
+      ((uintptr_t)scores & 3u) || ((uintptr_t)est_opt & 3u))
+    return MOE_ERR_INVALID;
+  const int sms = sm_count();
+  if (sms <= 0) return MOE_ERR_CUDA;
+  // about two CTAs per SM over the batch, each CTA at least 8 channels
+  const int nq = d->k * d->I, wpc = kRdScreenThreads / 32;
+  const int gx = std::max(1, std::min((nq + wpc - 1) / wpc, (2 * sms + B - 1) / B));
+  reader_screen_kernel<<<dim3((unsigned)gx, (unsigned)B), kRdScreenThreads, 0, (cudaStream_t)stream>>>(
+      static_cast<const uint16_t*>(x), d->H, d->E, d->I, d->k, ids, w, signs, codes, scales, dnorm, scores,
+      est_opt);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

@@ -1,0 +1,179 @@
+// Weight-only channel screen of the channel-sparse reader: the rotated
+// ternary sketch of every channel's gate and up rows, built once per layer
+// from the weights, and the per-token screen that turns it into output-unit
+// scores for the top-keep selection ([Reader] "가중치만으로 만든 reader",
+// step 1 and step 2, eq. 1).
+#pragma once
+
+#include <cuda_fp16.h>
+
+#include "small_kernels.cuh"
+
+namespace moedec {
+
+constexpr int kRdBlock = 128;        // coordinates per rotation block
+constexpr int kRdMaxWords = 4;       // 2-bit code words per lane and row (H <= 2048)
+constexpr int kRdScreenThreads = 256;
+
+// Sketch builder: one CTA of 128 threads per channel j = e*I + c of a
+// channel-major layer [E][I][3][H] bf16 (gate row, up row, down column).
+// For the gate and the up row, block by block (thread t = coordinate t):
+//   u = H_128 (s * v) in fp64 by the Sylvester butterfly (unnormalised, so
+//       R v = u / sqrt(128) for the orthogonal R = H_128 diag(s) / sqrt(128));
+//       every sum is exact while the block's bf16 values span < 2^38;
+//   delta = 0.7 * (sum |u| / 128); code = sign(u) where |u| > delta, else 0;
+//   scale = fp16(fp32(sum of |u| over the coded coordinates / their count));
+//   rho = sum((u - scale * code)^2) / 128 / 128 (mean squared error of the
+//       block in the orthogonal rotation's units).
+// Codes of row r of channel j: words (2j + r) * H/16 .., coordinate h at
+// bits 2(h % 16) (nonzero) and 2(h % 16) + 1 (negative) of word h / 16.
+// dnorm[j] = fp32(sqrt(sum of the squared down column)), summed in fp64.
+__global__ void __launch_bounds__(kRdBlock) reader_build_kernel(const uint16_t* __restrict__ cm,
+                                                                const int8_t* __restrict__ signs, int H,
+                                                                uint32_t* __restrict__ codes,
+                                                                uint16_t* __restrict__ scales,
+                                                                float* __restrict__ rho,
+                                                                float* __restrict__ dnorm) {
+  __shared__ double u[kRdBlock];
+  __shared__ double red[3][kRdBlock / 32];
+  __shared__ int rcnt[kRdBlock / 32];
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const size_t j = blockIdx.x;
+  const uint16_t* rows = cm + j * 3 * (size_t)H;
+  const int nb = H / kRdBlock, words = H / 16;
+  auto block_sum = [&](double v, int slot) -> double {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0) red[slot][warp] = v;
+    __syncthreads();
+    return (red[slot][0] + red[slot][1]) + (red[slot][2] + red[slot][3]);
+  };
+  for (int r = 0; r < 2; ++r) {
+    const uint16_t* v = rows + (size_t)r * H;
+    const size_t row = 2 * j + r;
+    for (int b = 0; b < nb; ++b) {
+      const int h = b * kRdBlock + t;
+      u[t] = (double)bf16_to_f(v[h]) * (double)signs[h];
+      __syncthreads();
+      // stage m: (x_i, x_{i+m}) <- (x_i + x_{i+m}, x_i - x_{i+m}) for i & m == 0
+      for (int m = 1; m < kRdBlock; m <<= 1) {
+        const double a = u[t], p = u[t ^ m];
+        const double nv = (t & m) ? (p - a) : (a + p);
+        __syncthreads();
+        u[t] = nv;
+        __syncthreads();
+      }
+      const double ut = u[t], au = fabs(ut);
+      const double delta = 0.7 * (block_sum(au, 0) / 128.0);
+      const bool nz = au > delta, neg = ut < 0.0;
+      const double ssum = block_sum(nz ? au : 0.0, 1);
+      int c = nz ? 1 : 0;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+      if (lane == 0) rcnt[warp] = c;
+      __syncthreads();
+      const int cnt = rcnt[0] + rcnt[1] + rcnt[2] + rcnt[3];
+      const double scale64 = cnt ? ssum / (double)cnt : 0.0;
+      const __half s16 = __float2half_rn(__double2float_rn(scale64));
+      const double sc = (double)__half2float(s16);
+      const double err = ut - (nz ? (neg ? -sc : sc) : 0.0);
+      const double esum = block_sum(err * err, 2);
+      // 2-bit fields of 16 coordinates OR-ed into one word
+      uint32_t bits = (nz ? (neg ? 3u : 1u) : 0u) << (2 * (t & 15));
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) bits |= __shfl_xor_sync(0xffffffffu, bits, o);
+      if ((t & 15) == 0) codes[row * words + b * (kRdBlock / 16) + (t >> 4)] = bits;
+      if (t == 0) {
+        scales[row * nb + b] = __half_as_ushort(s16);
+        rho[row * nb + b] = (float)(esum / 128.0 / 128.0);
+      }
+      __syncthreads();  // u and red are rewritten by the next block
+    }
+  }
+  const uint16_t* d = rows + 2 * (size_t)H;
+  double q = 0.0;
+  for (int h = t; h < H; h += kRdBlock) {
+    const double dv = (double)bf16_to_f(d[h]);
+    q += dv * dv;
+  }
+  const double tot = block_sum(q, 0);
+  if (t == 0) dnorm[j] = (float)sqrt(tot);
+}
+
+// Screen: token b = blockIdx.y. The CTA rotates x_b once, ux = H_128 (s * x_b)
+// per block in fp32 (shared memory), then each warp takes channels q of the
+// k*I candidates (slot q / I, channel q % I of expert ids[b, slot]):
+//   g_hat = sum_blocks scale_b * (codes_b . ux_b) / 128, v_hat likewise,
+//   scores[b, e, c] = w[b, slot] * dnorm[e*I + c] * |SiLU(g_hat) * v_hat|.
+// Lane l holds the coordinates of code words l + 32 t (t < H/512) in
+// registers, so each row is read as H/16 coalesced words. est_opt[b, slot,
+// c] = {g_hat, v_hat} when given. Rows of unrouted experts, and of ids
+// outside [0, E), are not written.
+__global__ void __launch_bounds__(kRdScreenThreads) reader_screen_kernel(
+    const uint16_t* __restrict__ x, int H, int E, int I, int k, const int32_t* __restrict__ ids,
+    const float* __restrict__ w, const int8_t* __restrict__ signs, const uint32_t* __restrict__ codes,
+    const uint16_t* __restrict__ scales, const float* __restrict__ dnorm, float* __restrict__ scores,
+    float* __restrict__ est) {
+  __shared__ float ux[2048];
+  const int b = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int i = tid; i < H; i += kRdScreenThreads) ux[i] = bf16_to_f(x[(size_t)b * H + i]) * (float)signs[i];
+  __syncthreads();
+  for (int lg = 0; lg < 7; ++lg) {
+    const int m = 1 << lg;
+    for (int p = tid; p < H / 2; p += kRdScreenThreads) {
+      const int i = ((p >> lg) << (lg + 1)) | (p & (m - 1));
+      const float a0 = ux[i], a1 = ux[i + m];
+      ux[i] = a0 + a1;
+      ux[i + m] = a0 - a1;
+    }
+    __syncthreads();
+  }
+  const int words = H / 16, nb = H / kRdBlock;
+  float xr[kRdMaxWords][16];
+#pragma unroll
+  for (int t = 0; t < kRdMaxWords; ++t) {
+    const int wd = lane + 32 * t;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) xr[t][i] = wd < words ? ux[16 * wd + i] : 0.f;
+  }
+  const int nq = k * I, wpc = kRdScreenThreads / 32;
+  for (int q = blockIdx.x * wpc + warp; q < nq; q += gridDim.x * wpc) {
+    const int slot = q / I, c = q - slot * I;
+    const int e = ids[b * k + slot];
+    if ((unsigned)e >= (unsigned)E) continue;  // an id out of range is skipped (warp-uniform)
+    const size_t j = (size_t)e * I + c;
+    float gv[2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const uint32_t* cw = codes + (2 * j + r) * (size_t)words;
+      const uint16_t* sc = scales + (2 * j + r) * (size_t)nb;
+      float acc = 0.f;
+#pragma unroll
+      for (int t = 0; t < kRdMaxWords; ++t) {
+        const int wd = lane + 32 * t;
+        if (wd < words) {
+          const uint32_t word = __ldg(cw + wd);
+          const float s = __half2float(__ushort_as_half(__ldg(sc + (wd >> 3))));
+          float pt = 0.f;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const uint32_t f = word >> (2 * i);
+            if (f & 1u) pt += (f & 2u) ? -xr[t][i] : xr[t][i];
+          }
+          acc = fmaf(s, pt, acc);
+        }
+      }
+      gv[r] = warp_sum(acc) * (1.0f / 128.0f);
+    }
+    if (lane == 0) {
+      scores[((size_t)b * E + e) * I + c] = w[b * k + slot] * __ldg(dnorm + j) * fabsf(silu_f(gv[0]) * gv[1]);
+      if (est != nullptr) {
+        float* o = est + (((size_t)b * k + slot) * I + c) * 2;
+        o[0] = gv[0];
+        o[1] = gv[1];
+      }
+    }
+  }
+}
+
+}  // namespace moedec

@@ -34,7 +34,7 @@ EXPORTS = [
     "moe_abi_version", "moe_status_string", "moe_workspace_bytes", "moe_workspace_init",
     "moe_get_status", "moe_route_topk", "moe_expert_forward", "moe_layer_forward",
     "moe_stack_forward", "moe_channel_topk_forward", "moe_touched_experts",
-    "moe_layer_forward_static", "moe_channel_stack_forward",
+    "moe_layer_forward_static", "moe_channel_stack_forward", "moe_reader_build", "moe_reader_screen",
 ]
 
 
@@ -70,6 +70,8 @@ _lib.moe_touched_experts.argtypes = [_P, _I, _I, _I, _P, _P, _P, _P, _P]
 _lib.moe_channel_stack_forward.argtypes = [ctypes.POINTER(LayerDesc), _I, _P, ctypes.c_uint32, _P, _I, _P, _P, _P,
                                            _P, _P, _P, _P, _P, _S, _P]
 _lib.moe_layer_forward_static.argtypes = [ctypes.POINTER(LayerDesc), _P, _I, _P, _P, _P, _P, _P, _P]
+_lib.moe_reader_build.argtypes = [ctypes.POINTER(LayerDesc), _P, _P, _P, _P, _P, _P]
+_lib.moe_reader_screen.argtypes = [ctypes.POINTER(LayerDesc), _P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P]
 for _f in EXPORTS[3:]:
     getattr(_lib, _f).restype = ctypes.c_int
 
@@ -193,3 +195,21 @@ def moe_layer_forward_static(desc, x, y, x_next=None, ids_out=None, w_out=None, 
     _check(_lib.moe_layer_forward_static(ctypes.byref(desc), _ptr(x), x.shape[0], _ptr(y), _ptr(x_next),
                                          _ptr(ids_out), _ptr(w_out), _ptr(status_out), _stream(stream)),
            "moe_layer_forward_static")
+
+
+def reader_sketch_shapes(desc: LayerDesc) -> dict:
+    """Shapes of the channel screen's sketch buffers for one layer."""
+    n = desc.E * desc.I
+    return {"codes": (n, 2, desc.H // 16), "scales": (n, 2, desc.H // 128), "rho": (n, 2, desc.H // 128),
+            "dnorm": (n,)}
+
+
+def moe_reader_build(desc, signs, codes, scales, rho, dnorm, stream=None):
+    _check(_lib.moe_reader_build(ctypes.byref(desc), _ptr(signs), _ptr(codes), _ptr(scales), _ptr(rho),
+                                 _ptr(dnorm), _stream(stream)), "moe_reader_build")
+
+
+def moe_reader_screen(desc, x, ids, w, signs, codes, scales, dnorm, scores, est=None, stream=None):
+    _check(_lib.moe_reader_screen(ctypes.byref(desc), _ptr(x), x.shape[0], _ptr(ids), _ptr(w), _ptr(signs),
+                                  _ptr(codes), _ptr(scales), _ptr(dnorm), _ptr(scores), _ptr(est),
+                                  _stream(stream)), "moe_reader_screen")

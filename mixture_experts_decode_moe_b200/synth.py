@@ -153,6 +153,19 @@ def channel_scores(B, E, I, scale: torch.Tensor, seed, device="cpu") -> torch.Te
     return (z * scale.to(device)).contiguous()
 
 
+def reader_signs(H: int, seed: int, device="cpu") -> torch.Tensor:
+    """The channel screen's random rotation signs: H values of +-1, int8."""
+    g = _gen(seed, device)
+    return (torch.randint(0, 2, (H,), generator=g, device=device, dtype=torch.int8) * 2 - 1).to(torch.int8)
+
+
+def router_weights(B: int, k: int, seed: int, device="cpu") -> torch.Tensor:
+    """Positive per-slot expert weights U(0.05, 1), fp32 [B, k] (an input
+    of the screen; the screen does not require them to sum to 1)."""
+    g = _gen(seed, device)
+    return (0.05 + 0.95 * torch.rand((B, k), generator=g, device=device)).contiguous()
+
+
 def linear_experts(E, H, seed, device="cpu") -> torch.Tensor:
     """E expert matrices [E, H, H] bf16 N(0, 0.02)."""
     return _chunked_normal((E, H, H), W_STD, _gen(seed, device), device)

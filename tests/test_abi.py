@@ -84,3 +84,29 @@ def test_invalid_arguments_rejected_before_launch(M):
     cm = desc(M, E=128, I=768, layout=1)
     assert lib.moe_channel_topk_forward(ctypes.byref(cm), dummy, 1, dummy, dummy, dummy, 8 * 768 + 1,
                                         dummy, None, dummy, dummy, 1 << 20, None) == 1
+
+
+def test_reader_entries_reject_bad_arguments_before_launch(M):
+    lib = M._lib
+    P = ctypes.c_void_p
+    dummy = P(4096)  # never dereferenced: every call below fails validation first
+    cm = desc(M, E=128, I=768, layout=1)
+    cm.gate = dummy
+    planar = desc(M, E=128, I=768)
+    planar.gate = dummy
+    odd_h = desc(M, H=192, E=16, I=64, k=2, layout=1)  # H % 128 != 0
+    odd_h.gate = dummy
+    wide = desc(M, H=4096, E=16, I=64, k=2, layout=1)
+    wide.gate = dummy
+    b = ctypes.byref
+    assert lib.moe_reader_build(b(planar), dummy, dummy, dummy, dummy, dummy, None) == M.MOE_ERR_INVALID
+    assert lib.moe_reader_build(b(cm), None, dummy, dummy, dummy, dummy, None) == M.MOE_ERR_INVALID
+    assert lib.moe_reader_build(b(cm), dummy, P(4098), dummy, dummy, dummy, None) == M.MOE_ERR_INVALID
+    assert lib.moe_reader_build(b(odd_h), dummy, dummy, dummy, dummy, dummy, None) == M.MOE_ERR_UNSUPPORTED
+    assert lib.moe_reader_build(b(wide), dummy, dummy, dummy, dummy, dummy, None) == M.MOE_ERR_UNSUPPORTED
+    args = (dummy, dummy, dummy, dummy, dummy, dummy, dummy, None, None)
+    assert lib.moe_reader_screen(b(cm), dummy, 0, *args) == M.MOE_ERR_INVALID
+    assert lib.moe_reader_screen(b(cm), dummy, 257, *args) == M.MOE_ERR_INVALID
+    assert lib.moe_reader_screen(b(planar), dummy, 1, *args) == M.MOE_ERR_INVALID
+    assert lib.moe_reader_screen(b(cm), None, 1, *args) == M.MOE_ERR_INVALID
+    assert lib.moe_reader_screen(b(odd_h), dummy, 1, *args) == M.MOE_ERR_UNSUPPORTED
