@@ -106,15 +106,20 @@ __global__ void __launch_bounds__(kRdBlock) reader_build_kernel(const uint16_t* 
 //   g_hat = sum_blocks scale_b * (codes_b . ux_b) / 128, v_hat likewise,
 //   scores[b, e, c] = w[b, slot] * dnorm[e*I + c] * |SiLU(g_hat) * v_hat|.
 // Lane l holds the coordinates of code words l + 32 t (t < H/512) in
-// registers, so each row is read as H/16 coalesced words. est_opt[b, slot,
-// c] = {g_hat, v_hat} when given. Rows of unrouted experts, and of ids
-// outside [0, E), are not written.
+// registers (read from a copy of ux padded by one float per 16, so that the
+// 32 lanes hit 32 banks), and each row is read as H/16 coalesced words. A
+// warp fetches its next channel's words, scales, weight and norm before it
+// decodes the current one. A code adds x with its sign bit flipped when the
+// code is negative, selected away when it is zero (no branches).
+// est_opt[b, slot, c] = {g_hat, v_hat} when given. Rows of unrouted experts,
+// and of ids outside [0, E), are not written.
 __global__ void __launch_bounds__(kRdScreenThreads) reader_screen_kernel(
     const uint16_t* __restrict__ x, int H, int E, int I, int k, const int32_t* __restrict__ ids,
     const float* __restrict__ w, const int8_t* __restrict__ signs, const uint32_t* __restrict__ codes,
     const uint16_t* __restrict__ scales, const float* __restrict__ dnorm, float* __restrict__ scores,
     float* __restrict__ est) {
   __shared__ float ux[2048];
+  __shared__ float uxp[2048 + 2048 / 16];
   const int b = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   for (int i = tid; i < H; i += kRdScreenThreads) ux[i] = bf16_to_f(x[(size_t)b * H + i]) * (float)signs[i];
   __syncthreads();
@@ -128,51 +133,79 @@ __global__ void __launch_bounds__(kRdScreenThreads) reader_screen_kernel(
     }
     __syncthreads();
   }
+  for (int i = tid; i < H; i += kRdScreenThreads) uxp[i + (i >> 4)] = ux[i];
+  __syncthreads();
   const int words = H / 16, nb = H / kRdBlock;
   float xr[kRdMaxWords][16];
 #pragma unroll
   for (int t = 0; t < kRdMaxWords; ++t) {
     const int wd = lane + 32 * t;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) xr[t][i] = wd < words ? ux[16 * wd + i] : 0.f;
+    for (int i = 0; i < 16; ++i) xr[t][i] = wd < words ? uxp[17 * wd + i] : 0.f;
   }
-  const int nq = k * I, wpc = kRdScreenThreads / 32;
-  for (int q = blockIdx.x * wpc + warp; q < nq; q += gridDim.x * wpc) {
-    const int slot = q / I, c = q - slot * I;
-    const int e = ids[b * k + slot];
-    if ((unsigned)e >= (unsigned)E) continue;  // an id out of range is skipped (warp-uniform)
-    const size_t j = (size_t)e * I + c;
-    float gv[2];
+  // one channel's inputs, fetched a channel ahead
+  struct Fetch {
+    int e, slot, c;
+    float wt, dn;
+    uint32_t wv[2][kRdMaxWords];
+    float sv[2][kRdMaxWords];
+  };
+  const int nq = k * I, wpc = kRdScreenThreads / 32, qstride = gridDim.x * wpc;
+  auto fetch = [&](int q, Fetch& f) {
+    f.e = -1;
+    if (q >= nq) return;
+    f.slot = q / I;
+    f.c = q - f.slot * I;
+    const int e = __ldg(ids + b * k + f.slot);
+    if ((unsigned)e >= (unsigned)E) return;  // an id out of range is skipped (warp-uniform)
+    f.e = e;
+    const size_t j = (size_t)e * I + f.c;
+    f.wt = __ldg(w + b * k + f.slot);
+    f.dn = __ldg(dnorm + j);
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const uint32_t* cw = codes + (2 * j + r) * (size_t)words;
-      const uint16_t* sc = scales + (2 * j + r) * (size_t)nb;
-      float acc = 0.f;
+    for (int r = 0; r < 2; ++r)
 #pragma unroll
       for (int t = 0; t < kRdMaxWords; ++t) {
         const int wd = lane + 32 * t;
-        if (wd < words) {
-          const uint32_t word = __ldg(cw + wd);
-          const float s = __half2float(__ushort_as_half(__ldg(sc + (wd >> 3))));
+        f.wv[r][t] = wd < words ? __ldg(codes + (2 * j + r) * (size_t)words + wd) : 0u;
+        f.sv[r][t] = wd < words ? __half2float(__ushort_as_half(__ldg(scales + (2 * j + r) * (size_t)nb + (wd >> 3))))
+                                : 0.f;
+      }
+  };
+  Fetch cur, nxt;
+  int q = blockIdx.x * wpc + warp;
+  fetch(q, cur);
+  for (; q < nq; q += qstride) {
+    fetch(q + qstride, nxt);
+    if (cur.e >= 0) {
+      float gv[2];
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        float acc = 0.f;
+#pragma unroll
+        for (int t = 0; t < kRdMaxWords; ++t) {
+          const uint32_t word = cur.wv[r][t];
           float pt = 0.f;
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const uint32_t f = word >> (2 * i);
-            if (f & 1u) pt += (f & 2u) ? -xr[t][i] : xr[t][i];
+            const uint32_t sgn = (word << (30 - 2 * i)) & 0x80000000u;  // bit 2i+1 -> sign
+            const float xv = __uint_as_float(__float_as_uint(xr[t][i]) ^ sgn);
+            pt += ((word >> (2 * i)) & 1u) ? xv : 0.f;
           }
-          acc = fmaf(s, pt, acc);
+          acc = fmaf(cur.sv[r][t], pt, acc);
+        }
+        gv[r] = warp_sum(acc) * (1.0f / 128.0f);
+      }
+      if (lane == 0) {
+        scores[((size_t)b * E + cur.e) * I + cur.c] = cur.wt * cur.dn * fabsf(silu_f(gv[0]) * gv[1]);
+        if (est != nullptr) {
+          float* o = est + (((size_t)b * k + cur.slot) * I + cur.c) * 2;
+          o[0] = gv[0];
+          o[1] = gv[1];
         }
       }
-      gv[r] = warp_sum(acc) * (1.0f / 128.0f);
     }
-    if (lane == 0) {
-      scores[((size_t)b * E + e) * I + c] = w[b * k + slot] * __ldg(dnorm + j) * fabsf(silu_f(gv[0]) * gv[1]);
-      if (est != nullptr) {
-        float* o = est + (((size_t)b * k + slot) * I + c) * 2;
-        o[0] = gv[0];
-        o[1] = gv[1];
-      }
-    }
+    cur = nxt;
   }
 }
 
