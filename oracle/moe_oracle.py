@@ -550,6 +550,67 @@ def reader_screen(x: np.ndarray, ids: Sequence[int], w: Sequence[float], sketch,
 
 
 # ----------------------------------------------------------------------------
+# Partial screen and recovery of dropped channels. [Reader] "가중치만으로 만든
+# reader": step 1's partial scan (at low budgets only the ternary codes of
+# the 80 coordinates with the largest |Rx| in each block are read) and step 3
+# ("버린 채널을 rank-32 맵으로 복구한다", eq. 2): U = the top 32 left singular
+# vectors of the layer's stacked down columns, b_j = U^T d_j per channel, and
+#   y_hat = sum_{j in K} w_j d_j a_j + U sum_{j in S} w_j b_j p_j,
+# K the kept channels (exact a_j), S the dropped ones with the screen's
+# estimate p_j = phi(g_hat_j) v_hat_j.
+# Readings: ties in |Rx| go to the lower coordinate; "all down columns of the
+# layer" are the E*I columns d_{e,c} of every expert.
+# ----------------------------------------------------------------------------
+
+PARTIAL_COORDS = 80
+RECOVERY_RANK = 32
+
+
+def reader_partial_mask(x: np.ndarray, signs: np.ndarray, m: int = PARTIAL_COORDS) -> np.ndarray:
+    """Boolean [H]: in each block, the m coordinates with the largest |u_x|
+    (u_x = H_128 (s * x), the same order as |R x|), ties to the lower index."""
+    ux = np.abs(reader_rotate(x, signs)).reshape(-1, READER_BLOCK)
+    mask = np.zeros_like(ux, dtype=bool)
+    for b in range(ux.shape[0]):
+        order = sorted(range(READER_BLOCK), key=lambda i: (-ux[b, i], i))
+        mask[b, order[:m]] = True
+    return mask.reshape(-1)
+
+
+def reader_estimate_partial(x: np.ndarray, codes: np.ndarray, scales: np.ndarray, signs: np.ndarray,
+                            m: int = PARTIAL_COORDS) -> float:
+    """The estimate of reader_estimate over the masked coordinates only."""
+    keep = reader_partial_mask(x, signs, m)
+    c = np.where(keep, np.asarray(codes, dtype=np.float64), 0.0)
+    return reader_estimate(x, c, scales, signs)
+
+
+def recovery_basis(down_cols: np.ndarray, rank: int = RECOVERY_RANK) -> np.ndarray:
+    """U [H, rank]: the top `rank` left singular vectors of D = [d_1 ... d_n]
+    (down_cols [n, H], one down column per row), by the library SVD."""
+    u, _, _ = np.linalg.svd(np.asarray(down_cols, dtype=np.float64).T, full_matrices=False)
+    return u[:, :rank]
+
+
+def recovery_coeffs(U: np.ndarray, d: np.ndarray) -> np.ndarray:
+    """b_j = U^T d_j."""
+    return np.asarray(U).T @ np.asarray(d, dtype=np.float64)
+
+
+def reader_output(kept_terms: Iterable[tuple], dropped_terms: Iterable[tuple], U: np.ndarray) -> np.ndarray:
+    """Eq. 2. kept_terms: (w_j, a_j, d_j) of the kept channels; dropped_terms:
+    (w_j, p_j, b_j) of the dropped ones."""
+    H = U.shape[0]
+    y = np.zeros(H)
+    for wj, aj, dj in kept_terms:
+        y = y + wj * aj * np.asarray(dj, dtype=np.float64)
+    r = np.zeros(U.shape[1])
+    for wj, pj, bj in dropped_terms:
+        r = r + wj * pj * np.asarray(bj, dtype=np.float64)
+    return y + U @ r
+
+
+# ----------------------------------------------------------------------------
 # Bytes-per-token accounting and decode ceiling.
 # [MoE-arith] "Two Numbers Instead of One" / moe_promise.py: ceiling =
 # achieved bandwidth / bytes per token. [Beam] §2 memory table: resident =

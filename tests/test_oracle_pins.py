@@ -619,3 +619,88 @@ def test_eq1_score_hand_values():
     # the sign of v_hat and of phi(g_hat) do not matter; a zero estimate scores 0
     assert O.reader_score(0.5, 2.0, -1.0, 3.0) == O.reader_score(0.5, 2.0, -1.0, -3.0)
     assert O.reader_score(0.5, 2.0, 0.0, 5.0) == 0.0
+
+
+def test_partial_mask_bruteforce_and_ties():
+    # The mask against a direct count per coordinate: i is kept iff fewer than
+    # m coordinates of its block beat it (larger |u|, or equal and lower index).
+    r = rng(46)
+    H = 256
+    s = r.choice([-1.0, 1.0], H)
+    x = O.bf16_round(r.normal(0, 1, H))
+    for m in (0, 1, 80, 127, 128):
+        mask = O.reader_partial_mask(x, s, m).reshape(-1, 128)
+        ua = np.abs(O.reader_rotate(x, s)).reshape(-1, 128)
+        for b in range(ua.shape[0]):
+            for i in range(128):
+                beat = np.sum(ua[b] > ua[b, i]) + np.sum((ua[b] == ua[b, i]) & (np.arange(128) < i))
+                assert mask[b, i] == (beat < m)
+    # ties: x = e_0 rotates to +-1 everywhere in block 0; the first 80 indices win
+    e0 = np.zeros(H)
+    e0[0] = 1.0
+    mk = O.reader_partial_mask(e0, s, 80).reshape(-1, 128)
+    assert mk[0, :80].all() and not mk[0, 80:].any()
+
+
+def test_partial_estimate_special_cases():
+    # m = 128 reads every code (the full estimate); m = 0 reads none.
+    r = rng(47)
+    H = 256
+    s = r.choice([-1.0, 1.0], H)
+    g = O.bf16_round(r.normal(0, 0.02, H))
+    x = O.bf16_round(r.normal(0, 1, H))
+    codes, sc, _ = O.reader_sketch_row(g, s)
+    assert O.reader_estimate_partial(x, codes, sc, s, 128) == O.reader_estimate(x, codes, sc, s)
+    assert O.reader_estimate_partial(x, codes, sc, s, 0) == 0.0
+    # the dropped coordinates are those of smallest |Rx|: with codes all +1
+    # and unit scales, the partial estimate is the sum of the kept u_x / 128
+    ones = np.ones(H, dtype=np.int8)
+    ux = O.reader_rotate(x, s)
+    keep = O.reader_partial_mask(x, s, 80)
+    got = O.reader_estimate_partial(x, ones, np.ones(2), s, 80)
+    assert abs(got - ux[keep].sum() / 128) <= 1e-12 * np.abs(ux).sum()
+
+
+def test_recovery_full_rank_is_exact():
+    # Eq. 2 with rank = H (U square, orthogonal): U b_j = U U^T d_j = d_j, so the
+    # recovered part is sum_S w_j p_j d_j exactly; with p_j = a_j the output is
+    # the all-kept (dense) channel output.
+    r = rng(48)
+    H, n = 16, 40
+    D = r.normal(0, 1, (n, H))
+    U = O.recovery_basis(D, rank=H)
+    assert np.allclose(U.T @ U, np.eye(H), atol=1e-12)
+    w = r.uniform(0.1, 1.0, n)
+    a = r.normal(0, 1, n)
+    kept = [0, 3, 7]
+    dropped = [j for j in range(n) if j not in kept]
+    y = O.reader_output([(w[j], a[j], D[j]) for j in kept],
+                        [(w[j], a[j], O.recovery_coeffs(U, D[j])) for j in dropped], U)
+    dense = sum(w[j] * a[j] * D[j] for j in range(n))
+    assert np.allclose(y, dense, atol=1e-10)
+
+
+def test_recovery_exact_on_low_rank_columns_and_eckart_young():
+    # Down columns inside a 3-dim subspace: a rank-3 basis spans them, so the
+    # recovery of every dropped channel is exact. And the residual of the
+    # rank-r projection of D is the sum of the squared trailing singular values.
+    r = rng(49)
+    H, n, k = 24, 60, 3
+    A = r.normal(0, 1, (H, k))
+    D = (A @ r.normal(0, 1, (k, n))).T
+    U = O.recovery_basis(D, rank=k)
+    for j in range(n):
+        assert np.allclose(U @ O.recovery_coeffs(U, D[j]), D[j], atol=1e-10)
+    D2 = r.normal(0, 1, (n, H))
+    s = np.linalg.svd(D2.T, compute_uv=False)
+    for rank in (1, 5, 12):
+        U2 = O.recovery_basis(D2, rank=rank)
+        resid = D2.T - U2 @ (U2.T @ D2.T)
+        assert abs(np.sum(resid ** 2) - np.sum(s[rank:] ** 2)) <= 1e-9 * np.sum(s ** 2)
+
+
+def test_recovery_map_is_half_a_percent_of_a_channel():
+    # [Reader] step 3: the map adds about 0.5% of resident memory. With 32 fp16
+    # coefficients per channel against its 3 bf16 rows of H = 2048 (Qwen3-Thinking):
+    frac = 32 * 2 / (3 * 2048 * 2)
+    assert abs(frac - 0.005) < 0.0005
