@@ -416,6 +416,17 @@ def channel_stack_layer(x: np.ndarray, router: np.ndarray, channel: Callable[[in
     return residual_bf16(x, y), y, ids, w, logits, kept
 
 
+def channel_union(kept_lists: Iterable[Iterable[int]]) -> np.ndarray:
+    """Channels a batch reads once: the union of every token's kept channel
+    indices e*I + c, ascending ([Reader] "속도": at batch > 1 the tokens' kept
+    channels are read as their union, which grows with the batch)."""
+    parts = [np.asarray(list(k), dtype=np.int64) for k in kept_lists]
+    parts = [q for q in parts if q.size]
+    if not parts:
+        return np.zeros(0, dtype=np.int64)
+    return np.unique(np.concatenate(parts))
+
+
 def sectors_touched(ranges: Iterable[tuple]) -> int:
     """Distinct 32-byte sectors covering the half-open byte ranges [lo, hi).
 

@@ -704,3 +704,20 @@ def test_recovery_map_is_half_a_percent_of_a_channel():
     # coefficients per channel against its 3 bf16 rows of H = 2048 (Qwen3-Thinking):
     frac = 32 * 2 / (3 * 2048 * 2)
     assert abs(frac - 0.005) < 0.0005
+
+
+def test_channel_union_of_a_batch():
+    # brute force against a set; one token gives its own kept list; tokens
+    # with the same kept list read it once; disjoint lists add up
+    r = rng(50)
+    lists = [sorted(r.choice(600, 37, replace=False).tolist()) for _ in range(5)]
+    u = O.channel_union(lists)
+    assert u.tolist() == sorted(set().union(*map(set, lists)))
+    assert O.channel_union(lists[:1]).tolist() == lists[0]
+    assert O.channel_union([lists[0]] * 4).tolist() == lists[0]
+    a, b = list(range(0, 10)), list(range(10, 25))
+    assert O.channel_union([a, b]).size == 25
+    assert O.channel_union([[], []]).size == 0
+    # read bytes of the union: 384 sectors per aligned channel-major channel
+    H = 2048
+    assert O.sectors_touched(O.channel_major_ranges(u, H)) == 384 * u.size
