@@ -110,3 +110,28 @@ def test_reader_entries_reject_bad_arguments_before_launch(M):
     assert lib.moe_reader_screen(b(planar), dummy, 1, *args) == M.MOE_ERR_INVALID
     assert lib.moe_reader_screen(b(cm), None, 1, *args) == M.MOE_ERR_INVALID
     assert lib.moe_reader_screen(b(odd_h), dummy, 1, *args) == M.MOE_ERR_UNSUPPORTED
+
+
+def test_plain_c_program_links_and_calls_the_abi(M, tmp_path):
+    """The boundary is usable from C: the header compiles as C99, and a C
+    program linked against libmoedec.so gets the ABI version and a host-side
+    argument rejection (no GPU work)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "abi.c"
+    src.write_text(
+        '#include <stdio.h>\n#include "moedec.h"\n'
+        "int main(void) {\n"
+        "  moe_layer_desc d = {0};\n"
+        "  moe_status st = moe_layer_forward(&d, 0, 1, 0, 0, 0, 0, 0, 0, 0);\n"
+        '  printf("%d %d %s\\n", moe_abi_version(), (int)st, moe_status_string(st));\n'
+        "  return 0;\n}\n")
+    exe = tmp_path / "abi"
+    libdir = os.path.dirname(M.LIB_PATH)
+    subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe),
+                    "-L", libdir, "-l:" + os.path.basename(M.LIB_PATH), "-Wl,-rpath," + libdir], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
+    assert out[0] == "1" and out[1] == str(M.MOE_ERR_INVALID)
