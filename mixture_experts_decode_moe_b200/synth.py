@@ -139,6 +139,26 @@ def channel_major_layer(H, E, I, seed, device="cpu", router_scale=1.0):
     return {"router": router, "cm": _chunked_normal((E, I, 3, H), W_STD, g, device)}
 
 
+def channel_major_layer_lowrank(H, E, I, seed, rank=32, noise=0.3, device="cpu", router_scale=1.0):
+    """Channel-major layer like channel_major_layer, except that the down
+    columns share a planted rank-`rank` subspace: d = W_STD (sqrt(1 - noise^2)
+    B z + noise eps), B [H, rank] with orthonormal columns scaled by
+    sqrt(H / rank), z ~ N(0, I_rank), eps ~ N(0, I_H) per channel, so each
+    coordinate still has standard deviation W_STD and a fraction of about
+    1 - noise^2 of each column's energy lies in span(B). Stands in for trained
+    down projections, whose columns concentrate in few directions."""
+    g = _gen(seed, device)
+    router = normal_bf16((E, H), W_STD * router_scale, g, device)
+    gu = _chunked_normal((E, I, 2, H), W_STD, g, device)
+    q, _ = torch.linalg.qr(torch.randn((H, rank), generator=g, device=device, dtype=torch.float32))
+    basis = q * (H / rank) ** 0.5
+    z = torch.randn((E * I, rank), generator=g, device=device)
+    eps = torch.randn((E * I, H), generator=g, device=device)
+    d = W_STD * ((1.0 - noise * noise) ** 0.5 * (z @ basis.T) + noise * eps)
+    cm = torch.cat([gu, d.to(torch.bfloat16).view(E, I, 1, H)], dim=2).contiguous()
+    return {"router": router, "cm": cm, "basis": basis}
+
+
 def channel_scale(E, I, seed, device="cpu") -> torch.Tensor:
     """Per-channel Pareto(alpha=1.5, x_m=1) scale: U^(-1/1.5), U ~ U(0, 1]."""
     g = _gen(seed, device)

@@ -51,3 +51,24 @@ def test_channel_scores_and_keep():
     assert S.keep_count(0.13, 8, 768) == 799 and S.keep_count(0.18, 8, 768) == 1106
     cm = S.channel_major_layer(64, 2, 3, seed=6)
     assert cm["cm"].shape == (2, 3, 3, 64)
+
+
+def test_lowrank_down_columns_concentrate_in_the_planted_subspace():
+    # the oracle's rank-32 basis of the generated down columns spans the
+    # planted subspace (principal angles near 0), and captures about
+    # 1 - noise^2 of the columns' energy
+    import numpy as np
+    from oracle import moe_oracle as O
+    from mixture_experts_decode_moe_b200 import synth as S
+    H, E, I, r, nu = 256, 4, 96, 8, 0.3
+    L = S.channel_major_layer_lowrank(H, E, I, seed=5, rank=r, noise=nu)
+    cm = L["cm"].float().double().numpy()
+    assert cm.shape == (E, I, 3, H)
+    D = cm[:, :, 2, :].reshape(E * I, H)
+    assert abs(D.std() / S.W_STD - 1.0) < 0.05
+    U = O.recovery_basis(D, rank=r)
+    B = np.linalg.qr(L["basis"].double().numpy())[0]
+    cosines = np.linalg.svd(U.T @ B, compute_uv=False)
+    assert cosines.min() > 0.97
+    captured = np.sum((D @ U) ** 2) / np.sum(D ** 2)
+    assert abs(captured - (1 - nu ** 2 + nu ** 2 * r / H)) < 0.03
