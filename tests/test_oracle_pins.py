@@ -721,3 +721,76 @@ def test_channel_union_of_a_batch():
     # read bytes of the union: 384 sectors per aligned channel-major channel
     H = 2048
     assert O.sectors_touched(O.channel_major_ranges(u, H)) == 384 * u.size
+
+
+def test_reader_screen_pairs_each_slot_with_its_own_weight_and_expert():
+    # Two routed experts in slots (1, 0) with distinct slot weights, two
+    # channels each. With x = e_0 and s_0 = +1 the rotated token is all ones in
+    # block 0 (column 0 of H_128), so an estimate is scale * (sum of codes) / 128;
+    # the sketch below gives every (expert, channel) its own (g_hat, v_hat), so
+    # the eq. 1 scores follow in closed form. Pairing slot t with w[e] instead
+    # of w[t], reading expert t instead of ids[t], or swapping the gate and up
+    # sketches gives other numbers.
+    H, I = 128, 2
+    s = np.ones(H)
+    x = np.zeros(H)
+    x[0] = 1.0
+    ids, w = [1, 0], [0.25, 0.75]
+    half = np.zeros(H, dtype=np.int8)
+    half[:64] = 1                                   # sum of codes = 64: estimate = scale / 2
+    g_hat = {(0, 0): 1.0, (0, 1): -0.5, (1, 0): 2.0, (1, 1): 0.25}
+    v_hat = {(0, 0): 3.0, (0, 1): 1.5, (1, 0): -1.0, (1, 1): 4.0}
+    dn = {(0, 0): 1.0, (0, 1): 2.0, (1, 0): 0.5, (1, 1): 3.0}
+
+    def sketch(e, c):
+        return half, np.array([2 * g_hat[e, c]]), half, np.array([2 * v_hat[e, c]]), dn[e, c]
+
+    scores, est = O.reader_screen(x, ids, w, sketch, I, s)
+    sil = lambda z: z / (1.0 + math.exp(-z))
+    for t, e in enumerate(ids):
+        for c in range(I):
+            assert est[t, c].tolist() == [g_hat[e, c], v_hat[e, c]]
+            want = w[t] * dn[e, c] * abs(sil(g_hat[e, c]) * v_hat[e, c])
+            assert abs(scores[t, c] - want) <= 1e-15 * want
+    # the closed forms above are not symmetric in the plausible slips
+    assert abs(scores[0, 0] - 0.25 * 0.5 * abs(sil(2.0) * -1.0)) < 1e-15
+    assert scores[0, 0] != 0.75 * 0.5 * abs(sil(2.0) * -1.0)   # w[e] for e = 1 would be 0.75
+    assert scores[0, 0] != 0.25 * 0.5 * abs(sil(-1.0) * 2.0)   # gate and up swapped
+    assert scores[1, 0] != 0.75 * 1.0 * abs(sil(2.0) * -1.0)   # slot 1 read as expert 1
+
+
+def test_channel_stack_layer_routes_and_computes_on_u_and_adds_y_to_x():
+    # H = 4, E = 3, k = 2, I = 2 with one-hot router rows (logit of expert e =
+    # u[h_e]), one-hot gate rows, scaled one-hot up rows and one-hot down
+    # columns, so every a_j and y are closed forms of u = rmsnorm_bf16(x).
+    # x has rms sqrt(10) != 1: routing on x (weights from 4, 2 instead of u's
+    # 1.27, 0.63), experts fed x, or the residual added to u all change the result.
+    H, E, I, k, keep = 4, 3, 2, 2, 3
+    x = np.array([4.0, -4.0, 2.0, -2.0])
+    u = O.rmsnorm_bf16(x)
+    onehot = np.eye(H)
+    R = onehot[[0, 2, 1]]                             # logits = (u0, u2, u1)
+    scores = np.array([[5.0, 1.0], [4.0, 3.0], [9.0, 9.0]])  # expert 2 is not routed
+
+    def channel(e, c):
+        return np.stack([onehot[c], (e + 1) * onehot[c + 2], onehot[(e + c) % H]])
+
+    xn, y, ids, w, logits, kept = O.channel_stack_layer(x, R, channel, scores, k, keep, I)
+    assert np.array_equal(logits, u[[0, 2, 1]])
+    assert ids.tolist() == [0, 1]
+    w0 = 1.0 / (1.0 + math.exp(u[2] - u[0]))
+    assert np.allclose(w, [w0, 1.0 - w0], rtol=0, atol=1e-15)
+    assert kept.tolist() == [0, 2, 3]                 # scores 5, 4, 3 of the routed rows
+    sil = lambda z: z / (1.0 + math.exp(-z))
+    want = np.zeros(H)
+    for e, c in ((0, 0), (1, 0), (1, 1)):
+        a = sil(u[c]) * (e + 1) * u[c + 2]
+        want[(e + c) % H] += w[list(ids).index(e)] * a
+    assert np.allclose(y, want, rtol=0, atol=1e-14)
+    assert np.array_equal(xn, O.residual_bf16(x, want))
+    assert not np.array_equal(xn, O.residual_bf16(u, want))
+    wx = 1.0 / (1.0 + math.exp(x[2] - x[0]))
+    assert abs(w[0] - wx) > 0.1                       # routing on x is told apart
+    # without the pre-norm the layer works on x itself
+    _, y0, _, w_raw, l0, _ = O.channel_stack_layer(x, R, channel, scores, k, keep, I, pre_norm=False)
+    assert np.array_equal(l0, x[[0, 2, 1]]) and abs(w_raw[0] - wx) < 1e-15
