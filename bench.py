@@ -183,6 +183,9 @@ class A3BStack:
         self.tokens_per_step = B
         self.launches_per_step = 1
         self.kernel = f"decode_kernel<layers,B{B},{wtype},planar>"
+        self.sources = DECODE_KERNEL_SOURCES
+        self.dtype = "bf16" if wtype == "bf16" else "int4"
+        self.wtype = wtype
         self.record = 0
 
     def _x(self, i):
@@ -221,6 +224,14 @@ class A3BStack:
     def config(self):
         return a3b_config(self.name, self.w, self.B, self.nl)
 
+    def oracle_sample(self, budget_s):
+        """The fp64 oracle on whole layers of this stack (batch 1 token by token)."""
+        tps, done, dt = oracle_rate(self.layers, self.w, self.xs, budget_s=budget_s, wtype=self.wtype)
+        return {"value": tps, "unit": "tok/s", "cores": blas_threads(), "kind": "oracle",
+                "sample": f"{done} layer passes of one token in {dt:.1f} s, scaled to tokens through "
+                          f"{self.nl} layers (fp64; the router, shared and routed experts' slices copied "
+                          "from the device; RMS pre-norm as on the device)"}
+
 
 class ChannelStack:
     """48-layer channel-major stack, batch 1, channel top-k keep over given scores."""
@@ -247,6 +258,8 @@ class ChannelStack:
         self.tokens_per_step = 1
         self.launches_per_step = 1
         self.kernel = "decode_kernel<layers,B1,bf16,channel-major>"
+        self.sources = DECODE_KERNEL_SOURCES
+        self.dtype = "bf16"
 
     def step(self, i, stream):
         self.M.moe_channel_stack_forward(self.descs, self.xs[i % 256:][:1], self.scores[i % self.nsc], self.keep,
@@ -269,6 +282,29 @@ class ChannelStack:
     def nbytes(self, r):
         # router + kept channels (gate row, up row, down column) + the 8 score rows read
         return self.nl * (2 * self.E * self.H + self.keep * 3 * self.H * 2 + self.k * self.I * 4)
+
+    def oracle_sample(self, budget_s):
+        """The fp64 oracle's channel-stack layer, token 0 through the layers in order."""
+        from oracle import moe_oracle as O
+
+        def f64(t):
+            return t.detach().cpu().float().double().numpy()
+        t0 = time.perf_counter()
+        x = f64(self.xs[0])
+        done = 0
+        while True:
+            l = done % self.nl
+            cm = self.layers[l]["cm"]
+            R = f64(self.layers[l]["router"])
+            sc = f64(self.scores[0, l])
+            x, *_ = O.channel_stack_layer(x, R, lambda e, c, cm=cm: f64(cm[e, c]), sc, self.k, self.keep, self.I)
+            done += 1
+            if time.perf_counter() - t0 >= budget_s:
+                break
+        dt = time.perf_counter() - t0
+        return {"value": (done / self.nl) / dt, "unit": "tok/s", "cores": blas_threads(), "kind": "oracle",
+                "sample": f"{done} channel-sparse layer passes of one token in {dt:.1f} s, scaled to tokens "
+                          f"through {self.nl} layers (fp64; kept channels copied from the device)"}
 
     def config(self):
         return {"workload": f"channel_topk_{int(round(100 * self.frac))}pct", "layers": self.nl, "hidden": self.H,
@@ -297,6 +333,9 @@ class BatchSweep:
         self.tokens_per_step = B
         self.launches_per_step = 4  # plan, gather, GEMV engine, tensor-core engine (+ a memset)
         self.kernel = "linear plan+gather+gemv+tcgen05"
+        self.sources = LINEAR_KERNEL_SOURCES
+        self.dtype = "bf16"
+        self.record = 0
 
     def step(self, i, stream):
         t = i % self.nsets
@@ -321,10 +360,134 @@ class BatchSweep:
     def nbytes(self, r):
         return self.touched[r % self.nsets] * self.H * self.H * 2
 
+    def touched_record(self):
+        """Touched experts of the step inputs against E[1 - (1 - k/E)^B]."""
+        return {"mean_touched": statistics.mean(self.touched), "expected": self.E * (1 - (1 - self.k / self.E) ** self.B),
+                "input_sets": self.nsets}
+
+    def oracle_sample(self, budget_s):
+        """The fp64 oracle on whole tokens of step 0 (each token through its k experts)."""
+        from oracle import moe_oracle as O
+        t0 = time.perf_counter()
+        x = self.xs[0].detach().cpu().float().double().numpy()
+        ids = self.ids[0].cpu().numpy()
+        done = 0
+        while True:
+            b = done % self.B
+            O.linear_experts(x[b], lambda e: self.W[e].detach().cpu().float().double().numpy(),
+                             ids[b].tolist(), [1.0] * self.k)
+            done += 1
+            if time.perf_counter() - t0 >= budget_s:
+                break
+        dt = time.perf_counter() - t0
+        return {"value": done / dt, "unit": "tok/s", "cores": blas_threads(), "kind": "oracle",
+                "sample": f"{done} tokens of one batch in {dt:.1f} s, each through its {self.k} experts of "
+                          f"{self.H} x {self.H} (fp64; expert matrices copied from the device)"}
+
     def config(self):
         return {"workload": f"batch_sweep_b{self.B}", "experts": self.E, "top_k": self.k, "hidden": self.H,
                 "batch": self.B, "expected_touched": self.E * (1 - (1 - self.k / self.E) ** self.B),
                 "l2": "inputs larger than L2 (8.6 GB of expert matrices)"}
+
+
+class ChannelBatch:
+    """Channel-sparse layers of the 48-layer channel-major stack at batch B
+    (4 or 8): per layer, B tokens with their own routed experts (k distinct
+    uniform ids) and scores select their kept channels, and the batch reads
+    the union of the kept channels once (one launch per layer). The bytes of
+    a step are the union's 32-byte sectors the kernel reports, plus the
+    score rows; they are compared with reading the touched experts whole
+    (the full-read column of the pages' Table 7)."""
+
+    def __init__(self, torch, M, S, device, rank, B=4, frac=0.13, steps=0):
+        self.torch, self.M, self.S, self.dev = torch, M, S, device
+        w = S.WORKLOADS["channel_topk"]
+        H, E, I, k, nl = w["H"], w["E"], w["I"], w["k"], w["layers"]
+        self.H, self.E, self.I, self.k, self.nl, self.B, self.frac = H, E, I, k, nl, B, frac
+        self.keep = S.keep_count(frac, k, I)
+        self.layers = [S.channel_major_layer(H, E, I, seed=S.weight_seed(5, l), device=device) for l in range(nl)]
+        self.descs = [M.make_desc(H, E, I, k, layout=M.MOE_LAYOUT_CHANNEL_MAJOR, router=L["router"], gate=L["cm"])
+                      for L in self.layers]
+        self.nsets = 4
+        scale = [S.channel_scale(E, I, seed=S.weight_seed(5, l) + 7, device=device) for l in range(nl)]
+        self.scores = [[S.channel_scores(B, E, I, scale[l], seed=S.act_seed(5, l) + 1000 * t + 97 * rank,
+                                         device=device) for l in range(nl)] for t in range(self.nsets)]
+        self.ids = [[S.uniform_ids(B, E, k, seed=S.act_seed(5, l) + 2000 + 1000 * t + 97 * rank, device=device)
+                     for l in range(nl)] for t in range(self.nsets)]
+        self.wts = [torch.softmax(torch.randn((B, k), device=device), dim=1) for _ in range(nl)]
+        self.xs = [S.tokens(B, H, seed=S.act_seed(5) + 31 * t + 97 * rank, device=device) for t in range(self.nsets)]
+        self.ws = M.alloc_workspace(self.descs[0], B, device)
+        self.y = torch.empty((B, H), dtype=torch.float32, device=device)
+        self.sec = torch.empty((B,), dtype=torch.int64, device=device)
+        self.ucount = torch.zeros((max(steps, 1), nl), dtype=torch.int32, device=device)
+        self.usec = torch.zeros((max(steps, 1), nl), dtype=torch.int64, device=device)
+        self.tokens_per_step = B
+        self.launches_per_step = nl
+        self.kernel = f"channel_batch_kernel<B{B}> x {nl} layers"
+        self.sources = ("common.cuh", "decode.cuh", "decode_kernel.cuh", "channel_batch.cuh")
+        self.dtype = "bf16"
+        self.record = 0
+
+    def step(self, i, stream):
+        t = i % self.nsets
+        r = self.record
+        for l in range(self.nl):
+            kw = {"union_count": self.ucount[r, l:l + 1], "union_sectors": self.usec[r, l:l + 1]} \
+                if r < self.ucount.shape[0] else {}
+            self.M.moe_channel_topk_forward(self.descs[l], self.xs[t], self.ids[t][l], self.wts[l], self.scores[t][l],
+                                            self.keep, self.y, self.sec, self.ws, stream=stream, **kw)
+
+    def host_buffers(self):
+        return 0, 0
+
+    def e2e_step(self, i, stream):
+        self.step(i, stream)
+
+    def nbytes(self, r):
+        """Union sectors x 32 (what the batch read) + the B x k score rows read."""
+        return int(self.usec[r].sum().item()) * 32 + self.nl * self.B * self.k * self.I * 4
+
+    def touched_record(self):
+        """Bytes per layer of the union read against reading the touched
+        experts whole (the pages' Table 7 full-read column)."""
+        import statistics as st
+        u = self.ucount[: min(self.ucount.shape[0], 1 << 30)].float()
+        touched = [len(set(self.ids[t][l].reshape(-1).tolist())) for t in range(self.nsets) for l in range(self.nl)]
+        full_mb = st.mean(touched) * self.I * 3 * self.H * 2 / 1e6
+        union_mb = float(u[u > 0].mean().item()) * 3 * self.H * 2 / 1e6 if bool((u > 0).any()) else 0.0
+        return {"union_channels_per_layer": float(u[u > 0].mean().item()) if bool((u > 0).any()) else 0.0,
+                "kept_per_token": self.keep, "union_mb_per_layer": union_mb, "full_read_mb_per_layer": full_mb,
+                "union_share_of_full": union_mb / full_mb if full_mb else None,
+                "table7_reference_share": {"B4": 49.9 / 229.1, "B8": 92.3 / 359.3}}
+
+    def oracle_sample(self, budget_s):
+        from oracle import moe_oracle as O
+
+        def f64(t):
+            return t.detach().cpu().float().double().numpy()
+        t0 = time.perf_counter()
+        done = 0
+        while True:
+            l = done % self.nl
+            cm = self.layers[l]["cm"]
+            for b in range(self.B):
+                ids = self.ids[0][l][b].tolist()
+                kept = O.channel_topk_select(f64(self.scores[0][l][b]), ids, self.keep)
+                O.channel_sparse_forward(f64(self.xs[0][b]), lambda e, c: f64(cm[e, c]), ids, f64(self.wts[l][b]),
+                                         kept, self.I)
+            done += 1
+            if time.perf_counter() - t0 >= budget_s:
+                break
+        dt = time.perf_counter() - t0
+        return {"value": done * self.B / self.nl / dt, "unit": "tok/s", "cores": blas_threads(), "kind": "oracle",
+                "sample": f"{done} layers of a batch of {self.B} in {dt:.1f} s, scaled to tokens through "
+                          f"{self.nl} layers (fp64; kept channels copied from the device)"}
+
+    def config(self):
+        return {"workload": f"channel_topk_{int(round(100 * self.frac))}pct_b{self.B}", "layers": self.nl,
+                "hidden": self.H, "experts": self.E, "top_k": self.k, "channels": self.I, "keep": self.keep,
+                "batch": self.B, "routing": "k distinct uniform ids per token and layer",
+                "l2": "inputs larger than L2 (58 GB of channel-major weights)"}
 
 
 def make_workload(name, torch, M, S, device, rank, args):
@@ -336,13 +499,15 @@ def make_workload(name, torch, M, S, device, rank, args):
         return ChannelStack(torch, M, S, device, rank, args.keep_frac, steps=args.steps)
     if name == "batch_sweep":
         return BatchSweep(torch, M, S, device, rank, args.batch or 256, steps=args.steps, experts=args.experts)
+    if name == "channel_batch":
+        return ChannelBatch(torch, M, S, device, rank, args.batch or 4, args.keep_frac, steps=args.steps)
     raise SystemExit(f"unknown workload {name}")
 
 
 # ---------------------------------------------------------------- CPU oracle timing
 
 
-def oracle_rate(layers, w, xs, budget_s=12.0, max_layers=None, start_token=0):
+def oracle_rate(layers, w, xs, budget_s=12.0, max_layers=None, start_token=0, wtype="bf16"):
     """Time the fp64 oracle (as it stands) layer by layer on whole tokens.
 
     Token t goes through layers 0..L-1 (RMS pre-norm, MoE, residual: the same
@@ -363,7 +528,13 @@ def oracle_rate(layers, w, xs, budget_s=12.0, max_layers=None, start_token=0):
         Ld = layers[done % nl]
         R = f64(Ld["router"])
         shared = (f64(Ld["sh_gate"]), f64(Ld["sh_up"]), f64(Ld["sh_down_t"]))
-        experts = lambda e, Ld=Ld: (f64(Ld["gate"][e]), f64(Ld["up"][e]), f64(Ld["down_t"][e]))
+        if wtype == "bf16":
+            experts = lambda e, Ld=Ld: (f64(Ld["gate"][e]), f64(Ld["up"][e]), f64(Ld["down_t"][e]))
+        else:
+            experts = lambda e, Ld=Ld: (
+                O.dequant_rows_int4(Ld["gate"][e].cpu().numpy(), f64(Ld["gate_s"][e])),
+                O.dequant_rows_int4(Ld["up"][e].cpu().numpy(), f64(Ld["up_s"][e])),
+                O.dequant_down_t_int4(Ld["down_t"][e].cpu().numpy(), f64(Ld["down_s"][e])))
         x, *_ = O.stack_layer(x, R, experts, k, shared=shared, pre_norm=True)
         done += 1
         if done % nl == 0:
@@ -388,7 +559,14 @@ def blas_threads():
 
 
 def run_reference(args):
-    """The oracle arm: the fp64 CPU oracle timed on this host's cores."""
+    """The oracle arm: the fp64 CPU oracle timed on this host's cores.
+
+    One step of this arm is one token through one layer of the stack (a
+    bounded sample: 1/40 of a token), so that K steps take seconds rather
+    than the tens of minutes 40-layer tokens would; ms_per_step is the time
+    of one such step and steps x ms_per_step is the time actually spent.
+    The value is scaled to the metric's unit: tok/s = 1 / (layers x step time).
+    """
     ws_n, rank, local = dist_env()
     if rank != 0:
         return 0
@@ -397,6 +575,7 @@ def run_reference(args):
                           f"({WORKLOAD}, batch 1) only"}), flush=True)
         return 0
     import torch
+    from oracle import moe_oracle as O
     from mixture_experts_decode_moe_b200 import synth as S
     w = S.WORKLOADS[WORKLOAD]
     H, E, I, k, I_sh, nl = w["H"], w["E"], w["I"], w["k"], w["I_shared"], w["layers"]
@@ -406,25 +585,40 @@ def run_reference(args):
     layers = [S.swiglu_layer_bf16(H, E, I, I_sh, seed=S.weight_seed(w["cfg"], l), device=dev,
                                   router_scale=w["router_scale"]) for l in range(nl)]
     xs = S.tokens(w["tokens"], H, seed=S.act_seed(w["cfg"]), device=dev)
-    per_step = max(0.2, 90.0 / max(1, args.steps + args.warmup))
-    secs, n_layers = [], 0
+
+    def f64(t):
+        return t.detach().cpu().float().double().numpy()
+
+    x = f64(xs[0])
+    tok = 0
+    secs = []
     for i in range(args.warmup + args.steps):
-        tps, done, dt = oracle_rate(layers, w, xs, budget_s=per_step, start_token=i)
+        l = i % nl
+        if i and l == 0:
+            tok += 1
+            x = f64(xs[tok % xs.shape[0]])
+        Ld = layers[l]
+        t0 = time.perf_counter()
+        R = f64(Ld["router"])
+        shared = (f64(Ld["sh_gate"]), f64(Ld["sh_up"]), f64(Ld["sh_down_t"]))
+        experts = lambda e, Ld=Ld: (f64(Ld["gate"][e]), f64(Ld["up"][e]), f64(Ld["down_t"][e]))
+        x, *_ = O.stack_layer(x, R, experts, k, shared=shared, pre_norm=True)
+        dt = time.perf_counter() - t0
         if i >= args.warmup:
-            secs.append(1.0 / tps)
-            n_layers += done
-    sec = sum(secs) / len(secs)
-    value = 1.0 / sec
+            secs.append(dt)
+    step_s = sum(secs) / len(secs)
+    value = 1.0 / (nl * step_s)
     cores = blas_threads()
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": 1,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sec, "higher_is_better": True,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * step_s, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "step_unit": f"one token through one layer of the {nl}-layer stack",
         "config": dict(a3b_config(WORKLOAD, w, 1), parallelism="single"),
         "cpu_baseline": {"value": value, "unit": "tok/s", "cores": cores, "kind": "oracle",
-                         "sample": f"per step >= {per_step:.2f} s of whole layers ({n_layers} layer passes "
-                                   f"timed in all), scaled to tokens through {nl} layers; routed-expert "
-                                   "slices fetched from the device"},
+                         "sample": f"{args.steps} timed layer passes (after {args.warmup} untimed), one token "
+                                   f"through the layers in order, scaled to tokens through {nl} layers; "
+                                   "router, shared and routed-expert slices fetched from the device"},
         "e2e": {"value": value, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -446,20 +640,10 @@ def nvtx_pop(torch):
         pass
 
 
-def run_ours(args):
-    import torch
-    ws_n, rank, local = dist_env()
-    torch.cuda.set_device(local)
-    device = torch.device("cuda", local)
-    init_dist(ws_n, "nccl")
-    from mixture_experts_decode_moe_b200 import build as Bld
-    Bld.build()
-    from mixture_experts_decode_moe_b200 import moedec as M
-    from mixture_experts_decode_moe_b200 import synth as S
-
-    wl = make_workload(args.workload, torch, M, S, device, rank, args)
-    stream = torch.cuda.current_stream(device)
-    torch.cuda.synchronize()
+def measure(torch, M, wl, args, stream, ws_n, device, local, nvtx_name="timed"):
+    """W untimed warm-up steps, then K steps timed with CUDA events on the
+    launching stream (barrier + synchronize on both sides), clocks sampled
+    during the timed region. Returns the timing record of the workload."""
     wl.record = 10 ** 9  # no routing record during warm-up
     for i in range(args.warmup):
         wl.step(i, stream)
@@ -467,12 +651,10 @@ def run_ours(args):
     st = M.moe_get_status(wl.ws, stream)
     if st != M.MOE_OK:
         raise SystemExit(f"device status after warm-up: {M.moe_status_string(st)}")
-
-    # ---- device-timed region: inputs resident in HBM (larger than L2)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     barrier(ws_n)
     torch.cuda.synchronize()
-    nvtx_push(torch, "timed")
+    nvtx_push(torch, nvtx_name)
     with ClockSampler(local) as clk:
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
@@ -487,12 +669,57 @@ def run_ours(args):
     nvtx_pop(torch)
     barrier(ws_n)
     wl.record = 10 ** 9
-    total_ms = max_over_ranks(t0.elapsed_time(t1), ws_n, device)
-    launch_ms = [a.elapsed_time(b) for a, b in ev]
-    clocks = clk.summary()
     if M.moe_get_status(wl.ws, stream) != M.MOE_OK:
         raise SystemExit("device status error in timed region")
-    step_bytes = [wl.nbytes(i) for i in range(args.steps)]
+    return {"total_ms": max_over_ranks(t0.elapsed_time(t1), ws_n, device),
+            "launch_ms": [a.elapsed_time(b) for a, b in ev],
+            "step_bytes": [wl.nbytes(i) for i in range(args.steps)],
+            "clocks": clk.summary()}
+
+
+def roofline(wl, t):
+    """Roofline record of a workload: algorithmic bytes of each step / that
+    step's device time, averaged; peak = measured HBM copy bandwidth."""
+    hbm, hbm_kind = peaks()
+    achieved = statistics.mean(b / (ms * 1e-3) / 1e9 for b, ms in zip(t["step_bytes"], t["launch_ms"]))
+    rec = recorded_profile(wl)
+    r = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+         "traffic": rec.get("dram_bytes_per_launch"), "peak_kind": hbm_kind,
+         "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS, "kernel": wl.kernel,
+         "algorithmic_bytes_per_launch": statistics.mean(t["step_bytes"])}
+    if getattr(wl, "launches_per_step", 1) > 1:
+        r["timed_unit"] = f"whole step ({wl.launches_per_step} launches)"
+    if "tensor_pipe_active_pct" in rec:
+        r["tensor_pipe_active_pct"] = rec["tensor_pipe_active_pct"]
+    return r
+
+
+# Every other configuration of the workload list, timed after the headline in
+# the default run (each built, timed and freed in turn).
+EXTRA_WORKLOADS = ([("a3b_int4", {"batch": 1}), ("a3b_int4", {"batch": 8}),
+                    ("channel_topk", {"keep_frac": 0.13}), ("channel_topk", {"keep_frac": 0.18})] +
+                   [("batch_sweep", {"batch": b}) for b in (1, 4, 16, 64, 256)] +
+                   [("channel_batch", {"batch": 4, "keep_frac": 0.13}), ("channel_batch", {"batch": 8, "keep_frac": 0.18})])
+
+
+def run_ours(args):
+    import torch
+    ws_n, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    init_dist(ws_n, "nccl")
+    from mixture_experts_decode_moe_b200 import build as Bld
+    Bld.build()
+    from mixture_experts_decode_moe_b200 import moedec as M
+    from mixture_experts_decode_moe_b200 import synth as S
+
+    wl = make_workload(args.workload, torch, M, S, device, rank, args)
+    stream = torch.cuda.current_stream(device)
+    torch.cuda.synchronize()
+
+    # ---- device-timed region: inputs resident in HBM (larger than L2)
+    t = measure(torch, M, wl, args, stream, ws_n, device, local)
+    total_ms = t["total_ms"]
 
     # ---- end to end through the C ABI with host buffers (pinned), copies timed
     h2d, d2h = wl.host_buffers()
@@ -510,20 +737,6 @@ def run_ours(args):
     barrier(ws_n)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), ws_n, device)
 
-    hbm, hbm_kind = peaks()
-    # achieved = algorithmic bytes of each launch / its device time, averaged
-    achieved = statistics.mean(b / (ms * 1e-3) / 1e9 for b, ms in zip(step_bytes, launch_ms))
-    traffic = None
-    tfile = os.path.join(ROOT, "profiles", f"traffic_{wl.config()['workload']}.json")
-    if os.path.exists(tfile):
-        try:
-            with open(tfile) as f:
-                tj = json.load(f)
-            if tj.get("kernel_source_hash") == source_hash():
-                traffic = tj.get("dram_bytes_per_launch")
-        except Exception:
-            traffic = None
-
     tokens_total = args.steps * wl.tokens_per_step * ws_n
     value = tokens_total / (total_ms * 1e-3)
     cfg = wl.config()
@@ -531,23 +744,44 @@ def run_ours(args):
     line = {
         "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": ws_n, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": cfg,
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved / hbm, "traffic": traffic, "peak_kind": hbm_kind,
-                     "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS, "kernel": wl.kernel,
-                     "algorithmic_bytes_per_launch": statistics.mean(step_bytes)},
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if wl.dtype == "bf16" else wl.dtype,
+        "data": "synthetic", "config": cfg,
+        "roofline": roofline(wl, t),
         "e2e": {"value": tokens_total / (e2e_ms * 1e-3), "unit": "tok/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": args.steps * wl.launches_per_step,
-        "clocks": clocks,
+        "clocks": t["clocks"],
     }
-    if args.workload == "a3b_bf16" and rank == 0 and ws_n == 1 and not args.no_cpu_baseline:
-        tps, done, dt = oracle_rate(wl.layers, wl.w, wl.xs, budget_s=args.cpu_budget)
-        line["cpu_baseline"] = {"value": tps, "unit": "tok/s", "cores": blas_threads(), "kind": "oracle",
-                                "sample": f"{done} layer passes of the stack in {dt:.1f} s, scaled to tokens "
-                                          f"through {wl.nl} layers (fp64; routed-expert slices copied from the "
-                                          "device; RMS pre-norm as on the device)"}
+    if rank == 0 and ws_n == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = wl.oracle_sample(args.cpu_budget)
+
+    # ---- the other configurations (one GPU): same timing, each freed in turn
+    if ws_n == 1 and args.workload == WORKLOAD and not args.no_workloads:
+        del wl
+        import gc
+        gc.collect()
+        torch.cuda.empty_cache()
+        entries = []
+        for name, over in EXTRA_WORKLOADS:
+            a = argparse.Namespace(**vars(args))
+            for key, v in over.items():
+                setattr(a, key, v)
+            w2 = make_workload(name, torch, M, S, device, rank, a)
+            t2 = measure(torch, M, w2, a, stream, ws_n, device, local, nvtx_name="timed_" + name)
+            c2 = w2.config()
+            e = {"workload": c2["workload"], "value": a.steps * w2.tokens_per_step / (t2["total_ms"] * 1e-3),
+                 "unit": "tok/s", "ms_per_step": t2["total_ms"] / a.steps, "steps": a.steps, "warmup": a.warmup,
+                 "tokens_per_step": w2.tokens_per_step, "dtype": w2.dtype, "roofline": roofline(w2, t2),
+                 "gpu_launches": a.steps * w2.launches_per_step, "clocks": t2["clocks"], "config": c2}
+            if hasattr(w2, "touched_record"):
+                e["touched"] = w2.touched_record()
+            if not args.no_cpu_baseline:
+                e["cpu_baseline"] = w2.oracle_sample(args.extra_cpu_budget)
+            entries.append(e)
+            del w2
+            gc.collect()
+            torch.cuda.empty_cache()
+        line["workloads"] = entries
     if rank == 0:
         print(json.dumps(line), flush=True)
     if ws_n > 1:
@@ -559,16 +793,30 @@ def run_ours(args):
 # the sources decode_kernel is compiled from: a recorded DRAM traffic figure
 # stays valid while these are unchanged
 DECODE_KERNEL_SOURCES = ("common.cuh", "decode.cuh", "decode_kernel.cuh")
+LINEAR_KERNEL_SOURCES = ("common.cuh", "small_kernels.cuh", "linear.cuh")
 
 
-def source_hash():
+def source_hash(sources=DECODE_KERNEL_SOURCES):
     import hashlib
     h = hashlib.sha256()
     cs = os.path.join(ROOT, "mixture_experts_decode_moe_b200", "csrc")
-    for f in DECODE_KERNEL_SOURCES:
+    for f in sources:
         with open(os.path.join(cs, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
+
+
+def recorded_profile(wl):
+    """The ncu figures recorded for this workload's kernel (DRAM bytes per
+    launch, tensor-pipe activity), valid only while the kernel's sources hash
+    to the value recorded with them; {} otherwise."""
+    tfile = os.path.join(ROOT, "profiles", f"traffic_{wl.config()['workload']}.json")
+    try:
+        with open(tfile) as f:
+            tj = json.load(f)
+    except Exception:
+        return {}
+    return tj if tj.get("kernel_source_hash") == source_hash(wl.sources) else {}
 
 
 def main():
@@ -579,7 +827,12 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default=WORKLOAD, choices=["a3b_bf16", "a3b_int4", "channel_topk", "batch_sweep"])
+    ap.add_argument("--extra-cpu-budget", type=float, default=4.0,
+                    help="seconds of oracle time per extra configuration's cpu_baseline")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="time the headline configuration only (no workloads array)")
+    ap.add_argument("--workload", default=WORKLOAD, choices=["a3b_bf16", "a3b_int4", "channel_topk", "batch_sweep",
+                                                            "channel_batch"])
     ap.add_argument("--batch", type=int, default=0, help="batch (a3b_int4: 1 or 8; batch_sweep: 1..256)")
     ap.add_argument("--layers", type=int, default=0,
                     help="fewer stack layers (profiling captures only; the metric is quoted on the full stack)")

@@ -66,7 +66,7 @@
 extern "C" {
 #endif
 
-#define MOEDEC_ABI_VERSION 1
+#define MOEDEC_ABI_VERSION 2
 
 typedef struct CUstream_st* moe_stream_t; /* a cudaStream_t */
 
@@ -124,6 +124,24 @@ moe_status moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t stream);
  * `stream`. Returns MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_INVALID (bad ids). */
 moe_status moe_get_status(const void* ws, moe_stream_t stream);
 
+/* Time budget of every device-side wait of later calls on this workspace, in
+ * SM clock cycles (a wait that runs out ends the call with MOE_ERR_TIMEOUT in
+ * the status word; the kernels then drain their copies in flight and return).
+ * 0 restores the default of 2e9 cycles (about 1 s). moe_workspace_init()
+ * also restores it. Asynchronous on stream; returns MOE_ERR_INVALID for a
+ * NULL or misaligned workspace. */
+moe_status moe_workspace_set_wait_budget(void* ws, unsigned long long cycles, moe_stream_t stream);
+
+/* Fault injection for tests of the timeout path. With
+ * MOE_INJECT_BARRIER_EXTRA_ARRIVAL set, every grid-wide barrier of later
+ * calls on this workspace waits for one arrival more than the grid makes, so
+ * the wait runs out after the workspace's budget and the call reports
+ * MOE_ERR_TIMEOUT (no GPU fault is involved). 0 clears it, and so does
+ * moe_workspace_init(). Asynchronous on stream; unknown bits are rejected
+ * with MOE_ERR_INVALID. */
+#define MOE_INJECT_BARRIER_EXTRA_ARRIVAL 1u
+moe_status moe_workspace_set_inject(void* ws, uint32_t flags, moe_stream_t stream);
+
 /* Router only: for each token b, logits = router @ x[b] (fp32 accumulate),
  * ids[b, :] = the k experts with the largest logits in descending order,
  * ties to the lowest index; w[b, i] = softmax over all E logits restricted to
@@ -174,32 +192,55 @@ moe_status moe_stack_forward(const moe_layer_desc* layers, int32_t L, const void
                              int32_t* ids_hist_opt, float* w_hist_opt,
                              void* ws, size_t ws_bytes, moe_stream_t stream);
 
-/* Channel-sparse routed experts (CHANNEL_MAJOR bf16 SWIGLU, batch 1 per
- * call row): for token b the candidates are the k*I channels (e, c) of its
- * routed experts e = ids[b, :], indexed e*I + c. Keep the `keep` largest
- * scores[b, e, c] (ties to the lowest index); dropped channels are not read
- * and contribute 0:  y[b] = sum_{kept (e,c)} w_e a_{e,c} d_{e,c}.
+/* Channel-sparse routed experts (CHANNEL_MAJOR bf16 SWIGLU): for token b the
+ * candidates are the k*I channels (e, c) of its routed experts e = ids[b, :],
+ * indexed e*I + c. Keep the `keep` largest scores[b, e, c] (ties to the lowest
+ * index); dropped channels are not read and contribute 0:
+ *   y[b] = sum_{kept (e,c)} w[b, e] a_{b,e,c} d_{e,c}
+ * (review of arXiv:2610.37386, keep-rule table and "2단계"). A batch (B >= 2)
+ * reads the UNION of its tokens' kept channels once, in one launch, and
+ * applies each union channel to every token that kept it (same review,
+ * Table 7 rows B = 4 and 8, "속도").
  *   scores [B, E, I] fp32 (only the routed rows are read);
- *   kept_opt [B, keep] int32 = kept indices in ascending order, or NULL;
+ *   kept_opt [B, keep] int32 = each token's kept indices, ascending, or NULL;
  *   sectors [B] uint64 = distinct 32-byte sectors of routed-expert weights
- *   the kernel read for that token. 0 <= keep <= k*I, 1 <= B <= 8. */
+ *     covered by that token's kept channels;
+ *   union_count_opt [1] int32 = channels in the union (what the batch read);
+ *   union_sectors_opt [1] uint64 = distinct 32-byte sectors the batch read.
+ * ids distinct per token and < E (else MOE_ERR_INVALID in the status word and
+ * y undefined). 0 <= keep <= k*I <= 8192, 1 <= B <= 8, H <= 2048; for B >= 2
+ * also min(E, B*k) * I <= 65536 (else MOE_ERR_UNSUPPORTED). */
 moe_status moe_channel_topk_forward(const moe_layer_desc* desc, const void* x, int32_t B,
                                     const int32_t* ids, const float* w, const float* scores,
                                     int32_t keep, float* y, int32_t* kept_opt,
-                                    unsigned long long* sectors,
+                                    unsigned long long* sectors, int32_t* union_count_opt,
+                                    unsigned long long* union_sectors_opt,
                                     void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* One layer's channel-screen sketch (the buffers moe_reader_build writes). */
+typedef struct {
+  const uint32_t* codes;   /* [E*I][2][H/16] 2-bit codes */
+  const uint16_t* scales;  /* [E*I][2][H/128] fp16 bit patterns */
+  const float* dnorm;      /* [E*I] down-column norms */
+} moe_sketch_desc;
 
 /* Channel-sparse decode stack (one token): per layer l, u_l = x_l (or its RMS
  * normalisation with MOE_STACK_PRE_RMSNORM), the router picks k experts of u_l
  * as in moe_route_topk, then only the `keep` best channels of those experts by
- * scores[l, e, c] are read and applied as in moe_channel_topk_forward;
+ * their scores are read and applied as in moe_channel_topk_forward;
  * x_{l+1} = bf16_rne(x_l + y_l). layers[L]: CHANNEL_MAJOR bf16 SWIGLU with a
- * router, same shape. x [1, H] bf16; scores [L, E, I] fp32; x_out [1, H];
- * optional x_hist [L+1, H], y_hist [L, H], ids_hist / w_hist [L, k],
- * kept_hist [L, keep] (ascending); sectors [L] = 32-byte sectors of routed
- * weights read per layer. 1 <= L <= 64, 0 <= keep <= k*I. */
+ * router, same shape. The scores come from exactly one of:
+ *   scores [L, E, I] fp32, given; or
+ *   sketches [L] + signs [H]: computed in the kernel for each layer by the
+ *   weight-only screen of moe_reader_screen on u_l (eq. 1 with the layer's
+ *   routing weights); needs H % 128 == 0 (else MOE_ERR_UNSUPPORTED).
+ * x [1, H] bf16; x_out [1, H]; optional x_hist [L+1, H], y_hist [L, H],
+ * ids_hist / w_hist [L, k], kept_hist [L, keep] (ascending); sectors [L] =
+ * 32-byte sectors of routed weights read per layer. 1 <= L <= 64,
+ * 0 <= keep <= k*I. */
 moe_status moe_channel_stack_forward(const moe_layer_desc* layers, int32_t L, const void* x, uint32_t flags,
-                                     const float* scores, int32_t keep, void* x_out, void* x_hist_opt,
+                                     const float* scores, const moe_sketch_desc* sketches, const int8_t* signs,
+                                     int32_t keep, void* x_out, void* x_hist_opt,
                                      float* y_hist_opt, int32_t* ids_hist_opt, float* w_hist_opt,
                                      int32_t* kept_hist_opt, unsigned long long* sectors,
                                      void* ws, size_t ws_bytes, moe_stream_t stream);
@@ -231,9 +272,12 @@ moe_status moe_touched_experts(const int32_t* ids, int32_t B, int32_t k, int32_t
  *  - The scratch needed is moe_workspace_bytes(desc, B); a shape that needs
  *    more than MOE_STATIC_SCRATCH_BYTES is rejected with MOE_ERR_UNSUPPORTED
  *    before anything is launched.
- *  - The first call on a device looks up the array's device address (once per
- *    device, with that device current). Make that first call outside any
- *    stream capture.
+ *  - Every call looks up the array's device address in the context current on
+ *    the calling thread (a host-side lookup). The first call in a context,
+ *    the first after a device reset included, may load the library's device
+ *    code there: make that call outside any stream capture.
+ *  - Every argument is checked before the array is touched: a call that
+ *    returns an error launches nothing and leaves the array as it was.
  *  - All calls on a device share the one array and it keeps the previous
  *    call's contents; each call first clears the part that must start at zero
  *    (the status word and barrier counter). Calls whose executions overlap on
@@ -288,6 +332,59 @@ moe_status moe_reader_screen(const moe_layer_desc* desc, const void* x, int32_t 
                              const float* w, const int8_t* signs, const uint32_t* codes,
                              const uint16_t* scales, const float* dnorm, float* scores, float* est_opt,
                              moe_stream_t stream);
+
+/* Partial screen ([Reader] "가중치만으로 만든 reader", step 1, partial scan):
+ * in each block of 128 rotated coordinates only the codes of the m coordinates
+ * with the largest |R x_b| (ties to the lower coordinate; the page uses m =
+ * 80) are read; otherwise as moe_reader_screen. It reads the codes in the
+ * coordinate-major layout, where skipping a coordinate skips its bytes:
+ *   codes_cmaj [E][2][H][I/16] uint32: coordinate h of row r (0 gate, 1 up) of
+ *   expert e, channel c at bits 2(c%16) (nonzero) and 2(c%16)+1 (negative)
+ *   of word c/16 (moe_reader_codes_coordinate_major builds it from codes).
+ * Codes read per token and routed expert: 2 * (H/128) * m * (I/16) words.
+ * 0 <= m <= 128, I % 16 == 0, I <= 1024, (I/16) * (H/128) <= 1024, else
+ * MOE_ERR_UNSUPPORTED. est_opt [B, k, I, 2] or NULL. */
+moe_status moe_reader_codes_coordinate_major(const moe_layer_desc* desc, const uint32_t* codes,
+                                             uint32_t* codes_cmaj, moe_stream_t stream);
+moe_status moe_reader_screen_partial(const moe_layer_desc* desc, const void* x, int32_t B, const int32_t* ids,
+                                     const float* w, const int8_t* signs, const uint32_t* codes_cmaj,
+                                     const uint16_t* scales, const float* dnorm, int32_t m, float* scores,
+                                     float* est_opt, moe_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Rank-32 recovery of dropped channels ([Reader] "가중치만으로 만든 reader",
+ * step 3, eq. 2): y_hat = sum_{kept j} w_j a_j d_j + U sum_{dropped j} w_j p_j
+ * b_j, with U [H, 32] an orthonormal basis of the top-32 left singular
+ * subspace of the layer's stacked down columns D = [d_1 .. d_n] (n = E*I, all
+ * experts' channels), b_j = U^T d_j, and p_j = SiLU(g_hat_j) v_hat_j the
+ * channel screen's estimate. desc: CHANNEL_MAJOR bf16 SWIGLU, H <= 2048. */
+#define MOE_RECOVERY_RANK 32
+
+/* Device scratch (bytes) moe_recovery_build needs for this layer shape
+ * (H*H fp32 plus two H x 32 fp64 blocks); 0 for an unsupported descriptor. */
+size_t moe_recovery_scratch_bytes(const moe_layer_desc* desc);
+
+/* Load time, once per layer: U [H, 32] fp32 row-major (U[h * 32 + i]) from
+ * the Gram matrix D D^T by 12 rounds of subspace iteration (fp64 CholeskyQR2
+ * orthonormalisation); coeffs [E*I, 32] fp16 bit patterns, coeffs[j] =
+ * U^T d_j rounded to nearest. Eq. 2 depends on U only through U U^T: any
+ * orthonormal basis of the subspace gives the same output. scratch is
+ * caller-owned (moe_recovery_scratch_bytes), 16-byte aligned; U 16-byte
+ * aligned, coeffs 16-byte aligned. Asynchronous on stream. */
+moe_status moe_recovery_build(const moe_layer_desc* desc, float* U, uint16_t* coeffs, void* scratch,
+                              size_t scratch_bytes, moe_stream_t stream);
+
+/* Decode time: for each token b (1 <= B <= 256), with ids [B, k] and w
+ * [B, k] its routing, est [B, k, I, 2] the screen's {g_hat, v_hat} of its
+ * routed experts' channels (moe_reader_screen's est_opt, same slot order),
+ * kept [B, keep] the channels the sparse forward kept (indices e*I + c, as
+ * moe_channel_topk_forward writes them): y[b] += U r_b with
+ * r_b = sum over the routed candidates (e, c) not kept of
+ * w[b, slot(e)] SiLU(g_hat) v_hat coeffs[e*I + c]. y [B, H] fp32 (added to).
+ * 0 <= keep <= k*I <= 8192; est 8-byte and coeffs 16-byte aligned. */
+moe_status moe_channel_recover(const moe_layer_desc* desc, int32_t B, const int32_t* ids, const float* w,
+                               const float* est, const int32_t* kept, int32_t keep, const float* U,
+                               const uint16_t* coeffs, float* y, moe_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -5,12 +5,15 @@
 
 #include <cmath>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
 #include "small_kernels.cuh"
 #include "linear.cuh"
 #include "reader.cuh"
+#include "channel_batch.cuh"
+#include "recovery.cuh"
 
 using namespace moedec;
 
@@ -29,13 +32,26 @@ struct WsLayout {
 inline WsLayout ws_layout(int B, int H, int E) {
   WsLayout w;
   size_t off = sizeof(WsControl);
-  w.logits = off;  // 8 bytes per logit: {value, tag} on the batch-1 path
-  off = align_up(off + (size_t)B * E * sizeof(unsigned long long));
+  // 8 bytes per logit: {value, tag} on the batch-1 path; B*E words, then two
+  // buffers of E words for the next layer's predicted logits (batch-1
+  // stacks, alternating by layer)
+  w.logits = off;
+  off = align_up(off + (size_t)(B + 2) * E * sizeof(unsigned long long));
   w.yacc = off;     // three layer accumulators in rotation
   off = align_up(off + 3 * (size_t)B * H * sizeof(float));
   w.total = off;
   return w;
 }
+
+// Channel-major batches (2..8 tokens): the tokens' kept lists follow the
+// common workspace parts ([B, min(k*I, 8192)] int32).
+inline size_t chan_kept_offset(int B, const moe_layer_desc* d) { return ws_layout(B, d->H, d->E).total; }
+inline size_t chan_kept_bytes(int B, const moe_layer_desc* d) {
+  return align_up((size_t)B * std::min((size_t)d->k * d->I, (size_t)kMaxCand) * sizeof(int32_t));
+}
+// ... then the screened scores of a channel-major stack layer ([E*I] fp32).
+inline size_t chan_scr_offset(int B, const moe_layer_desc* d) { return chan_kept_offset(B, d) + chan_kept_bytes(B, d); }
+inline size_t chan_scr_bytes(const moe_layer_desc* d) { return align_up((size_t)d->E * d->I * sizeof(float)); }
 
 // LINEAR experts: control block, the plan, and the packed token rows of the
 // tensor-core units (at most B*k + 32*min(E, B*k) rows of H bf16).
@@ -131,6 +147,7 @@ bool plan_smem(DecodeParams* p, int static_bytes, bool fast) {
   // keys: router top-k keys [B*E] and channel-sparse candidates [k*I]
   size_t nkeys = (p->mode == MODE_LAYERS) ? (size_t)B * p->E : 0;
   if (cm) nkeys = std::max(nkeys, (size_t)p->k * p->I + (size_t)p->k * p->I / 32 + 1);  // padded q + q / 32
+  if (cm && p->screen) nkeys = std::max(nkeys, (size_t)(2 * H + H / 16));  // rotated u and its padded copy
   const int keys_bytes = (int)align_up(std::max<size_t>(nkeys, 1) * 4, 128);
   const int kept_bytes = cm ? (int)align_up((size_t)std::max(p->keep, 1) * 4, 128) : 0;
   const int ysum_bytes = fast ? (int)align_up((size_t)H * 4, 128) : 0;
@@ -259,6 +276,7 @@ void fill_common(DecodeParams* p, const moe_layer_desc* d, int B, void* ws) {
   uint8_t* base = static_cast<uint8_t*>(ws);
   p->ctl = reinterpret_cast<WsControl*>(base);
   p->logits = reinterpret_cast<float*>(base + w.logits);
+  p->plogits = reinterpret_cast<unsigned long long*>(base + w.logits) + (size_t)B * d->E;
   p->yacc = reinterpret_cast<float*>(base + w.yacc);
 }
 
@@ -332,9 +350,42 @@ moe_status linear_forward(const moe_layer_desc* d, const void* x, int B, const i
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// Argument checks of moe_layer_forward that do not involve the workspace.
+moe_status layer_forward_args(const moe_layer_desc* d, const void* x, int B, const float* y, const void* x_next_opt,
+                              const int32_t* ids_out_opt, const float* w_out_opt) {
+  if (!y || !aligned16(y)) return MOE_ERR_INVALID;
+  if (!valid_shape(d) || B < 1 || B > 256) return MOE_ERR_INVALID;
+  if (d->kind != MOE_EXPERT_SWIGLU || d->layout != MOE_LAYOUT_PLANAR) return MOE_ERR_UNSUPPORTED;
+  if (B > kMaxB || d->H > 2048) return MOE_ERR_UNSUPPORTED;
+  if ((ids_out_opt == nullptr) != (w_out_opt == nullptr)) return MOE_ERR_INVALID;
+  if (!x || !aligned16(x) || (x_next_opt && !aligned16(x_next_opt))) return MOE_ERR_INVALID;
+  return check_weights(d, true);
+}
+
+// Experts of layer l+1 that a batch-1 stack predicts in layer l and
+// prefetches into L2 (the tagged-word routing path: planar, k <= 8, E <= 256,
+// H = 2048). k + 2 by default; the environment variable
+// MOEDEC_PREFETCH_EXPERTS (0..32) overrides it for tuning (0 = off).
+int prefetch_experts(const moe_layer_desc* d, int B, int L) {
+  if (B != 1 || L < 2 || !fast_path(d, B) || d->layout != MOE_LAYOUT_PLANAR || d->k > kWarps || d->E > 256)
+    return 0;
+  int n = d->k + 2;
+  if (const char* env = std::getenv("MOEDEC_PREFETCH_EXPERTS")) n = std::atoi(env);
+  return std::max(0, std::min(std::min(n, kMaxPred), d->E));
+}
+
 bool same_shape(const moe_layer_desc* a, const moe_layer_desc* b) {
   return a->H == b->H && a->E == b->E && a->I == b->I && a->k == b->k && a->kind == b->kind &&
          a->wtype == b->wtype && a->layout == b->layout && a->I_shared == b->I_shared;
+}
+
+__global__ void set_i32_kernel(int32_t* dst, int32_t v) { *dst = v; }
+
+// Sets one field of a workspace's control block, stream-ordered with the
+// calls around it (what = 1: the wait budget, 2: the injection bits).
+__global__ void ctl_set_kernel(WsControl* ctl, int what, unsigned long long budget, uint32_t inject) {
+  if (what == 1) ctl->wait_budget = budget;
+  else ctl->inject = inject;
 }
 
 }  // namespace
@@ -357,6 +408,7 @@ const char* moe_status_string(moe_status s) {
 size_t moe_workspace_bytes(const moe_layer_desc* d, int32_t B) {
   if (!valid_shape(d) || B < 1 || B > 256) return 0;
   if (d->kind == MOE_EXPERT_LINEAR) return std::max(ws_layout(B, d->H, d->E).total, lin_ws_layout(B, d->H, d->E, d->k).total);
+  if (d->layout == MOE_LAYOUT_CHANNEL_MAJOR) return chan_scr_offset(B, d) + chan_scr_bytes(d);
   return ws_layout(B, d->H, d->E).total;
 }
 
@@ -372,6 +424,20 @@ moe_status moe_get_status(const void* ws, moe_stream_t stream) {
     return MOE_ERR_CUDA;
   if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return MOE_ERR_CUDA;
   return (moe_status)st;
+}
+
+moe_status moe_workspace_set_wait_budget(void* ws, unsigned long long cycles, moe_stream_t stream) {
+  if (ws == nullptr || !aligned16(ws)) return MOE_ERR_INVALID;
+  WsControl* ctl = static_cast<WsControl*>(ws);
+  ctl_set_kernel<<<1, 1, 0, (cudaStream_t)stream>>>(ctl, 1, cycles, 0u);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status moe_workspace_set_inject(void* ws, uint32_t flags, moe_stream_t stream) {
+  if (ws == nullptr || !aligned16(ws) || (flags & ~(uint32_t)MOE_INJECT_BARRIER_EXTRA_ARRIVAL)) return MOE_ERR_INVALID;
+  WsControl* ctl = static_cast<WsControl*>(ws);
+  ctl_set_kernel<<<1, 1, 0, (cudaStream_t)stream>>>(ctl, 2, 0ull, flags);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 moe_status moe_route_topk(const void* x, const void* router, int32_t B, int32_t H, int32_t E, int32_t k,
@@ -501,6 +567,7 @@ moe_status moe_stack_forward(const moe_layer_desc* layers, int32_t L, const void
   fill_common(&p, d, B, ws);
   p.L = L;
   p.mode = MODE_LAYERS;
+  p.npred = prefetch_experts(d, B, L);
   p.pre_norm = pre_norm ? 1 : 0;
   p.x_in = static_cast<const uint16_t*>(x);
   p.x_out = static_cast<uint16_t*>(x_out);
@@ -513,11 +580,13 @@ moe_status moe_stack_forward(const moe_layer_desc* layers, int32_t L, const void
 }
 
 moe_status moe_channel_stack_forward(const moe_layer_desc* layers, int32_t L, const void* x, uint32_t flags,
-                                     const float* scores, int32_t keep, void* x_out, void* x_hist_opt,
+                                     const float* scores, const moe_sketch_desc* sketches, const int8_t* signs,
+                                     int32_t keep, void* x_out, void* x_hist_opt,
                                      float* y_hist_opt, int32_t* ids_hist_opt, float* w_hist_opt,
                                      int32_t* kept_hist_opt, unsigned long long* sectors, void* ws,
                                      size_t ws_bytes, moe_stream_t stream) {
-  if (layers == nullptr || L < 1 || L > kMaxLayers || !x || !scores || !sectors || !ws) return MOE_ERR_INVALID;
+  if (layers == nullptr || L < 1 || L > kMaxLayers || !x || !sectors || !ws) return MOE_ERR_INVALID;
+  if ((scores == nullptr) == (sketches == nullptr) || (sketches != nullptr && signs == nullptr)) return MOE_ERR_INVALID;
   if (flags & ~(uint32_t)MOE_STACK_PRE_RMSNORM) return MOE_ERR_INVALID;
   const moe_layer_desc* d = &layers[0];
   if (!valid_shape(d)) return MOE_ERR_INVALID;
@@ -525,8 +594,9 @@ moe_status moe_channel_stack_forward(const moe_layer_desc* layers, int32_t L, co
     return MOE_ERR_INVALID;
   if (keep < 0 || keep > d->k * d->I) return MOE_ERR_INVALID;
   if ((long long)d->k * d->I > kMaxCand || d->H > 2048) return MOE_ERR_UNSUPPORTED;
+  if (sketches != nullptr && d->H % kRdBlock != 0) return MOE_ERR_UNSUPPORTED;
   if ((ids_hist_opt == nullptr) != (w_hist_opt == nullptr)) return MOE_ERR_INVALID;
-  if (!aligned16(x) || !aligned16(ws) || !aligned16(scores) || (x_out && !aligned16(x_out)) ||
+  if (!aligned16(x) || !aligned16(ws) || (scores && !aligned16(scores)) || (x_out && !aligned16(x_out)) ||
       (x_hist_opt && !aligned16(x_hist_opt)) || (y_hist_opt && !aligned16(y_hist_opt)))
     return MOE_ERR_INVALID;
   if (ws_bytes < moe_workspace_bytes(d, 1)) return MOE_ERR_INVALID;
@@ -551,7 +621,22 @@ moe_status moe_channel_stack_forward(const moe_layer_desc* layers, int32_t L, co
   p.sectors_out = sectors;
   for (int l = 0; l < L; ++l) {
     fill_layer(&p.layer[l], &layers[l]);
-    p.layer[l].scores = scores + (size_t)l * d->E * d->I;
+    if (scores != nullptr) {
+      p.layer[l].scores = scores + (size_t)l * d->E * d->I;
+    } else {
+      const moe_sketch_desc& sk = sketches[l];
+      if (!sk.codes || !sk.scales || !sk.dnorm || ((uintptr_t)sk.codes & 3u) || ((uintptr_t)sk.scales & 1u) ||
+          ((uintptr_t)sk.dnorm & 3u))
+        return MOE_ERR_INVALID;
+      p.layer[l].sk_codes = sk.codes;
+      p.layer[l].sk_scales = sk.scales;
+      p.layer[l].sk_dnorm = sk.dnorm;
+    }
+  }
+  if (sketches != nullptr) {
+    p.screen = 1;
+    p.signs = signs;
+    p.scr = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + chan_scr_offset(1, d));
   }
   return launch_decode(p, 1, (cudaStream_t)stream);
 }
@@ -559,16 +644,10 @@ moe_status moe_channel_stack_forward(const moe_layer_desc* layers, int32_t L, co
 moe_status moe_layer_forward(const moe_layer_desc* d, const void* x, int32_t B, float* y, void* x_next_opt,
                              int32_t* ids_out_opt, float* w_out_opt, void* ws, size_t ws_bytes,
                              moe_stream_t stream) {
-  if (!y || !aligned16(y)) return MOE_ERR_INVALID;
-  if (!valid_shape(d) || B < 1 || B > 256) return MOE_ERR_INVALID;
-  if (d->kind != MOE_EXPERT_SWIGLU || d->layout != MOE_LAYOUT_PLANAR) return MOE_ERR_UNSUPPORTED;
-  if (B > kMaxB || d->H > 2048) return MOE_ERR_UNSUPPORTED;
-  if ((ids_out_opt == nullptr) != (w_out_opt == nullptr)) return MOE_ERR_INVALID;
-  if (!x || !ws || !aligned16(x) || !aligned16(ws) || (x_next_opt && !aligned16(x_next_opt)))
-    return MOE_ERR_INVALID;
-  if (ws_bytes < moe_workspace_bytes(d, B)) return MOE_ERR_INVALID;
-  moe_status st = check_weights(d, true);
+  moe_status st = layer_forward_args(d, x, B, y, x_next_opt, ids_out_opt, w_out_opt);
   if (st != MOE_OK) return st;
+  if (!ws || !aligned16(ws)) return MOE_ERR_INVALID;
+  if (ws_bytes < moe_workspace_bytes(d, B)) return MOE_ERR_INVALID;
   DecodeParams p;
   fill_common(&p, d, B, ws);
   p.L = 1;
@@ -584,7 +663,8 @@ moe_status moe_layer_forward(const moe_layer_desc* d, const void* x, int32_t B, 
 
 moe_status moe_channel_topk_forward(const moe_layer_desc* d, const void* x, int32_t B, const int32_t* ids,
                                     const float* w, const float* scores, int32_t keep, float* y,
-                                    int32_t* kept_opt, unsigned long long* sectors, void* ws, size_t ws_bytes,
+                                    int32_t* kept_opt, unsigned long long* sectors, int32_t* union_count_opt,
+                                    unsigned long long* union_sectors_opt, void* ws, size_t ws_bytes,
                                     moe_stream_t stream) {
   if (!valid_shape(d) || !x || !ids || !w || !scores || !y || !sectors || !ws) return MOE_ERR_INVALID;
   if (B < 1 || B > kMaxB) return MOE_ERR_INVALID;
@@ -593,27 +673,171 @@ moe_status moe_channel_topk_forward(const moe_layer_desc* d, const void* x, int3
   if (keep < 0 || keep > d->k * d->I) return MOE_ERR_INVALID;
   if ((long long)d->k * d->I > kMaxCand || d->H > 2048) return MOE_ERR_UNSUPPORTED;
   if (!aligned16(x) || !aligned16(y) || !aligned16(ws) || !aligned16(d->gate)) return MOE_ERR_INVALID;
-  if (ws_bytes < moe_workspace_bytes(d, 1)) return MOE_ERR_INVALID;
-  // tokens run one after another through the same workspace
-  for (int b = 0; b < B; ++b) {
+  if (ws_bytes < moe_workspace_bytes(d, B)) return MOE_ERR_INVALID;
+  cudaStream_t s = (cudaStream_t)stream;
+  const int nk = std::min(keep, d->k * d->I);
+  if (B == 1) {
+    // one token: the persistent decode kernel's channel-major path; its
+    // union is its own kept set
     DecodeParams p;
     fill_common(&p, d, 1, ws);
     p.L = 1;
     p.mode = MODE_EXPERTS;
     p.I_sh = 0;
     p.keep = keep;
-    p.x_in = static_cast<const uint16_t*>(x) + (size_t)b * d->H;
-    p.y_out = y + (size_t)b * d->H;
-    p.ids_in = ids + (size_t)b * d->k;
-    p.w_in = w + (size_t)b * d->k;
-    p.kept_out = kept_opt ? kept_opt + (size_t)b * keep : nullptr;
-    p.sectors_out = sectors + b;
+    p.x_in = static_cast<const uint16_t*>(x);
+    p.y_out = y;
+    p.ids_in = ids;
+    p.w_in = w;
+    p.kept_out = kept_opt;
+    p.sectors_out = sectors;
     fill_layer(&p.layer[0], d);
-    p.layer[0].scores = scores + (size_t)b * d->E * d->I;
-    moe_status st = launch_decode(p, 1, (cudaStream_t)stream);
+    p.layer[0].scores = scores;
+    moe_status st = launch_decode(p, 1, s);
     if (st != MOE_OK) return st;
+    if (union_count_opt) set_i32_kernel<<<1, 1, 0, s>>>(union_count_opt, nk);
+    if (union_sectors_opt &&
+        cudaMemcpyAsync(union_sectors_opt, sectors, sizeof(unsigned long long), cudaMemcpyDeviceToDevice, s) !=
+            cudaSuccess)
+      return MOE_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
   }
-  return MOE_OK;
+  // 2..8 tokens: one cooperative launch that reads the union once
+  const int G = sm_count();
+  if (G <= 0) return MOE_ERR_CUDA;
+  const long long units = std::min<long long>(d->E, (long long)B * d->k);
+  if (units > kCbMaxUnits || units * d->I > kCbMaxUnionBits) return MOE_ERR_UNSUPPORTED;
+  if (((long long)B * nk + G - 1) / G > kCbMaxSlice) return MOE_ERR_UNSUPPORTED;
+  ChanBatchParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.B = B; p.H = d->H; p.E = d->E; p.I = d->I; p.k = d->k; p.keep = keep;
+  p.x = static_cast<const uint16_t*>(x);
+  p.ids = ids;
+  p.w = w;
+  p.scores = scores;
+  p.cm = static_cast<const uint8_t*>(d->gate);
+  p.y = y;
+  p.kept_out = kept_opt;
+  p.sectors = sectors;
+  p.union_count = union_count_opt;
+  p.union_sectors = union_sectors_opt;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  p.ctl = reinterpret_cast<WsControl*>(base);
+  p.kept_ws = reinterpret_cast<int32_t*>(base + chan_kept_offset(B, d));
+  const long long nq = (long long)d->k * d->I;
+  const long long uw = (units * d->I + 31) / 32;
+  size_t ring = (size_t)kCbStages * kCbNch * 3 * d->H * 2;
+  ring = std::max(ring, (size_t)(nq + nq / 32 + 1) * 4);
+  ring = std::max(ring, (size_t)(B + 2) * (size_t)uw * 4);
+  ring = std::max(ring, (size_t)(d->E + 31) / 32 * 4);
+  ring = align_up(ring, (size_t)128);
+  p.ring_bytes = (int)ring;
+  p.smem_bytes = (int)(ring + (size_t)B * d->H * 2);
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, channel_batch_kernel) != cudaSuccess) return MOE_ERR_CUDA;
+  if (p.smem_bytes + (int)fa.sharedSizeBytes + 1024 > max_dyn_smem()) return MOE_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(channel_batch_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem_bytes) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(G);
+  cfg.blockDim = dim3(kCbThreads);
+  cfg.dynamicSmemBytes = p.smem_bytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, channel_batch_kernel, p) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+static bool partial_shape_ok(const moe_layer_desc* d) {
+  // one thread per (code word, block) in one CTA; per-channel sums in shared memory (I <= 1024)
+  return d->H % kRdBlock == 0 && d->H <= 2048 && d->I % 16 == 0 && d->I <= 1024 &&
+         (d->I / 16) * (d->H / kRdBlock) <= 1024;
+}
+
+moe_status moe_reader_codes_coordinate_major(const moe_layer_desc* d, const uint32_t* codes, uint32_t* codes_cmaj,
+                                             moe_stream_t stream) {
+  if (!valid_shape(d) || !reader_shape_ok(d) || !codes || !codes_cmaj) return MOE_ERR_INVALID;
+  if (!partial_shape_ok(d)) return MOE_ERR_UNSUPPORTED;
+  if (((uintptr_t)codes & 3u) || ((uintptr_t)codes_cmaj & 3u)) return MOE_ERR_INVALID;
+  const int sms = sm_count();
+  if (sms <= 0) return MOE_ERR_CUDA;
+  reader_cmaj_kernel<<<sms * 8, 256, 0, (cudaStream_t)stream>>>(codes, d->E, d->I, d->H, codes_cmaj);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status moe_reader_screen_partial(const moe_layer_desc* d, const void* x, int32_t B, const int32_t* ids,
+                                     const float* w, const int8_t* signs, const uint32_t* codes_cmaj,
+                                     const uint16_t* scales, const float* dnorm, int32_t m, float* scores,
+                                     float* est_opt, moe_stream_t stream) {
+  if (!valid_shape(d) || !reader_shape_ok(d) || !x || !ids || !w || !signs || !codes_cmaj || !scales || !dnorm ||
+      !scores)
+    return MOE_ERR_INVALID;
+  if (B < 1 || B > 256 || m < 0 || m > kRdBlock) return MOE_ERR_INVALID;
+  if (!partial_shape_ok(d)) return MOE_ERR_UNSUPPORTED;
+  if (((uintptr_t)x & 1u) || ((uintptr_t)codes_cmaj & 3u) || ((uintptr_t)dnorm & 3u) || ((uintptr_t)scales & 1u) ||
+      ((uintptr_t)scores & 3u) || ((uintptr_t)est_opt & 3u))
+    return MOE_ERR_INVALID;
+  const int nt = (d->I / 16) * (d->H / kRdBlock);
+  reader_screen_partial_kernel<<<dim3((unsigned)d->k, (unsigned)B), std::max(nt, d->H / kRdBlock), 0,
+                                 (cudaStream_t)stream>>>(static_cast<const uint16_t*>(x), d->H, d->E, d->I, d->k,
+                                                         ids, w, signs, codes_cmaj, scales, dnorm, m, scores,
+                                                         est_opt);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+static bool recovery_shape_ok(const moe_layer_desc* d) {
+  return valid_shape(d) && reader_shape_ok(d) && d->H <= 2048 && (long long)d->E * d->I < 0x7fffffffLL;
+}
+
+size_t moe_recovery_scratch_bytes(const moe_layer_desc* d) {
+  if (!recovery_shape_ok(d)) return 0;
+  return align_up((size_t)d->H * d->H * sizeof(float)) + 2 * align_up((size_t)d->H * kRecRank * sizeof(double));
+}
+
+moe_status moe_recovery_build(const moe_layer_desc* d, float* U, uint16_t* coeffs, void* scratch, size_t scratch_bytes,
+                              moe_stream_t stream) {
+  if (!recovery_shape_ok(d)) return valid_shape(d) && reader_shape_ok(d) ? MOE_ERR_UNSUPPORTED : MOE_ERR_INVALID;
+  if (!d->gate || !U || !coeffs || !scratch || !aligned16(d->gate) || !aligned16(U) || !aligned16(coeffs) ||
+      !aligned16(scratch))
+    return MOE_ERR_INVALID;
+  if (scratch_bytes < moe_recovery_scratch_bytes(d)) return MOE_ERR_INVALID;
+  const int H = d->H, n = d->E * d->I;
+  const int sms = sm_count();
+  if (sms <= 0) return MOE_ERR_CUDA;
+  cudaStream_t s = (cudaStream_t)stream;
+  uint8_t* base = static_cast<uint8_t*>(scratch);
+  float* C = reinterpret_cast<float*>(base);
+  double* Q = reinterpret_cast<double*>(base + align_up((size_t)H * H * sizeof(float)));
+  double* Y = Q + align_up((size_t)H * kRecRank * sizeof(double)) / sizeof(double);
+  const uint16_t* cm = static_cast<const uint16_t*>(d->gate);
+  const int nt = H / kGramTile;
+  gram_kernel<<<nt * (nt + 1) / 2, 256, 0, s>>>(cm, H, n, C);
+  subspace_init_kernel<<<(H * kRecRank + 255) / 256, 256, 0, s>>>(H, Q);
+  for (int r = 0; r < kRecRounds; ++r) {
+    subspace_mul_kernel<<<(H + 7) / 8, 256, 0, s>>>(C, H, Q, Y);
+    subspace_qr_kernel<<<1, 256, 0, s>>>(H, Y);
+    std::swap(Q, Y);
+  }
+  subspace_store_kernel<<<(H * kRecRank + 255) / 256, 256, 0, s>>>(H, Q, U);
+  coeff_kernel<<<sms * 4, 256, 0, s>>>(cm, H, n, U, coeffs);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status moe_channel_recover(const moe_layer_desc* d, int32_t B, const int32_t* ids, const float* w,
+                               const float* est, const int32_t* kept, int32_t keep, const float* U,
+                               const uint16_t* coeffs, float* y, moe_stream_t stream) {
+  if (!valid_shape(d) || !reader_shape_ok(d) || !ids || !w || !est || !U || !coeffs || !y) return MOE_ERR_INVALID;
+  if (B < 1 || B > 256 || keep < 0 || keep > d->k * d->I || (keep > 0 && !kept)) return MOE_ERR_INVALID;
+  if ((long long)d->k * d->I > kMaxCand) return MOE_ERR_UNSUPPORTED;
+  if (((uintptr_t)est & 7u) || !aligned16(coeffs) || ((uintptr_t)U & 3u) || ((uintptr_t)y & 3u))
+    return MOE_ERR_INVALID;
+  recover_kernel<<<B, 256, 0, (cudaStream_t)stream>>>(d->H, d->E, d->I, d->k, ids, w, est, kept, keep, U, coeffs,
+                                                      y);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 }  // extern "C"
@@ -622,27 +846,19 @@ moe_status moe_channel_topk_forward(const moe_layer_desc* d, const void* x, int3
 //
 // A library-owned scratch array stands in for the caller's workspace. In host
 // code the symbol below is only a handle: its device address is looked up with
-// cudaGetSymbolAddress (per device, with that device current) and that
-// address is what the kernel receives.
+// cudaGetSymbolAddress, with the caller's device current, and that address is
+// what the kernel receives. The lookup runs on every call (it is a host-side
+// table lookup once the library's device code is loaded in the current
+// context), so the address always belongs to the context that is current now,
+// also after a device reset has replaced the context.
 namespace {
 
 static __device__ __align__(256) unsigned char g_static_scratch[MOE_STATIC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_static_mu;
-void* g_static_addr[kMaxDevices] = {};
-
 moe_status static_scratch_address(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
-  if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_static_mu);
-  if (g_static_addr[dev] == nullptr) {
-    void* addr = nullptr;
-    if (cudaGetSymbolAddress(&addr, g_static_scratch) != cudaSuccess || addr == nullptr) return MOE_ERR_CUDA;
-    g_static_addr[dev] = addr;
-  }
-  *out = g_static_addr[dev];
+  void* addr = nullptr;
+  if (cudaGetSymbolAddress(&addr, g_static_scratch) != cudaSuccess || addr == nullptr) return MOE_ERR_CUDA;
+  *out = addr;
   return MOE_OK;
 }
 
@@ -654,8 +870,12 @@ extern "C" moe_status moe_layer_forward_static(const moe_layer_desc* desc, const
   const size_t need = moe_workspace_bytes(desc, B);
   if (need == 0) return MOE_ERR_INVALID;
   if (need > MOE_STATIC_SCRATCH_BYTES) return MOE_ERR_UNSUPPORTED;  // beyond the fixed scratch size
+  // every argument check runs before the shared scratch is touched: a
+  // rejected call launches nothing and leaves the previous contents alone
+  moe_status st = layer_forward_args(desc, x, B, y, x_next_opt, ids_out_opt, w_out_opt);
+  if (st != MOE_OK) return st;
   void* scratch = nullptr;
-  moe_status st = static_scratch_address(&scratch);
+  st = static_scratch_address(&scratch);
   if (st != MOE_OK) return st;
   cudaStream_t s = (cudaStream_t)stream;
   // the previous call's status word and barrier counter must not leak into

@@ -19,16 +19,22 @@ constexpr int kWarps = kThreads / 32;
 constexpr uint32_t kStatusTimeout = MOE_ERR_TIMEOUT;
 constexpr uint32_t kStatusBadIds = MOE_ERR_INVALID;
 
-// Budget for any device-side wait, in SM clock cycles (~1 s at 2 GHz). A wait
-// that runs out records MOE_ERR_TIMEOUT and the kernel returns.
+// Default budget for any device-side wait, in SM clock cycles (~1 s at
+// 2 GHz). A wait that runs out records MOE_ERR_TIMEOUT and the kernel returns.
+// A workspace may carry its own budget (WsControl::wait_budget, 0 = this).
 constexpr long long kWaitBudgetCycles = 2000000000LL;
+
+// WsControl::inject bits (set from the host for tests of the timeout path):
+// every grid-wide barrier waits for one arrival more than the grid makes.
+constexpr uint32_t kInjectBarrierExtraArrival = MOE_INJECT_BARRIER_EXTRA_ARRIVAL;
 
 // Workspace control block (first 256 bytes of every workspace).
 struct alignas(16) WsControl {
   uint32_t status;          // 0 = ok, else a moe_status
-  uint32_t pad0;
+  uint32_t inject;          // fault-injection bits (kInject*), 0 = none
   unsigned long long bar;   // grid-barrier arrival counter (monotonic)
-  unsigned long long pad[14];
+  unsigned long long wait_budget;  // cycles per bounded wait, 0 = kWaitBudgetCycles
+  unsigned long long pad[13];
   // batch-1 decode: routed jobs handed out per layer (layer l uses
   // pool[l % 3]), in a cache line of their own
   uint32_t pool[4];
@@ -114,12 +120,18 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
   return ok != 0;
 }
 
+// The wait budget of a workspace (read once per kernel).
+__device__ __forceinline__ long long ctl_wait_budget(const WsControl* ctl) {
+  const unsigned long long b = ctl->wait_budget;
+  return b ? (long long)(b > 0x7fffffffffffffffull ? 0x7fffffffffffffffull : b) : kWaitBudgetCycles;
+}
+
 // Bounded wait on an mbarrier phase. Returns false if the budget ran out.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long long budget = kWaitBudgetCycles) {
   if (mbar_try_wait_sleep(bar, parity, 20000)) return true;
   long long t0 = clock64();
   while (!mbar_try_wait_sleep(bar, parity, 20000)) {
-    if (clock64() - t0 > kWaitBudgetCycles) return false;
+    if (clock64() - t0 > budget) return false;
   }
   return true;
 }
@@ -127,6 +139,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t pol;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ uint64_t policy_evict_normal() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(pol));
   return pol;
 }
 __device__ __forceinline__ uint64_t policy_evict_last() {
@@ -144,6 +161,13 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
           smem_u32(dst)),
       "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
       : "memory");
+}
+
+// Prefetch [src, src + bytes) from global memory into L2 (no shared memory
+// involved, no completion to wait for). src 16-byte aligned, bytes a
+// multiple of 16.
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
 __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
@@ -165,36 +189,6 @@ __device__ __forceinline__ unsigned long long ld_acquire_gpu(const unsigned long
 
 __device__ __forceinline__ void set_status(WsControl* ctl, uint32_t code) {
   atomicCAS(&ctl->status, 0u, code);
-}
-
-// Grid-wide barrier for a cooperative launch (all CTAs co-resident). The
-// counter is monotonic across launches; every launch adds a multiple of
-// gridDim.x, so the target of this barrier is the next multiple above the
-// ticket. Returns false (and records MOE_ERR_TIMEOUT) if the wait ran out.
-__device__ __forceinline__ bool grid_barrier(WsControl* ctl) {
-  __shared__ int ok_s;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    const unsigned long long n = gridDim.x;
-    unsigned long long ticket = atom_add_release_gpu(&ctl->bar, 1ull);
-    unsigned long long target = (ticket / n + 1ull) * n;
-    int ok = 1;
-    if (ld_acquire_gpu(&ctl->bar) < target) {
-      long long t0 = clock64();
-      while (ld_acquire_gpu(&ctl->bar) < target) {
-        if (clock64() - t0 > kWaitBudgetCycles) {
-          ok = 0;
-          set_status(ctl, kStatusTimeout);
-          break;
-        }
-      }
-    }
-    __threadfence();
-    ok_s = ok;
-  }
-  __syncthreads();
-  return ok_s != 0;
 }
 
 }  // namespace moedec

@@ -28,6 +28,8 @@
 //    into the ring while the current layer drains.
 #pragma once
 
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 
 namespace moedec {
@@ -37,6 +39,7 @@ constexpr int kMaxB = 8;
 constexpr int kMaxK = 32;
 constexpr int kMaxE = 1024;
 constexpr int kMaxCand = 8192;  // channel-sparse candidates per token (k*I)
+constexpr int kMaxPred = 32;    // experts of the next layer prefetched into L2
 
 enum DecodeMode : int { MODE_EXPERTS = 0, MODE_LAYERS = 1 };
 
@@ -52,6 +55,11 @@ struct LayerW {
   const uint8_t* sh_up;
   const uint8_t* sh_down;
   const float* scores;    // channel-sparse scores [B, E, I] fp32
+  // channel screen sketch of the layer (channel-major stacks that compute
+  // their scores): codes [E*I][2][H/16], fp16 scales [E*I][2][H/128], dnorm [E*I]
+  const uint32_t* sk_codes;
+  const uint16_t* sk_scales;
+  const float* sk_dnorm;
 };
 
 struct DecodeParams {
@@ -66,6 +74,14 @@ struct DecodeParams {
   int rows_per_job;  // router rows per job
   int nstages;
   int stage_bytes;
+  // batch-1 stack: experts of layer l+1 predicted in layer l from
+  // R_{l+1} u_l and prefetched into L2 (0 = off), at most kMaxPred
+  int npred;
+  // channel-major stack: scores from the weight-only screen, computed in the
+  // kernel per layer into scr [E*I] (0 = scores are an input)
+  int screen;
+  const int8_t* signs;    // [H] rotation signs of the screen
+  float* scr;             // ws [E*I]
   // shared-memory carve-up (byte offsets from the dynamic smem base)
   int off_x, off_u, off_lg, off_keys, off_kept, off_ysum, off_xf, off_bar, smem_bytes;
   // io
@@ -82,6 +98,7 @@ struct DecodeParams {
   unsigned long long* sectors_out;  // channel-sparse [B] (or null)
   WsControl* ctl;
   float* logits;          // ws [B, E]
+  unsigned long long* plogits;  // ws [E]: predicted logits of the next layer, {value, tag} words
   float* yacc;            // ws [2, B, H]
   LayerW layer[kMaxLayers];
 };

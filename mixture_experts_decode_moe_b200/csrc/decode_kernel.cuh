@@ -205,9 +205,12 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
   __shared__ RouteSmem<BMAX> rs;
   __shared__ int route_ready_s, prod_layer_s[kProducers], abort_s, bad_s, okw_s;
   __shared__ uint32_t ltag_s;  // logit tag of layer 0 in this launch (fast path)
+  __shared__ long long budget_s;  // cycles per bounded wait (the workspace's budget)
+  __shared__ uint32_t inject_s;   // fault-injection bits of the workspace
   __shared__ long long jp_s[kProducers], jc_s, jcg_s[kProducers];
   __shared__ Job jdesc[8];     // fast path: the job held by each stage
   __shared__ int rcnt_s[2 * kProducers];  // fast path: router-partial counters
+  __shared__ int pred_s[kProducers][kMaxPred];  // fast path: predicted experts of the next layer
   __shared__ float dotbuf[16][NV];
   __shared__ float hbuf[kWarps][NCH * BMAX];
   __shared__ uint32_t cand_key[kWarps * kMaxK];
@@ -247,6 +250,8 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
       jp_s[q] = 0;           // jobs producer q has passed (its own ones issued)
     }
     abort_s = 0;
+    budget_s = ctl_wait_budget(ctl);
+    inject_s = ctl->inject;
     jc_s = 0;
     for (int q = 0; q < kProducers; ++q) jcg_s[q] = 0;
     for (int q = 0; q < 2 * kProducers; ++q) rcnt_s[q] = 0;
@@ -262,6 +267,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
       reinterpret_cast<uint4*>(p.x_hist)[i] = reinterpret_cast<const uint4*>(p.x_in)[i];
   }
   __syncthreads();
+  const long long budget = budget_s;
 
   // At batch 1 the routed channel count is the same every layer (k * I, or
   // the kept count), so this CTA's routed range {t0, t1, unit, channel} is
@@ -338,6 +344,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
     // next one grabbed while the current one is issued), then an end marker.
     const int pi = warp - kWarps;
     const uint64_t pol = policy_evict_first();
+    const uint64_t pol_n = policy_evict_normal();
     const int nps = (p.nstages - pi + kPipes - 1) / kPipes;
     int pm = 0;
     uint32_t pph = 0;
@@ -356,7 +363,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
       if (lq >= nps) {
         const long long t0 = clock64();
         while (!mbar_try_wait_sleep(&empty[slot], pph ^ 1u, 20000)) {
-          if (*(volatile int*)&abort_s || clock64() - t0 > kWaitBudgetCycles) return -1;
+          if (*(volatile int*)&abort_s || clock64() - t0 > budget) return -1;
         }
       }
       if (lane == 0) jdesc[slot] = jb;
@@ -366,6 +373,136 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
       ++lq;
       if (++pm == nps) { pm = 0; pph ^= 1u; }
       if (lane == 0) *(volatile long long*)&jp_s[pi] = lq;
+    };
+    // Prediction of layer ln's experts: the tagged words R_ln u_{ln-1} (E <=
+    // 256, written by every CTA's prediction jobs in layer ln - 1) are polled
+    // like the routing words, and the npred largest taken by rounds of a
+    // warp-wide argmax (ties to the lower index). Then the chunks of those
+    // experts' weights (gate, up, down, and int4 scales; 16 KB chunks) are
+    // spread over the CTAs, and this producer's lanes prefetch every other
+    // chunk of this CTA's share into L2. Returns false on a poll timeout or
+    // an abort. The prefetch only warms L2: results do not depend on it.
+    auto predict_prefetch = [&](int ln) -> bool {
+      // the words of layer ln sit in buffer ln % 2: the next writes of that
+      // buffer (layer ln + 2's prediction, made in layer ln + 1) come after
+      // the grid barrier that ends layer ln, which this CTA reaches only
+      // after this producer has issued layer ln's routed jobs
+      const unsigned long long* wb = p.plogits + (size_t)(ln & 1) * E;
+      const uint32_t want = 0x80000000u | (ltag_s + (uint32_t)ln);
+      uint32_t key[8];
+      bool done[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        done[q] = 64 * q + 2 * lane >= E;
+        key[2 * q] = 0u;
+        key[2 * q + 1] = 0u;
+      }
+      const long long t0 = clock64();
+      for (;;) {
+        unsigned long long a[4], b[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (!done[q]) ld_relaxed_gpu_v2(wb + 64 * q + 2 * lane, a[q], b[q]);
+        bool all = true;
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (!done[q]) {
+            const bool has_b = 64 * q + 2 * lane + 1 < E;
+            if ((uint32_t)(a[q] >> 32) == want && (!has_b || (uint32_t)(b[q] >> 32) == want)) {
+              done[q] = true;
+              key[2 * q] = float_key(__uint_as_float((uint32_t)a[q]));
+              key[2 * q + 1] = has_b ? float_key(__uint_as_float((uint32_t)b[q])) : 0u;
+            } else {
+              all = false;
+            }
+          }
+        if (__all_sync(0xffffffffu, all)) break;
+        if (__any_sync(0xffffffffu, *(volatile int*)&abort_s != 0 || clock64() - t0 > budget)) {
+          if (lane == 0 && !*(volatile int*)&abort_s) set_status(ctl, kStatusTimeout);
+          return false;
+        }
+        __nanosleep(32);
+      }
+      auto slot_idx = [&](int s) { return 64 * (s >> 1) + 2 * lane + (s & 1); };
+      const int np = min(p.npred, E);
+      uint32_t bk = key[0];
+      int bs = 0;
+#pragma unroll
+      for (int s = 1; s < 8; ++s)
+        if (key[s] > bk) { bk = key[s]; bs = s; }
+      for (int r = 0; r < np; ++r) {
+        const uint32_t M = __reduce_max_sync(0xffffffffu, bk);
+        const uint32_t tie = __ballot_sync(0xffffffffu, bk == M);
+        int wl = __ffs(tie) - 1;
+        if (tie & (tie - 1)) {
+          const uint32_t mi = __reduce_min_sync(0xffffffffu, bk == M ? (uint32_t)slot_idx(bs) : 0xffffffffu);
+          wl = __ffs(__ballot_sync(0xffffffffu, bk == M && (uint32_t)slot_idx(bs) == mi)) - 1;
+        }
+        if (lane == wl) {
+          pred_s[pi][r] = slot_idx(bs);
+#pragma unroll
+          for (int s = 0; s < 8; ++s)
+            if (s == bs) key[s] = 0u;
+          bk = key[0];
+          bs = 0;
+#pragma unroll
+          for (int s = 1; s < 8; ++s)
+            if (key[s] > bk) { bk = key[s]; bs = s; }
+        }
+      }
+      __syncwarp();
+      // byte ranges of one expert: gate, up, down (+ int4 gate, up, down scales)
+      constexpr int NRNG = (WT == MOE_W_BF16) ? 3 : 6;
+      constexpr uint32_t kChunk = 16384;
+      const LayerW& Ln = p.layer[ln];
+      auto range_of = [&](int e, int r, const uint8_t*& ptr, uint32_t& bytes) {
+        if constexpr (WT == MOE_W_BF16) {
+          const uint8_t* base = r == 0 ? Ln.gate : (r == 1 ? Ln.up : Ln.down);
+          bytes = (uint32_t)I * (uint32_t)rowb;
+          ptr = base + (size_t)e * bytes;
+        } else {
+          if (r < 3) {
+            const uint8_t* base = r == 0 ? Ln.gate : (r == 1 ? Ln.up : Ln.down);
+            bytes = (uint32_t)I * (uint32_t)(H >> 1);
+            ptr = base + (size_t)e * bytes;
+          } else if (r < 5) {
+            bytes = (uint32_t)I * (uint32_t)(H >> 5);
+            ptr = (r == 3 ? Ln.gate_s : Ln.up_s) + (size_t)e * bytes;
+          } else {
+            bytes = (uint32_t)(I >> 6) * (uint32_t)rowb;
+            ptr = Ln.down_s + (size_t)e * bytes;
+          }
+        }
+      };
+      int cpe = 0;  // chunks per expert
+#pragma unroll
+      for (int r = 0; r < NRNG; ++r) {
+        const uint8_t* ptr;
+        uint32_t bytes;
+        range_of(0, r, ptr, bytes);
+        cpe += (int)((bytes + kChunk - 1) / kChunk);
+      }
+      const long long Q = (long long)np * cpe;
+      const long long q0 = (long long)cta * Q / G, q1 = (long long)(cta + 1) * Q / G;
+      for (long long q = q0 + pi + kProducers * lane; q < q1; q += kProducers * 32) {
+        const int e = pred_s[pi][(int)(q / cpe)];
+        int w = (int)(q % cpe);
+#pragma unroll
+        for (int r = 0; r < NRNG; ++r) {
+          const uint8_t* ptr;
+          uint32_t bytes;
+          range_of(e, r, ptr, bytes);
+          const int nc = (int)((bytes + kChunk - 1) / kChunk);
+          if (w < nc) {
+            const uint32_t off = (uint32_t)w * kChunk;
+            prefetch_l2(ptr + off, min(kChunk, bytes - off));
+            break;
+          }
+          w -= nc;
+        }
+      }
+      __syncwarp();
+      return true;
     };
     for (int l = 0; l < p.L; ++l) {
       const LayerW& Lw = p.layer[l];
@@ -400,11 +537,31 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
         __syncwarp();
         next_stage();
       }
+      if (p.npred > 0 && l + 1 < p.L) {
+        // the next layer's router rows, applied to this layer's input by the
+        // consumers: a prediction of the next layer's experts (job u = 1).
+        // Read with normal L2 priority, so that the next layer's own router
+        // job finds them in L2.
+        const LayerW& Ln = p.layer[l + 1];
+        for (int r = rr0; r < rr1; r += p.rows_per_job, ++sidx) {
+          if (sidx % kPipes != pi) continue;
+          const Job jb{JOB_ROUTER, l, 1, r, min(p.rows_per_job, rr1 - r)};
+          const int slot = take_stage(jb);
+          if (slot < 0) goto producer_done;
+          if (lane == 0) {
+            const uint32_t bytes = (uint32_t)jb.n * rowb;
+            mbar_expect_tx(&full[slot], bytes);
+            bulk_g2s(ring + (size_t)slot * p.stage_bytes, Ln.router + (size_t)r * rowb, bytes, &full[slot], pol_n);
+          }
+          __syncwarp();
+          next_stage();
+        }
+      }
       {
         // routing of layer l (plain polls with short sleeps, then one acquire)
         const long long t0 = clock64();
         while (*(volatile int*)&route_ready_s < l) {
-          if (*(volatile int*)&abort_s || clock64() - t0 > kWaitBudgetCycles) goto producer_done;
+          if (*(volatile int*)&abort_s || clock64() - t0 > budget) goto producer_done;
           __nanosleep(20);
         }
         (void)ld_acquire_cta(&route_ready_s);
@@ -496,6 +653,12 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
         v = __shfl_sync(0xffffffffu, v, 0);
         held = (l + 1 < p.L) ? (int)v : -1;
       }
+      // every routed copy of layer l is issued: while the layer drains, and
+      // through the barrier, epilogue, router and top-k of layer l + 1 (when
+      // HBM would idle), prefetch this CTA's share of the experts layer
+      // l + 1 is predicted to route to into L2
+      if (p.npred > 0 && l + 1 < p.L)
+        if (!predict_prefetch(l + 1)) goto producer_done;
     }
     } else {
     // producer pi issues the jobs q with q % kProducers == pi; both walk the
@@ -529,7 +692,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
         // routing after it. The published value only grows.
         const long long t0 = clock64();
         while (*(volatile int*)&route_ready_s < pc.layer) {
-          if (*(volatile int*)&abort_s || clock64() - t0 > kWaitBudgetCycles) goto producer_done;
+          if (*(volatile int*)&abort_s || clock64() - t0 > budget) goto producer_done;
           __nanosleep(20);
         }
         (void)ld_acquire_cta(&route_ready_s);
@@ -547,7 +710,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
         const uint32_t par = pph ^ 1u;
         const long long t0 = clock64();
         while (!mbar_try_wait_sleep(&empty[slot], par, 20000)) {
-          if (*(volatile int*)&abort_s || clock64() - t0 > kWaitBudgetCycles) goto producer_done;
+          if (*(volatile int*)&abort_s || clock64() - t0 > budget) goto producer_done;
         }
       }
       {
@@ -680,7 +843,8 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
         xw[(seg * 32 + 4 * (tid & 7) + m) * 4 + comp] = w;
         uwp[m] = w;
       }
-      if constexpr (kFastI4) reinterpret_cast<uint4*>(us)[tid] = uw;  // u for the int4 rows' FMA dots
+      // u as plain bf16 for the int4 rows' FMA dots and for the channel screen
+      if (kFastI4 || (LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR && p.screen)) reinterpret_cast<uint4*>(us)[tid] = uw;
       cbar();
     };
     auto load_xfrag = [&]() {
@@ -700,10 +864,12 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
       return bar_base + nbar * (unsigned long long)G;
     };
     auto wait_grid = [&](unsigned long long target) -> bool {  // thread 0 only
+      // (an injected fault asks for one arrival that never comes)
+      if (inject_s & kInjectBarrierExtraArrival) target += 1;
       if (ld_acquire_gpu(&ctl->bar) >= target) return true;
       const long long t0 = clock64();
       while (ld_acquire_gpu(&ctl->bar) < target)
-        if (clock64() - t0 > kWaitBudgetCycles) return false;
+        if (clock64() - t0 > budget) return false;
       return true;
     };
     auto grid_sync = [&]() -> bool {
@@ -717,7 +883,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
       if (mbar_try_wait_sleep(bar, parity, 20000)) return true;
       const long long t0 = clock64();
       while (!mbar_try_wait_sleep(bar, parity, 20000)) {
-        if (*(volatile int*)&abort_s || clock64() - t0 > kWaitBudgetCycles) return false;
+        if (*(volatile int*)&abort_s || clock64() - t0 > budget) return false;
       }
       return true;
     };
@@ -1028,10 +1194,15 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
                 float t = 0.f;
                 for (int w = 0; w < NCH; ++w) t += dotbuf[my_group * NCH + w + kWarps * buf][r];
                 if (k <= kWarps) {
-                  // {value, tag}: readers poll the word itself, no router barrier
-                  const unsigned long long tag = (unsigned long long)(0x80000000u | (ltag_s + (uint32_t)j.layer));
-                  st_relaxed_gpu_u64(reinterpret_cast<unsigned long long*>(p.logits) + j.c0 + r,
-                                     (tag << 32) | __float_as_uint(t));
+                  // {value, tag}: readers poll the word itself, no router barrier.
+                  // A prediction job (u = 1) holds the next layer's router
+                  // rows: its words carry the next layer's tag.
+                  const bool pred = j.u != 0;
+                  const unsigned long long tag =
+                      (unsigned long long)(0x80000000u | (ltag_s + (uint32_t)(j.layer + (pred ? 1 : 0))));
+                  unsigned long long* dw = pred ? p.plogits + (size_t)((j.layer + 1) & 1) * E
+                                                : reinterpret_cast<unsigned long long*>(p.logits);
+                  st_relaxed_gpu_u64(dw + j.c0 + r, (tag << 32) | __float_as_uint(t));
                 } else {
                   p.logits[j.c0 + r] = t;  // read after the router barrier
                 }
@@ -1289,7 +1460,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
             }
           }
         if (__all_sync(0xffffffffu, all)) break;
-        if (__any_sync(0xffffffffu, clock64() - t0 > kWaitBudgetCycles)) return false;  // warp-uniform
+        if (__any_sync(0xffffffffu, clock64() - t0 > budget)) return false;  // warp-uniform
       }
       // slot s of lane l holds expert 64 (s / 2) + 2 l + s % 2: slots in
       // ascending index order, so a strict > keeps the lowest index of a tie
@@ -1379,7 +1550,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
               const long long t0 = clock64();
               do {
                 t[q] = ld_relaxed_gpu(wb + i);
-              } while ((uint32_t)(t[q] >> 32) != want && clock64() - t0 < kWaitBudgetCycles);
+              } while ((uint32_t)(t[q] >> 32) != want && clock64() - t0 < budget);
               if ((uint32_t)(t[q] >> 32) != want) okw_s = 0;
             }
             lg[i] = __uint_as_float((uint32_t)t[q]);
@@ -1573,11 +1744,99 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
     // The ascending list comes from contiguous per-thread chunks and one
     // prefix scan. Keys sit in shared memory at q + q / 32 (conflict-free for
     // both the row and the chunk walks).
+    // ---- weight-only channel screen of layer l inside the stack ([Reader]
+    // "가중치만으로 만든 reader", steps 1-2, eq. 1): every CTA rotates u (fp32
+    // butterfly per block of 128, u_x = H_128 (s * u), in the keys buffer,
+    // then a copy padded by one float per 16 coordinates), then scores its
+    // share of the k*I candidates (candidate q = unit * I + c): warp per
+    // channel, lane l holding code words l + 32t of each row, the next
+    // channel's words fetched before the current one is decoded;
+    //   s_j = w_e ||d_j|| |SiLU(g_hat) v_hat|, g_hat = sum_b scale_b codes_b . u_x,b / 128
+    // written to scr[e*I + c]. A grid barrier then makes every CTA's scores
+    // visible to the selection. Returns false when the barrier ran out.
+    auto screen_layer = [&](int l) -> bool {
+      if constexpr (LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR) {
+        const LayerW& Lw = p.layer[l];
+        float* ux = reinterpret_cast<float*>(keys);
+        float* uxp = ux + H;
+        for (int i = tid; i < H; i += kConsumers) ux[i] = bf16_to_f(us[i]) * (float)p.signs[i];
+        cbar();
+        for (int lg2 = 0; lg2 < 7; ++lg2) {
+          const int mm = 1 << lg2;
+          for (int q = tid; q < H / 2; q += kConsumers) {
+            const int i = ((q >> lg2) << (lg2 + 1)) | (q & (mm - 1));
+            const float a0 = ux[i], a1 = ux[i + mm];
+            ux[i] = a0 + a1;
+            ux[i + mm] = a0 - a1;
+          }
+          cbar();
+        }
+        for (int i = tid; i < H; i += kConsumers) uxp[i + (i >> 4)] = ux[i];
+        cbar();
+        const int words = H >> 4, nb = H >> 7;
+        const int N = k * I;
+        const int q0 = (int)((long long)cta * N / G), q1 = (int)((long long)(cta + 1) * N / G);
+        struct Fetch {
+          int j, u;
+          uint32_t wv[2][4];
+          float sv[2][4];
+        };
+        auto fetch = [&](int q, Fetch& f) {
+          f.j = -1;
+          if (q >= q1) return;
+          const int u = q / I;
+          f.u = u;
+          f.j = rs.unit_e[u] * I + (q - u * I);
+#pragma unroll
+          for (int r = 0; r < 2; ++r)
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+              const int wd = lane + 32 * t;
+              f.wv[r][t] = wd < words ? __ldg(Lw.sk_codes + ((size_t)f.j * 2 + r) * words + wd) : 0u;
+              f.sv[r][t] = wd < words ? __half2float(__ushort_as_half(__ldg(Lw.sk_scales + ((size_t)f.j * 2 + r) * nb + (wd >> 3))))
+                                      : 0.f;
+            }
+        };
+        Fetch cur, nxt;
+        fetch(q0 + warp, cur);
+        for (int q = q0 + warp; q < q1; q += kWarps) {
+          fetch(q + kWarps, nxt);
+          float gv[2];
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            float acc = 0.f;
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+              const int wd = lane + 32 * t;
+              if (wd < words) {
+                const uint32_t word = cur.wv[r][t];
+                float pt = 0.f;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                  const uint32_t sgn = (word << (30 - 2 * i)) & 0x80000000u;
+                  const float xv = __uint_as_float(__float_as_uint(uxp[17 * wd + i]) ^ sgn);
+                  pt += ((word >> (2 * i)) & 1u) ? xv : 0.f;
+                }
+                acc = fmaf(cur.sv[r][t], pt, acc);
+              }
+            }
+            gv[r] = warp_sum(acc) * (1.0f / 128.0f);
+          }
+          if (lane == 0)
+            p.scr[cur.j] = rs.unit_w[cur.u][0] * __ldg(Lw.sk_dnorm + cur.j) * fabsf(silu_f(gv[0]) * gv[1]);
+          cur = nxt;
+        }
+        return grid_sync();
+      } else {
+        return true;
+      }
+    };
+
     auto select_channels = [&](int l) {
       constexpr int KR = kMaxCand / kConsumers;  // key rows per thread
       const int N = rs.U * I;
       const int rows = (N + kConsumers - 1) / kConsumers;
-      const float* sc = p.layer[l].scores;
+      const float* sc = p.screen ? p.scr : p.layer[l].scores;
       const float invI = 1.0f / (float)I;
       auto pad = [](int q) { return q + (q >> 5); };
       // 1. keys: row-major q = i * 256 + tid, all loads in flight at once
@@ -1590,7 +1849,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
           kv[i] = 0.f;
           if (i < rows && q < N) {
             const int u = __float2int_rz(((float)q + 0.5f) * invI);
-            kv[i] = __ldg(sc + (size_t)rs.unit_e[u] * I + (q - u * I));
+            kv[i] = __ldcg(sc + (size_t)rs.unit_e[u] * I + (q - u * I));  // written in this launch when screened
           }
         }
 #pragma unroll
@@ -1706,15 +1965,20 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
     // fast path: this group's static jobs per layer (router rows in jobs of
     // rows_per_job, shared channels in jobs of NCH; static job s belongs to
     // pipe s % kPipes)
-    int own_router = 0, own_shared = 0;
+    int own_router = 0, own_shared = 0, own_pred = 0;
     const int nj_pool = ((LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR) ? (p.keep > 0 ? min(k * I, p.keep) : 0) : k * I) / NCH + 1;
     if constexpr (kFast && MODE == MODE_LAYERS) {
       const unsigned Gu = (unsigned)G, cu = (unsigned)cta;
       const int nr = (int)((cu + 1) * (unsigned)E / Gu) - (int)(cu * (unsigned)E / Gu);
       const int ns = (int)((cu + 1) * (unsigned)p.I_sh / Gu) - (int)(cu * (unsigned)p.I_sh / Gu);
       const int nrj = (nr + p.rows_per_job - 1) / p.rows_per_job, nsj = (ns + NCH - 1) / NCH;
-      for (int sx = 0; sx < nrj + nsj; ++sx)
-        if (sx % kPipes == my_group) { if (sx < nrj) ++own_router; else ++own_shared; }
+      const int npj = p.npred > 0 ? nrj : 0;  // prediction jobs (all layers but the last)
+      for (int sx = 0; sx < nrj + nsj + npj; ++sx)
+        if (sx % kPipes == my_group) {
+          if (sx < nrj) ++own_router;
+          else if (sx < nrj + nsj) ++own_shared;
+          else ++own_pred;
+        }
     }
     // this CTA's slice [ys0, ys1) of the B*H/4 float4 slots of an accumulator
     // (outputs, zeroing); B*H/4 <= 2^14, so 32-bit products suffice
@@ -1763,7 +2027,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
         if (tid == 0 && l > 0) {
           const long long t0 = clock64();
           while (min(*(volatile int*)&prod_layer_s[0], *(volatile int*)&prod_layer_s[1]) < l - 1) {
-            if (clock64() - t0 > kWaitBudgetCycles) { set_status(ctl, kStatusTimeout); break; }
+            if (clock64() - t0 > budget) { set_status(ctl, kStatusTimeout); break; }
             __nanosleep(20);
           }
           (void)ld_acquire_cta(&prod_layer_s[0]);
@@ -1817,6 +2081,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
         }
         if (!units_done && !build_units() && cta == 0 && tid == 0) set_status(ctl, kStatusBadIds);
         if constexpr (LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR) {
+          if (p.screen && !screen_layer(l)) { if (tid == 0) set_status(ctl, kStatusTimeout); return false; }
           select_channels(l);
           if (cta == 0) {
             if (p.kept_out != nullptr)
@@ -1845,6 +2110,8 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
           if (!do_route()) { failed = true; break; }
         }
         for (int i = 0; i < own_shared && !fl; ++i) fl = consume_pipe() != JOB_SHARED;
+        if (l + 1 < p.L)
+          for (int i = 0; i < own_pred && !fl; ++i) fl = consume_pipe() != JOB_ROUTER;
         for (int it = 0; !fl; ++it) {
           const int ty = consume_pipe();
           if (ty == JOB_END) break;
@@ -1984,6 +2251,9 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
       }
     }
     if (failed && tid == 0) {
+      // every failure is a wait that ran out (bad ids do not stop the
+      // kernel); the first status recorded stays
+      set_status(ctl, kStatusTimeout);
       jc_s = jc;
       st_release_cta(&abort_s, 1);
     }
@@ -1997,13 +2267,13 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
       for (int g = 0; g < kPipes; ++g) {
         const int n = (p.nstages - g + kPipes - 1) / kPipes;
         for (long long q = jcg_s[g]; q < jp_s[g]; ++q)
-          mbar_wait(&full[g + kPipes * (int)(q % n)], (uint32_t)((q / n) & 1));
+          mbar_wait(&full[g + kPipes * (int)(q % n)], (uint32_t)((q / n) & 1), budget);
       }
     } else {
       // job q was issued iff producer q % kProducers got past it
       const long long issued = max(jp_s[0], jp_s[1]);
       for (long long q = jc_s; q < issued; ++q)
-        if (q < jp_s[q % kProducers]) mbar_wait(&full[q % p.nstages], (uint32_t)((q / p.nstages) & 1));
+        if (q < jp_s[q % kProducers]) mbar_wait(&full[q % p.nstages], (uint32_t)((q / p.nstages) & 1), budget);
     }
   }
 }

@@ -335,6 +335,8 @@ __global__ void __launch_bounds__(kThreads, 1) linear_tc_kernel(const __grid_con
   __shared__ __align__(8) uint64_t full[kTcStages], empty[kTcStages], tfull[2], tempty[2], done_bar;
   __shared__ uint32_t tmem_base_s;
   __shared__ int abort_s;
+  __shared__ long long issued_s;  // loads the producer issued
+  __shared__ long long budget_s;  // cycles per bounded wait (the workspace's budget)
   const LinParams& p = tp.lp;
   const LinPlan* pl = p.plan;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -351,6 +353,8 @@ __global__ void __launch_bounds__(kThreads, 1) linear_tc_kernel(const __grid_con
     mbar_init(&done_bar, 1);
     fence_mbar_init();
     abort_s = 0;
+    issued_s = 0;
+    budget_s = ctl_wait_budget(p.ctl);
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_base_s)),
@@ -361,6 +365,7 @@ __global__ void __launch_bounds__(kThreads, 1) linear_tc_kernel(const __grid_con
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_s;
+  const long long budget = budget_s;
 
   auto unit_info = [&](int unit, int& e, int& xrow, int& npad, int& n_u, int& uoff, int& m0, int& k0) {
     const int i = unit / per_unit, rem = unit - i * per_unit;
@@ -376,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1) linear_tc_kernel(const __grid_con
   auto bounded_wait = [&](uint64_t* bar, uint32_t par) -> bool {
     const long long t0 = clock64();
     while (!mbar_try_wait_sleep(bar, par, 20000)) {
-      if (*(volatile int*)&abort_s || clock64() - t0 > kWaitBudgetCycles) {
+      if (*(volatile int*)&abort_s || clock64() - t0 > budget) {
         *(volatile int*)&abort_s = 1;
         return false;
       }
@@ -406,6 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1) linear_tc_kernel(const __grid_con
           if (++slot == kTcStages) { slot = 0; ph ^= 1u; }
         }
       }
+      issued_s = issued;
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer
@@ -435,9 +441,10 @@ __global__ void __launch_bounds__(kThreads, 1) linear_tc_kernel(const __grid_con
         ++ucount;
         if (++buf == 2) { buf = 0; tph ^= 1u; }
       }
-      // all issued MMAs done before the teardown
+      // all issued MMAs done before the teardown (waited for even after an
+      // abort: the accumulator is deallocated below)
       tc_commit(&done_bar);
-      bounded_wait(&done_bar, 0);
+      if (!mbar_wait(&done_bar, 0, budget)) *(volatile int*)&abort_s = 1;
     }
   } else if (warp >= 4) {
     // ---------------- epilogue warpgroup
@@ -469,6 +476,15 @@ __global__ void __launch_bounds__(kThreads, 1) linear_tc_kernel(const __grid_con
     }
   }
   tc_fence_before();
+  __syncthreads();
+  // after an abort, loads may still be landing in stages that no MMA read:
+  // the producer waits (bounded) for the last kTcStages it issued, the only
+  // ones whose phase can still be open, before the shared memory is released
+  if (tid == 0 && abort_s) {
+    const long long n = issued_s < kTcStages ? issued_s : kTcStages;
+    for (long long q = issued_s - n; q < issued_s; ++q)
+      (void)mbar_wait(&full[q % kTcStages], (uint32_t)((q / kTcStages) & 1), budget);
+  }
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();

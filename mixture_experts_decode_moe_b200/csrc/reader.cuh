@@ -209,4 +209,139 @@ __global__ void __launch_bounds__(kRdScreenThreads) reader_screen_kernel(
   }
 }
 
+// ---------------------------------------------------------------- partial screen
+//
+// [Reader] "가중치만으로 만든 reader", step 1, partial scan: at low budgets the
+// screen reads, in each block of 128 rotated coordinates, only the codes of
+// the m (80 on the page) coordinates with the largest |R x|. In the
+// channel-major code layout a block's 128 codes of one row are a single
+// 32-byte sector, so skipping coordinates saves nothing; in the
+// coordinate-major layout below the codes of one coordinate of all of an
+// expert's channels are contiguous, so a skipped coordinate is bytes not read.
+
+// Coordinate-major codes: [E][2][H][I/16] uint32, coordinate h of row r of
+// expert e, channel c at bits 2(c % 16) (nonzero) and 2(c % 16) + 1
+// (negative) of word c / 16 -- the same 2-bit code as the channel-major
+// sketch, transposed. One thread per output word (load time).
+__global__ void reader_cmaj_kernel(const uint32_t* __restrict__ codes, int E, int I, int H,
+                                   uint32_t* __restrict__ codes_cmaj) {
+  const int wpr = I / 16, wpc = H / 16;
+  const size_t total = (size_t)E * 2 * H * wpr;
+  for (size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total; idx += (size_t)gridDim.x * blockDim.x) {
+    const int w = (int)(idx % wpr);
+    const size_t t = idx / wpr;
+    const int h = (int)(t % H);
+    const size_t er = t / H;
+    const int r = (int)(er % 2), e = (int)(er / 2);
+    uint32_t bits = 0u;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const size_t j = (size_t)e * I + 16 * w + i;
+      const uint32_t word = __ldg(codes + (j * 2 + r) * wpc + (h >> 4));
+      bits |= ((word >> (2 * (h & 15))) & 3u) << (2 * i);
+    }
+    codes_cmaj[idx] = bits;
+  }
+}
+
+// Partial screen: CTA (slot t, token b), (I/16) x (H/128) threads: thread
+// (w = tid % (I/16), block bl = tid / (I/16)) handles code word w (channels
+// 16w .. 16w + 15) in block bl. The token is rotated in fp64 (every sum of
+// the bf16 inputs is exact there), so the m largest |u_x| of each block --
+// ties to the lower coordinate -- are exactly the oracle's choice; the kept
+// coordinates' codes are then read (one coalesced word per lane and
+// coordinate) and accumulated in fp32 against u_x, scaled per block by the
+// channel's fp16 scale, and summed over blocks:
+//   g_hat = sum_bl scale_bl * sum_{h kept in bl} code_h u_x,h / 128,
+// likewise v_hat; scores[b, e, c] = w[b, t] dnorm[e*I + c] |SiLU(g_hat) v_hat|
+// and est_opt[b, t, c] = {g_hat, v_hat}. Rows of unrouted experts and ids
+// outside [0, E) are not written.
+__global__ void __launch_bounds__(1024) reader_screen_partial_kernel(
+    const uint16_t* __restrict__ x, int H, int E, int I, int k, const int32_t* __restrict__ ids,
+    const float* __restrict__ w, const int8_t* __restrict__ signs, const uint32_t* __restrict__ codes_cmaj,
+    const uint16_t* __restrict__ scales, const float* __restrict__ dnorm, int m, float* __restrict__ scores,
+    float* __restrict__ est) {
+  __shared__ double u64[2048];
+  __shared__ float uf[2048];
+  __shared__ short kc[16][128];
+  __shared__ int nkc[16];
+  __shared__ float gsum[1024], vsum[1024];
+  const int t = blockIdx.x, b = blockIdx.y, tid = threadIdx.x, nt = blockDim.x;
+  const int e = __ldg(ids + b * k + t);
+  if (e < 0 || e >= E) return;  // uniform over the CTA
+  const int wpr = I / 16, nb = H / kRdBlock;
+  for (int i = tid; i < H; i += nt) u64[i] = (double)bf16_to_f(x[(size_t)b * H + i]) * (double)signs[i];
+  for (int i = tid; i < I; i += nt) { gsum[i] = 0.f; vsum[i] = 0.f; }
+  __syncthreads();
+  for (int lg = 0; lg < 7; ++lg) {
+    const int mm = 1 << lg;
+    for (int p = tid; p < H / 2; p += nt) {
+      const int i = ((p >> lg) << (lg + 1)) | (p & (mm - 1));
+      const double a0 = u64[i], a1 = u64[i + mm];
+      u64[i] = a0 + a1;
+      u64[i + mm] = a0 - a1;
+    }
+    __syncthreads();
+  }
+  // keep flag of each coordinate: fewer than m of its block beat it
+  for (int i = tid; i < H; i += nt) {
+    const int blk = i / kRdBlock, o = i - blk * kRdBlock;
+    const double ai = fabs(u64[i]);
+    int beat = 0;
+    for (int j = 0; j < kRdBlock; ++j) {
+      const double aj = fabs(u64[blk * kRdBlock + j]);
+      beat += (aj > ai) || (aj == ai && j < o);
+    }
+    uf[i] = (float)u64[i];
+    kc[blk][o] = (short)(beat < m ? 1 : 0);
+  }
+  __syncthreads();
+  if (tid < nb) {  // each block's kept coordinates, ascending
+    int n = 0;
+    for (int o = 0; o < kRdBlock; ++o)
+      if (kc[tid][o]) kc[tid][n++] = (short)(tid * kRdBlock + o);
+    nkc[tid] = n;
+  }
+  __syncthreads();
+  const int wd = tid % wpr, bl = tid / wpr;
+  if (bl < nb) {
+    const int n = nkc[bl];
+    for (int r = 0; r < 2; ++r) {
+      const uint32_t* cw = codes_cmaj + ((size_t)e * 2 + r) * H * wpr + wd;
+      float acc[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+      for (int q = 0; q < n; ++q) {
+        const int h = kc[bl][q];
+        const uint32_t word = __ldg(cw + (size_t)h * wpr);
+        const float xv = uf[h];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const uint32_t sgn = (word << (30 - 2 * i)) & 0x80000000u;
+          const float v = __uint_as_float(__float_as_uint(xv) ^ sgn);
+          acc[i] += ((word >> (2 * i)) & 1u) ? v : 0.f;
+        }
+      }
+      float* dst = r ? vsum : gsum;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int c = 16 * wd + i;
+        const float sc = __half2float(__ushort_as_half(__ldg(scales + (((size_t)e * I + c) * 2 + r) * nb + bl)));
+        atomicAdd(&dst[c], sc * acc[i]);
+      }
+    }
+  }
+  __syncthreads();
+  const float wt = __ldg(w + b * k + t);
+  for (int c = tid; c < I; c += nt) {
+    const float gh = gsum[c] * (1.0f / 128.0f), vh = vsum[c] * (1.0f / 128.0f);
+    scores[((size_t)b * E + e) * I + c] = wt * __ldg(dnorm + (size_t)e * I + c) * fabsf(silu_f(gh) * vh);
+    if (est != nullptr) {
+      float* o = est + (((size_t)b * k + t) * I + c) * 2;
+      o[0] = gh;
+      o[1] = vh;
+    }
+  }
+}
+
 }  // namespace moedec

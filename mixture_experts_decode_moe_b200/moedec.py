@@ -28,6 +28,8 @@ MOE_W_BF16, MOE_W_INT4_G64 = 0, 1
 MOE_EXPERT_SWIGLU, MOE_EXPERT_LINEAR = 0, 1
 MOE_LAYOUT_PLANAR, MOE_LAYOUT_CHANNEL_MAJOR = 0, 1
 MOE_STACK_PRE_RMSNORM = 1
+MOE_INJECT_BARRIER_EXTRA_ARRIVAL = 1
+MOE_RECOVERY_RANK = 32
 MOE_STATIC_SCRATCH_BYTES = 256 * 1024
 
 EXPORTS = [
@@ -35,6 +37,9 @@ EXPORTS = [
     "moe_get_status", "moe_route_topk", "moe_expert_forward", "moe_layer_forward",
     "moe_stack_forward", "moe_channel_topk_forward", "moe_touched_experts",
     "moe_layer_forward_static", "moe_channel_stack_forward", "moe_reader_build", "moe_reader_screen",
+    "moe_workspace_set_wait_budget", "moe_workspace_set_inject", "moe_recovery_scratch_bytes",
+    "moe_recovery_build", "moe_channel_recover", "moe_reader_codes_coordinate_major",
+    "moe_reader_screen_partial",
 ]
 
 
@@ -65,15 +70,29 @@ _lib.moe_expert_forward.argtypes = [ctypes.POINTER(LayerDesc), _P, _I, _P, _P, _
 _lib.moe_layer_forward.argtypes = [ctypes.POINTER(LayerDesc), _P, _I, _P, _P, _P, _P, _P, _S, _P]
 _lib.moe_stack_forward.argtypes = [ctypes.POINTER(LayerDesc), _I, _P, _I, ctypes.c_uint32, _P, _P, _P, _P, _P, _P, _S, _P]
 _lib.moe_channel_topk_forward.argtypes = [ctypes.POINTER(LayerDesc), _P, _I, _P, _P, _P, _I, _P, _P, _P,
-                                          _P, _S, _P]
+                                          _P, _P, _P, _S, _P]
 _lib.moe_touched_experts.argtypes = [_P, _I, _I, _I, _P, _P, _P, _P, _P]
-_lib.moe_channel_stack_forward.argtypes = [ctypes.POINTER(LayerDesc), _I, _P, ctypes.c_uint32, _P, _I, _P, _P, _P,
-                                           _P, _P, _P, _P, _P, _S, _P]
+class SketchDesc(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("dnorm", ctypes.c_void_p)]
+
+
+_lib.moe_channel_stack_forward.argtypes = [ctypes.POINTER(LayerDesc), _I, _P, ctypes.c_uint32, _P,
+                                           ctypes.POINTER(SketchDesc), _P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _S,
+                                           _P]
 _lib.moe_layer_forward_static.argtypes = [ctypes.POINTER(LayerDesc), _P, _I, _P, _P, _P, _P, _P, _P]
 _lib.moe_reader_build.argtypes = [ctypes.POINTER(LayerDesc), _P, _P, _P, _P, _P, _P]
 _lib.moe_reader_screen.argtypes = [ctypes.POINTER(LayerDesc), _P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P]
+_lib.moe_reader_codes_coordinate_major.argtypes = [ctypes.POINTER(LayerDesc), _P, _P, _P]
+_lib.moe_reader_screen_partial.argtypes = [ctypes.POINTER(LayerDesc), _P, _I, _P, _P, _P, _P, _P, _P, _I, _P, _P,
+                                           _P]
+_lib.moe_recovery_scratch_bytes.argtypes = [ctypes.POINTER(LayerDesc)]
+_lib.moe_recovery_build.argtypes = [ctypes.POINTER(LayerDesc), _P, _P, _P, _S, _P]
+_lib.moe_channel_recover.argtypes = [ctypes.POINTER(LayerDesc), _I, _P, _P, _P, _P, _I, _P, _P, _P, _P]
+_lib.moe_workspace_set_wait_budget.argtypes = [_P, ctypes.c_ulonglong, _P]
+_lib.moe_workspace_set_inject.argtypes = [_P, ctypes.c_uint32, _P]
 for _f in EXPORTS[3:]:
     getattr(_lib, _f).restype = ctypes.c_int
+_lib.moe_recovery_scratch_bytes.restype = _S
 
 
 class MoeError(RuntimeError):
@@ -141,6 +160,14 @@ def moe_get_status(ws: torch.Tensor, stream=None) -> int:
     return int(_lib.moe_get_status(_ptr(ws), _stream(stream)))
 
 
+def moe_workspace_set_wait_budget(ws: torch.Tensor, cycles: int, stream=None):
+    _check(_lib.moe_workspace_set_wait_budget(_ptr(ws), cycles, _stream(stream)), "moe_workspace_set_wait_budget")
+
+
+def moe_workspace_set_inject(ws: torch.Tensor, flags: int, stream=None):
+    _check(_lib.moe_workspace_set_inject(_ptr(ws), flags, _stream(stream)), "moe_workspace_set_inject")
+
+
 def moe_route_topk(x, router, k, ids, w, margin=None, ws=None, stream=None):
     B, H = x.shape
     E = router.shape[0]
@@ -167,16 +194,27 @@ def moe_stack_forward(descs, x, x_out, ws, x_hist=None, y_hist=None, ids_hist=No
                                   _stream(stream)), "moe_stack_forward")
 
 
-def moe_channel_topk_forward(desc, x, ids, w, scores, keep, y, sectors, ws, kept=None, stream=None):
+def moe_channel_topk_forward(desc, x, ids, w, scores, keep, y, sectors, ws, kept=None, union_count=None,
+                             union_sectors=None, stream=None):
     _check(_lib.moe_channel_topk_forward(ctypes.byref(desc), _ptr(x), x.shape[0], _ptr(ids), _ptr(w),
-                                         _ptr(scores), keep, _ptr(y), _ptr(kept), _ptr(sectors), _ptr(ws),
-                                         ws.numel(), _stream(stream)), "moe_channel_topk_forward")
+                                         _ptr(scores), keep, _ptr(y), _ptr(kept), _ptr(sectors),
+                                         _ptr(union_count), _ptr(union_sectors), _ptr(ws), ws.numel(),
+                                         _stream(stream)), "moe_channel_topk_forward")
+
+
+def make_sketch(codes, scales, dnorm) -> SketchDesc:
+    """One layer's channel-screen sketch (moe_reader_build's buffers)."""
+    return SketchDesc(codes.data_ptr(), scales.data_ptr(), dnorm.data_ptr())
 
 
 def moe_channel_stack_forward(descs, x, scores, keep, x_out, sectors, ws, x_hist=None, y_hist=None, ids_hist=None,
-                              w_hist=None, kept_hist=None, flags=0, stream=None):
+                              w_hist=None, kept_hist=None, flags=0, sketches=None, signs=None, stream=None):
+    """scores [L, E, I] given, or scores=None with sketches (one make_sketch()
+    per layer) and signs: the kernel screens every layer itself."""
     arr = (LayerDesc * len(descs))(*descs)
-    _check(_lib.moe_channel_stack_forward(arr, len(descs), _ptr(x), flags, _ptr(scores), keep, _ptr(x_out),
+    sk = None if sketches is None else (SketchDesc * len(sketches))(*sketches)
+    _check(_lib.moe_channel_stack_forward(arr, len(descs), _ptr(x), flags, _ptr(scores), sk, _ptr(signs), keep,
+                                          _ptr(x_out),
                                           _ptr(x_hist), _ptr(y_hist), _ptr(ids_hist), _ptr(w_hist),
                                           _ptr(kept_hist), _ptr(sectors), _ptr(ws), ws.numel(), _stream(stream)),
            "moe_channel_stack_forward")
@@ -213,3 +251,38 @@ def moe_reader_screen(desc, x, ids, w, signs, codes, scales, dnorm, scores, est=
     _check(_lib.moe_reader_screen(ctypes.byref(desc), _ptr(x), x.shape[0], _ptr(ids), _ptr(w), _ptr(signs),
                                   _ptr(codes), _ptr(scales), _ptr(dnorm), _ptr(scores), _ptr(est),
                                   _stream(stream)), "moe_reader_screen")
+
+
+def moe_recovery_build(desc, U, coeffs, stream=None):
+    """Load-time recovery map of one channel-major layer: U [H, 32] fp32 and
+    coeffs [E*I, 32] (fp16 bit patterns, any 2-byte dtype). The build's
+    scratch is allocated through torch and released when the call returns
+    (stream-ordered by torch's allocator)."""
+    n = int(_lib.moe_recovery_scratch_bytes(ctypes.byref(desc)))
+    if n == 0:
+        raise MoeError(MOE_ERR_UNSUPPORTED, "moe_recovery_scratch_bytes")
+    scratch = torch.empty(n, dtype=torch.uint8, device=U.device)
+    _check(_lib.moe_recovery_build(ctypes.byref(desc), _ptr(U), _ptr(coeffs), _ptr(scratch), n, _stream(stream)),
+           "moe_recovery_build")
+    return scratch
+
+
+def moe_channel_recover(desc, ids, w, est, kept, keep, U, coeffs, y, stream=None):
+    _check(_lib.moe_channel_recover(ctypes.byref(desc), ids.shape[0], _ptr(ids), _ptr(w), _ptr(est), _ptr(kept),
+                                    keep, _ptr(U), _ptr(coeffs), _ptr(y), _stream(stream)), "moe_channel_recover")
+
+
+def reader_cmaj_shape(desc: LayerDesc) -> tuple:
+    """Shape of the coordinate-major code buffer of one layer."""
+    return (desc.E, 2, desc.H, desc.I // 16)
+
+
+def moe_reader_codes_coordinate_major(desc, codes, codes_cmaj, stream=None):
+    _check(_lib.moe_reader_codes_coordinate_major(ctypes.byref(desc), _ptr(codes), _ptr(codes_cmaj),
+                                                  _stream(stream)), "moe_reader_codes_coordinate_major")
+
+
+def moe_reader_screen_partial(desc, x, ids, w, signs, codes_cmaj, scales, dnorm, m, scores, est=None, stream=None):
+    _check(_lib.moe_reader_screen_partial(ctypes.byref(desc), _ptr(x), x.shape[0], _ptr(ids), _ptr(w), _ptr(signs),
+                                          _ptr(codes_cmaj), _ptr(scales), _ptr(dnorm), m, _ptr(scores), _ptr(est),
+                                          _stream(stream)), "moe_reader_screen_partial")

@@ -36,7 +36,7 @@ def test_every_declared_symbol_is_exported(M):
 
 
 def test_abi_version_and_status_strings(M):
-    assert M.moe_abi_version() == 1
+    assert M.moe_abi_version() == 2
     for s in range(5):
         assert M.moe_status_string(s)
     assert M.moe_status_string(99) == "unknown status"
@@ -83,7 +83,10 @@ def test_invalid_arguments_rejected_before_launch(M):
     assert lib.moe_get_status(None, None) == 1
     cm = desc(M, E=128, I=768, layout=1)
     assert lib.moe_channel_topk_forward(ctypes.byref(cm), dummy, 1, dummy, dummy, dummy, 8 * 768 + 1,
-                                        dummy, None, dummy, dummy, 1 << 20, None) == 1
+                                        dummy, None, dummy, None, None, dummy, 1 << 20, None) == 1
+    # batches of more than 8 tokens are rejected
+    assert lib.moe_channel_topk_forward(ctypes.byref(cm), dummy, 9, dummy, dummy, dummy, 10,
+                                        dummy, None, dummy, None, None, dummy, 1 << 30, None) == 1
 
 
 def test_reader_entries_reject_bad_arguments_before_launch(M):
@@ -134,4 +137,13 @@ def test_plain_c_program_links_and_calls_the_abi(M, tmp_path):
     subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe),
                     "-L", libdir, "-l:" + os.path.basename(M.LIB_PATH), "-Wl,-rpath," + libdir], check=True)
     out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
-    assert out[0] == "1" and out[1] == str(M.MOE_ERR_INVALID)
+    assert out[0] == "2" and out[1] == str(M.MOE_ERR_INVALID)
+
+
+def test_budget_and_injection_reject_bad_arguments_before_launch(M):
+    lib = M._lib
+    P = ctypes.c_void_p
+    assert lib.moe_workspace_set_wait_budget(None, 5, None) == M.MOE_ERR_INVALID
+    assert lib.moe_workspace_set_wait_budget(P(4097), 5, None) == M.MOE_ERR_INVALID
+    assert lib.moe_workspace_set_inject(None, 1, None) == M.MOE_ERR_INVALID
+    assert lib.moe_workspace_set_inject(P(4096), 2, None) == M.MOE_ERR_INVALID  # unknown bit

@@ -148,7 +148,7 @@ def cm_desc(M, cm, H, E, I, k):
 
 def run_channel(M, desc, x, ids, wt, scores, keep, H):
     B = x.shape[0]
-    ws = M.alloc_workspace(desc, 1)
+    ws = M.alloc_workspace(desc, B)
     y = torch.empty((B, H), dtype=torch.float32, device=DEV)
     kept = torch.empty((B, max(keep, 1)), dtype=torch.int32, device=DEV)
     sec = torch.empty((B,), dtype=torch.int64, device=DEV)

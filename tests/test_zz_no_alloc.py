@@ -32,13 +32,23 @@ def M():
     return moedec
 
 
-@pytest.mark.parametrize("B", [1, 4])
-def test_static_scratch_matches_workspace_entry_point(M, B):
-    from mixture_experts_decode_moe_b200 import synth as S
+def layer(M, S, wtype):
     H, E, I, k, I_sh = 2048, 64, 256, 8, 128
-    L = S.swiglu_layer_bf16(H, E, I, I_sh, seed=4242, device=DEV, router_scale=0.1)
+    if wtype == "int4":
+        L = S.swiglu_layer_int4(H, E, I, I_sh, seed=4244, device=DEV, router_scale=0.1)
+        extra = {"wtype": M.MOE_W_INT4_G64, "gate_s": L["gate_s"], "up_s": L["up_s"], "down_s": L["down_s"]}
+    else:
+        L = S.swiglu_layer_bf16(H, E, I, I_sh, seed=4242, device=DEV, router_scale=0.1)
+        extra = {}
     desc = M.make_desc(H, E, I, k, router=L["router"], gate=L["gate"], up=L["up"], down_t=L["down_t"],
-                       sh_gate=L["sh_gate"], sh_up=L["sh_up"], sh_down_t=L["sh_down_t"])
+                       sh_gate=L["sh_gate"], sh_up=L["sh_up"], sh_down_t=L["sh_down_t"], **extra)
+    return L, desc, H, k
+
+
+@pytest.mark.parametrize("wtype,B", [("bf16", 1), ("bf16", 4), ("int4", 1), ("int4", 8)])
+def test_static_scratch_matches_workspace_entry_point(M, wtype, B):
+    from mixture_experts_decode_moe_b200 import synth as S
+    L, desc, H, k = layer(M, S, wtype)
     x = S.tokens(B, H, seed=4243, device=DEV)
 
     def outputs():
@@ -53,14 +63,43 @@ def test_static_scratch_matches_workspace_entry_point(M, B):
     for call in range(2):
         y, xn, ids, w = outputs()
         status = torch.full((1,), -1, dtype=torch.int32, device=DEV)
+        torch.cuda.synchronize()
+        free0, used0 = torch.cuda.mem_get_info()[0], torch.cuda.memory_allocated()
+        allocs0 = torch.cuda.memory_stats().get("allocation.all.allocated", 0)
         M.moe_layer_forward_static(desc, x, y, x_next=xn, ids_out=ids, w_out=w, status_out=status)
         torch.cuda.synchronize()
+        # nothing was allocated: not through torch, and not from the device
+        # (the second call runs with the library already loaded in this context)
+        assert torch.cuda.memory_allocated() == used0, call
+        assert torch.cuda.memory_stats().get("allocation.all.allocated", 0) == allocs0, call
+        if call == 1:
+            assert torch.cuda.mem_get_info()[0] == free0
         assert int(status) == M.MOE_OK, (call, int(status))
         assert torch.equal(ids, ids0), call
         assert np.allclose(f64(w), f64(w0), rtol=1e-6), call
         assert rel_err(f64(y), f64(y0)) <= REL_TOL, call
         assert rel_err(f64(xn), f64(xn0)) <= REL_TOL, call
     assert M.moe_get_status(ws) == M.MOE_OK
+
+
+def test_static_scratch_rejected_call_leaves_scratch_alone(M):
+    """A call with a bad argument returns an error before anything is
+    launched; the next valid call still matches the workspace entry point."""
+    from mixture_experts_decode_moe_b200 import synth as S
+    L, desc, H, k = layer(M, S, "bf16")
+    x = S.tokens(1, H, seed=4245, device=DEV)
+    y0 = torch.empty((1, H), dtype=torch.float32, device=DEV)
+    ws = M.alloc_workspace(desc, 1)
+    M.moe_layer_forward(desc, x, y0, ws)
+    # ids without weights: rejected on the host
+    ids = torch.empty((1, k), dtype=torch.int32, device=DEV)
+    st = M._lib.moe_layer_forward_static(ctypes.byref(desc), M._ptr(x), 1, M._ptr(y0), None, M._ptr(ids), None,
+                                         None, M._stream(None))
+    assert st == M.MOE_ERR_INVALID
+    y = torch.empty((1, H), dtype=torch.float32, device=DEV)
+    M.moe_layer_forward_static(desc, x, y)
+    torch.cuda.synchronize()
+    assert rel_err(f64(y), f64(y0)) <= REL_TOL
 
 
 def test_static_scratch_rejects_shapes_beyond_its_size(M):
