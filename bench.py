@@ -26,6 +26,8 @@ import sys
 import tempfile
 import time
 
+import numpy as np
+
 ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
@@ -234,12 +236,14 @@ class A3BStack:
 
 
 class ChannelStack:
-    """48-layer channel-major stack, batch 1, channel top-k keep over given scores."""
+    """48-layer channel-major stack, batch 1, channel top-k keep over given
+    scores, or (screen=True) over scores the kernel computes per layer from
+    the weight-only sketch of each layer (the screen inside the stack)."""
 
-    def __init__(self, torch, M, S, device, rank, frac=0.13, steps=0):
+    def __init__(self, torch, M, S, device, rank, frac=0.13, steps=0, layers=0, screen=False):
         self.torch, self.M, self.S, self.dev = torch, M, S, device
         w = S.WORKLOADS["channel_topk"]
-        H, E, I, k, nl = w["H"], w["E"], w["I"], w["k"], w["layers"]
+        H, E, I, k, nl = w["H"], w["E"], w["I"], w["k"], layers or w["layers"]
         self.H, self.E, self.I, self.k, self.nl = H, E, I, k, nl
         self.keep = S.keep_count(frac, k, I)
         self.frac = frac
@@ -257,13 +261,33 @@ class ChannelStack:
         self.sectors = torch.empty((nl,), dtype=torch.int64, device=device)
         self.tokens_per_step = 1
         self.launches_per_step = 1
-        self.kernel = "decode_kernel<layers,B1,bf16,channel-major>"
+        self.kernel = "decode_kernel<layers,B1,bf16,channel-major>" + (" + in-kernel screen" if screen else "")
         self.sources = DECODE_KERNEL_SOURCES
         self.dtype = "bf16"
+        self.screen = screen
+        self.sketches = None
+        if screen:
+            self.signs = S.reader_signs(H, seed=S.weight_seed(5, 0) + 11, device=device)
+            shp = M.reader_sketch_shapes(self.descs[0])
+            self.sk_bufs = []
+            for d in self.descs:
+                codes = torch.empty(shp["codes"], dtype=torch.int32, device=device)
+                scales = torch.empty(shp["scales"], dtype=torch.int16, device=device)
+                rho = torch.empty(shp["rho"], dtype=torch.float32, device=device)
+                dnorm = torch.empty(shp["dnorm"], dtype=torch.float32, device=device)
+                M.moe_reader_build(d, self.signs, codes, scales, rho, dnorm)
+                self.sk_bufs.append((codes, scales, dnorm))
+                del rho
+            self.sketches = [M.make_sketch(c, sc, dn) for (c, sc, dn) in self.sk_bufs]
+            torch.cuda.synchronize()
+
+    def _scores(self, i):
+        return None if self.screen else self.scores[i % self.nsc]
 
     def step(self, i, stream):
-        self.M.moe_channel_stack_forward(self.descs, self.xs[i % 256:][:1], self.scores[i % self.nsc], self.keep,
+        self.M.moe_channel_stack_forward(self.descs, self.xs[i % 256:][:1], self._scores(i), self.keep,
                                          self.x_out, self.sectors, self.ws, flags=self.M.MOE_STACK_PRE_RMSNORM,
+                                         sketches=self.sketches, signs=self.signs if self.screen else None,
                                          stream=stream)
 
     def host_buffers(self):
@@ -275,13 +299,19 @@ class ChannelStack:
 
     def e2e_step(self, i, stream):
         self.x_dev.copy_(self.x_host[i % 256:][:1], non_blocking=True)
-        self.M.moe_channel_stack_forward(self.descs, self.x_dev, self.scores[i % self.nsc], self.keep, self.x_out,
-                                         self.sectors, self.ws, flags=self.M.MOE_STACK_PRE_RMSNORM, stream=stream)
+        self.M.moe_channel_stack_forward(self.descs, self.x_dev, self._scores(i), self.keep, self.x_out,
+                                         self.sectors, self.ws, flags=self.M.MOE_STACK_PRE_RMSNORM,
+                                         sketches=self.sketches, signs=self.signs if self.screen else None,
+                                         stream=stream)
         self.out_host.copy_(self.x_out, non_blocking=True)
 
     def nbytes(self, r):
-        # router + kept channels (gate row, up row, down column) + the 8 score rows read
-        return self.nl * (2 * self.E * self.H + self.keep * 3 * self.H * 2 + self.k * self.I * 4)
+        # router + kept channels (gate row, up row, down column) + the 8 score rows read;
+        # screened: + the routed experts' codes, scales and down-column norms
+        b = 2 * self.E * self.H + self.keep * 3 * self.H * 2 + self.k * self.I * 4
+        if self.screen:
+            b += self.k * self.I * (2 * (self.H // 4 + 2 * (self.H // 128)) + 4)
+        return self.nl * b
 
     def oracle_sample(self, budget_s):
         """The fp64 oracle's channel-stack layer, token 0 through the layers in order."""
@@ -292,11 +322,27 @@ class ChannelStack:
         t0 = time.perf_counter()
         x = f64(self.xs[0])
         done = 0
+        sg = f64(self.signs) if self.screen else None
         while True:
             l = done % self.nl
             cm = self.layers[l]["cm"]
             R = f64(self.layers[l]["router"])
-            sc = f64(self.scores[0, l])
+            if self.screen:
+                # the screen from the oracle's own sketch of the routed experts' channels
+                u = O.rmsnorm_bf16(x)
+                ids, w, _, _ = O.route_topk(u, R, self.k)
+
+                def sketch(e, c, cm=cm):
+                    g, v, d = f64(cm[e, c])
+                    cg, scg, _ = O.reader_sketch_row(g, sg)
+                    cv, scv, _ = O.reader_sketch_row(v, sg)
+                    return cg, scg, cv, scv, float(np.sqrt(np.sum(d ** 2)))
+                o_sc, _ = O.reader_screen(u, ids.tolist(), w, sketch, self.I, sg)
+                sc = np.full((self.E, self.I), -np.inf)
+                for t, e in enumerate(ids.tolist()):
+                    sc[e] = o_sc[t]
+            else:
+                sc = f64(self.scores[0, l])
             x, *_ = O.channel_stack_layer(x, R, lambda e, c, cm=cm: f64(cm[e, c]), sc, self.k, self.keep, self.I)
             done += 1
             if time.perf_counter() - t0 >= budget_s:
@@ -304,10 +350,13 @@ class ChannelStack:
         dt = time.perf_counter() - t0
         return {"value": (done / self.nl) / dt, "unit": "tok/s", "cores": blas_threads(), "kind": "oracle",
                 "sample": f"{done} channel-sparse layer passes of one token in {dt:.1f} s, scaled to tokens "
-                          f"through {self.nl} layers (fp64; kept channels copied from the device)"}
+                          f"through {self.nl} layers (fp64; kept channels copied from the device"
+                          + ("; scores from the oracle's own screen)" if self.screen else ")")}
 
     def config(self):
-        return {"workload": f"channel_topk_{int(round(100 * self.frac))}pct", "layers": self.nl, "hidden": self.H,
+        return {"workload": f"channel_topk_{int(round(100 * self.frac))}pct" + ("_screened" if self.screen else ""),
+                "scores": "computed in the kernel from per-layer sketches" if self.screen else "input",
+                "layers": self.nl, "hidden": self.H,
                 "experts": self.E, "top_k": self.k, "channels": self.I, "keep": self.keep, "batch": 1,
                 "pre_norm": "rms", "l2": "inputs larger than L2 (58 GB of channel-major weights)"}
 
@@ -399,10 +448,10 @@ class ChannelBatch:
     score rows; they are compared with reading the touched experts whole
     (the full-read column of the pages' Table 7)."""
 
-    def __init__(self, torch, M, S, device, rank, B=4, frac=0.13, steps=0):
+    def __init__(self, torch, M, S, device, rank, B=4, frac=0.13, steps=0, layers=0):
         self.torch, self.M, self.S, self.dev = torch, M, S, device
         w = S.WORKLOADS["channel_topk"]
-        H, E, I, k, nl = w["H"], w["E"], w["I"], w["k"], w["layers"]
+        H, E, I, k, nl = w["H"], w["E"], w["I"], w["k"], layers or w["layers"]
         self.H, self.E, self.I, self.k, self.nl, self.B, self.frac = H, E, I, k, nl, B, frac
         self.keep = S.keep_count(frac, k, I)
         self.layers = [S.channel_major_layer(H, E, I, seed=S.weight_seed(5, l), device=device) for l in range(nl)]
@@ -496,11 +545,13 @@ def make_workload(name, torch, M, S, device, rank, args):
     if name == "a3b_int4":
         return A3BStack(torch, M, S, device, rank, "int4", args.batch or 1, steps=args.steps, layers=args.layers)
     if name == "channel_topk":
-        return ChannelStack(torch, M, S, device, rank, args.keep_frac, steps=args.steps)
+        return ChannelStack(torch, M, S, device, rank, args.keep_frac, steps=args.steps, layers=args.layers,
+                            screen=getattr(args, "screen", False))
     if name == "batch_sweep":
         return BatchSweep(torch, M, S, device, rank, args.batch or 256, steps=args.steps, experts=args.experts)
     if name == "channel_batch":
-        return ChannelBatch(torch, M, S, device, rank, args.batch or 4, args.keep_frac, steps=args.steps)
+        return ChannelBatch(torch, M, S, device, rank, args.batch or 4, args.keep_frac, steps=args.steps,
+                            layers=args.layers)
     raise SystemExit(f"unknown workload {name}")
 
 
@@ -699,7 +750,8 @@ def roofline(wl, t):
 EXTRA_WORKLOADS = ([("a3b_int4", {"batch": 1}), ("a3b_int4", {"batch": 8}),
                     ("channel_topk", {"keep_frac": 0.13}), ("channel_topk", {"keep_frac": 0.18})] +
                    [("batch_sweep", {"batch": b}) for b in (1, 4, 16, 64, 256)] +
-                   [("channel_batch", {"batch": 4, "keep_frac": 0.13}), ("channel_batch", {"batch": 8, "keep_frac": 0.18})])
+                   [("channel_batch", {"batch": 4, "keep_frac": 0.13}), ("channel_batch", {"batch": 8, "keep_frac": 0.18}),
+                    ("channel_topk", {"keep_frac": 0.13, "screen": True})])
 
 
 def run_ours(args):
@@ -839,6 +891,8 @@ def main():
     ap.add_argument("--experts", type=int, default=0,
                     help="fewer batch-sweep experts (profiling captures only; the sweep is quoted on 64)")
     ap.add_argument("--keep-frac", type=float, default=0.13, help="channel_topk budget (0.13 or 0.18)")
+    ap.add_argument("--screen", action="store_true",
+                    help="channel_topk: scores computed in the kernel from per-layer sketches")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 warm-up steps
     if args.impl == "reference":

@@ -32,9 +32,9 @@ struct WsLayout {
 inline WsLayout ws_layout(int B, int H, int E) {
   WsLayout w;
   size_t off = sizeof(WsControl);
-  // 8 bytes per logit: {value, tag} on the batch-1 path; B*E words, then two
-  // buffers of E words for the next layer's predicted logits (batch-1
-  // stacks, alternating by layer)
+  // 8 bytes per logit: {value, tag} on the batch-1 path (plain floats
+  // [B, E] at batch > 1), then two buffers of E words for the next layer's
+  // predicted logits (batch-1 stacks, alternating by layer)
   w.logits = off;
   off = align_up(off + (size_t)(B + 2) * E * sizeof(unsigned long long));
   w.yacc = off;     // three layer accumulators in rotation
@@ -150,6 +150,7 @@ bool plan_smem(DecodeParams* p, int static_bytes, bool fast) {
   if (cm && p->screen) nkeys = std::max(nkeys, (size_t)(2 * H + H / 16));  // rotated u and its padded copy
   const int keys_bytes = (int)align_up(std::max<size_t>(nkeys, 1) * 4, 128);
   const int kept_bytes = cm ? (int)align_up((size_t)std::max(p->keep, 1) * 4, 128) : 0;
+  const int hist_bytes = cm ? kSelBins * 4 : 0;  // radix-select histogram
   const int ysum_bytes = fast ? (int)align_up((size_t)H * 4, 128) : 0;
   const int xf_bytes = fast ? H * 2 : 0;  // x fragments, [segment][lane] x 16 B
   int stage;
@@ -158,7 +159,7 @@ bool plan_smem(DecodeParams* p, int static_bytes, bool fast) {
   stage = std::max(stage, p->rows_per_job * rowb);
   if (p->I_sh > 0) stage = std::max(stage, NCH * 3 * rowb);
   stage = (int)align_up(stage, 128);
-  const int fixed = x_bytes + u_bytes + lg_bytes + keys_bytes + kept_bytes + ysum_bytes + xf_bytes;
+  const int fixed = x_bytes + u_bytes + lg_bytes + keys_bytes + kept_bytes + hist_bytes + ysum_bytes + xf_bytes;
   const int nst = std::min(8, (budget - fixed - 256) / stage);
   if (nst < 2) return false;
   p->stage_bytes = stage;
@@ -169,6 +170,7 @@ bool plan_smem(DecodeParams* p, int static_bytes, bool fast) {
   p->off_lg = off; off += lg_bytes;
   p->off_keys = off; off += keys_bytes;
   p->off_kept = off; off += kept_bytes;
+  p->off_hist = off; off += hist_bytes;
   p->off_ysum = off; off += ysum_bytes;
   p->off_xf = off; off += xf_bytes;
   p->off_bar = off; off += (int)align_up((size_t)3 * nst * 8, 128);  // full, empty, dots-ready
@@ -364,12 +366,14 @@ moe_status layer_forward_args(const moe_layer_desc* d, const void* x, int B, con
 
 // Experts of layer l+1 that a batch-1 stack predicts in layer l and
 // prefetches into L2 (the tagged-word routing path: planar, k <= 8, E <= 256,
-// H = 2048). k + 2 by default; the environment variable
-// MOEDEC_PREFETCH_EXPERTS (0..32) overrides it for tuning (0 = off).
+// H = 2048). 0 (off) by default; the environment variable
+// MOEDEC_PREFETCH_EXPERTS (0..32) sets it for tuning.
 int prefetch_experts(const moe_layer_desc* d, int B, int L) {
   if (B != 1 || L < 2 || !fast_path(d, B) || d->layout != MOE_LAYOUT_PLANAR || d->k > kWarps || d->E > 256)
     return 0;
-  int n = d->k + 2;
+  // off by default: measured on the A3B stack, the prefetch flood delays the
+  // grid barrier and the next layer's serial chain by more than it saves
+  int n = 0;
   if (const char* env = std::getenv("MOEDEC_PREFETCH_EXPERTS")) n = std::atoi(env);
   return std::max(0, std::min(std::min(n, kMaxPred), d->E));
 }
@@ -727,7 +731,7 @@ moe_status moe_channel_topk_forward(const moe_layer_desc* d, const void* x, int3
   const long long nq = (long long)d->k * d->I;
   const long long uw = (units * d->I + 31) / 32;
   size_t ring = (size_t)kCbStages * kCbNch * 3 * d->H * 2;
-  ring = std::max(ring, (size_t)(nq + nq / 32 + 1) * 4);
+  ring = std::max(ring, align_up((size_t)(nq + nq / 32 + 1) * 4, 128) + (size_t)kSelBins * 4);  // keys + histogram
   ring = std::max(ring, (size_t)(B + 2) * (size_t)uw * 4);
   ring = std::max(ring, (size_t)(d->E + 31) / 32 * 4);
   ring = align_up(ring, (size_t)128);

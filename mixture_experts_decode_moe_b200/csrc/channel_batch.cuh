@@ -134,7 +134,6 @@ __global__ void __launch_bounds__(kCbThreads, 1) channel_batch_kernel(const __gr
     const int rows = (N + kCbConsumers - 1) / kCbConsumers;
     uint32_t* keys = reinterpret_cast<uint32_t*>(ring);  // padded q + q / 32
     auto pad = [](int q) { return q + (q >> 5); };
-    uint32_t kr[KR];
     {
       float kv[KR];
 #pragma unroll
@@ -149,56 +148,19 @@ __global__ void __launch_bounds__(kCbThreads, 1) channel_batch_kernel(const __gr
 #pragma unroll
       for (int i = 0; i < KR; ++i) {
         const int q = i * kCbConsumers + tid;
-        kr[i] = 0u;
-        if (i < rows && q < N) {
-          kr[i] = float_key(kv[i]);
-          keys[pad(q)] = kr[i];
-        }
+        if (i < rows && q < N) keys[pad(q)] = float_key(kv[i]);
       }
     }
     const bool all = keep >= N;
     uint32_t T = 0u;
     int r = 0;
-    int par = 0;
-    // (absent keys are 0 and every threshold tried is >= 1)
-    auto count_ge = [&](uint32_t c) -> int {
-      int n = 0;
-#pragma unroll
-      for (int i0 = 0; i0 < KR; i0 += 8)
-        if (i0 < rows) {
-#pragma unroll
-          for (int i = i0; i < i0 + 8; ++i) n += kr[i] >= c ? 1 : 0;
-        }
-      n = (int)__reduce_add_sync(0xffffffffu, (uint32_t)n);
-      if (lane == 0) scan_s[kWarps * par + warp] = n;
-      cbar();
-      int t = 0;
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) t += scan_s[kWarps * par + w];
-      par ^= 1;
-      return t;
-    };
+    cbar();
     if (keep > 0 && !all) {
-      uint32_t kmax = 0u, kmin = 0xffffffffu;
-#pragma unroll
-      for (int i = 0; i < KR; ++i)
-        if (i < rows && i * kCbConsumers + tid < N) { kmax = max(kmax, kr[i]); kmin = min(kmin, max(kr[i], 1u)); }
-      kmax = __reduce_max_sync(0xffffffffu, kmax);
-      kmin = __reduce_min_sync(0xffffffffu, kmin);
-      if (lane == 0) { red_s[warp] = kmax; red_s[kWarps + warp] = kmin; }
-      cbar();
-      kmax = 0u;
-      kmin = 0xffffffffu;
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) { kmax = max(kmax, red_s[w]); kmin = min(kmin, red_s[kWarps + w]); }
-      const uint32_t diff = kmax ^ kmin;
-      const int top = diff ? 31 - __clz(diff) : -1;
-      T = top >= 0 ? kmax & ~(0xffffffffu >> (31 - top)) : kmax;
-      for (int bit = top; bit >= 0; --bit) {
-        const uint32_t c = T | (1u << bit);
-        if (count_ge(c) >= keep) T = c;
-      }
-      r = keep - (T == 0xffffffffu ? 0 : count_ge(T + 1u));
+      // the keep-th largest key and the count above it (histogram after the keys)
+      int* hist = reinterpret_cast<int*>(ring + ((size_t)(N + N / 32 + 1) * 4 + 127) / 128 * 128);
+      int n_gt = 0;
+      T = radix_select(keys, N, keep, hist, scan_s, &n_gt);
+      r = keep - n_gt;
     }
     cbar();  // keys[] complete
     int* kws = p.kept_ws + (size_t)b * keep;

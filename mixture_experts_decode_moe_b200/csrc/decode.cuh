@@ -83,7 +83,7 @@ struct DecodeParams {
   const int8_t* signs;    // [H] rotation signs of the screen
   float* scr;             // ws [E*I]
   // shared-memory carve-up (byte offsets from the dynamic smem base)
-  int off_x, off_u, off_lg, off_keys, off_kept, off_ysum, off_xf, off_bar, smem_bytes;
+  int off_x, off_u, off_lg, off_keys, off_kept, off_hist, off_ysum, off_xf, off_bar, smem_bytes;
   // io
   const uint16_t* x_in;   // [B, H]
   uint16_t* x_out;        // [B, H] final x (or null)

@@ -15,6 +15,7 @@ namespace moedec {
 constexpr int kConsumers = kThreads;          // 256 consumer threads
 constexpr int kProducers = 2;                // producer warps (alternate jobs)
 constexpr int kCtaThreads = kThreads + 32 * kProducers;
+static_assert(kCtaThreads * 200 <= 65536, "decode_kernel's register cap must fit one CTA per SM");
 
 __device__ __forceinline__ void cbar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 __device__ __forceinline__ int cbar_or(int pred) {
@@ -123,6 +124,68 @@ __device__ __forceinline__ void warp_reduce_multi(float (&v)[NV], float* out) {
   }
 }
 
+// ---------------------------------------------------------------- key selection
+
+constexpr int kSelBins = 2048;  // histogram bins of the radix select (11-bit digits)
+
+// The keep-th largest of n 32-bit keys (0 < keep < n <= kMaxCand), by a radix
+// select over the 256 consumer threads: three passes over digits of 11, 11
+// and 10 bits from the top; each pass counts, among the keys whose higher
+// digits equal the prefix found so far, how many have each digit (shared
+// atomics into hist[kSelBins]), then finds the digit where the count of
+// larger keys crosses keep (one block scan over the bins, largest first).
+// Keys are read from shared memory at keys[q + q / 32]. Returns T (the
+// keep-th largest key) and sets *n_gt to the number of keys > T, so that the
+// kept set is every key > T plus the first keep - n_gt keys == T in index
+// order. scratch: at least kWarps + 4 ints.
+__device__ __forceinline__ uint32_t radix_select(const uint32_t* keys, int n, int keep, int* hist, int* scratch,
+                                                 int* n_gt) {
+  const int tid = threadIdx.x;
+  uint32_t prefix = 0u;
+  int need = keep;  // keys still to take from the current prefix class
+  constexpr int kShift[3] = {21, 10, 0};
+  constexpr int kWidth[3] = {11, 11, 10};
+#pragma unroll
+  for (int pass = 0; pass < 3; ++pass) {
+    const int sh = kShift[pass], nb = 1 << kWidth[pass];
+    for (int i = tid; i < nb; i += kConsumers) hist[i] = 0;
+    cbar();
+    for (int q = tid; q < n; q += kConsumers) {
+      const uint32_t kv = keys[q + (q >> 5)];
+      const bool in_class = pass == 0 || (kv >> (sh + kWidth[pass])) == prefix;
+      if (in_class) atomicAdd(&hist[(kv >> sh) & (uint32_t)(nb - 1)], 1);
+    }
+    cbar();
+    // thread t owns the bins [(255 - t) * per, (256 - t) * per): thread 0 the
+    // largest digits; an exclusive scan over t counts the keys above its bins
+    const int per = nb / kConsumers;
+    const int b_hi = (kConsumers - tid) * per;  // one past this thread's largest bin
+    int mine = 0;
+    for (int b = b_hi - per; b < b_hi; ++b) mine += hist[b];
+    int total;
+    const int above = block_excl_scan(mine, scratch, &total);
+    if (above < need && above + mine >= need) {
+      int acc = above;
+      for (int b = b_hi - 1; b >= b_hi - per; --b) {
+        const int h = hist[b];
+        if (acc + h >= need) {
+          scratch[kWarps + 1] = b;
+          scratch[kWarps + 2] = acc;  // keys of the class with a larger digit
+          break;
+        }
+        acc += h;
+      }
+    }
+    cbar();
+    const int d = scratch[kWarps + 1];
+    need -= scratch[kWarps + 2];
+    prefix = (prefix << kWidth[pass]) | (uint32_t)d;
+    cbar();  // scratch and hist are rewritten by the next pass
+  }
+  *n_gt = keep - need;
+  return prefix;
+}
+
 // ---------------------------------------------------------------- top-k
 
 // One warp: the kk largest keys among keys[0, n) (n <= 1024), ties to the
@@ -186,8 +249,12 @@ __device__ __forceinline__ void ysum_steps(float (&acc)[64], float* ysum, int la
 
 // ---------------------------------------------------------------- the kernel
 
+// One CTA of kCtaThreads (320) threads per SM: up to 200 registers per thread
+// (64,000 of the SM's 65,536). With the 168 that a 1-block launch bound
+// gives, the channel-major instance spills to local memory, which goes to L2
+// because shared memory takes nearly all of L1.
 template <int MODE, int BMAX, int WT, int LAYOUT, int NCH, int HV>
-__global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_constant__ DecodeParams p) {
+__global__ void __maxnreg__(200) decode_kernel(const __grid_constant__ DecodeParams p) {
   constexpr int NR = 2 * NCH;        // dot rows per job (gate+up rows; router rows)
   constexpr int NV = NR * BMAX;      // values reduced per job
   // Batch-1 bf16 rows of 2048 elements: every warp owns whole channels (see
@@ -205,6 +272,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
   __shared__ RouteSmem<BMAX> rs;
   __shared__ int route_ready_s, prod_layer_s[kProducers], abort_s, bad_s, okw_s;
   __shared__ uint32_t ltag_s;  // logit tag of layer 0 in this launch (fast path)
+  __shared__ unsigned long long bar_base_s;  // grid-barrier count at launch (a multiple of G)
   __shared__ long long budget_s;  // cycles per bounded wait (the workspace's budget)
   __shared__ uint32_t inject_s;   // fault-injection bits of the workspace
   __shared__ long long jp_s[kProducers], jc_s, jcg_s[kProducers];
@@ -250,6 +318,15 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
       jp_s[q] = 0;           // jobs producer q has passed (its own ones issued)
     }
     abort_s = 0;
+    // every launch passes at least one grid barrier, so bar_base / G differs
+    // between launches on a workspace and the tags (launch * 64 + layer, top
+    // bit set so that a cleared word never matches) do not repeat; a slot is
+    // rewritten only after the grid barrier that follows every reader's
+    // routing, so a reader never meets a later layer's tag. (Other CTAs may
+    // already have arrived at this launch's first barrier: fewer than G
+    // arrivals do not change the quotient.)
+    bar_base_s = (ld_relaxed_gpu(&ctl->bar) / (unsigned long long)G) * (unsigned long long)G;
+    ltag_s = 0x80000000u | ((uint32_t)(bar_base_s / (unsigned long long)G) * (uint32_t)kMaxLayers);
     budget_s = ctl_wait_budget(ctl);
     inject_s = ctl->inject;
     jc_s = 0;
@@ -268,6 +345,108 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
   }
   __syncthreads();
   const long long budget = budget_s;
+
+  // Batch-1 planar stacks are routed by consumer warp 0 alone (route_warp
+  // below) while the other warps go on with their shared-expert jobs.
+  // (Measured: routing in a producer warp, and writing the tagged logits to
+  // several copies polled by different CTAs, were both slower.)
+  const bool warp_routes = kFast && LAYOUT == MOE_LAYOUT_PLANAR && MODE == MODE_LAYERS && k <= kWarps && E <= 256;
+
+  // ---- B = 1, k <= 8, E <= 256, tagged logit words of layer `lay`: one
+  // warp routes alone, with no CTA barrier, while the other warps go on
+  // with their jobs. Lane l polls words 64q + 2l and 64q + 2l + 1 (q < 4;
+  // the warp's four 16-byte loads cover the 2 KB once) until all carry the
+  // layer's tag, then the k largest are taken by k rounds of a warp-wide
+  // argmax (ties: the lower expert index), followed by the softmax over the
+  // k and the units in ascending expert id. Returns false on a poll timeout.
+  // A logit whose key is 0 (a NaN with every bit set) is never selected.
+  auto route_warp = [&](int lay) -> bool {
+    const unsigned long long* wb = reinterpret_cast<const unsigned long long*>(p.logits);
+    const uint32_t want = 0x80000000u | (ltag_s + (uint32_t)lay);
+    uint32_t key[8];
+    bool done[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      done[q] = 64 * q + 2 * lane >= E;
+      key[2 * q] = 0u;
+      key[2 * q + 1] = 0u;
+    }
+    const long long t0 = clock64();
+    for (;;) {
+      unsigned long long a[4], b[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (!done[q]) ld_relaxed_gpu_v2(wb + 64 * q + 2 * lane, a[q], b[q]);
+      bool all = true;
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (!done[q]) {
+          const int i = 64 * q + 2 * lane;
+          const bool has_b = i + 1 < E;
+          if ((uint32_t)(a[q] >> 32) == want && (!has_b || (uint32_t)(b[q] >> 32) == want)) {
+            done[q] = true;
+            key[2 * q] = float_key(__uint_as_float((uint32_t)a[q]));
+            key[2 * q + 1] = has_b ? float_key(__uint_as_float((uint32_t)b[q])) : 0u;
+          } else {
+            all = false;
+          }
+        }
+      if (__all_sync(0xffffffffu, all)) break;
+      if (__any_sync(0xffffffffu, clock64() - t0 > budget)) return false;  // warp-uniform
+    }
+    // slot s of lane l holds expert 64 (s / 2) + 2 l + s % 2: slots in
+    // ascending index order, so a strict > keeps the lowest index of a tie
+    auto slot_idx = [&](int s) { return 64 * (s >> 1) + 2 * lane + (s & 1); };
+    uint32_t bk = key[0];
+    int bs = 0;
+#pragma unroll
+    for (int s = 1; s < 8; ++s)
+      if (key[s] > bk) { bk = key[s]; bs = s; }
+    for (int r = 0; r < k; ++r) {
+      const uint32_t M = __reduce_max_sync(0xffffffffu, bk);
+      const uint32_t tie = __ballot_sync(0xffffffffu, bk == M);
+      int wl = __ffs(tie) - 1;
+      if (tie & (tie - 1)) {
+        // several lanes hold M: the lowest expert index wins
+        const uint32_t mi = __reduce_min_sync(0xffffffffu, bk == M ? (uint32_t)slot_idx(bs) : 0xffffffffu);
+        wl = __ffs(__ballot_sync(0xffffffffu, bk == M && (uint32_t)slot_idx(bs) == mi)) - 1;
+      }
+      if (lane == wl) {
+        cand_key[kWarps + r] = M;
+        cand_idx[r] = slot_idx(bs);
+#pragma unroll
+        for (int s = 0; s < 8; ++s)
+          if (s == bs) key[s] = 0u;
+        bk = key[0];
+        bs = 0;
+#pragma unroll
+        for (int s = 1; s < 8; ++s)
+          if (key[s] > bk) { bk = key[s]; bs = s; }
+      }
+    }
+    __syncwarp();
+    const bool sel = lane < k;
+    const uint32_t kc = sel ? cand_key[kWarps + lane] : 0u;
+    const int ic = sel ? cand_idx[lane] : 0x7fffffff;
+    const float e = sel ? __expf(key_float(kc) - key_float(cand_key[kWarps])) : 0.f;
+    const float wl = e / warp_sum(e);
+    int urank = 0;
+    for (int m = 0; m < k; ++m) urank += cand_idx[m] < ic;
+    if (sel) {
+      rs.ids[0][lane] = ic;
+      rs.w[0][lane] = wl;
+      rs.unit_e[urank] = ic;
+      rs.unit_mask[urank] = 1u;
+      rs.unit_w[urank][0] = wl;
+      if (cta == 0 && p.ids_out != nullptr) {
+        p.ids_out[(size_t)lay * k + lane] = ic;
+        p.w_out[(size_t)lay * k + lane] = wl;
+      }
+    }
+    if (lane == 0) rs.U = k;
+    __syncwarp();
+    return true;
+  };
 
   // At batch 1 the routed channel count is the same every layer (k * I, or
   // the kept count), so this CTA's routed range {t0, t1, unit, channel} is
@@ -788,16 +967,8 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
     int cslot = 0;          // stage of the next job
     uint32_t cph = 0;       // its phase parity
     long long jc = 0;       // jobs consumed
-    unsigned long long bar_base = 0, nbar = 0;
-    if (tid == 0) {
-      bar_base = (ld_relaxed_gpu(&ctl->bar) / (unsigned long long)G) * (unsigned long long)G;
-      // every launch passes at least one grid barrier, so bar_base / G differs
-      // between launches on a workspace and the tags (launch * 64 + layer,
-      // top bit set so that a cleared word never matches) do not repeat; a
-      // slot is rewritten only after the grid barrier that follows every
-      // reader's routing, so a reader never meets a later layer's tag
-      ltag_s = 0x80000000u | ((uint32_t)(bar_base / (unsigned long long)G) * (uint32_t)kMaxLayers);
-    }
+    const unsigned long long bar_base = bar_base_s;
+    unsigned long long nbar = 0;
 
     float acc[BMAX][8];
 #pragma unroll
@@ -1029,7 +1200,47 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
                              : nullptr;
           if (r < ndot) nr = i + 1;
         }
-        if (nr > 0) {
+        if (BMAX > 1 && HV > 0 && int4_rows && nr > 0) {
+          // int4 rows at batch > 1: each weight vector is dequantised once
+          // and applied to every token of the job
+          float sacc[RPW][BMAX];
+#pragma unroll
+          for (int r = 0; r < RPW; ++r)
+#pragma unroll
+            for (int b = 0; b < BMAX; ++b) sacc[r][b] = 0.f;
+#pragma unroll
+          for (int i = 0; i < (HV > 0 ? HV : 1); ++i) {
+            const int v = i * 32 + lane;
+#pragma unroll
+            for (int r = 0; r < RPW; ++r)
+              if (r < nr) {
+                float wf[8];
+                int4x8_to_f(reinterpret_cast<const uint32_t*>(rowp[r])[v], wf);
+                const float sv = bf16_to_f(scp[r][v >> 3]);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) wf[e] *= sv;
+#pragma unroll
+                for (int b = 0; b < BMAX; ++b)
+                  if ((mask_any >> b) & 1u) {
+                    float xf[8];
+                    unpack8(us4[b * H8c + v], xf);
+                    float d = 0.f;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) d = fmaf(wf[e], xf[e], d);
+                    sacc[r][b] += d;
+                  }
+              }
+          }
+#pragma unroll
+          for (int b = 0; b < BMAX; ++b)
+            if ((mask_any >> b) & 1u)
+#pragma unroll
+              for (int r = 0; r < RPW; ++r)
+                if (r < nr) {
+                  const float t = warp_sum(sacc[r][b]);
+                  if (lane == 0) db[(warp + kWarps * r) * BMAX + b] = t;
+                }
+        } else if (nr > 0) {
 #pragma unroll
           for (int b = 0; b < BMAX; ++b)
             if ((mask_any >> b) & 1u) {
@@ -1084,29 +1295,23 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
               const int rows = H >> 5;
               float s[8];
               unpack8(reinterpret_cast<const uint4*>(st + 3 * NCH * (H >> 1) + 2 * NCH * rows)[tid], s);
-              float inner[BMAX][8];
-#pragma unroll
-              for (int b = 0; b < BMAX; ++b)
-#pragma unroll
-                for (int i = 0; i < 8; ++i) inner[b][i] = 0.f;
+              // the output's scale (one per 64-channel group, the job's group)
+              // folded into each product, so no second accumulator set is live
 #pragma unroll
               for (int ch = 0; ch < NCH; ++ch)
                 if (ch < j.n) {
                   float q[8];
                   int4x8_to_f(reinterpret_cast<const uint32_t*>(st + down_off + ch * ch_stride)[tid], q);
 #pragma unroll
+                  for (int i = 0; i < 8; ++i) q[i] *= s[i];
+#pragma unroll
                   for (int b = 0; b < BMAX; ++b)
                     if ((mask0 >> b) & 1u) {
                       const float h = hbuf[warp][ch * BMAX + b];
 #pragma unroll
-                      for (int i = 0; i < 8; ++i) inner[b][i] = fmaf(h, q[i], inner[b][i]);
+                      for (int i = 0; i < 8; ++i) acc[b][i] = fmaf(h, q[i], acc[b][i]);
                     }
                 }
-#pragma unroll
-              for (int b = 0; b < BMAX; ++b)
-                if ((mask0 >> b) & 1u)
-#pragma unroll
-                  for (int i = 0; i < 8; ++i) acc[b][i] = fmaf(s[i], inner[b][i], acc[b][i]);
             }
           }
         }
@@ -1200,9 +1405,12 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
                   const bool pred = j.u != 0;
                   const unsigned long long tag =
                       (unsigned long long)(0x80000000u | (ltag_s + (uint32_t)(j.layer + (pred ? 1 : 0))));
-                  unsigned long long* dw = pred ? p.plogits + (size_t)((j.layer + 1) & 1) * E
-                                                : reinterpret_cast<unsigned long long*>(p.logits);
-                  st_relaxed_gpu_u64(dw + j.c0 + r, (tag << 32) | __float_as_uint(t));
+                  const unsigned long long word = (tag << 32) | __float_as_uint(t);
+                  if (pred) {
+                    st_relaxed_gpu_u64(p.plogits + (size_t)((j.layer + 1) & 1) * E + j.c0 + r, word);
+                  } else {
+                    st_relaxed_gpu_u64(reinterpret_cast<unsigned long long*>(p.logits) + j.c0 + r, word);
+                  }
                 } else {
                   p.logits[j.c0 + r] = t;  // read after the router barrier
                 }
@@ -1418,102 +1626,6 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
       cbar();
       return bad_s == 0;
       }
-    };
-
-    // ---- B = 1, k <= 8, E <= 256, tagged logit words of layer `lay`: one
-    // warp routes alone, with no CTA barrier, while the other warps go on
-    // with their jobs. Lane l polls words 64q + 2l and 64q + 2l + 1 (q < 4;
-    // the warp's four 16-byte loads cover the 2 KB once) until all carry the
-    // layer's tag, then the k largest are taken by k rounds of a warp-wide
-    // argmax (ties: the lower expert index), followed by the softmax over the
-    // k and the units in ascending expert id. Returns false on a poll timeout.
-    // A logit whose key is 0 (a NaN with every bit set) is never selected.
-    auto route_warp = [&](int lay) -> bool {
-      const unsigned long long* wb = reinterpret_cast<const unsigned long long*>(p.logits);
-      const uint32_t want = 0x80000000u | (ltag_s + (uint32_t)lay);
-      uint32_t key[8];
-      bool done[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        done[q] = 64 * q + 2 * lane >= E;
-        key[2 * q] = 0u;
-        key[2 * q + 1] = 0u;
-      }
-      const long long t0 = clock64();
-      for (;;) {
-        unsigned long long a[4], b[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-          if (!done[q]) ld_relaxed_gpu_v2(wb + 64 * q + 2 * lane, a[q], b[q]);
-        bool all = true;
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-          if (!done[q]) {
-            const int i = 64 * q + 2 * lane;
-            const bool has_b = i + 1 < E;
-            if ((uint32_t)(a[q] >> 32) == want && (!has_b || (uint32_t)(b[q] >> 32) == want)) {
-              done[q] = true;
-              key[2 * q] = float_key(__uint_as_float((uint32_t)a[q]));
-              key[2 * q + 1] = has_b ? float_key(__uint_as_float((uint32_t)b[q])) : 0u;
-            } else {
-              all = false;
-            }
-          }
-        if (__all_sync(0xffffffffu, all)) break;
-        if (__any_sync(0xffffffffu, clock64() - t0 > budget)) return false;  // warp-uniform
-      }
-      // slot s of lane l holds expert 64 (s / 2) + 2 l + s % 2: slots in
-      // ascending index order, so a strict > keeps the lowest index of a tie
-      auto slot_idx = [&](int s) { return 64 * (s >> 1) + 2 * lane + (s & 1); };
-      uint32_t bk = key[0];
-      int bs = 0;
-#pragma unroll
-      for (int s = 1; s < 8; ++s)
-        if (key[s] > bk) { bk = key[s]; bs = s; }
-      for (int r = 0; r < k; ++r) {
-        const uint32_t M = __reduce_max_sync(0xffffffffu, bk);
-        const uint32_t tie = __ballot_sync(0xffffffffu, bk == M);
-        int wl = __ffs(tie) - 1;
-        if (tie & (tie - 1)) {
-          // several lanes hold M: the lowest expert index wins
-          const uint32_t mi = __reduce_min_sync(0xffffffffu, bk == M ? (uint32_t)slot_idx(bs) : 0xffffffffu);
-          wl = __ffs(__ballot_sync(0xffffffffu, bk == M && (uint32_t)slot_idx(bs) == mi)) - 1;
-        }
-        if (lane == wl) {
-          cand_key[kWarps + r] = M;
-          cand_idx[r] = slot_idx(bs);
-#pragma unroll
-          for (int s = 0; s < 8; ++s)
-            if (s == bs) key[s] = 0u;
-          bk = key[0];
-          bs = 0;
-#pragma unroll
-          for (int s = 1; s < 8; ++s)
-            if (key[s] > bk) { bk = key[s]; bs = s; }
-        }
-      }
-      __syncwarp();
-      const bool sel = lane < k;
-      const uint32_t kc = sel ? cand_key[kWarps + lane] : 0u;
-      const int ic = sel ? cand_idx[lane] : 0x7fffffff;
-      const float e = sel ? __expf(key_float(kc) - key_float(cand_key[kWarps])) : 0.f;
-      const float wl = e / warp_sum(e);
-      int urank = 0;
-      for (int m = 0; m < k; ++m) urank += cand_idx[m] < ic;
-      if (sel) {
-        rs.ids[0][lane] = ic;
-        rs.w[0][lane] = wl;
-        rs.unit_e[urank] = ic;
-        rs.unit_mask[urank] = 1u;
-        rs.unit_w[urank][0] = wl;
-        if (cta == 0 && p.ids_out != nullptr) {
-          p.ids_out[(size_t)lay * k + lane] = ic;
-          p.w_out[(size_t)lay * k + lane] = wl;
-        }
-      }
-      if (lane == 0) rs.U = k;
-      __syncwarp();
-      return true;
     };
 
     // ---- top-k of every token from lg[B][E]
@@ -1839,8 +1951,8 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
       const float* sc = p.screen ? p.scr : p.layer[l].scores;
       const float invI = 1.0f / (float)I;
       auto pad = [](int q) { return q + (q >> 5); };
-      // 1. keys: row-major q = i * 256 + tid, all loads in flight at once
-      uint32_t kr[KR];
+      // 1. keys: row-major q = i * 256 + tid, all loads in flight at once,
+      // stored at keys[q + q / 32] (conflict-free for the row and chunk walks)
       {
         float kv[KR];
 #pragma unroll
@@ -1855,60 +1967,19 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
 #pragma unroll
         for (int i = 0; i < KR; ++i) {
           const int q = i * kConsumers + tid;
-          kr[i] = 0u;
-          if (i < rows && q < N) {
-            kr[i] = float_key(kv[i]);
-            keys[pad(q)] = kr[i];
-          }
+          if (i < rows && q < N) keys[pad(q)] = float_key(kv[i]);
         }
       }
       const int keep = p.keep;
       const bool all = keep >= N;
       uint32_t T = 0u;
       int r = 0;
-      int* cnt_s = rs.scan;  // [2][8] per-warp counts, double-buffered
-      int par = 0;
-      // (absent keys are 0 and every threshold tried is >= 1)
-      auto count_ge = [&](uint32_t c) -> int {
-        int n = 0;
-#pragma unroll
-        for (int i0 = 0; i0 < KR; i0 += 8)
-          if (i0 < rows) {
-#pragma unroll
-            for (int i = i0; i < i0 + 8; ++i) n += kr[i] >= c ? 1 : 0;
-          }
-        n = (int)__reduce_add_sync(0xffffffffu, (uint32_t)n);
-        if (lane == 0) cnt_s[8 * par + warp] = n;
-        cbar();
-        int t = 0;
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) t += cnt_s[8 * par + w];
-        par ^= 1;
-        return t;
-      };
+      cbar();
       if (keep > 0 && !all) {
-        // 2. common prefix of all keys (from the smallest and largest key)
-        uint32_t kmax = 0u, kmin = 0xffffffffu;
-#pragma unroll
-        for (int i = 0; i < KR; ++i)
-          if (i < rows && i * kConsumers + tid < N) { kmax = max(kmax, kr[i]); kmin = min(kmin, max(kr[i], 1u)); }
-        kmax = __reduce_max_sync(0xffffffffu, kmax);
-        kmin = __reduce_min_sync(0xffffffffu, kmin);
-        if (lane == 0) { cand_key[warp] = kmax; cand_key[kWarps + warp] = kmin; }
-        cbar();
-        kmax = 0u;
-        kmin = 0xffffffffu;
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) { kmax = max(kmax, cand_key[w]); kmin = min(kmin, cand_key[kWarps + w]); }
-        const uint32_t diff = kmax ^ kmin;
-        const int top = diff ? 31 - __clz(diff) : -1;
-        T = top >= 0 ? kmax & ~(0xffffffffu >> (31 - top)) : kmax;  // the prefix, zeros below
-        // 3. largest T with #{key >= T} >= keep: the keep-th largest key
-        for (int bit = top; bit >= 0; --bit) {
-          const uint32_t c = T | (1u << bit);
-          if (count_ge(c) >= keep) T = c;
-        }
-        r = keep - (T == 0xffffffffu ? 0 : count_ge(T + 1u));
+        // 2. the keep-th largest key T and the count of keys above it
+        int n_gt = 0;
+        T = radix_select(keys, N, keep, reinterpret_cast<int*>(smem + p.off_hist), rs.scan + 32, &n_gt);
+        r = keep - n_gt;
       }
       cbar();  // keys[] complete
       // 4. ordered compaction over contiguous chunks: thread t takes
@@ -2020,6 +2091,29 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
       // ids -> routed units (and kept channels), published to the producer
       auto do_route = [&]() -> bool {
         constexpr bool kWarpRoute = MODE == MODE_LAYERS && BMAX == 1;
+        if (warp_routes) {
+          // warp 0 routes; the other warps need nothing from it and go on.
+          // The producers must be done with layer l - 1's units first.
+          ready = l;
+          if (warp != 0) return true;
+          if (lane == 0 && l > 0) {
+            const long long t0 = clock64();
+            while (min(*(volatile int*)&prod_layer_s[0], *(volatile int*)&prod_layer_s[1]) < l - 1) {
+              if (clock64() - t0 > budget) { set_status(ctl, kStatusTimeout); break; }
+              __nanosleep(20);
+            }
+            (void)ld_acquire_cta(&prod_layer_s[0]);
+            (void)ld_acquire_cta(&prod_layer_s[1]);
+          }
+          __syncwarp();
+          if (!route_warp(l)) {
+            // the others learn of it through the abort flag
+            if (lane == 0) { set_status(ctl, kStatusTimeout); st_release_cta(&abort_s, 1); }
+            return false;
+          }
+          if (lane == 0) st_release_cta(&route_ready_s, l);
+          return true;
+        }
         bool units_done = false;
         // the producer must be done with the previous layer's routing
         // before it is overwritten (it always is, unless this CTA had no
@@ -2033,21 +2127,10 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
           (void)ld_acquire_cta(&prod_layer_s[0]);
           (void)ld_acquire_cta(&prod_layer_s[1]);
         }
-        bool ids_done = false;
         if constexpr (MODE == MODE_LAYERS) {
-          if (kFast && LAYOUT == MOE_LAYOUT_PLANAR && k <= kWarps && E <= 256) {
-            // warp 0 routes; the other warps need nothing from it and go on
-            if constexpr (kFast && LAYOUT == MOE_LAYOUT_PLANAR) {
-              if (warp != 0) return true;
-              if (!route_warp(l)) {
-                // the others learn of it through the abort flag
-                if (lane == 0) { set_status(ctl, kStatusTimeout); st_release_cta(&abort_s, 1); }
-                return false;
-              }
-            }
-            units_done = true;
-            ids_done = true;
-          } else if (kFast && k <= kWarps) {
+          // (planar batch-1 stacks with k <= 8, E <= 256 are routed by
+          // warp 0 above and never get here)
+          if (kFast && k <= kWarps) {
             // logits straight from their tagged words (okw_s = 1 was set
             // before the phase barrier)
             if (!route_b1_small_k(2, l)) { if (tid == 0) set_status(ctl, kStatusTimeout); return false; }
@@ -2067,7 +2150,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
             if (BMAX == 1 && k <= kWarps) { route_b1_small_k(0, l); units_done = true; }
             else route();
           }
-          if (cta == 0 && p.ids_out != nullptr && !ids_done)
+          if (cta == 0 && p.ids_out != nullptr)
             for (int t = tid; t < B * k; t += kConsumers) {
               p.ids_out[(size_t)l * B * k + t] = rs.ids[t / k][t % k];
               p.w_out[(size_t)l * B * k + t] = rs.w[t / k][t % k];
