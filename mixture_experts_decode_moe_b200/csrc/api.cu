@@ -178,9 +178,9 @@ bool plan_smem(DecodeParams* p, int static_bytes, bool fast) {
   return true;
 }
 
-template <int MODE, int BMAX, int WT, int LAYOUT, int NCH, int HV>
+template <int MODE, int BMAX, int WT, int LAYOUT, int NCH, int HV, bool SCREEN>
 cudaError_t launch_decode_h(const DecodeParams& p0, int grid, cudaStream_t s) {
-  auto kern = decode_kernel<MODE, BMAX, WT, LAYOUT, NCH, HV>;
+  auto kern = decode_kernel<MODE, BMAX, WT, LAYOUT, NCH, HV, SCREEN>;
   cudaFuncAttributes fa;
   cudaError_t err = cudaFuncGetAttributes(&fa, kern);
   if (err != cudaSuccess) return err;
@@ -204,29 +204,34 @@ cudaError_t launch_decode_h(const DecodeParams& p0, int grid, cudaStream_t s) {
 
 // Full-row dot loops are specialised for H = 2048 (HV = H/256 = 8 vectors per
 // lane); other hidden sizes use the guarded generic loop.
-template <int MODE, int BMAX, int WT, int LAYOUT, int NCH>
+template <int MODE, int BMAX, int WT, int LAYOUT, int NCH, bool SCREEN>
 cudaError_t launch_decode_n(const DecodeParams& p, int grid, cudaStream_t s) {
   if (p.H == 2048) {
     // batch-1 H = 2048 kernels are the pipelined fast path: 4 channels per job
     if constexpr (BMAX == 1 && NCH != 4) return cudaErrorInvalidValue;
-    else return launch_decode_h<MODE, BMAX, WT, LAYOUT, NCH, 8>(p, grid, s);
+    else return launch_decode_h<MODE, BMAX, WT, LAYOUT, NCH, 8, SCREEN>(p, grid, s);
   }
-  return launch_decode_h<MODE, BMAX, WT, LAYOUT, NCH, 0>(p, grid, s);
+  return launch_decode_h<MODE, BMAX, WT, LAYOUT, NCH, 0, SCREEN>(p, grid, s);
 }
 
-template <int MODE, int BMAX, int WT, int LAYOUT>
+template <int MODE, int BMAX, int WT, int LAYOUT, bool SCREEN>
 cudaError_t launch_decode_m(const DecodeParams& p, int grid, cudaStream_t s) {
   if constexpr (BMAX == 1 && WT == MOE_W_BF16) {
-    if (p.nch == 8) return launch_decode_n<MODE, BMAX, WT, LAYOUT, 8>(p, grid, s);
+    if (p.nch == 8) return launch_decode_n<MODE, BMAX, WT, LAYOUT, 8, SCREEN>(p, grid, s);
   }
   if (p.nch != 4) return cudaErrorInvalidValue;
-  return launch_decode_n<MODE, BMAX, WT, LAYOUT, 4>(p, grid, s);
+  return launch_decode_n<MODE, BMAX, WT, LAYOUT, 4, SCREEN>(p, grid, s);
 }
 
-template <int BMAX, int WT, int LAYOUT>
+template <int BMAX, int WT, int LAYOUT, bool SCREEN = false>
 cudaError_t launch_decode_t(const DecodeParams& p, int grid, cudaStream_t s) {
-  if (p.mode == MODE_LAYERS) return launch_decode_m<MODE_LAYERS, BMAX, WT, LAYOUT>(p, grid, s);
-  return launch_decode_m<MODE_EXPERTS, BMAX, WT, LAYOUT>(p, grid, s);
+  if constexpr (SCREEN) {  // the screened channel stack (layers mode only)
+    if (p.mode != MODE_LAYERS) return cudaErrorInvalidValue;
+    return launch_decode_m<MODE_LAYERS, BMAX, WT, LAYOUT, true>(p, grid, s);
+  } else {
+    if (p.mode == MODE_LAYERS) return launch_decode_m<MODE_LAYERS, BMAX, WT, LAYOUT, false>(p, grid, s);
+    return launch_decode_m<MODE_EXPERTS, BMAX, WT, LAYOUT, false>(p, grid, s);
+  }
 }
 
 moe_status launch_decode(const DecodeParams& p, int bmax, cudaStream_t s) {
@@ -235,7 +240,8 @@ moe_status launch_decode(const DecodeParams& p, int bmax, cudaStream_t s) {
   cudaError_t err;
   if (p.layout == MOE_LAYOUT_CHANNEL_MAJOR) {
     if (bmax != 1) return MOE_ERR_UNSUPPORTED;
-    err = launch_decode_t<1, MOE_W_BF16, MOE_LAYOUT_CHANNEL_MAJOR>(p, grid, s);
+    err = p.screen ? launch_decode_t<1, MOE_W_BF16, MOE_LAYOUT_CHANNEL_MAJOR, true>(p, grid, s)
+                   : launch_decode_t<1, MOE_W_BF16, MOE_LAYOUT_CHANNEL_MAJOR, false>(p, grid, s);
   } else if (p.wtype == MOE_W_BF16) {
     err = (bmax == 1) ? launch_decode_t<1, MOE_W_BF16, MOE_LAYOUT_PLANAR>(p, grid, s)
                       : launch_decode_t<kMaxB, MOE_W_BF16, MOE_LAYOUT_PLANAR>(p, grid, s);

@@ -129,26 +129,26 @@ __global__ void __launch_bounds__(kCbThreads, 1) channel_batch_kernel(const __gr
       }
     }
     cbar();
-    constexpr int KR = kMaxCand / kCbConsumers;  // key rows per thread
     const int N = k * I;
     const int rows = (N + kCbConsumers - 1) / kCbConsumers;
     uint32_t* keys = reinterpret_cast<uint32_t*>(ring);  // padded q + q / 32
     auto pad = [](int q) { return q + (q >> 5); };
-    {
-      float kv[KR];
+#pragma unroll 1
+    for (int i0 = 0; i0 < rows; i0 += 4) {
+      float kv[4];
 #pragma unroll
-      for (int i = 0; i < KR; ++i) {
-        const int q = i * kCbConsumers + tid;
+      for (int i = 0; i < 4; ++i) {
+        const int q = (i0 + i) * kCbConsumers + tid;
         kv[i] = 0.f;
-        if (i < rows && q < N) {
+        if (i0 + i < rows && q < N) {
           const int u = q / I;
           kv[i] = __ldg(p.scores + ((size_t)b * E + tu_e[u]) * I + (q - u * I));
         }
       }
 #pragma unroll
-      for (int i = 0; i < KR; ++i) {
-        const int q = i * kCbConsumers + tid;
-        if (i < rows && q < N) keys[pad(q)] = float_key(kv[i]);
+      for (int i = 0; i < 4; ++i) {
+        const int q = (i0 + i) * kCbConsumers + tid;
+        if (i0 + i < rows && q < N) keys[pad(q)] = float_key(kv[i]);
       }
     }
     const bool all = keep >= N;
@@ -165,32 +165,14 @@ __global__ void __launch_bounds__(kCbThreads, 1) channel_batch_kernel(const __gr
     cbar();  // keys[] complete
     int* kws = p.kept_ws + (size_t)b * keep;
     if (keep > 0) {
-      const int chunk = rows;
-      const int q0 = min(N, tid * chunk), q1 = min(N, q0 + chunk);
-      int ng = 0, ne = 0;
-      for (int q = q0; q < q1; ++q) {
-        const uint32_t kk = keys[pad(q)];
-        ng += (all || kk > T) ? 1 : 0;
-        ne += (!all && kk == T) ? 1 : 0;
-      }
-      int tot;
-      const int pre = block_excl_scan(ng | (ne << 16), scan_s, &tot);
-      int pg = pre & 0xffff, pe = pre >> 16;
-      int u = q0 / I, c = q0 - u * I;
-      for (int q = q0; q < q1; ++q) {
-        const uint32_t kk = keys[pad(q)];
-        const bool gt = all || kk > T;
-        const bool eq = !all && kk == T;
-        if (gt || (eq && pe < r)) {
-          const int pos = pg + min(pe, r);
-          const int j = tu_e[u] * I + c;
-          kws[pos] = j;
-          if (p.kept_out) p.kept_out[(size_t)b * keep + pos] = j;
-        }
-        pg += gt ? 1 : 0;
-        pe += eq ? 1 : 0;
-        if (++c == I) { c = 0; ++u; }
-      }
+      // the kept list, ascending (ballot compaction; counts in the histogram's space)
+      int* cnt = reinterpret_cast<int*>(ring + ((size_t)(N + N / 32 + 1) * 4 + 127) / 128 * 128);
+      compact_kept(keys, N, all, T, r, cnt, scan_s, [&](int pos, int q) {
+        const int u = q / I;
+        const int j = tu_e[u] * I + (q - u * I);
+        kws[pos] = j;
+        if (p.kept_out) p.kept_out[(size_t)b * keep + pos] = j;
+      });
     }
     cbar();  // the kept list is complete (global writes of this CTA, ordered by the barrier)
     // sectors of the token's kept channels (channel-major ranges, a sector

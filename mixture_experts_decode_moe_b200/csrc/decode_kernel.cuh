@@ -15,7 +15,6 @@ namespace moedec {
 constexpr int kConsumers = kThreads;          // 256 consumer threads
 constexpr int kProducers = 2;                // producer warps (alternate jobs)
 constexpr int kCtaThreads = kThreads + 32 * kProducers;
-static_assert(kCtaThreads * 200 <= 65536, "decode_kernel's register cap must fit one CTA per SM");
 
 __device__ __forceinline__ void cbar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 __device__ __forceinline__ int cbar_or(int pred) {
@@ -143,16 +142,18 @@ __device__ __forceinline__ uint32_t radix_select(const uint32_t* keys, int n, in
   const int tid = threadIdx.x;
   uint32_t prefix = 0u;
   int need = keep;  // keys still to take from the current prefix class
-  constexpr int kShift[3] = {21, 10, 0};
-  constexpr int kWidth[3] = {11, 11, 10};
-#pragma unroll
+  // (a rolled loop: this runs once per layer, so short code beats unrolled
+  // code, whose instructions would be fetched cold every time)
+#pragma unroll 1
   for (int pass = 0; pass < 3; ++pass) {
-    const int sh = kShift[pass], nb = 1 << kWidth[pass];
+    const int sh = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+    const int wd = pass < 2 ? 11 : 10;
+    const int nb = 1 << wd;
     for (int i = tid; i < nb; i += kConsumers) hist[i] = 0;
     cbar();
     for (int q = tid; q < n; q += kConsumers) {
       const uint32_t kv = keys[q + (q >> 5)];
-      const bool in_class = pass == 0 || (kv >> (sh + kWidth[pass])) == prefix;
+      const bool in_class = pass == 0 || (kv >> (sh + wd)) == prefix;
       if (in_class) atomicAdd(&hist[(kv >> sh) & (uint32_t)(nb - 1)], 1);
     }
     cbar();
@@ -179,11 +180,53 @@ __device__ __forceinline__ uint32_t radix_select(const uint32_t* keys, int n, in
     cbar();
     const int d = scratch[kWarps + 1];
     need -= scratch[kWarps + 2];
-    prefix = (prefix << kWidth[pass]) | (uint32_t)d;
+    prefix = (prefix << wd) | (uint32_t)d;
     cbar();  // scratch and hist are rewritten by the next pass
   }
   *n_gt = keep - need;
   return prefix;
+}
+
+// Ordered compaction of the kept candidates over the 256 consumer threads:
+// candidate q (0 <= q < n, key at keys[q + q / 32]) is kept iff all, or its
+// key > T, or its key == T and fewer than r keys == T precede it. Thread t
+// visits q = 256 i + t; per row i each warp's ballots give its counts of
+// larger and equal keys, one block scan over the (row, warp) counts in row
+// order gives each warp's base, and a kept candidate's place in the
+// ascending list is (larger keys before it) + min(equal keys before it, r).
+// emit(pos, q) is called once per kept candidate. cnt: (n / 256 + 1) * kWarps
+// ints of scratch; scratch: kWarps + 1 ints.
+template <class Emit>
+__device__ __forceinline__ void compact_kept(const uint32_t* keys, int n, bool all, uint32_t T, int r, int* cnt,
+                                             int* scratch, Emit emit) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int rows = (n + kConsumers - 1) / kConsumers;
+  const uint32_t lt = (1u << lane) - 1u;
+  for (int i = 0; i < rows; ++i) {
+    const int q = i * kConsumers + tid;
+    const uint32_t kk = q < n ? keys[q + (q >> 5)] : 0u;
+    const uint32_t bg = __ballot_sync(0xffffffffu, q < n && (all || kk > T));
+    const uint32_t be = __ballot_sync(0xffffffffu, q < n && !all && kk == T);
+    if (lane == 0) cnt[i * kWarps + warp] = __popc(bg) | (__popc(be) << 16);
+  }
+  cbar();
+  const int m = rows * kWarps;  // <= 256 entries, one per thread
+  const int v = tid < m ? cnt[tid] : 0;
+  int total;
+  const int pre = block_excl_scan(v, scratch, &total);
+  if (tid < m) cnt[tid] = pre;  // each thread rewrites only the entry it read
+  cbar();
+  for (int i = 0; i < rows; ++i) {
+    const int q = i * kConsumers + tid;
+    const uint32_t kk = q < n ? keys[q + (q >> 5)] : 0u;
+    const bool g = q < n && (all || kk > T);
+    const bool e = q < n && !all && kk == T;
+    const uint32_t bg = __ballot_sync(0xffffffffu, g);
+    const uint32_t be = __ballot_sync(0xffffffffu, e);
+    const int base = cnt[i * kWarps + warp];
+    const int pg = (base & 0xffff) + __popc(bg & lt), pe = (base >> 16) + __popc(be & lt);
+    if (g || (e && pe < r)) emit(pg + min(pe, r), q);
+  }
 }
 
 // ---------------------------------------------------------------- top-k
@@ -231,7 +274,9 @@ __device__ __forceinline__ void warp_weights(const float* l, int k, float* w) {
 // 256 c + 8 lane + e in acc[8 c + e]) into ysum (element 256 c + 8 lane + e
 // at 256 c + 32 e + lane): at step st warp W adds its chunk (W + st) % 8, so
 // no two warps touch a chunk at once; one barrier per step. W is a template
-// argument so that every register index is a constant.
+// argument so that every register index is a constant. (The accumulators
+// are zeroed by the caller just before the next layer's first job that adds
+// to them, so that they are not live through routing and selection.)
 template <int W>
 __device__ __forceinline__ void ysum_steps(float (&acc)[64], float* ysum, int lane) {
 #pragma unroll
@@ -241,7 +286,6 @@ __device__ __forceinline__ void ysum_steps(float (&acc)[64], float* ysum, int la
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       yc[32 * e] = st == 0 ? acc[8 * c + e] : yc[32 * e] + acc[8 * c + e];
-      acc[8 * c + e] = 0.f;
     }
     cbar();
   }
@@ -249,12 +293,15 @@ __device__ __forceinline__ void ysum_steps(float (&acc)[64], float* ysum, int la
 
 // ---------------------------------------------------------------- the kernel
 
-// One CTA of kCtaThreads (320) threads per SM: up to 200 registers per thread
-// (64,000 of the SM's 65,536). With the 168 that a 1-block launch bound
-// gives, the channel-major instance spills to local memory, which goes to L2
-// because shared memory takes nearly all of L1.
-template <int MODE, int BMAX, int WT, int LAYOUT, int NCH, int HV>
-__global__ void __maxnreg__(200) decode_kernel(const __grid_constant__ DecodeParams p) {
+// One CTA of kCtaThreads (320) threads per SM. Ten warps put three on some of
+// the SM's four sub-partitions of 16K registers each, so a thread gets at
+// most 168 registers; spills would go to local memory, i.e. to L2, since
+// shared memory takes nearly all of L1 (live ranges are kept short instead).
+// SCREEN (channel-major stacks only): the scores are screened in the kernel
+// from per-layer sketches (a separate instance: the screen's registers would
+// make the plain channel-major instance spill).
+template <int MODE, int BMAX, int WT, int LAYOUT, int NCH, int HV, bool SCREEN = false>
+__global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_constant__ DecodeParams p) {
   constexpr int NR = 2 * NCH;        // dot rows per job (gate+up rows; router rows)
   constexpr int NV = NR * BMAX;      // values reduced per job
   // Batch-1 bf16 rows of 2048 elements: every warp owns whole channels (see
@@ -832,6 +879,15 @@ __global__ void __maxnreg__(200) decode_kernel(const __grid_constant__ DecodePar
         v = __shfl_sync(0xffffffffu, v, 0);
         held = (l + 1 < p.L) ? (int)v : -1;
       }
+      // channel-major stacks with given scores: this CTA's 1/G of the next
+      // layer's score tensor [E, I] into L2 (every CTA's selection reads the
+      // routed rows of it right after routing)
+      if (LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR && !SCREEN && l + 1 < p.L && pi == 0 && lane == 0) {
+        const size_t bytes = (size_t)E * I * 4;
+        const size_t b0 = ((size_t)cta * bytes / G) & ~(size_t)15, b1 = ((size_t)(cta + 1) * bytes / G) & ~(size_t)15;
+        const uint8_t* sc1 = reinterpret_cast<const uint8_t*>(p.layer[l + 1].scores);
+        if (b1 > b0 && ((uintptr_t)sc1 & 15u) == 0) prefetch_l2(sc1 + b0, (uint32_t)(b1 - b0));
+      }
       // every routed copy of layer l is issued: while the layer drains, and
       // through the barrier, epilogue, router and top-k of layer l + 1 (when
       // HBM would idle), prefetch this CTA's share of the experts layer
@@ -1015,7 +1071,7 @@ __global__ void __maxnreg__(200) decode_kernel(const __grid_constant__ DecodePar
         uwp[m] = w;
       }
       // u as plain bf16 for the int4 rows' FMA dots and for the channel screen
-      if (kFastI4 || (LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR && p.screen)) reinterpret_cast<uint4*>(us)[tid] = uw;
+      if (kFastI4 || (LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR && SCREEN)) reinterpret_cast<uint4*>(us)[tid] = uw;
       cbar();
     };
     auto load_xfrag = [&]() {
@@ -1200,47 +1256,7 @@ __global__ void __maxnreg__(200) decode_kernel(const __grid_constant__ DecodePar
                              : nullptr;
           if (r < ndot) nr = i + 1;
         }
-        if (BMAX > 1 && HV > 0 && int4_rows && nr > 0) {
-          // int4 rows at batch > 1: each weight vector is dequantised once
-          // and applied to every token of the job
-          float sacc[RPW][BMAX];
-#pragma unroll
-          for (int r = 0; r < RPW; ++r)
-#pragma unroll
-            for (int b = 0; b < BMAX; ++b) sacc[r][b] = 0.f;
-#pragma unroll
-          for (int i = 0; i < (HV > 0 ? HV : 1); ++i) {
-            const int v = i * 32 + lane;
-#pragma unroll
-            for (int r = 0; r < RPW; ++r)
-              if (r < nr) {
-                float wf[8];
-                int4x8_to_f(reinterpret_cast<const uint32_t*>(rowp[r])[v], wf);
-                const float sv = bf16_to_f(scp[r][v >> 3]);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) wf[e] *= sv;
-#pragma unroll
-                for (int b = 0; b < BMAX; ++b)
-                  if ((mask_any >> b) & 1u) {
-                    float xf[8];
-                    unpack8(us4[b * H8c + v], xf);
-                    float d = 0.f;
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) d = fmaf(wf[e], xf[e], d);
-                    sacc[r][b] += d;
-                  }
-              }
-          }
-#pragma unroll
-          for (int b = 0; b < BMAX; ++b)
-            if ((mask_any >> b) & 1u)
-#pragma unroll
-              for (int r = 0; r < RPW; ++r)
-                if (r < nr) {
-                  const float t = warp_sum(sacc[r][b]);
-                  if (lane == 0) db[(warp + kWarps * r) * BMAX + b] = t;
-                }
-        } else if (nr > 0) {
+        if (nr > 0) {
 #pragma unroll
           for (int b = 0; b < BMAX; ++b)
             if ((mask_any >> b) & 1u) {
@@ -1867,7 +1883,7 @@ __global__ void __maxnreg__(200) decode_kernel(const __grid_constant__ DecodePar
     // written to scr[e*I + c]. A grid barrier then makes every CTA's scores
     // visible to the selection. Returns false when the barrier ran out.
     auto screen_layer = [&](int l) -> bool {
-      if constexpr (LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR) {
+      if constexpr (LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR && SCREEN) {
         const LayerW& Lw = p.layer[l];
         float* ux = reinterpret_cast<float*>(keys);
         float* uxp = ux + H;
@@ -1945,29 +1961,30 @@ __global__ void __maxnreg__(200) decode_kernel(const __grid_constant__ DecodePar
     };
 
     auto select_channels = [&](int l) {
-      constexpr int KR = kMaxCand / kConsumers;  // key rows per thread
       const int N = rs.U * I;
       const int rows = (N + kConsumers - 1) / kConsumers;
-      const float* sc = p.screen ? p.scr : p.layer[l].scores;
+      const float* sc = SCREEN ? p.scr : p.layer[l].scores;
       const float invI = 1.0f / (float)I;
       auto pad = [](int q) { return q + (q >> 5); };
-      // 1. keys: row-major q = i * 256 + tid, all loads in flight at once,
-      // stored at keys[q + q / 32] (conflict-free for the row and chunk walks)
-      {
-        float kv[KR];
+      // 1. keys: row-major q = i * 256 + tid, stored at keys[q + q / 32]
+      // (conflict-free for the row walks); a rolled loop with four loads in
+      // flight (short code: it runs once per layer)
+#pragma unroll 1
+      for (int i0 = 0; i0 < rows; i0 += 4) {
+        float kv[4];
 #pragma unroll
-        for (int i = 0; i < KR; ++i) {
-          const int q = i * kConsumers + tid;
+        for (int i = 0; i < 4; ++i) {
+          const int q = (i0 + i) * kConsumers + tid;
           kv[i] = 0.f;
-          if (i < rows && q < N) {
+          if (i0 + i < rows && q < N) {
             const int u = __float2int_rz(((float)q + 0.5f) * invI);
             kv[i] = __ldcg(sc + (size_t)rs.unit_e[u] * I + (q - u * I));  // written in this launch when screened
           }
         }
 #pragma unroll
-        for (int i = 0; i < KR; ++i) {
-          const int q = i * kConsumers + tid;
-          if (i < rows && q < N) keys[pad(q)] = float_key(kv[i]);
+        for (int i = 0; i < 4; ++i) {
+          const int q = (i0 + i) * kConsumers + tid;
+          if (i0 + i < rows && q < N) keys[pad(q)] = float_key(kv[i]);
         }
       }
       const int keep = p.keep;
@@ -1982,31 +1999,12 @@ __global__ void __maxnreg__(200) decode_kernel(const __grid_constant__ DecodePar
         r = keep - n_gt;
       }
       cbar();  // keys[] complete
-      // 4. ordered compaction over contiguous chunks: thread t takes
-      // q in [t * chunk, (t + 1) * chunk)
-      if (keep > 0) {
-        const int chunk = rows;  // ceil(N / 256)
-        const int q0 = min(N, tid * chunk), q1 = min(N, q0 + chunk);
-        int ng = 0, ne = 0;
-        for (int q = q0; q < q1; ++q) {
-          const uint32_t kk = keys[pad(q)];
-          ng += (all || kk > T) ? 1 : 0;
-          ne += (!all && kk == T) ? 1 : 0;
-        }
-        int tot;
-        const int pre = block_excl_scan(ng | (ne << 16), rs.scan + 16, &tot);
-        int pg = pre & 0xffff, pe = pre >> 16;
-        int u = __float2int_rz(((float)q0 + 0.5f) * invI), c = q0 - u * I;
-        for (int q = q0; q < q1; ++q) {
-          const uint32_t kk = keys[pad(q)];
-          const bool gt = all || kk > T;
-          const bool eq = !all && kk == T;
-          if (gt || (eq && pe < r)) kept[pg + min(pe, r)] = rs.unit_e[u] * I + c;
-          pg += gt ? 1 : 0;
-          pe += eq ? 1 : 0;
-          if (++c == I) { c = 0; ++u; }
-        }
-      }
+      // 4. the kept list, ascending (ballot compaction)
+      if (keep > 0)
+        compact_kept(keys, N, all, T, r, rs.scan, reinterpret_cast<int*>(smem + p.off_hist), [&](int pos, int q) {
+          const int u = __float2int_rz(((float)q + 0.5f) * invI);
+          kept[pos] = rs.unit_e[u] * I + (q - u * I);
+        });
       if (tid == 0) rs.ncand = keep > 0 ? min(N, keep) : 0;
       cbar();
       // sectors: each kept channel's byte range, less a sector shared with
@@ -2130,7 +2128,13 @@ __global__ void __maxnreg__(200) decode_kernel(const __grid_constant__ DecodePar
         if constexpr (MODE == MODE_LAYERS) {
           // (planar batch-1 stacks with k <= 8, E <= 256 are routed by
           // warp 0 above and never get here)
-          if (kFast && k <= kWarps) {
+          if (kFast && k <= kWarps && E <= 256) {
+            // channel-major: warp 0 routes from the tagged words, the others
+            // wait; every warp learns the outcome from one barrier reduction
+            const int bad = (warp == 0) ? (route_warp(l) ? 0 : 1) : 0;
+            if (cbar_or(bad)) { if (tid == 0) set_status(ctl, kStatusTimeout); return false; }
+            units_done = true;
+          } else if (kFast && k <= kWarps) {
             // logits straight from their tagged words (okw_s = 1 was set
             // before the phase barrier)
             if (!route_b1_small_k(2, l)) { if (tid == 0) set_status(ctl, kStatusTimeout); return false; }
@@ -2164,7 +2168,7 @@ __global__ void __maxnreg__(200) decode_kernel(const __grid_constant__ DecodePar
         }
         if (!units_done && !build_units() && cta == 0 && tid == 0) set_status(ctl, kStatusBadIds);
         if constexpr (LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR) {
-          if (p.screen && !screen_layer(l)) { if (tid == 0) set_status(ctl, kStatusTimeout); return false; }
+          if (SCREEN && !screen_layer(l)) { if (tid == 0) set_status(ctl, kStatusTimeout); return false; }
           select_channels(l);
           if (cta == 0) {
             if (p.kept_out != nullptr)
@@ -2192,6 +2196,9 @@ __global__ void __maxnreg__(200) decode_kernel(const __grid_constant__ DecodePar
         } else {
           if (!do_route()) { failed = true; break; }
         }
+        // the output accumulators start from zero here: not live before
+#pragma unroll
+        for (int i = 0; i < (kFast ? 64 : 1); ++i) accf[i] = 0.f;
         for (int i = 0; i < own_shared && !fl; ++i) fl = consume_pipe() != JOB_SHARED;
         if (l + 1 < p.L)
           for (int i = 0; i < own_pred && !fl; ++i) fl = consume_pipe() != JOB_ROUTER;
