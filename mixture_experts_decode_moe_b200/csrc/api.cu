@@ -146,11 +146,11 @@ bool plan_smem(DecodeParams* p, int static_bytes, bool fast) {
   const int lg_bytes = (p->mode == MODE_LAYERS) ? (int)align_up((size_t)B * p->E * 4, 128) : 0;
   // keys: router top-k keys [B*E] and channel-sparse candidates [k*I]
   size_t nkeys = (p->mode == MODE_LAYERS) ? (size_t)B * p->E : 0;
-  if (cm) nkeys = std::max(nkeys, (size_t)p->k * p->I + (size_t)p->k * p->I / 32 + 1);  // padded q + q / 32
+  if (cm) nkeys = std::max(nkeys, (size_t)p->k * p->I);
   if (cm && p->screen) nkeys = std::max(nkeys, (size_t)(2 * H + H / 16));  // rotated u and its padded copy
   const int keys_bytes = (int)align_up(std::max<size_t>(nkeys, 1) * 4, 128);
   const int kept_bytes = cm ? (int)align_up((size_t)std::max(p->keep, 1) * 4, 128) : 0;
-  const int hist_bytes = cm ? kSelBins * 4 : 0;  // radix-select histogram
+  const int hist_bytes = cm ? (int)align_up((size_t)(2 * kSelBins + kSelScratch) * 4, 128) : 0;  // the channel select's bins and scratch
   const int ysum_bytes = fast ? (int)align_up((size_t)H * 4, 128) : 0;
   const int xf_bytes = fast ? H * 2 : 0;  // x fragments, [segment][lane] x 16 B
   int stage;
@@ -734,10 +734,9 @@ moe_status moe_channel_topk_forward(const moe_layer_desc* d, const void* x, int3
   uint8_t* base = static_cast<uint8_t*>(ws);
   p.ctl = reinterpret_cast<WsControl*>(base);
   p.kept_ws = reinterpret_cast<int32_t*>(base + chan_kept_offset(B, d));
-  const long long nq = (long long)d->k * d->I;
   const long long uw = (units * d->I + 31) / 32;
   size_t ring = (size_t)kCbStages * kCbNch * 3 * d->H * 2;
-  ring = std::max(ring, align_up((size_t)(nq + nq / 32 + 1) * 4, 128) + (size_t)kSelBins * 4);  // keys + histogram
+  ring = std::max(ring, align_up((size_t)d->k * d->I * 4, 128) + (size_t)(2 * kSelBins + kSelScratch) * 4);  // keys, the select's bins and scratch
   ring = std::max(ring, (size_t)(B + 2) * (size_t)uw * 4);
   ring = std::max(ring, (size_t)(d->E + 31) / 32 * 4);
   ring = align_up(ring, (size_t)128);

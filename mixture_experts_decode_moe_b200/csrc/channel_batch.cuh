@@ -13,9 +13,8 @@
 // applied to every token that kept it.
 //
 // How (B200 design), one CTA per SM, 8 consumer warps + 1 producer warp:
-//  A. CTA b < B selects token b's kept channels (keys in registers, the
-//     keep-th largest key found bit by bit below the common prefix, ordered
-//     compaction), writes them ascending to the workspace (and the caller's
+//  A. CTA b < B selects token b's kept channels (the keep-th largest key
+//     by histogram passes over the keys' own range, ordered compaction), writes them ascending to the workspace (and the caller's
 //     kept list) with the token's sector count; every CTA zeroes its slice
 //     of y. One grid-wide barrier.
 //  B. Every CTA builds the batch's touched experts (ascending), one bitmap of
@@ -130,50 +129,24 @@ __global__ void __launch_bounds__(kCbThreads, 1) channel_batch_kernel(const __gr
     }
     cbar();
     const int N = k * I;
-    const int rows = (N + kCbConsumers - 1) / kCbConsumers;
-    uint32_t* keys = reinterpret_cast<uint32_t*>(ring);  // padded q + q / 32
-    auto pad = [](int q) { return q + (q >> 5); };
-#pragma unroll 1
-    for (int i0 = 0; i0 < rows; i0 += 4) {
-      float kv[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int q = (i0 + i) * kCbConsumers + tid;
-        kv[i] = 0.f;
-        if (i0 + i < rows && q < N) {
-          const int u = q / I;
-          kv[i] = __ldg(p.scores + ((size_t)b * E + tu_e[u]) * I + (q - u * I));
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int q = (i0 + i) * kCbConsumers + tid;
-        if (i0 + i < rows && q < N) keys[pad(q)] = float_key(kv[i]);
-      }
-    }
-    const bool all = keep >= N;
-    uint32_t T = 0u;
-    int r = 0;
+    // keys, then the select's bins and scratch, in the ring (unused until
+    // phase C)
+    uint32_t* keys = reinterpret_cast<uint32_t*>(ring);
+    int* hist = reinterpret_cast<int*>(ring + ((size_t)N * 4 + 127) / 128 * 128);
+    int* sel_sc = hist + 2 * kSelBins;
+    const float* srow = p.scores + (size_t)b * E * I;
+    const bool vec = (I & 3) == 0 && ((uintptr_t)p.scores & 15u) == 0;
+    sel_load_keys(keys, N, I, vec, [&](int u) { return srow + (size_t)tu_e[u] * I; }, hist, sel_sc);
     cbar();
-    if (keep > 0 && !all) {
-      // the keep-th largest key and the count above it (histogram after the keys)
-      int* hist = reinterpret_cast<int*>(ring + ((size_t)(N + N / 32 + 1) * 4 + 127) / 128 * 128);
-      int n_gt = 0;
-      T = radix_select(keys, N, keep, hist, scan_s, &n_gt);
-      r = keep - n_gt;
-    }
-    cbar();  // keys[] complete
     int* kws = p.kept_ws + (size_t)b * keep;
-    if (keep > 0) {
-      // the kept list, ascending (ballot compaction; counts in the histogram's space)
-      int* cnt = reinterpret_cast<int*>(ring + ((size_t)(N + N / 32 + 1) * 4 + 127) / 128 * 128);
-      compact_kept(keys, N, all, T, r, cnt, scan_s, [&](int pos, int q) {
+    if (keep > 0)
+      // the kept list, ascending
+      sel_kept(keys, N, keep, hist, sel_sc, [&](int pos, int q) {
         const int u = q / I;
         const int j = tu_e[u] * I + (q - u * I);
         kws[pos] = j;
         if (p.kept_out) p.kept_out[(size_t)b * keep + pos] = j;
       });
-    }
     cbar();  // the kept list is complete (global writes of this CTA, ordered by the barrier)
     // sectors of the token's kept channels (channel-major ranges, a sector
     // shared with the previous kept channel counted once)

@@ -125,107 +125,340 @@ __device__ __forceinline__ void warp_reduce_multi(float (&v)[NV], float* out) {
 
 // ---------------------------------------------------------------- key selection
 
-constexpr int kSelBins = 2048;  // histogram bins of the radix select (11-bit digits)
+constexpr int kSelBins = 2048;                    // histogram bins of one select pass
+constexpr int kSelGather = 64;                    // class size ranked directly
+constexpr int kSelScratch = 160 + kConsumers;     // ints of scratch the select needs
 
-// The keep-th largest of n 32-bit keys (0 < keep < n <= kMaxCand), by a radix
-// select over the 256 consumer threads: three passes over digits of 11, 11
-// and 10 bits from the top; each pass counts, among the keys whose higher
-// digits equal the prefix found so far, how many have each digit (shared
-// atomics into hist[kSelBins]), then finds the digit where the count of
-// larger keys crosses keep (one block scan over the bins, largest first).
-// Keys are read from shared memory at keys[q + q / 32]. Returns T (the
-// keep-th largest key) and sets *n_gt to the number of keys > T, so that the
-// kept set is every key > T plus the first keep - n_gt keys == T in index
-// order. scratch: at least kWarps + 4 ints.
-__device__ __forceinline__ uint32_t radix_select(const uint32_t* keys, int n, int keep, int* hist, int* scratch,
-                                                 int* n_gt) {
-  const int tid = threadIdx.x;
-  uint32_t prefix = 0u;
-  int need = keep;  // keys still to take from the current prefix class
-  // (a rolled loop: this runs once per layer, so short code beats unrolled
-  // code, whose instructions would be fetched cold every time)
-#pragma unroll 1
-  for (int pass = 0; pass < 3; ++pass) {
-    const int sh = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
-    const int wd = pass < 2 ? 11 : 10;
-    const int nb = 1 << wd;
-    for (int i = tid; i < nb; i += kConsumers) hist[i] = 0;
-    cbar();
-    for (int q = tid; q < n; q += kConsumers) {
-      const uint32_t kv = keys[q + (q >> 5)];
-      const bool in_class = pass == 0 || (kv >> (sh + wd)) == prefix;
-      if (in_class) atomicAdd(&hist[(kv >> sh) & (uint32_t)(nb - 1)], 1);
-    }
-    cbar();
-    // thread t owns the bins [(255 - t) * per, (256 - t) * per): thread 0 the
-    // largest digits; an exclusive scan over t counts the keys above its bins
-    const int per = nb / kConsumers;
-    const int b_hi = (kConsumers - tid) * per;  // one past this thread's largest bin
-    int mine = 0;
-    for (int b = b_hi - per; b < b_hi; ++b) mine += hist[b];
-    int total;
-    const int above = block_excl_scan(mine, scratch, &total);
-    if (above < need && above + mine >= need) {
-      int acc = above;
-      for (int b = b_hi - 1; b >= b_hi - per; --b) {
-        const int h = hist[b];
-        if (acc + h >= need) {
-          scratch[kWarps + 1] = b;
-          scratch[kWarps + 2] = acc;  // keys of the class with a larger digit
-          break;
-        }
-        acc += h;
-      }
-    }
-    cbar();
-    const int d = scratch[kWarps + 1];
-    need -= scratch[kWarps + 2];
-    prefix = (prefix << wd) | (uint32_t)d;
-    cbar();  // scratch and hist are rewritten by the next pass
+// The channel select runs once per layer on 256 threads; its costs here are
+// shared-memory wavefronts, shared atomics (about three per cycle per SM),
+// warp collectives (30-60 cycles of latency, about 19 cycles apart when
+// independent) and divergent branches. So: few passes over the keys, branch-
+// free per-key code, ballots only where they do not chain.
+//
+// The loader places key q at keys[q], warp w loading candidates
+// [w * kw, (w + 1) * kw), kw = ceil(n / 8) rounded up to a multiple of 128.
+__device__ __forceinline__ int sel_kw(int n) { return (((n + kWarps - 1) / kWarps) + 127) & ~127; }
+
+// The select's own walk: thread t owns the contiguous chunk q in
+// [t * c, min(n, t * c + c)), c = ceil(n / 256) rounded up to a multiple of
+// 4 (at most 32), read as 16-byte words.
+__device__ __forceinline__ int sel_chunk(int n) { return ((n + kConsumers - 1) / kConsumers + 3) & ~3; }
+
+// Exclusive prefix over the warp's lanes of v < 2^NB, and the warp total,
+// from NB ballots that do not depend on one another (a shuffle scan would
+// chain five 50-cycle steps).
+template <int NB>
+__device__ __forceinline__ int warp_scan_bits(uint32_t v, int* total) {
+  const uint32_t lt = (1u << (threadIdx.x & 31)) - 1u;
+  uint32_t m[NB];
+#pragma unroll
+  for (int b = 0; b < NB; ++b) m[b] = __ballot_sync(0xffffffffu, (v >> b) & 1u);
+  int pre = 0, tot = 0;
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+    pre += __popc(m[b] & lt) << b;
+    tot += __popc(m[b]) << b;
   }
-  *n_gt = keep - need;
-  return prefix;
+  *total = tot;
+  return pre;
 }
 
-// Ordered compaction of the kept candidates over the 256 consumer threads:
-// candidate q (0 <= q < n, key at keys[q + q / 32]) is kept iff all, or its
-// key > T, or its key == T and fewer than r keys == T precede it. Thread t
-// visits q = 256 i + t; per row i each warp's ballots give its counts of
-// larger and equal keys, one block scan over the (row, warp) counts in row
-// order gives each warp's base, and a kept candidate's place in the
-// ascending list is (larger keys before it) + min(equal keys before it, r).
-// emit(pos, q) is called once per kept candidate. cnt: (n / 256 + 1) * kWarps
-// ints of scratch; scratch: kWarps + 1 ints.
-template <class Emit>
-__device__ __forceinline__ void compact_kept(const uint32_t* keys, int n, bool all, uint32_t T, int r, int* cnt,
-                                             int* scratch, Emit emit) {
+// A predicated shared-memory add of 1 (no branch around it).
+__device__ __forceinline__ void red_shared_add_if(bool p, int* addr) {
+  asm volatile("{ .reg .pred q; setp.ne.u32 q, %0, 0; @q red.shared.add.u32 [%1], 1; }" ::"r"((int)p), "r"(smem_u32(addr))
+               : "memory");
+}
+#ifndef CLK
+#define CLK(i)
+#endif
+// keys[q] = float_key(score of candidate q), candidate q = u * I + c being
+// channel c of unit u, row(u) its unit's I scores. With vec (I % 4 == 0 and
+// every row 16-byte aligned) each lane copies up to eight 16-byte groups of
+// its warp's range straight into shared memory (cp.async through L2, no
+// registers held), then turns its own groups into keys in place; otherwise a
+// rolled loop of four loads per lane. It also starts the select: sc[w] /
+// sc[8 + w] = min / max key of warp w's share, hist[0, kSelBins) and the
+// class-bit words zeroed. The caller synchronises before sel_kept.
+template <class Row>
+__device__ __forceinline__ void sel_load_keys(uint32_t* keys, int n, int I, bool vec, Row row, int* hist, int* sc) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int rows = (n + kConsumers - 1) / kConsumers;
-  const uint32_t lt = (1u << lane) - 1u;
-  for (int i = 0; i < rows; ++i) {
-    const int q = i * kConsumers + tid;
-    const uint32_t kk = q < n ? keys[q + (q >> 5)] : 0u;
-    const uint32_t bg = __ballot_sync(0xffffffffu, q < n && (all || kk > T));
-    const uint32_t be = __ballot_sync(0xffffffffu, q < n && !all && kk == T);
-    if (lane == 0) cnt[i * kWarps + warp] = __popc(bg) | (__popc(be) << 16);
+  const int kw = sel_kw(n);
+  const int q1 = min(n, (warp + 1) * kw);
+  const float invI = 1.0f / (float)I;
+  uint32_t mn = 0xffffffffu, mx = 0u;
+  if (vec) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int q = warp * kw + 4 * (lane + 32 * j);
+      if (q < q1) {
+        const int u = __float2int_rz(((float)q + 0.5f) * invI);
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(keys + q)), "l"(row(u) + (q - u * I))
+                     : "memory");
+      }
+    }
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int q = warp * kw + 4 * (lane + 32 * j);
+      if (q < q1) {
+        uint4 w = *reinterpret_cast<const uint4*>(keys + q);
+        w.x = float_key(__uint_as_float(w.x));
+        w.y = float_key(__uint_as_float(w.y));
+        w.z = float_key(__uint_as_float(w.z));
+        w.w = float_key(__uint_as_float(w.w));
+        mn = min(min(mn, min(w.x, w.y)), min(w.z, w.w));
+        mx = max(max(mx, max(w.x, w.y)), max(w.z, w.w));
+        *reinterpret_cast<uint4*>(keys + q) = w;
+      }
+    }
+  } else {
+#pragma unroll 1
+    for (int q0 = warp * kw + lane; q0 < q1; q0 += 128) {
+      float v[4];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const int q = q0 + 32 * t;
+        v[t] = 0.f;
+        if (q < q1) {
+          const int u = __float2int_rz(((float)q + 0.5f) * invI);
+          v[t] = __ldcg(row(u) + (q - u * I));
+        }
+      }
+#pragma unroll
+      for (int t = 0; t < 4; ++t)
+        if (q0 + 32 * t < q1) {
+          const uint32_t k = float_key(v[t]);
+          keys[q0 + 32 * t] = k;
+          mn = min(mn, k);
+          mx = max(mx, k);
+        }
+    }
   }
+  mn = __reduce_min_sync(0xffffffffu, mn);
+  mx = __reduce_max_sync(0xffffffffu, mx);
+  for (int b = tid; b < kSelBins; b += kConsumers) hist[b] = 0;
+  sc[160 + tid] = 0;
+  if (lane == 0) {
+    sc[warp] = (int)mn;
+    sc[kWarps + warp] = (int)mx;
+  }
+  if (tid == 0) sc[27] = 0;
+}
+
+// The kept channels of one token, exact: every key > T plus the first
+// keep - #{> T} keys == T in index order, T the keep-th largest key, listed
+// ascending through emit(pos, q). 0 < keep; n <= kMaxCand; keys and sc as
+// sel_load_keys left them, after a barrier.
+//  1. The class of keys that can still hold T starts as [min, max]. A pass
+//     counts the class's keys in up to 2048 equal power-of-two-wide bins over
+//     its range (predicated shared adds; the bins follow the data's own
+//     range, so keys spread over them); warp totals of the bins (thread t
+//     owns bins [8t, 8t + 8)) locate the warp, and a ballot scan the thread,
+//     whose bins hold the rank still needed: that bin becomes the class. At
+//     most three passes, typically one; they stop once the class holds at
+//     most 64 keys or one value.
+//  2. One branch-free pass marks each thread's keys above the class (a
+//     32-bit mask per thread) and its class keys.
+//  3. A class of one value: its first `need` keys in index order are kept
+//     (ballot scan of the per-thread counts). Otherwise the class keys are
+//     gathered (a shared counter) and thread t < cnt ranks class key t
+//     against the class: T and, among keys == T, the index order; kept class
+//     keys set their bit in their owner's word.
+//  4. Positions: a ballot scan of the per-thread kept counts, one barrier for
+//     the warp totals, then each thread emits its set bits in order.
+template <class Emit>
+__device__ __forceinline__ void sel_kept(const uint32_t* keys, int n, int keep, int* hist, int* sc, Emit emit) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int c = sel_chunk(n);
+  const int q0 = tid * c, q1 = min(n, q0 + c);
+  const int nq = max(0, q1 - q0);
+  const uint4* kp = reinterpret_cast<const uint4*>(keys + q0);
+  int* xm = sc + 160;  // [256] kept bits of class keys, per owning thread
+  uint32_t mask = 0u;  // bit i: candidate q0 + i kept
+  if (keep >= n) {
+    mask = nq >= 32 ? 0xffffffffu : ((1u << nq) - 1u);
+  } else {
+    uint32_t lo = (uint32_t)sc[0], hi = (uint32_t)sc[kWarps];
+#pragma unroll
+    for (int w = 1; w < kWarps; ++w) {
+      lo = min(lo, (uint32_t)sc[w]);
+      hi = max(hi, (uint32_t)sc[kWarps + w]);
+    }
+    int need = keep;  // rank of T inside the class [lo, hi]
+    int cnt = n;      // keys in the class
+    // 2. histogram passes until the class is small or one value
+#pragma unroll 1
+    for (int pass = 0; pass < 3 && lo != hi && cnt > kSelGather; ++pass) {
+      int* h = hist + (pass & 1) * kSelBins;
+      int* hn = hist + ((pass + 1) & 1) * kSelBins;
+      const int sh = max(0, 32 - __clz(hi - lo) - 11);
+#pragma unroll 2
+      for (int j = 0; 4 * j < nq; ++j) {
+        const uint4 w = kp[j];
+        const uint32_t e[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const bool ok = 4 * j + t < nq && e[t] >= lo && e[t] <= hi;
+          red_shared_add_if(ok, &h[ok ? (e[t] - lo) >> sh : 0]);
+        }
+      }
+      for (int b = tid; b < kSelBins; b += kConsumers) hn[b] = 0;
+      cbar();
+      const int4 c0 = reinterpret_cast<const int4*>(h)[2 * tid];
+      const int4 c1 = reinterpret_cast<const int4*>(h)[2 * tid + 1];
+      const int mine = c0.x + c0.y + c0.z + c0.w + c1.x + c1.y + c1.z + c1.w;
+      const int wsum = __reduce_add_sync(0xffffffffu, mine);
+      if (lane == 0) sc[16 + warp] = wsum;
+      cbar();
+      int W = -1, wabove = 0;
+      {
+        int acc = 0;
+#pragma unroll
+        for (int w = kWarps - 1; w >= 0; --w) {
+          const int t = sc[16 + w];
+          if (W < 0 && acc + t >= need) {
+            W = w;
+            wabove = acc;
+          }
+          acc += t;
+        }
+      }
+      if (warp == W) {
+        const uint32_t gtm = ~((2u << lane) - 1u);
+        uint32_t m[14];
+#pragma unroll
+        for (int b = 0; b < 14; ++b) m[b] = __ballot_sync(0xffffffffu, ((uint32_t)mine >> b) & 1u);
+        int above = wabove;
+#pragma unroll
+        for (int b = 0; b < 14; ++b) above += __popc(m[b] & gtm) << b;
+        if (above < need && above + mine >= need) {
+          const int cv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+          int acc = above, dj = 0, aj = 0, cj = 0;
+          bool found = false;
+#pragma unroll
+          for (int j = 7; j >= 0; --j)
+            if (!found) {
+              if (acc + cv[j] >= need) {
+                found = true;
+                dj = 8 * tid + j;
+                aj = acc;
+                cj = cv[j];
+              } else {
+                acc += cv[j];
+              }
+            }
+          sc[24] = dj;
+          sc[25] = aj;
+          sc[26] = cj;
+        }
+      }
+      cbar();
+      const uint32_t d = (uint32_t)sc[24];
+      need -= sc[25];
+      cnt = sc[26];
+      lo += d << sh;
+      hi = min(hi, lo + ((1u << sh) - 1u));
+    }
+    // 3. classify: keys above the class are kept; the class's keys are
+    // gathered (at most kSelGather of them unless the class is one value)
+    uint32_t cm = 0u;  // this thread's class keys
+#pragma unroll 2
+    for (int j = 0; 4 * j < nq; ++j) {
+      const uint4 w = kp[j];
+      const uint32_t e[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const int i = 4 * j + t;
+        const bool ok = i < nq;
+        mask |= (ok && e[t] > hi) ? (1u << i) : 0u;
+        cm |= (ok && e[t] >= lo && e[t] <= hi) ? (1u << i) : 0u;
+      }
+    }
+    if (lo == hi) {
+      // one value T = lo: its first `need` keys in index order are kept
+      int tot;
+      int pre = warp_scan_bits<6>((uint32_t)__popc(cm), &tot);
+      if (lane == 0) sc[16 + warp] = tot;
+      cbar();
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w)
+        if (w < warp) pre += sc[16 + w];
+      for (int take = need - pre; cm != 0u && take > 0; --take) {
+        mask |= cm & (0u - cm);  // lowest remaining class key
+        cm &= cm - 1u;
+      }
+    } else {
+      // gather the class (at most kSelGather keys)
+      while (cm != 0u) {
+        const int i = __ffs(cm) - 1;
+        cm &= cm - 1u;
+        const int sl = atomicAdd(&sc[27], 1);
+        if (sl < kSelGather) {
+          sc[32 + sl] = (int)keys[q0 + i];
+          sc[96 + sl] = q0 + i;
+        }
+      }
+      cbar();
+      // threads t < cnt rank class key t against the whole class: T is the
+      // key with fewer than need larger and at least need larger-or-equal
+      // class keys (any such thread writes the same T); of the keys == T
+      // the first need - #{> T} in index order are kept
+      const bool ac = tid < cnt;
+      const uint32_t v = ac ? (uint32_t)sc[32 + tid] : 0u;
+      const int iv = ac ? sc[96 + tid] : 0;
+      int g = 0, e = 0;
+      if (ac) {
+#pragma unroll 1
+        for (int m = 0; m < cnt; m += 4) {
+          const int4 o4 = *reinterpret_cast<const int4*>(sc + 32 + m);
+          const uint32_t o[4] = {(uint32_t)o4.x, (uint32_t)o4.y, (uint32_t)o4.z, (uint32_t)o4.w};
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            g += (m + t < cnt && o[t] > v) ? 1 : 0;
+            e += (m + t < cnt && o[t] >= v) ? 1 : 0;
+          }
+        }
+        if (g < need && e >= need) {
+          sc[28] = (int)v;
+          sc[29] = g;
+        }
+      }
+      cbar();
+      if (ac) {
+        const uint32_t T = (uint32_t)sc[28];
+        const int r = need - sc[29];  // keys == T to keep
+        bool kept = v > T;
+        if (v == T) {
+          int t0 = 0;
+#pragma unroll 1
+          for (int m = 0; m < cnt; m += 4) {
+            const int4 o4 = *reinterpret_cast<const int4*>(sc + 32 + m);
+            const int4 p4 = *reinterpret_cast<const int4*>(sc + 96 + m);
+            const uint32_t o[4] = {(uint32_t)o4.x, (uint32_t)o4.y, (uint32_t)o4.z, (uint32_t)o4.w};
+            const int oq[4] = {p4.x, p4.y, p4.z, p4.w};
+#pragma unroll
+            for (int t = 0; t < 4; ++t) t0 += (m + t < cnt && o[t] == T && oq[t] < iv) ? 1 : 0;
+          }
+          kept = t0 < r;
+        }
+        if (kept) atomicOr(&xm[iv / c], 1 << (iv % c));
+      }
+      cbar();
+      mask |= (uint32_t)xm[tid];
+    }
+  }
+  // 4. positions: exclusive prefix of the per-thread kept counts
+  int tot;
+  int pos = warp_scan_bits<6>((uint32_t)__popc(mask), &tot);
+  if (lane == 0) sc[16 + warp] = tot;
   cbar();
-  const int m = rows * kWarps;  // <= 256 entries, one per thread
-  const int v = tid < m ? cnt[tid] : 0;
-  int total;
-  const int pre = block_excl_scan(v, scratch, &total);
-  if (tid < m) cnt[tid] = pre;  // each thread rewrites only the entry it read
-  cbar();
-  for (int i = 0; i < rows; ++i) {
-    const int q = i * kConsumers + tid;
-    const uint32_t kk = q < n ? keys[q + (q >> 5)] : 0u;
-    const bool g = q < n && (all || kk > T);
-    const bool e = q < n && !all && kk == T;
-    const uint32_t bg = __ballot_sync(0xffffffffu, g);
-    const uint32_t be = __ballot_sync(0xffffffffu, e);
-    const int base = cnt[i * kWarps + warp];
-    const int pg = (base & 0xffff) + __popc(bg & lt), pe = (base >> 16) + __popc(be & lt);
-    if (g || (e && pe < r)) emit(pg + min(pe, r), q);
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w)
+    if (w < warp) pos += sc[16 + w];
+  while (mask) {
+    const int b = __ffs(mask) - 1;
+    emit(pos++, q0 + b);
+    mask &= mask - 1u;
   }
 }
 
@@ -272,20 +505,32 @@ __device__ __forceinline__ void warp_weights(const float* l, int k, float* w) {
 
 // Cross-warp sum of per-warp output accumulators (64 per lane, element
 // 256 c + 8 lane + e in acc[8 c + e]) into ysum (element 256 c + 8 lane + e
-// at 256 c + 32 e + lane): at step st warp W adds its chunk (W + st) % 8, so
-// no two warps touch a chunk at once; one barrier per step. W is a template
-// argument so that every register index is a constant. (The accumulators
-// are zeroed by the caller just before the next layer's first job that adds
-// to them, so that they are not live through routing and selection.)
-template <int W>
-__device__ __forceinline__ void ysum_steps(float (&acc)[64], float* ysum, int lane) {
+// at 256 c + 32 e + lane): at step st warp w adds its chunk (w + st) % 8, so
+// no two warps touch a chunk at once; one barrier per step. Every warp runs
+// the same code (a switch picks the chunk, so that every register index is a
+// constant): it runs once per layer, and one shared copy is fetched once
+// instead of eight. (The accumulators are zeroed by the caller just before
+// the next layer's first job that adds to them, so that they are not live
+// through routing and selection.)
+template <int C>
+__device__ __forceinline__ void ysum_chunk(const float (&acc)[64], float* ysum, int lane, bool first) {
+  float* yc = ysum + 256 * C + lane;
 #pragma unroll
+  for (int e = 0; e < 8; ++e) yc[32 * e] = first ? acc[8 * C + e] : yc[32 * e] + acc[8 * C + e];
+}
+__device__ __forceinline__ void ysum_all(const float (&acc)[64], float* ysum, int lane, int warp) {
+#pragma unroll 1
   for (int st = 0; st < 8; ++st) {
-    const int c = (W + st) & 7;
-    float* yc = ysum + 256 * c + lane;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      yc[32 * e] = st == 0 ? acc[8 * c + e] : yc[32 * e] + acc[8 * c + e];
+    const bool first = st == 0;
+    switch ((warp + st) & 7) {
+      case 0: ysum_chunk<0>(acc, ysum, lane, first); break;
+      case 1: ysum_chunk<1>(acc, ysum, lane, first); break;
+      case 2: ysum_chunk<2>(acc, ysum, lane, first); break;
+      case 3: ysum_chunk<3>(acc, ysum, lane, first); break;
+      case 4: ysum_chunk<4>(acc, ysum, lane, first); break;
+      case 5: ysum_chunk<5>(acc, ysum, lane, first); break;
+      case 6: ysum_chunk<6>(acc, ysum, lane, first); break;
+      default: ysum_chunk<7>(acc, ysum, lane, first); break;
     }
     cbar();
   }
@@ -403,10 +648,11 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
   // warp routes alone, with no CTA barrier, while the other warps go on
   // with their jobs. Lane l polls words 64q + 2l and 64q + 2l + 1 (q < 4;
   // the warp's four 16-byte loads cover the 2 KB once) until all carry the
-  // layer's tag, then the k largest are taken by k rounds of a warp-wide
-  // argmax (ties: the lower expert index), followed by the softmax over the
-  // k and the units in ascending expert id. Returns false on a poll timeout.
-  // A logit whose key is 0 (a NaN with every bit set) is never selected.
+  // layer's tag, then the k largest are taken by k rounds over per-lane
+  // sorted lists (ties: the lower expert index), followed by the softmax over
+  // the k and the units in ascending expert id. Returns false on a poll
+  // timeout. Warp-wide steps cost 30-60 cycles each here, so each round has
+  // two on its dependent path and the rest stays in registers.
   auto route_warp = [&](int lay) -> bool {
     const unsigned long long* wb = reinterpret_cast<const unsigned long long*>(p.logits);
     const uint32_t want = 0x80000000u | (ltag_s + (uint32_t)lay);
@@ -441,44 +687,62 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
       if (__all_sync(0xffffffffu, all)) break;
       if (__any_sync(0xffffffffu, clock64() - t0 > budget)) return false;  // warp-uniform
     }
-    // slot s of lane l holds expert 64 (s / 2) + 2 l + s % 2: slots in
-    // ascending index order, so a strict > keeps the lowest index of a tie
-    auto slot_idx = [&](int s) { return 64 * (s >> 1) + 2 * lane + (s & 1); };
-    uint32_t bk = key[0];
-    int bs = 0;
+    // Slot s of lane l holds expert 64 (s / 2) + 2 l + s % 2. Each lane
+    // sorts its 8 slots best first as 64-bit values key << 32 | ~expert
+    // (larger key, then lower index; empty slots 0) with a 19-comparator
+    // network; then each of the k rounds takes the best head over the warp
+    // (one max reduction over the head keys and one ballot; a second
+    // reduction, on the index, only when several heads tie) and the winner
+    // drops its head. Every lane follows the chosen keys, so the softmax
+    // needs no exchange.
+    unsigned long long v[8];
 #pragma unroll
-    for (int s = 1; s < 8; ++s)
-      if (key[s] > bk) { bk = key[s]; bs = s; }
+    for (int s = 0; s < 8; ++s) {
+      const int e = 64 * (s >> 1) + 2 * lane + (s & 1);
+      v[s] = e < E ? (((unsigned long long)key[s] << 32) | (unsigned long long)(~(uint32_t)e)) : 0ull;
+    }
+    auto cas = [&](int i, int j) {
+      const unsigned long long a = v[i], b = v[j];
+      v[i] = a < b ? b : a;
+      v[j] = a < b ? a : b;
+    };
+    cas(0, 1); cas(2, 3); cas(4, 5); cas(6, 7);
+    cas(0, 2); cas(1, 3); cas(4, 6); cas(5, 7);
+    cas(1, 2); cas(5, 6);
+    cas(0, 4); cas(1, 5); cas(2, 6); cas(3, 7);
+    cas(2, 4); cas(3, 5);
+    cas(1, 2); cas(3, 4); cas(5, 6);
+    float m0 = 0.f, esum = 0.f, my_e = 0.f;
     for (int r = 0; r < k; ++r) {
-      const uint32_t M = __reduce_max_sync(0xffffffffu, bk);
-      const uint32_t tie = __ballot_sync(0xffffffffu, bk == M);
-      int wl = __ffs(tie) - 1;
+      const uint32_t hk = (uint32_t)(v[0] >> 32);
+      const uint32_t M = __reduce_max_sync(0xffffffffu, hk);
+      uint32_t tie = __ballot_sync(0xffffffffu, hk == M);
       if (tie & (tie - 1)) {
-        // several lanes hold M: the lowest expert index wins
-        const uint32_t mi = __reduce_min_sync(0xffffffffu, bk == M ? (uint32_t)slot_idx(bs) : 0xffffffffu);
-        wl = __ffs(__ballot_sync(0xffffffffu, bk == M && (uint32_t)slot_idx(bs) == mi)) - 1;
+        // several heads hold the key M: the lowest expert index wins
+        const uint32_t lo = __reduce_max_sync(0xffffffffu, hk == M ? (uint32_t)v[0] : 0u);
+        tie = __ballot_sync(0xffffffffu, hk == M && (uint32_t)v[0] == lo);
       }
-      if (lane == wl) {
+      const bool win = lane == __ffs(tie) - 1;
+      if (win) {
         cand_key[kWarps + r] = M;
-        cand_idx[r] = slot_idx(bs);
-#pragma unroll
-        for (int s = 0; s < 8; ++s)
-          if (s == bs) key[s] = 0u;
-        bk = key[0];
-        bs = 0;
-#pragma unroll
-        for (int s = 1; s < 8; ++s)
-          if (key[s] > bk) { bk = key[s]; bs = s; }
+        cand_idx[r] = (int)~(uint32_t)v[0];
       }
+#pragma unroll
+      for (int s = 0; s < 7; ++s) v[s] = win ? v[s + 1] : v[s];
+      v[7] = win ? 0ull : v[7];
+      const float lm = key_float(M);
+      if (r == 0) m0 = lm;
+      const float er = __expf(lm - m0);
+      esum += er;
+      if (lane == r) my_e = er;
     }
     __syncwarp();
     const bool sel = lane < k;
-    const uint32_t kc = sel ? cand_key[kWarps + lane] : 0u;
     const int ic = sel ? cand_idx[lane] : 0x7fffffff;
-    const float e = sel ? __expf(key_float(kc) - key_float(cand_key[kWarps])) : 0.f;
-    const float wl = e / warp_sum(e);
+    const float wl = my_e / esum;
     int urank = 0;
-    for (int m = 0; m < k; ++m) urank += cand_idx[m] < ic;
+#pragma unroll
+    for (int m = 0; m < 8; ++m) urank += (m < k && cand_idx[m] < ic) ? 1 : 0;
     if (sel) {
       rs.ids[0][lane] = ic;
       rs.w[0][lane] = wl;
@@ -1865,13 +2129,10 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
 
     // ---- channel-sparse selection (B = 1): kept[] ascending, rs.ncand
     // Candidate q = u * I + c (routed unit u in ascending expert order,
-    // channel c). The keep-th largest key T is found bit by bit below the
-    // common prefix of all keys (count of keys >= T | bit, one warp reduction
-    // and one barrier per bit, keys held in registers); the kept set is every
-    // key > T plus the first r keys == T in index order (r = keep - #{> T}).
-    // The ascending list comes from contiguous per-thread chunks and one
-    // prefix scan. Keys sit in shared memory at q + q / 32 (conflict-free for
-    // both the row and the chunk walks).
+    // channel c). The keys are loaded into shared memory (sel_load_keys);
+    // sel_kept finds the keep-th largest key T by histogram passes over the
+    // keys' own range and lists the kept set (every key > T plus the first
+    // keep - #{> T} keys == T in index order) ascending.
     // ---- weight-only channel screen of layer l inside the stack ([Reader]
     // "가중치만으로 만든 reader", steps 1-2, eq. 1): every CTA rotates u (fp32
     // butterfly per block of 128, u_x = H_128 (s * u), in the keys buffer,
@@ -1962,49 +2223,23 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
 
     auto select_channels = [&](int l) {
       const int N = rs.U * I;
-      const int rows = (N + kConsumers - 1) / kConsumers;
       const float* sc = SCREEN ? p.scr : p.layer[l].scores;
-      const float invI = 1.0f / (float)I;
-      auto pad = [](int q) { return q + (q >> 5); };
-      // 1. keys: row-major q = i * 256 + tid, stored at keys[q + q / 32]
-      // (conflict-free for the row walks); a rolled loop with four loads in
-      // flight (short code: it runs once per layer)
-#pragma unroll 1
-      for (int i0 = 0; i0 < rows; i0 += 4) {
-        float kv[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int q = (i0 + i) * kConsumers + tid;
-          kv[i] = 0.f;
-          if (i0 + i < rows && q < N) {
-            const int u = __float2int_rz(((float)q + 0.5f) * invI);
-            kv[i] = __ldcg(sc + (size_t)rs.unit_e[u] * I + (q - u * I));  // written in this launch when screened
-          }
-        }
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int q = (i0 + i) * kConsumers + tid;
-          if (i0 + i < rows && q < N) keys[pad(q)] = float_key(kv[i]);
-        }
-      }
+      int* hist = reinterpret_cast<int*>(smem + p.off_hist);
+      int* ssc = hist + 2 * kSelBins;
+      // 1. the candidates' keys (written in this launch when screened: read
+      // through L2)
+      const bool vec = (I & 3) == 0 && ((uintptr_t)sc & 15u) == 0;
+      sel_load_keys(keys, N, I, vec, [&](int u) { return sc + (size_t)rs.unit_e[u] * I; }, hist, ssc);
       const int keep = p.keep;
-      const bool all = keep >= N;
-      uint32_t T = 0u;
-      int r = 0;
       cbar();
-      if (keep > 0 && !all) {
-        // 2. the keep-th largest key T and the count of keys above it
-        int n_gt = 0;
-        T = radix_select(keys, N, keep, reinterpret_cast<int*>(smem + p.off_hist), rs.scan + 32, &n_gt);
-        r = keep - n_gt;
-      }
-      cbar();  // keys[] complete
-      // 4. the kept list, ascending (ballot compaction)
-      if (keep > 0)
-        compact_kept(keys, N, all, T, r, rs.scan, reinterpret_cast<int*>(smem + p.off_hist), [&](int pos, int q) {
+      // 2. the kept list, ascending
+      if (keep > 0) {
+        const float invI = 1.0f / (float)I;
+        sel_kept(keys, N, keep, hist, ssc, [&](int pos, int q) {
           const int u = __float2int_rz(((float)q + 0.5f) * invI);
           kept[pos] = rs.unit_e[u] * I + (q - u * I);
         });
+      }
       if (tid == 0) rs.ncand = keep > 0 ? min(N, keep) : 0;
       cbar();
       // sectors: each kept channel's byte range, less a sector shared with
@@ -2247,16 +2482,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
         // lane), so no two warps touch a chunk at once; then thread t adds
         // elements 8t..8t+7 to the L2 accumulator
         float* ysum = reinterpret_cast<float*>(smem + p.off_ysum);
-        switch (warp) {
-          case 0: ysum_steps<0>(accf, ysum, lane); break;
-          case 1: ysum_steps<1>(accf, ysum, lane); break;
-          case 2: ysum_steps<2>(accf, ysum, lane); break;
-          case 3: ysum_steps<3>(accf, ysum, lane); break;
-          case 4: ysum_steps<4>(accf, ysum, lane); break;
-          case 5: ysum_steps<5>(accf, ysum, lane); break;
-          case 6: ysum_steps<6>(accf, ysum, lane); break;
-          default: ysum_steps<7>(accf, ysum, lane); break;
-        }
+        ysum_all(accf, ysum, lane, warp);
         float v[8];
         {
           const float* yt = ysum + 256 * (tid >> 5) + (tid & 31);
