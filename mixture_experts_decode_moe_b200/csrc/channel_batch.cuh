@@ -149,23 +149,30 @@ __global__ void __launch_bounds__(kCbThreads, 1) channel_batch_kernel(const __gr
       });
     cbar();  // the kept list is complete (global writes of this CTA, ordered by the barrier)
     // sectors of the token's kept channels (channel-major ranges, a sector
-    // shared with the previous kept channel counted once)
+    // shared with the previous kept channel counted once; channels that
+    // start and end on 32-byte boundaries share none)
     const unsigned long long base = (unsigned long long)(uintptr_t)p.cm;
-    uint32_t sec = 0;
     const int nk = keep < N ? keep : N;
-    for (int i = tid; i < nk; i += kCbConsumers) {
-      const unsigned long long s0 = (base + (unsigned long long)kws[i] * cb) >> 5;
-      const unsigned long long s1 = (base + (unsigned long long)(kws[i] + 1) * cb - 1) >> 5;
-      sec += (uint32_t)(s1 - s0 + 1);
-      if (i > 0 && ((base + (unsigned long long)(kws[i - 1] + 1) * cb - 1) >> 5) == s0) sec -= 1;
+    if (((base | (unsigned long long)cb) & 31ull) == 0) {
+      if (tid == 0) p.sectors[b] = (unsigned long long)nk * ((unsigned long long)cb >> 5);
+    } else {
+      uint32_t sec = 0;
+      for (int i = tid; i < nk; i += kCbConsumers) {
+        const unsigned long long s0 = (base + (unsigned long long)kws[i] * cb) >> 5;
+        const unsigned long long s1 = (base + (unsigned long long)(kws[i] + 1) * cb - 1) >> 5;
+        sec += (uint32_t)(s1 - s0 + 1);
+        if (i > 0 && ((base + (unsigned long long)(kws[i - 1] + 1) * cb - 1) >> 5) == s0) sec -= 1;
+      }
+      sec = __reduce_add_sync(0xffffffffu, sec);
+      if (lane == 0) red_s[warp] = sec;
+      cbar();
+      if (tid == 0) {
+        unsigned long long t = 0;
+        for (int w = 0; w < kWarps; ++w) t += red_s[w];
+        p.sectors[b] = t;
+      }
     }
-    sec = __reduce_add_sync(0xffffffffu, sec);
-    if (lane == 0) red_s[warp] = sec;
-    cbar();
     if (tid == 0) {
-      unsigned long long t = 0;
-      for (int w = 0; w < kWarps; ++w) t += red_s[w];
-      p.sectors[b] = t;
       if (bad_s) set_status(ctl, kStatusBadIds);
     }
   }

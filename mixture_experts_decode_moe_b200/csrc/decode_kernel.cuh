@@ -563,6 +563,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ RouteSmem<BMAX> rs;
   __shared__ int route_ready_s, prod_layer_s[kProducers], abort_s, bad_s, okw_s;
+  __shared__ int units_s;  // planar batch 1: layer * 64 + units of its routing published so far
   __shared__ uint32_t ltag_s;  // logit tag of layer 0 in this launch (fast path)
   __shared__ unsigned long long bar_base_s;  // grid-barrier count at launch (a multiple of G)
   __shared__ long long budget_s;  // cycles per bounded wait (the workspace's budget)
@@ -605,6 +606,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
     }
     fence_mbar_init();
     route_ready_s = -1;  // last layer whose routing the consumers published
+    units_s = -1;
     for (int q = 0; q < kProducers; ++q) {
       prod_layer_s[q] = -1;  // last layer whose routed jobs producer q issued
       jp_s[q] = 0;           // jobs producer q has passed (its own ones issued)
@@ -724,8 +726,16 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
       }
       const bool win = lane == __ffs(tie) - 1;
       if (win) {
+        const int ew = (int)~(uint32_t)v[0];
         cand_key[kWarps + r] = M;
-        cand_idx[r] = (int)~(uint32_t)v[0];
+        cand_idx[r] = ew;
+        if (warp_routes) {
+          // planar: unit r is the r-th chosen expert, published at once so
+          // that the producers can start its copies during the next rounds
+          rs.unit_e[r] = ew;
+          rs.unit_mask[r] = 1u;
+          st_release_cta(&units_s, lay * 64 + r + 1);
+        }
       }
 #pragma unroll
       for (int s = 0; s < 7; ++s) v[s] = win ? v[s + 1] : v[s];
@@ -740,9 +750,14 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
     const bool sel = lane < k;
     const int ic = sel ? cand_idx[lane] : 0x7fffffff;
     const float wl = my_e / esum;
-    int urank = 0;
+    // units: the chosen order (planar, published above) or ascending expert
+    // id (channel-major, whose candidate order must follow the channel ids)
+    int urank = lane;
+    if (!warp_routes) {
+      urank = 0;
 #pragma unroll
-    for (int m = 0; m < 8; ++m) urank += (m < k && cand_idx[m] < ic) ? 1 : 0;
+      for (int m = 0; m < 8; ++m) urank += (m < k && cand_idx[m] < ic) ? 1 : 0;
+    }
     if (sel) {
       rs.ids[0][lane] = ic;
       rs.w[0][lane] = wl;
@@ -858,6 +873,22 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
       }
       if (lane == 0) jdesc[slot] = jb;
       return slot;
+    };
+    // planar batch 1: until units_s (layer * 64 + units published) reaches
+    // want; lane 0 polls, the warp learns the outcome; false on an abort or
+    // when the wait runs out
+    auto wait_units = [&](int want) -> bool {
+      int ok = 1;
+      if (lane == 0) {
+        const long long tw = clock64();
+        while (*(volatile int*)&units_s < want)
+          if (*(volatile int*)&abort_s || clock64() - tw > budget) {
+            ok = 0;
+            break;
+          }
+        (void)ld_acquire_cta(&units_s);
+      }
+      return __shfl_sync(0xffffffffu, ok, 0) != 0;
     };
     auto next_stage = [&]() {
       ++lq;
@@ -1047,7 +1078,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
           next_stage();
         }
       }
-      {
+      if (!warp_routes) {
         // routing of layer l (plain polls with short sleeps, then one acquire)
         const long long t0 = clock64();
         while (*(volatile int*)&route_ready_s < l) {
@@ -1063,6 +1094,11 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
         int idx = held;
         held = -1;
         if (idx < 0) {
+          // a grab without one held from the previous layer (layer 0): on
+          // the planar batch-1 path nothing else orders it after the launch's
+          // reset of the pools, so wait for the layer's first unit, which is
+          // published after that reset's grid barrier
+          if (warp_routes && !wait_units(l * 64 + 1)) goto producer_done;
           unsigned v = 0;
           if (lane == 0) v = atomicAdd(&ctl->pool[l % 3], 1u);
           idx = (int)__shfl_sync(0xffffffffu, v, 0);
@@ -1088,6 +1124,9 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
         }
         const int slot = take_stage(jb);
         if (slot < 0) goto producer_done;
+        // planar batch 1: wait only for this job's units (published one by
+        // one during the top-k), not for the whole routing
+        if (warp_routes && !wait_units(l * 64 + (ch0 + n - 1) / I + 1)) goto producer_done;
         if (lane == 0) {
           uint64_t* bar = &full[slot];
           uint8_t* dst = ring + (size_t)slot * p.stage_bytes;
@@ -2242,26 +2281,33 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
       }
       if (tid == 0) rs.ncand = keep > 0 ? min(N, keep) : 0;
       cbar();
-      // sectors: each kept channel's byte range, less a sector shared with
-      // the previous kept channel; per-warp sums, then one add per warp
-      const unsigned long long base = (unsigned long long)(uintptr_t)p.layer[l].gate;
-      const unsigned long long cb = 3ull * rowb;
-      uint32_t sec = 0;
-      for (int i = tid; i < rs.ncand; i += kConsumers) {
-        const unsigned long long s0 = (base + (unsigned long long)kept[i] * cb) >> 5;
-        const unsigned long long s1 = (base + (unsigned long long)(kept[i] + 1) * cb - 1) >> 5;
-        sec += (uint32_t)(s1 - s0 + 1);
-        if (i > 0 && ((base + (unsigned long long)(kept[i - 1] + 1) * cb - 1) >> 5) == s0) sec -= 1;
+      // sectors (reported by CTA 0 only): each kept channel's byte range,
+      // less a sector shared with the previous kept channel; channels that
+      // start and end on 32-byte boundaries share none
+      if (cta == 0 && p.sectors_out != nullptr) {
+        const unsigned long long base = (unsigned long long)(uintptr_t)p.layer[l].gate;
+        const unsigned long long cb = 3ull * rowb;
+        if (((base | cb) & 31ull) == 0) {
+          if (tid == 0) rs.sectors = (unsigned long long)rs.ncand * (cb >> 5);
+        } else {
+          uint32_t sec = 0;
+          for (int i = tid; i < rs.ncand; i += kConsumers) {
+            const unsigned long long s0 = (base + (unsigned long long)kept[i] * cb) >> 5;
+            const unsigned long long s1 = (base + (unsigned long long)(kept[i] + 1) * cb - 1) >> 5;
+            sec += (uint32_t)(s1 - s0 + 1);
+            if (i > 0 && ((base + (unsigned long long)(kept[i - 1] + 1) * cb - 1) >> 5) == s0) sec -= 1;
+          }
+          sec = __reduce_add_sync(0xffffffffu, sec);
+          if (lane == 0) rs.scan[warp] = (int)sec;
+          cbar();
+          if (tid == 0) {
+            unsigned long long t = 0;
+            for (int w = 0; w < kWarps; ++w) t += (uint32_t)rs.scan[w];
+            rs.sectors = t;
+          }
+          cbar();
+        }
       }
-      sec = __reduce_add_sync(0xffffffffu, sec);
-      if (lane == 0) rs.scan[warp] = (int)sec;
-      cbar();
-      if (tid == 0) {
-        unsigned long long t = 0;
-        for (int w = 0; w < kWarps; ++w) t += (uint32_t)rs.scan[w];
-        rs.sectors = t;
-      }
-      cbar();
     };
 
     bool failed = false;
@@ -2437,6 +2483,23 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
         for (int i = 0; i < own_shared && !fl; ++i) fl = consume_pipe() != JOB_SHARED;
         if (l + 1 < p.L)
           for (int i = 0; i < own_pred && !fl; ++i) fl = consume_pipe() != JOB_ROUTER;
+        if (warp_routes && !fl) {
+          // the routed copies may start before the routing is complete (its
+          // units are published one by one); their weights come last
+          int ok = 1;
+          if (lane == 0) {
+            const long long tw = clock64();
+            while (*(volatile int*)&route_ready_s < l)
+              if (*(volatile int*)&abort_s || clock64() - tw > budget) {
+                ok = 0;
+                break;
+              }
+            (void)ld_acquire_cta(&route_ready_s);
+          }
+          __syncwarp();
+          fl = !__shfl_sync(0xffffffffu, ok, 0);
+          if (fl && lane == 0 && !*(volatile int*)&abort_s) set_status(ctl, kStatusTimeout);
+        }
         for (int it = 0; !fl; ++it) {
           const int ty = consume_pipe();
           if (ty == JOB_END) break;
