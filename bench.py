@@ -473,7 +473,7 @@ class ChannelBatch:
         self.tokens_per_step = B
         self.launches_per_step = nl
         self.kernel = f"channel_batch_kernel<B{B}> x {nl} layers"
-        self.sources = ("common.cuh", "decode.cuh", "decode_kernel.cuh", "channel_batch.cuh")
+        self.sources = DECODE_KERNEL_SOURCES + ("channel_batch.cuh",)
         self.dtype = "bf16"
         self.record = 0
 
@@ -844,7 +844,7 @@ def run_ours(args):
 
 # the sources decode_kernel is compiled from: a recorded DRAM traffic figure
 # stays valid while these are unchanged
-DECODE_KERNEL_SOURCES = ("common.cuh", "decode.cuh", "decode_kernel.cuh")
+DECODE_KERNEL_SOURCES = ("common.cuh", "decode.cuh", "screen_lut.cuh", "decode_kernel.cuh")
 LINEAR_KERNEL_SOURCES = ("common.cuh", "small_kernels.cuh", "linear.cuh")
 
 

@@ -217,7 +217,8 @@ moe_status moe_channel_topk_forward(const moe_layer_desc* desc, const void* x, i
                                     unsigned long long* union_sectors_opt,
                                     void* ws, size_t ws_bytes, moe_stream_t stream);
 
-/* One layer's channel-screen sketch (the buffers moe_reader_build writes). */
+/* One layer's channel-screen sketch (the buffers moe_reader_build writes);
+ * codes 16-byte, scales and dnorm 4-byte aligned, else MOE_ERR_INVALID. */
 typedef struct {
   const uint32_t* codes;   /* [E*I][2][H/16] 2-bit codes */
   const uint16_t* scales;  /* [E*I][2][H/128] fp16 bit patterns */
@@ -327,7 +328,9 @@ moe_status moe_reader_build(const moe_layer_desc* desc, const int8_t* signs, uin
  * routed experts e = ids[b, slot] (w[b, slot] its router weight), writes
  * scores[b, e, c] for c < I; rows of experts token b did not route to, and
  * of ids outside [0, E), are not written. est_opt [B, k, I, 2] fp32 receives {g_hat, v_hat} (or NULL).
- * x [B, H] bf16 is the expert input (the normalised x under pre-norm). */
+ * x [B, H] bf16 is the expert input (the normalised x under pre-norm).
+ * Here codes must be 16-byte and scales 4-byte aligned (the screen copies
+ * them with 16- and 4-byte pieces), else MOE_ERR_INVALID. */
 moe_status moe_reader_screen(const moe_layer_desc* desc, const void* x, int32_t B, const int32_t* ids,
                              const float* w, const int8_t* signs, const uint32_t* codes,
                              const uint16_t* scales, const float* dnorm, float* scores, float* est_opt,

@@ -147,7 +147,7 @@ bool plan_smem(DecodeParams* p, int static_bytes, bool fast) {
   // keys: router top-k keys [B*E] and channel-sparse candidates [k*I]
   size_t nkeys = (p->mode == MODE_LAYERS) ? (size_t)B * p->E : 0;
   if (cm) nkeys = std::max(nkeys, (size_t)p->k * p->I);
-  if (cm && p->screen) nkeys = std::max(nkeys, (size_t)(2 * H + H / 16));  // rotated u and its padded copy
+  if (cm && p->screen) nkeys = std::max(nkeys, (size_t)kLutFloats);  // the screen's subset-sum table
   const int keys_bytes = (int)align_up(std::max<size_t>(nkeys, 1) * 4, 128);
   const int kept_bytes = cm ? (int)align_up((size_t)std::max(p->keep, 1) * 4, 128) : 0;
   const int hist_bytes = cm ? (int)align_up((size_t)(2 * kSelBins + kSelScratch) * 4, 128) : 0;  // the channel select's bins and scratch
@@ -187,6 +187,13 @@ cudaError_t launch_decode_h(const DecodeParams& p0, int grid, cudaStream_t s) {
   DecodeParams p = p0;
   constexpr bool kFast = (BMAX == 1 && HV == 8 && (WT == MOE_W_BF16 || LAYOUT == MOE_LAYOUT_PLANAR));
   if (!plan_smem(&p, (int)fa.sharedSizeBytes, kFast)) return cudaErrorInvalidConfiguration;
+  if (p.screen) {
+    // the in-stack screen stages each CTA's candidates (code rows, scale
+    // rows, down-column norm) in the ring
+    const long long per_cand = (long long)p.H / 2 + p.H / 32 + 4;
+    const long long nmax = ((long long)p.k * p.I + grid - 1) / grid;
+    if (nmax * per_cand > (long long)p.nstages * p.stage_bytes) return cudaErrorInvalidConfiguration;
+  }
   err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem_bytes);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
@@ -511,15 +518,23 @@ moe_status moe_reader_screen(const moe_layer_desc* d, const void* x, int32_t B, 
     return MOE_ERR_INVALID;
   if (B < 1 || B > 256) return MOE_ERR_INVALID;
   if (d->H % kRdBlock != 0 || d->H > 2048) return MOE_ERR_UNSUPPORTED;
-  if (((uintptr_t)x & 1u) || ((uintptr_t)codes & 3u) || ((uintptr_t)dnorm & 3u) || ((uintptr_t)scales & 1u) ||
+  if (((uintptr_t)x & 1u) || ((uintptr_t)codes & 15u) || ((uintptr_t)dnorm & 3u) || ((uintptr_t)scales & 3u) ||
       ((uintptr_t)scores & 3u) || ((uintptr_t)est_opt & 3u))
     return MOE_ERR_INVALID;
   const int sms = sm_count();
   if (sms <= 0) return MOE_ERR_CUDA;
-  // about two CTAs per SM over the batch, each CTA at least 8 channels
+  // about two CTAs per SM over the batch, each CTA at least 8 channels; a
+  // CTA stages its candidates' code and scale rows in shared memory
   const int nq = d->k * d->I, wpc = kRdScreenThreads / 32;
-  const int gx = std::max(1, std::min((nq + wpc - 1) / wpc, (2 * sms + B - 1) / B));
-  reader_screen_kernel<<<dim3((unsigned)gx, (unsigned)B), kRdScreenThreads, 0, (cudaStream_t)stream>>>(
+  int gx = std::max(1, std::min((nq + wpc - 1) / wpc, (2 * sms + B - 1) / B));
+  const size_t per_cand = (size_t)d->H / 2 + (size_t)d->H / 32;  // bytes of one candidate's codes and scales
+  const size_t lut_bytes = sizeof(float) * kLutFloats + sizeof(int) * kMaxK;
+  const size_t room = (size_t)max_dyn_smem() - lut_bytes - 1024;
+  while ((size_t)((nq + gx - 1) / gx) * per_cand > room) ++gx;  // more CTAs, fewer candidates each
+  const size_t dyn = (size_t)((nq + gx - 1) / gx) * per_cand + 16;
+  if (cudaFuncSetAttribute(reader_screen_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  reader_screen_kernel<<<dim3((unsigned)gx, (unsigned)B), kRdScreenThreads, dyn, (cudaStream_t)stream>>>(
       static_cast<const uint16_t*>(x), d->H, d->E, d->I, d->k, ids, w, signs, codes, scales, dnorm, scores,
       est_opt);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
@@ -635,7 +650,7 @@ moe_status moe_channel_stack_forward(const moe_layer_desc* layers, int32_t L, co
       p.layer[l].scores = scores + (size_t)l * d->E * d->I;
     } else {
       const moe_sketch_desc& sk = sketches[l];
-      if (!sk.codes || !sk.scales || !sk.dnorm || ((uintptr_t)sk.codes & 3u) || ((uintptr_t)sk.scales & 1u) ||
+      if (!sk.codes || !sk.scales || !sk.dnorm || ((uintptr_t)sk.codes & 15u) || ((uintptr_t)sk.scales & 3u) ||
           ((uintptr_t)sk.dnorm & 3u))
         return MOE_ERR_INVALID;
       p.layer[l].sk_codes = sk.codes;

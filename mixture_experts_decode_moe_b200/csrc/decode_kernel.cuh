@@ -9,6 +9,7 @@
 #pragma once
 
 #include "decode.cuh"
+#include "screen_lut.cuh"
 
 namespace moedec {
 
@@ -2173,11 +2174,11 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
     // keys' own range and lists the kept set (every key > T plus the first
     // keep - #{> T} keys == T in index order) ascending.
     // ---- weight-only channel screen of layer l inside the stack ([Reader]
-    // "가중치만으로 만든 reader", steps 1-2, eq. 1): every CTA rotates u (fp32
-    // butterfly per block of 128, u_x = H_128 (s * u), in the keys buffer,
-    // then a copy padded by one float per 16 coordinates), then scores its
-    // share of the k*I candidates (candidate q = unit * I + c): warp per
-    // channel, lane l holding code words l + 32t of each row, the next
+    // "가중치만으로 만든 reader", steps 1-2, eq. 1): every CTA rotates u (fp32,
+    // u_x = H_128 (s * u) per block of 128, in registers and shuffles) into
+    // the subset-sum table of every 4 coordinates (in the keys buffer), then
+    // scores its share of the k*I candidates (candidate q = unit * I + c):
+    // warp per channel, lane l taking code words l + 32t of each row, the next
     // channel's words fetched before the current one is decoded;
     //   s_j = w_e ||d_j|| |SiLU(g_hat) v_hat|, g_hat = sum_b scale_b codes_b . u_x,b / 128
     // written to scr[e*I + c]. A grid barrier then makes every CTA's scores
@@ -2185,74 +2186,63 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
     auto screen_layer = [&](int l) -> bool {
       if constexpr (LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR && SCREEN) {
         const LayerW& Lw = p.layer[l];
-        float* ux = reinterpret_cast<float*>(keys);
-        float* uxp = ux + H;
-        for (int i = tid; i < H; i += kConsumers) ux[i] = bf16_to_f(us[i]) * (float)p.signs[i];
-        cbar();
-        for (int lg2 = 0; lg2 < 7; ++lg2) {
-          const int mm = 1 << lg2;
-          for (int q = tid; q < H / 2; q += kConsumers) {
-            const int i = ((q >> lg2) << (lg2 + 1)) | (q & (mm - 1));
-            const float a0 = ux[i], a1 = ux[i + mm];
-            ux[i] = a0 + a1;
-            ux[i + mm] = a0 - a1;
-          }
-          cbar();
-        }
-        for (int i = tid; i < H; i += kConsumers) uxp[i + (i >> 4)] = ux[i];
-        cbar();
-        const int words = H >> 4, nb = H >> 7;
+        // This CTA's candidates q in [q0, q1): their code rows, scale rows and
+        // down-column norms are copied into the ring (idle between the
+        // routing and the routed copies; cp.async through L2, one round trip
+        // for all of them) while every thread rotates u into the subset-sum
+        // table (in the keys buffer, free until the selection). Then a warp
+        // per candidate, 8 table lookups per code word.
+        float* lut = reinterpret_cast<float*>(keys);
+        const int words = H >> 4, nb = H >> 7, cw = 2 * words;
         const int N = k * I;
         const int q0 = (int)((long long)cta * N / G), q1 = (int)((long long)(cta + 1) * N / G);
-        struct Fetch {
-          int j, u;
-          uint32_t wv[2][4];
-          float sv[2][4];
-        };
-        auto fetch = [&](int q, Fetch& f) {
-          f.j = -1;
-          if (q >= q1) return;
+        const int n = q1 - q0;
+        uint32_t* st_codes = reinterpret_cast<uint32_t*>(ring);                       // [n][2][words]
+        uint16_t* st_scales = reinterpret_cast<uint16_t*>(ring + (size_t)n * cw * 4);  // [n][2][nb]
+        float* st_dn = reinterpret_cast<float*>(ring + (size_t)n * (cw * 4 + nb * 4));  // [n]
+        auto chan = [&](int q) {
           const int u = q / I;
-          f.u = u;
-          f.j = rs.unit_e[u] * I + (q - u * I);
+          return rs.unit_e[u] * I + (q - u * I);
+        };
+        // warp w copies candidates w, w + 8, ...: lane l the 16-byte pieces
+        // l + 32 i of the two code rows and the 4-byte pieces of the scale
+        // rows, lane 0 the norm
+        for (int i = warp; i < n; i += kWarps) {
+          const int j = chan(q0 + i);
+          for (int o = lane; o < cw / 4; o += 32)
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(st_codes + (size_t)i * cw + 4 * o)),
+                         "l"(Lw.sk_codes + (size_t)j * cw + 4 * o)
+                         : "memory");
+          for (int o = lane; o < nb; o += 32)
+            asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(st_scales + (size_t)i * 2 * nb + 2 * o)),
+                         "l"(Lw.sk_scales + (size_t)j * 2 * nb + 2 * o)
+                         : "memory");
+          if (lane == 0)
+            asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(st_dn + i)), "l"(Lw.sk_dnorm + j)
+                         : "memory");
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        screen_build_lut(H, [&](int h) { return bf16_to_f(us[h]) * (float)p.signs[h]; }, lut);
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+        cbar();
+        for (int i = warp; i < n; i += kWarps) {
+          const uint32_t* cr = st_codes + (size_t)i * cw;
+          const uint16_t* sr = st_scales + (size_t)i * 2 * nb;
+          float acc[2] = {0.f, 0.f};
 #pragma unroll
           for (int r = 0; r < 2; ++r)
 #pragma unroll
             for (int t = 0; t < 4; ++t) {
               const int wd = lane + 32 * t;
-              f.wv[r][t] = wd < words ? __ldg(Lw.sk_codes + ((size_t)f.j * 2 + r) * words + wd) : 0u;
-              f.sv[r][t] = wd < words ? __half2float(__ushort_as_half(__ldg(Lw.sk_scales + ((size_t)f.j * 2 + r) * nb + (wd >> 3))))
-                                      : 0.f;
+              if (wd < words)
+                acc[r] = fmaf(__half2float(__ushort_as_half(sr[r * nb + (wd >> 3)])), screen_word(lut, wd, cr[r * words + wd]),
+                              acc[r]);
             }
-        };
-        Fetch cur, nxt;
-        fetch(q0 + warp, cur);
-        for (int q = q0 + warp; q < q1; q += kWarps) {
-          fetch(q + kWarps, nxt);
-          float gv[2];
-#pragma unroll
-          for (int r = 0; r < 2; ++r) {
-            float acc = 0.f;
-#pragma unroll
-            for (int t = 0; t < 4; ++t) {
-              const int wd = lane + 32 * t;
-              if (wd < words) {
-                const uint32_t word = cur.wv[r][t];
-                float pt = 0.f;
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                  const uint32_t sgn = (word << (30 - 2 * i)) & 0x80000000u;
-                  const float xv = __uint_as_float(__float_as_uint(uxp[17 * wd + i]) ^ sgn);
-                  pt += ((word >> (2 * i)) & 1u) ? xv : 0.f;
-                }
-                acc = fmaf(cur.sv[r][t], pt, acc);
-              }
-            }
-            gv[r] = warp_sum(acc) * (1.0f / 128.0f);
+          const float gv0 = warp_sum(acc[0]) * (1.0f / 128.0f), gv1 = warp_sum(acc[1]) * (1.0f / 128.0f);
+          if (lane == 0) {
+            const int q = q0 + i, u = q / I;
+            p.scr[chan(q)] = rs.unit_w[u][0] * st_dn[i] * fabsf(silu_f(gv0) * gv1);
           }
-          if (lane == 0)
-            p.scr[cur.j] = rs.unit_w[cur.u][0] * __ldg(Lw.sk_dnorm + cur.j) * fabsf(silu_f(gv[0]) * gv[1]);
-          cur = nxt;
         }
         return grid_sync();
       } else {

@@ -7,6 +7,7 @@
 
 #include <cuda_fp16.h>
 
+#include "screen_lut.cuh"
 #include "small_kernels.cuh"
 
 namespace moedec {
@@ -100,112 +101,91 @@ __global__ void __launch_bounds__(kRdBlock) reader_build_kernel(const uint16_t* 
   if (t == 0) dnorm[j] = (float)sqrt(tot);
 }
 
-// Screen: token b = blockIdx.y. The CTA rotates x_b once, ux = H_128 (s * x_b)
-// per block in fp32 (shared memory), then each warp takes channels q of the
-// k*I candidates (slot q / I, channel q % I of expert ids[b, slot]):
+// Screen: token b = blockIdx.y; CTA x takes the contiguous candidates
+// q in [x * k*I / G, (x + 1) * k*I / G) (slot q / I, channel q % I of expert
+// ids[b, slot]):
 //   g_hat = sum_blocks scale_b * (codes_b . ux_b) / 128, v_hat likewise,
 //   scores[b, e, c] = w[b, slot] * dnorm[e*I + c] * |SiLU(g_hat) * v_hat|.
-// Lane l holds the coordinates of code words l + 32 t (t < H/512) in
-// registers (read from a copy of ux padded by one float per 16, so that the
-// 32 lanes hit 32 banks), and each row is read as H/16 coalesced words. A
-// warp fetches its next channel's words, scales, weight and norm before it
-// decodes the current one. A code adds x with its sign bit flipped when the
-// code is negative, selected away when it is zero (no branches).
-// est_opt[b, slot, c] = {g_hat, v_hat} when given. Rows of unrouted experts,
-// and of ids outside [0, E), are not written.
+// The CTA first copies its candidates' code rows and scales into shared
+// memory (cp.async through L2: one round trip for all of them, no registers
+// held) and, while they land, rotates x_b, ux = H_128 (s * x_b) per block in
+// fp32, into the table of subset sums of every 4 coordinates
+// (screen_build_lut). Then warp w decodes candidates w, w + 8, ...: lane l
+// takes code words l + 32 t of each row, 8 table lookups per word
+// (screen_word). est_opt[b, slot, c] = {g_hat, v_hat} when given. Rows of
+// unrouted experts, and of ids outside [0, E), are not written.
+// Dynamic shared memory: ceil(k*I / G) * (H / 2 + H / 32) bytes.
 __global__ void __launch_bounds__(kRdScreenThreads) reader_screen_kernel(
     const uint16_t* __restrict__ x, int H, int E, int I, int k, const int32_t* __restrict__ ids,
     const float* __restrict__ w, const int8_t* __restrict__ signs, const uint32_t* __restrict__ codes,
     const uint16_t* __restrict__ scales, const float* __restrict__ dnorm, float* __restrict__ scores,
     float* __restrict__ est) {
-  __shared__ float ux[2048];
-  __shared__ float uxp[2048 + 2048 / 16];
+  __shared__ float lut[kLutFloats];
+  __shared__ int ids_s[kMaxK];
+  extern __shared__ __align__(16) uint32_t staged[];
   const int b = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  for (int i = tid; i < H; i += kRdScreenThreads) ux[i] = bf16_to_f(x[(size_t)b * H + i]) * (float)signs[i];
-  __syncthreads();
-  for (int lg = 0; lg < 7; ++lg) {
-    const int m = 1 << lg;
-    for (int p = tid; p < H / 2; p += kRdScreenThreads) {
-      const int i = ((p >> lg) << (lg + 1)) | (p & (m - 1));
-      const float a0 = ux[i], a1 = ux[i + m];
-      ux[i] = a0 + a1;
-      ux[i + m] = a0 - a1;
-    }
-    __syncthreads();
-  }
-  for (int i = tid; i < H; i += kRdScreenThreads) uxp[i + (i >> 4)] = ux[i];
-  __syncthreads();
-  const int words = H / 16, nb = H / kRdBlock;
-  float xr[kRdMaxWords][16];
+  const int words = H / 16, nb = H / kRdBlock, cw = 2 * words;
+  const int nq = k * I, G = gridDim.x;
+  const int q0 = (int)((long long)blockIdx.x * nq / G), q1 = (int)((long long)(blockIdx.x + 1) * nq / G);
+  const int n = q1 - q0;
+  uint32_t* st_codes = staged;                                               // [n][2][words]
+  uint16_t* st_scales = reinterpret_cast<uint16_t*>(staged + (size_t)n * cw);  // [n][2][nb]
+  // x_b (s * x) into registers while the ids arrive
+  float xv[8];
 #pragma unroll
-  for (int t = 0; t < kRdMaxWords; ++t) {
-    const int wd = lane + 32 * t;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) xr[t][i] = wd < words ? uxp[17 * wd + i] : 0.f;
+  for (int i = 0; i < 8; ++i) {
+    const int h = 8 * tid + i;
+    xv[i] = h < H ? bf16_to_f(x[(size_t)b * H + h]) * (float)signs[h] : 0.f;
   }
-  // one channel's inputs, fetched a channel ahead
-  struct Fetch {
-    int e, slot, c;
-    float wt, dn;
-    uint32_t wv[2][kRdMaxWords];
-    float sv[2][kRdMaxWords];
+  if (tid < k) ids_s[tid] = __ldg(ids + b * k + tid);
+  __syncthreads();
+  auto chan = [&](int q) -> int {  // channel e*I + c of candidate q, or -1
+    const int slot = q / I, e = ids_s[slot];
+    return (unsigned)e < (unsigned)E ? e * I + (q - slot * I) : -1;
   };
-  const int nq = k * I, wpc = kRdScreenThreads / 32, qstride = gridDim.x * wpc;
-  auto fetch = [&](int q, Fetch& f) {
-    f.e = -1;
-    if (q >= nq) return;
-    f.slot = q / I;
-    f.c = q - f.slot * I;
-    const int e = __ldg(ids + b * k + f.slot);
-    if ((unsigned)e >= (unsigned)E) return;  // an id out of range is skipped (warp-uniform)
-    f.e = e;
-    const size_t j = (size_t)e * I + f.c;
-    f.wt = __ldg(w + b * k + f.slot);
-    f.dn = __ldg(dnorm + j);
+  // warp w copies candidates w, w + 8, ...: their two code rows (16-byte
+  // pieces, lane l taking pieces l + 32 i) and two scale rows (4-byte pieces)
+  for (int i = warp; i < n; i += kRdScreenThreads / 32) {
+    const int j = chan(q0 + i);
+    if (j < 0) continue;  // warp-uniform
+    for (int o = lane; o < cw / 4; o += 32)
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(st_codes + (size_t)i * cw + 4 * o)),
+                   "l"(codes + (size_t)j * cw + 4 * o)
+                   : "memory");
+    for (int o = lane; o < nb; o += 32)
+      asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(st_scales + (size_t)i * 2 * nb + 2 * o)),
+                   "l"(scales + (size_t)j * 2 * nb + 2 * o)
+                   : "memory");
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+  screen_rotate_lut(H, xv, lut);
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+  __syncthreads();
+  for (int i = warp; i < n; i += kRdScreenThreads / 32) {
+    const int q = q0 + i, j = chan(q);
+    if (j < 0) continue;  // warp-uniform
+    const uint32_t* cr = st_codes + (size_t)i * cw;
+    const uint16_t* sr = st_scales + (size_t)i * 2 * nb;
+    float acc[2] = {0.f, 0.f};
 #pragma unroll
     for (int r = 0; r < 2; ++r)
 #pragma unroll
       for (int t = 0; t < kRdMaxWords; ++t) {
         const int wd = lane + 32 * t;
-        f.wv[r][t] = wd < words ? __ldg(codes + (2 * j + r) * (size_t)words + wd) : 0u;
-        f.sv[r][t] = wd < words ? __half2float(__ushort_as_half(__ldg(scales + (2 * j + r) * (size_t)nb + (wd >> 3))))
-                                : 0.f;
+        if (wd < words)
+          acc[r] = fmaf(__half2float(__ushort_as_half(sr[r * nb + (wd >> 3)])), screen_word(lut, wd, cr[r * words + wd]),
+                        acc[r]);
       }
-  };
-  Fetch cur, nxt;
-  int q = blockIdx.x * wpc + warp;
-  fetch(q, cur);
-  for (; q < nq; q += qstride) {
-    fetch(q + qstride, nxt);
-    if (cur.e >= 0) {
-      float gv[2];
-#pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        float acc = 0.f;
-#pragma unroll
-        for (int t = 0; t < kRdMaxWords; ++t) {
-          const uint32_t word = cur.wv[r][t];
-          float pt = 0.f;
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const uint32_t sgn = (word << (30 - 2 * i)) & 0x80000000u;  // bit 2i+1 -> sign
-            const float xv = __uint_as_float(__float_as_uint(xr[t][i]) ^ sgn);
-            pt += ((word >> (2 * i)) & 1u) ? xv : 0.f;
-          }
-          acc = fmaf(cur.sv[r][t], pt, acc);
-        }
-        gv[r] = warp_sum(acc) * (1.0f / 128.0f);
-      }
-      if (lane == 0) {
-        scores[((size_t)b * E + cur.e) * I + cur.c] = cur.wt * cur.dn * fabsf(silu_f(gv[0]) * gv[1]);
-        if (est != nullptr) {
-          float* o = est + (((size_t)b * k + cur.slot) * I + cur.c) * 2;
-          o[0] = gv[0];
-          o[1] = gv[1];
-        }
+    const float g = warp_sum(acc[0]) * (1.0f / 128.0f), v = warp_sum(acc[1]) * (1.0f / 128.0f);
+    if (lane == 0) {
+      const int slot = q / I, c = q - slot * I;
+      scores[((size_t)b * E + ids_s[slot]) * I + c] = __ldg(w + b * k + slot) * __ldg(dnorm + j) * fabsf(silu_f(g) * v);
+      if (est != nullptr) {
+        float* o = est + (((size_t)b * k + slot) * I + c) * 2;
+        o[0] = g;
+        o[1] = v;
       }
     }
-    cur = nxt;
   }
 }
 

@@ -11,8 +11,9 @@ relative; dnorm within 2 fp32 ulps.
 Screen: the estimates g_hat, v_hat within 1e-5 x B, where B =
 sum_b scale_b n_b sum_{i in b}|x_i| / 128 (n_b nonzero codes) bounds every
 partial sum of the estimate, rotation included. The kernel rounds in fp32 at
-most ~32 times along any path (7 butterfly stages, 16 + 4 accumulations per
-lane, 5 shuffle steps): 32 x 2^-24 = 1.9e-6 x B, so 1e-5 leaves a factor 5.
+most ~32 times along any path (7 butterfly stages, 3 in a subset-sum table
+entry, 8 combining a code word's table lookups, 4 accumulations per lane, 5
+shuffle steps: 27): 32 x 2^-24 = 1.9e-6 x B, so 1e-5 leaves a factor 5.
 Scores within the propagated bound w ||d|| (1.1 |v| dg + |SiLU(g)| dv + dg dv)
 + 1e-5 s (|SiLU'| <= 1.1; the last term covers fp32 dnorm and SiLU).
 """
