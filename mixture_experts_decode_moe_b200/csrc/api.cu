@@ -731,7 +731,7 @@ moe_status moe_channel_topk_forward(const moe_layer_desc* d, const void* x, int3
   const int G = sm_count();
   if (G <= 0) return MOE_ERR_CUDA;
   const long long units = std::min<long long>(d->E, (long long)B * d->k);
-  if (units > kCbMaxUnits || units * d->I > kCbMaxUnionBits) return MOE_ERR_UNSUPPORTED;
+  if (units > kCbMaxUnits || (long long)d->E * d->I > kCbMaxChanBits) return MOE_ERR_UNSUPPORTED;
   if (((long long)B * nk + G - 1) / G > kCbMaxSlice) return MOE_ERR_UNSUPPORTED;
   ChanBatchParams p;
   std::memset(&p, 0, sizeof(p));
@@ -749,10 +749,17 @@ moe_status moe_channel_topk_forward(const moe_layer_desc* d, const void* x, int3
   uint8_t* base = static_cast<uint8_t*>(ws);
   p.ctl = reinterpret_cast<WsControl*>(base);
   p.kept_ws = reinterpret_cast<int32_t*>(base + chan_kept_offset(B, d));
-  const long long uw = (units * d->I + 31) / 32;
+  // the tokens' kept-channel bitmaps (B x jstride words) use the scores area
+  // of the channel workspace: B * E*I / 8 bytes <= E*I * 4 bytes
+  const long long jstride = (((long long)d->E * d->I + 31) / 32 + 3) / 4 * 4;
+  p.jstride = (int)jstride;
+  p.bits_ws = reinterpret_cast<uint32_t*>(base + chan_scr_offset(B, d));
+  if ((size_t)B * jstride * 4 > chan_scr_bytes(d)) return MOE_ERR_UNSUPPORTED;
   size_t ring = (size_t)kCbStages * kCbNch * 3 * d->H * 2;
-  ring = std::max(ring, align_up((size_t)d->k * d->I * 4, 128) + (size_t)(2 * kSelBins + kSelScratch) * 4);  // keys, the select's bins and scratch
-  ring = std::max(ring, (size_t)(B + 2) * (size_t)uw * 4);
+  // phase A: keys, the select's bins and scratch, the token's bitmap
+  ring = std::max(ring, align_up((size_t)d->k * d->I * 4, 128) + (size_t)(2 * kSelBins + kSelScratch) * 4 +
+                            (size_t)jstride * 4);
+  ring = std::max(ring, (size_t)(B + 2) * (size_t)jstride * 4);  // phase B: the bitmaps, the union, its prefix
   ring = std::max(ring, (size_t)(d->E + 31) / 32 * 4);
   ring = align_up(ring, (size_t)128);
   p.ring_bytes = (int)ring;

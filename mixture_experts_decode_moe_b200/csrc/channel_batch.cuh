@@ -14,14 +14,15 @@
 //
 // How (B200 design), one CTA per SM, 8 consumer warps + 1 producer warp:
 //  A. CTA b < B selects token b's kept channels (the keep-th largest key
-//     by histogram passes over the keys' own range, ordered compaction), writes them ascending to the workspace (and the caller's
-//     kept list) with the token's sector count; every CTA zeroes its slice
-//     of y. One grid-wide barrier.
-//  B. Every CTA builds the batch's touched experts (ascending), one bitmap of
-//     kept channels per token over (touched expert, channel), their union and
-//     its prefix counts, and takes a contiguous slice of the union list with
-//     each channel's token mask; it adds its slice's sectors to the union's
-//     sector count.
+//     by histogram passes over the keys' own range, ordered compaction),
+//     writes them ascending to the workspace (and the caller's kept list)
+//     and as a bitmap over the channel ids, with the token's sector count;
+//     every CTA zeroes its slice of y. One grid-wide barrier.
+//  B. Every CTA builds the batch's touched experts (ascending), ORs the
+//     tokens' kept-channel bitmaps (over channel ids j = e*I + c, written by
+//     phase A) into the union and its prefix counts, and takes a contiguous
+//     slice of the union list with each channel's token mask; it adds its
+//     slice's sectors to the union's sector count.
 //  C. The producer warp streams the slice's channels (12 KB each at H =
 //     2048, one bulk copy per run of consecutive channels) through a ring of
 //     shared-memory stages; per job of 4 channels, warp w computes half of
@@ -40,7 +41,7 @@ constexpr int kCbThreads = kCbConsumers + 32;    // + 1 producer warp
 constexpr int kCbNch = 4;                        // channels per job
 constexpr int kCbStages = 3;
 constexpr int kCbMaxUnits = kMaxB * kMaxK;       // touched experts of a batch (<= B * k <= 256)
-constexpr int kCbMaxUnionBits = 65536;           // touched experts x I
+constexpr int kCbMaxChanBits = 1 << 20;          // E * I (the union is kept over channel ids)
 constexpr int kCbMaxSlice = 1024;                // union channels per CTA
 
 struct ChanBatchParams {
@@ -57,6 +58,8 @@ struct ChanBatchParams {
   unsigned long long* union_sectors;  // [1] or null
   WsControl* ctl;
   int32_t* kept_ws;        // [B, keep] workspace
+  uint32_t* bits_ws;       // [B, jstride] workspace: each token's kept channels as bits of j = e*I + c
+  int jstride;             // words per token bitmap: ceil(E*I / 32) rounded up to a multiple of 4
   int ring_bytes;          // shared-memory ring (also the selection keys and the union bitmaps)
   int smem_bytes;          // ring + x
 };
@@ -134,6 +137,9 @@ __global__ void __launch_bounds__(kCbThreads, 1) channel_batch_kernel(const __gr
     uint32_t* keys = reinterpret_cast<uint32_t*>(ring);
     int* hist = reinterpret_cast<int*>(ring + ((size_t)N * 4 + 127) / 128 * 128);
     int* sel_sc = hist + 2 * kSelBins;
+    // the token's kept channels as bits of j = e*I + c, after the scratch
+    uint32_t* bm = reinterpret_cast<uint32_t*>(sel_sc + kSelScratch);
+    for (int i = tid; i < p.jstride; i += kCbConsumers) bm[i] = 0u;
     const float* srow = p.scores + (size_t)b * E * I;
     const bool vec = (I & 3) == 0 && ((uintptr_t)p.scores & 15u) == 0;
     sel_load_keys(keys, N, I, vec, [&](int u) { return srow + (size_t)tu_e[u] * I; }, hist, sel_sc);
@@ -145,9 +151,11 @@ __global__ void __launch_bounds__(kCbThreads, 1) channel_batch_kernel(const __gr
         const int u = q / I;
         const int j = tu_e[u] * I + (q - u * I);
         kws[pos] = j;
+        atomicOr(&bm[j >> 5], 1u << (j & 31));
         if (p.kept_out) p.kept_out[(size_t)b * keep + pos] = j;
       });
     cbar();  // the kept list is complete (global writes of this CTA, ordered by the barrier)
+    for (int i = tid; i < p.jstride; i += kCbConsumers) p.bits_ws[(size_t)b * p.jstride + i] = bm[i];
     // sectors of the token's kept channels (channel-major ranges, a sector
     // shared with the previous kept channel counted once; channels that
     // start and end on 32-byte boundaries share none)
@@ -201,14 +209,16 @@ __global__ void __launch_bounds__(kCbThreads, 1) channel_batch_kernel(const __gr
   // ---------------------------------------------------------------- B: union and this CTA's slice
   // every CTA checks the ids itself (in range, distinct per token): with a
   // bad id nothing is computed (CTA b recorded the status in phase A)
+  __shared__ int ids_s[kCbMaxUnits];
   if (!failed) {
     if (tid == 0) bad_s = 0;
+    for (int t = tid; t < B * k; t += kCbThreads) ids_s[t] = __ldg(p.ids + t);
     __syncthreads();
     for (int t = tid; t < B * k; t += kCbThreads) {
-      const int e = __ldg(p.ids + t), b = t / k;
+      const int e = ids_s[t], b = t / k;
       bool bad = e < 0 || e >= E;
       for (int s2 = 0; s2 < k; ++s2)
-        if (b * k + s2 != t && __ldg(p.ids + b * k + s2) == e) bad = true;
+        if (b * k + s2 != t && ids_s[b * k + s2] == e) bad = true;
       if (bad) bad_s = 1;
     }
     __syncthreads();
@@ -222,7 +232,7 @@ __global__ void __launch_bounds__(kCbThreads, 1) channel_batch_kernel(const __gr
     for (int i = tid; i < ne32; i += kCbThreads) ebits[i] = 0u;
     __syncthreads();
     for (int t = tid; t < B * k; t += kCbThreads) {
-      const int e = __ldg(p.ids + t);
+      const int e = ids_s[t];
       if (e >= 0 && e < E) atomicOr(&ebits[e >> 5], 1u << (e & 31));
     }
     __syncthreads();
@@ -254,35 +264,29 @@ __global__ void __launch_bounds__(kCbThreads, 1) channel_batch_kernel(const __gr
     for (int i = tid; i < U * kMaxB; i += kCbThreads) wt[i / kMaxB][i % kMaxB] = 0.f;
     __syncthreads();
     for (int t = tid; t < B * k; t += kCbThreads) {
-      const int e = __ldg(p.ids + t);
+      const int e = ids_s[t];
       if (e >= 0 && e < E) wt[unit_of_e[e]][t / k] = __ldg(p.w + t);
     }
-    // one bitmap of kept channels per token over (unit, channel), then the
-    // union; the words live in the (still unused) ring
-    const int UW = (U * I + 31) >> 5;
-    uint32_t* tb = reinterpret_cast<uint32_t*>(ring);          // [B][UW]
-    uint32_t* uw = tb + (size_t)B * UW;                          // [UW] union
-    int* upre = reinterpret_cast<int*>(uw + UW);                 // [UW] exclusive prefix of popc
-    for (int i = tid; i < B * UW; i += kCbThreads) tb[i] = 0u;
-    __syncthreads();
-    const int nk = min(keep, k * I);
-    for (int t = tid; t < B * nk; t += kCbThreads) {
-      const int b = t / nk;
-      const int j = __ldcg(p.kept_ws + (size_t)b * keep + (t - b * nk));
-      const int e = j / I;
-      const int bit = (int)unit_of_e[e] * I + (j - e * I);
-      atomicOr(&tb[(size_t)b * UW + (bit >> 5)], 1u << (bit & 31));
-    }
-    __syncthreads();
-    // union words and their prefix counts: thread t takes contiguous words
-    const int per = (UW + kCbThreads - 1) / kCbThreads;
-    const int w0 = min(UW, tid * per), w1 = min(UW, w0 + per);
+    // the union of the tokens' kept channels over j = e*I + c: thread t takes
+    // the contiguous words [w0, w1) (a multiple of 4: 16-byte loads of every
+    // token's bitmap, written by phase A), keeps them in the (still unused)
+    // ring for the slice below and ORs them
+    const int JS = p.jstride;
+    uint32_t* tb = reinterpret_cast<uint32_t*>(ring);          // [B][JS]
+    uint32_t* uw = tb + (size_t)B * JS;                          // [JS] union
+    int* upre = reinterpret_cast<int*>(uw + JS);                 // [JS] exclusive prefix of popc
+    const int per = ((JS + 4 * kCbThreads - 1) / (4 * kCbThreads)) * 4;
+    const int w0 = min(JS, tid * per), w1 = min(JS, w0 + per);
     int cnt = 0;
-    for (int i = w0; i < w1; ++i) {
-      uint32_t m = 0u;
-      for (int b = 0; b < B; ++b) m |= tb[(size_t)b * UW + i];
-      uw[i] = m;
-      cnt += __popc(m);
+    for (int i = w0; i < w1; i += 4) {
+      uint4 m = make_uint4(0u, 0u, 0u, 0u);
+      for (int b = 0; b < B; ++b) {
+        const uint4 v = __ldcg(reinterpret_cast<const uint4*>(p.bits_ws + (size_t)b * JS + i));
+        *reinterpret_cast<uint4*>(tb + (size_t)b * JS + i) = v;
+        m.x |= v.x; m.y |= v.y; m.z |= v.z; m.w |= v.w;
+      }
+      *reinterpret_cast<uint4*>(uw + i) = m;
+      cnt += __popc(m.x) + __popc(m.y) + __popc(m.z) + __popc(m.w);
     }
     // block-wide exclusive scan over all 288 threads (9 warps)
     {
@@ -312,23 +316,33 @@ __global__ void __launch_bounds__(kCbThreads, 1) channel_batch_kernel(const __gr
     __shared__ int prev_j_s;
     if (tid == 0) prev_j_s = -1;
     __syncthreads();
-    for (int i = w0; i < w1; ++i) {
-      int rk = upre[i];
-      for (uint32_t m = uw[i]; m; m &= m - 1) {
-        if (rk >= s0 - 1 && rk < s1) {
-          const int bit = i * 32 + __ffs(m) - 1;
-          const int u = bit / I, c = bit - u * I;
-          const int j = unit_e[u] * I + c;
-          if (rk == s0 - 1) {
-            prev_j_s = j;
-          } else {
-            uint32_t tm = 0u;
-            for (int b = 0; b < B; ++b) tm |= ((tb[(size_t)b * UW + i] >> (bit & 31)) & 1u) << b;
-            sl_j[rk - s0] = j;
-            sl_m[rk - s0] = (uint8_t)tm;
-          }
-        }
-        ++rk;
+    // thread t finds union channel s0 - 1 + t (its word: the last with
+    // prefix <= rank, by binary search; its bit: the rank's set bit of the
+    // word), so the slice is extracted in parallel
+    for (int t = tid; t <= ns; t += kCbThreads) {
+      const int rk = s0 - 1 + t;
+      if (rk < 0) continue;
+      int lo = 0, hi = JS - 1;  // upre[lo] <= rk < upre[hi + 1]
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (upre[mid] <= rk) lo = mid; else hi = mid - 1;
+      }
+      const uint32_t mw = uw[lo];
+      int nth = rk - upre[lo], bit = 0;
+      uint32_t m = mw;
+#pragma unroll
+      for (int wdt = 16; wdt >= 1; wdt >>= 1) {
+        const int c = __popc(m & ((1u << wdt) - 1u));
+        if (nth >= c) { nth -= c; m >>= wdt; bit += wdt; }
+      }
+      const int j = lo * 32 + bit;
+      if (t == 0) {
+        prev_j_s = j;
+      } else {
+        uint32_t tm = 0u;
+        for (int b = 0; b < B; ++b) tm |= ((tb[(size_t)b * JS + lo] >> bit) & 1u) << b;
+        sl_j[t - 1] = j;
+        sl_m[t - 1] = (uint8_t)tm;
       }
     }
     __syncthreads();
