@@ -71,8 +71,10 @@ __global__ void __launch_bounds__(kCbThreads, 1) channel_batch_kernel(const __gr
   __shared__ short unit_of_e[kMaxE];
   __shared__ float wt[kCbMaxUnits][kMaxB];
   __shared__ int tu_e[kMaxK];               // phase A: token's experts, ascending
-  __shared__ int sl_j[kCbMaxSlice];         // phase C: this CTA's union channels
-  __shared__ uint8_t sl_m[kCbMaxSlice];     //          and their token masks
+  __shared__ int sl_j[kCbMaxSlice];         // phase C: this CTA's union channels,
+  __shared__ uint8_t sl_m[kCbMaxSlice];     //          their token masks
+  __shared__ uint8_t sl_u[kCbMaxSlice];     //          and their units (touched experts)
+  __shared__ float hw[kWarps][kCbNch * kMaxB];  // per warp: a job's activations w * SiLU(g) * u
   __shared__ float part[2][kCbNch][2][kMaxB][2];
   __shared__ int scan_s[2 * kWarps + 2];
   __shared__ uint32_t red_s[2 * kWarps];
@@ -343,6 +345,7 @@ __global__ void __launch_bounds__(kCbThreads, 1) channel_batch_kernel(const __gr
         for (int b = 0; b < B; ++b) tm |= ((tb[(size_t)b * JS + lo] >> bit) & 1u) << b;
         sl_j[t - 1] = j;
         sl_m[t - 1] = (uint8_t)tm;
+        sl_u[t - 1] = (uint8_t)unit_of_e[j / I];
       }
     }
     __syncthreads();
@@ -441,11 +444,16 @@ __global__ void __launch_bounds__(kCbThreads, 1) channel_batch_kernel(const __gr
               if ((tm >> b) & 1u) {
                 float xf[8];
                 unpack8(xs4[b * H8 + v], xf);
+                float g0 = gf[0] * xf[0], g1 = gf[1] * xf[1], u0 = uf[0] * xf[0], u1 = uf[1] * xf[1];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                  dg[b] = fmaf(gf[e], xf[e], dg[b]);
-                  du[b] = fmaf(uf[e], xf[e], du[b]);
+                for (int e = 2; e < 8; e += 2) {
+                  g0 = fmaf(gf[e], xf[e], g0);
+                  g1 = fmaf(gf[e + 1], xf[e + 1], g1);
+                  u0 = fmaf(uf[e], xf[e], u0);
+                  u1 = fmaf(uf[e + 1], xf[e + 1], u1);
                 }
+                dg[b] += g0 + g1;
+                du[b] += u0 + u1;
               }
           }
         }
@@ -456,22 +464,31 @@ __global__ void __launch_bounds__(kCbThreads, 1) channel_batch_kernel(const __gr
           warp_reduce_multi<2 * kMaxB>(v16, &part[q & 1][ch][half][0][0]);
         }
         cbar();
-        // 2. the job's down columns on this warp's 1/8 of the outputs
+        // 2. the job's activations h = w * SiLU(g) * u, lane c * 8 + b of
+        // every warp taking channel c and token b (all in parallel), then the
+        // job's down columns on this warp's 1/8 of the outputs
+        {
+          const int c = lane >> 3, b = lane & 7;
+          float h = 0.f;
+          if (c < n && b < B && ((sl_m[i0 + c] >> b) & 1u)) {
+            const float g = part[q & 1][c][0][b][0] + part[q & 1][c][1][b][0];
+            const float uu = part[q & 1][c][0][b][1] + part[q & 1][c][1][b][1];
+            h = wt[sl_u[i0 + c]][b] * silu_f(g) * uu;
+          }
+          hw[warp][lane] = h;
+          __syncwarp();
+        }
         if (lane < dv) {
 #pragma unroll
           for (int c = 0; c < kCbNch; ++c)
             if (c < n) {
               const uint32_t m = sl_m[i0 + c];
-              const int j = sl_j[i0 + c];
-              const int u = unit_of_e[j / I];
               float d[8];
               unpack8(reinterpret_cast<const uint4*>(st + (size_t)c * cb + 2 * rowb)[vd], d);
 #pragma unroll
               for (int b = 0; b < kMaxB; ++b)
                 if ((m >> b) & 1u) {
-                  const float g = part[q & 1][c][0][b][0] + part[q & 1][c][1][b][0];
-                  const float uu = part[q & 1][c][0][b][1] + part[q & 1][c][1][b][1];
-                  const float h = wt[u][b] * silu_f(g) * uu;
+                  const float h = hw[warp][c * kMaxB + b];
 #pragma unroll
                   for (int e = 0; e < 8; ++e) acc[b][e] = fmaf(h, d[e], acc[b][e]);
                 }
