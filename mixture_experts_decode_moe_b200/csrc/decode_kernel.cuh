@@ -806,8 +806,32 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
       }
       if (cur.t1 < 0) {
         if (ready_layer < cur.layer) return false;
-        if constexpr (BMAX == 1) cur.set_routed_fixed(rfix);
-        else cur.set_routed(LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR ? rs.ncand : rs.U * I, I);
+        if constexpr (BMAX == 1) {
+          cur.set_routed_fixed(rfix);
+        } else if constexpr (LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR) {
+          cur.set_routed(rs.ncand, I);
+        } else {
+          // batch > 1: a routed channel of unit u costs 1 + (tokens routed
+          // to u) (its fetch plus one dot per token), so CTA c takes the
+          // channels whose cost offset falls in [c C / G, (c + 1) C / G)
+          const int U = rs.U;
+          long long C = 0;
+          for (int u = 0; u < U; ++u) C += (long long)I * (1 + __popc(rs.unit_mask[u]));
+          auto first_from = [&](long long x) -> int {  // first channel whose cost offset is >= x
+            long long acc = 0;
+            for (int u = 0; u < U; ++u) {
+              const long long wu = 1 + __popc(rs.unit_mask[u]), cu = (long long)I * wu;
+              if (x < acc + cu) return u * I + (int)((x - acc + wu - 1) / wu);
+              acc += cu;
+            }
+            return U * I;
+          };
+          const unsigned long long Gu = (unsigned long long)G;
+          cur.t = first_from((long long)((unsigned long long)cta * (unsigned long long)C / Gu));
+          cur.t1 = first_from((long long)((unsigned long long)(cta + 1) * (unsigned long long)C / Gu));
+          cur.u = cur.t / I;
+          cur.c = cur.t - cur.u * I;
+        }
       }
       if (cur.t >= cur.t1) { cur.begin_layer(p, cur.layer + 1); continue; }
       if (LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR) {
