@@ -43,6 +43,8 @@ constexpr int kCbStages = 3;
 constexpr int kCbMaxUnits = kMaxB * kMaxK;       // touched experts of a batch (<= B * k <= 256)
 constexpr int kCbMaxChanBits = 1 << 20;          // E * I (the union is kept over channel ids)
 constexpr int kCbMaxSlice = 1024;                // union channels per CTA
+static_assert(kCbNch * kMaxB == 32, "a job's activations: one lane per (channel, token)");
+static_assert(kCbMaxUnits <= 256, "slice units are stored as bytes");
 
 struct ChanBatchParams {
   int B, H, E, I, k, keep;
