@@ -136,7 +136,7 @@ inline int pick_nch(const moe_layer_desc* d, int B) {
 
 // Shared-memory carve-up of the persistent decode kernel: as many ring stages
 // as fit next to the fixed tiles, given the kernel's static shared memory.
-bool plan_smem(DecodeParams* p, int static_bytes, bool fast) {
+bool plan_smem(DecodeParams* p, int static_bytes, bool fast, bool tc_batch) {
   const int H = p->H, rowb = 2 * H, B = p->B, NCH = p->nch;
   const int budget = max_dyn_smem() - static_bytes - 1024;
   if (budget <= 0) return false;
@@ -151,13 +151,21 @@ bool plan_smem(DecodeParams* p, int static_bytes, bool fast) {
   const int keys_bytes = (int)align_up(std::max<size_t>(nkeys, 1) * 4, 128);
   const int kept_bytes = cm ? (int)align_up((size_t)std::max(p->keep, 1) * 4, 128) : 0;
   const int hist_bytes = cm ? (int)align_up((size_t)(2 * kSelBins + kSelScratch) * 4, 128) : 0;  // the channel select's bins and scratch
-  const int ysum_bytes = fast ? (int)align_up((size_t)H * 4, 128) : 0;
+  // output sums in shared memory: [H] (batch-1 fast path), [B][H] (int4 batch path)
+  const int ysum_bytes = fast ? (int)align_up((size_t)H * 4, 128) : (tc_batch ? (int)align_up((size_t)B * H * 4, 128) : 0);
   const int xf_bytes = fast ? H * 2 : 0;  // x fragments, [segment][lane] x 16 B
   int stage;
   if (cm || p->wtype == MOE_W_BF16) stage = NCH * 3 * rowb;
   else stage = NCH * (3 * (H / 2) + 2 * (H / 32)) + rowb;
-  stage = std::max(stage, p->rows_per_job * rowb);
-  if (p->I_sh > 0) stage = std::max(stage, NCH * 3 * rowb);
+  if (tc_batch) {
+    // stages sized for the int4 jobs: router jobs take as many rows, shared
+    // jobs one channel (three bf16 rows)
+    p->rows_per_job = std::max(1, std::min(p->rows_per_job, stage / rowb));
+    if (p->I_sh > 0) stage = std::max(stage, 3 * rowb);
+  } else {
+    stage = std::max(stage, p->rows_per_job * rowb);
+    if (p->I_sh > 0) stage = std::max(stage, NCH * 3 * rowb);
+  }
   stage = (int)align_up(stage, 128);
   const int fixed = x_bytes + u_bytes + lg_bytes + keys_bytes + kept_bytes + hist_bytes + ysum_bytes + xf_bytes;
   const int nst = std::min(8, (budget - fixed - 256) / stage);
@@ -186,7 +194,8 @@ cudaError_t launch_decode_h(const DecodeParams& p0, int grid, cudaStream_t s) {
   if (err != cudaSuccess) return err;
   DecodeParams p = p0;
   constexpr bool kFast = (BMAX == 1 && HV == 8 && (WT == MOE_W_BF16 || LAYOUT == MOE_LAYOUT_PLANAR));
-  if (!plan_smem(&p, (int)fa.sharedSizeBytes, kFast)) return cudaErrorInvalidConfiguration;
+  constexpr bool kTcB = WT == MOE_W_INT4_G64 && BMAX == 8 && HV == 8 && NCH == 4 && LAYOUT == MOE_LAYOUT_PLANAR;
+  if (!plan_smem(&p, (int)fa.sharedSizeBytes, kFast, kTcB)) return cudaErrorInvalidConfiguration;
   if (p.screen) {
     // the in-stack screen stages each CTA's candidates (code rows, scale
     // rows, down-column norm) in the ring

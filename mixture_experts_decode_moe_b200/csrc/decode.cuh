@@ -111,6 +111,7 @@ struct RouteSmem {
   int unit_e[BMAX * kMaxK];
   uint32_t unit_mask[BMAX * kMaxK];
   float unit_w[BMAX * kMaxK][BMAX];
+  int cpre[BMAX * kMaxK + 1];  // batch > 1: cost offset of each unit's first channel (cpre[U] = total)
   uint32_t bitmap[kMaxE / 32];
   int rank_base[kMaxE / 32];
   int ids[BMAX][kMaxK];
@@ -244,6 +245,22 @@ __device__ __forceinline__ float diag_part(const float (&d0)[4], const float (&d
 // in one 32-bit word, element 2i in the low nibble of byte i) -> float q.
 // (w ^ 0x88888888) turns q into q + 8 in [0, 15]; OR-ing that into the
 // mantissa of 2^23 gives 2^23 + q + 8 exactly; subtracting 2^23 + 8 leaves q.
+// a - b on packed bf16 pairs (round to nearest)
+__device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// Codes i and i + 4 of an int4 word (two's complement nibbles, element 8 v + i
+// in bits 4 i .. 4 i + 3) as a bf16 pair {lo: code i, hi: code i + 4}, exact:
+// the nibble flipped to c + 8 fills the low mantissa bits of 128.0, and
+// 136 is taken off.
+__device__ __forceinline__ uint32_t int4_pair_bf16(uint32_t w, int i) {
+  const uint32_t t = ((w ^ 0x88888888u) >> (4 * i)) & 0x000F000Fu;
+  return bf16x2_sub(t | 0x43004300u, 0x43084308u);
+}
+
 __device__ __forceinline__ void int4x8_to_f(uint32_t w, float* q) {
   const uint32_t t = w ^ 0x88888888u;
 #pragma unroll

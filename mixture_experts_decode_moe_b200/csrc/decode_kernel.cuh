@@ -555,6 +555,18 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
   // (int4 experts too, planar: their router and shared rows are bf16)
   constexpr bool kFast = (BMAX == 1 && HV == 8 && (WT == MOE_W_BF16 || LAYOUT == MOE_LAYOUT_PLANAR));
   constexpr bool kFastI4 = kFast && WT == MOE_W_INT4_G64;
+  // int4 experts at batch > 1 with H = 2048: a routed job's gate and up dots
+  // for all tokens on tensor cores (each code decoded once per job); the
+  // output sums live in shared memory (registers hold one token's at a time)
+  constexpr bool kTcB = WT == MOE_W_INT4_G64 && BMAX == 8 && HV == 8 && NCH == 4 && LAYOUT == MOE_LAYOUT_PLANAR;
+  static_assert(!kTcB || NCH * BMAX == 32, "one lane per (channel, token) activation");
+  // batch > 1: cost of a routed channel in units of one token's work is
+  // kJobW + (tokens routed to its expert): its fetch (and, on the int4 batch
+  // path, its tensor-core dots for all tokens at once) plus the per-token work
+  constexpr int kJobW = kTcB ? 3 : 1;
+  // channels per shared-expert job (bf16 rows): one on the int4 batch path,
+  // whose ring stages are sized for int4 jobs
+  constexpr int kShN = kTcB ? 1 : NCH;
   static_assert(!kFast || (NCH == 2 || NCH == 4 || NCH == 8), "warp groups of 2, 4 or 8 warps");
   constexpr int kGroups = kFast ? kWarps / NCH : 1;
   // fast path: warp group g and producer g form pipeline g with the ring
@@ -575,6 +587,8 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
   __shared__ int pred_s[kProducers][kMaxPred];  // fast path: predicted experts of the next layer
   __shared__ float dotbuf[16][NV];
   __shared__ float hbuf[kWarps][NCH * BMAX];
+  __shared__ float2 tcpart[kTcB ? 2 : 1][kWarps][32];  // per warp: (gate, up) partial dots [channel][token]
+  __shared__ float2 hb2[kTcB ? kWarps : 1][32];        // per warp: activations as pairs {h, h}
   __shared__ uint32_t cand_key[kWarps * kMaxK];
   __shared__ int cand_idx[kWarps * kMaxK];
   __shared__ int sel_pos[kWarps][kMaxK];
@@ -632,6 +646,8 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
     reinterpret_cast<uint4*>(xs)[i] = reinterpret_cast<const uint4*>(p.x_in)[i];
   if constexpr (kFast)
     for (int i = tid; i < H; i += kCtaThreads) reinterpret_cast<float*>(smem + p.off_ysum)[i] = 0.f;
+  if constexpr (kTcB)  // the batch path's output sums [B][H] (thread t owns 8 t .. 8 t + 7 of each token)
+    for (int i = tid; i < B * H; i += kCtaThreads) reinterpret_cast<float*>(smem + p.off_ysum)[i] = 0.f;
   if (p.x_hist != nullptr) {
     const long long n = (long long)B * H8;
     for (long long i = (unsigned)cta * (unsigned)n / (unsigned)G + tid; i < (unsigned)(cta + 1) * (unsigned)n / (unsigned)G;
@@ -798,7 +814,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
         return true;
       }
       if (cur.type == JOB_SHARED) {
-        const int n = min(NCH, cur.t1 - cur.t);
+        const int n = min(kShN, cur.t1 - cur.t);
         j = Job{JOB_SHARED, cur.layer, 0, cur.t, n};
         cur.t += n;
         if (cur.t >= cur.t1) { cur.type = JOB_ROUTED; cur.t = -1; cur.t1 = -1; }
@@ -811,20 +827,22 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
         } else if constexpr (LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR) {
           cur.set_routed(rs.ncand, I);
         } else {
-          // batch > 1: a routed channel of unit u costs 1 + (tokens routed
-          // to u) (its fetch plus one dot per token), so CTA c takes the
-          // channels whose cost offset falls in [c C / G, (c + 1) C / G)
+          // batch > 1: a routed channel of unit u costs kJobW + (tokens
+          // routed to u), so CTA c takes the channels whose cost offset falls
+          // in [c C / G, (c + 1) C / G); the units' cost offsets rs.cpre were
+          // summed when the units were built
           const int U = rs.U;
-          long long C = 0;
-          for (int u = 0; u < U; ++u) C += (long long)I * (1 + __popc(rs.unit_mask[u]));
+          const long long C = rs.cpre[U];
           auto first_from = [&](long long x) -> int {  // first channel whose cost offset is >= x
-            long long acc = 0;
-            for (int u = 0; u < U; ++u) {
-              const long long wu = 1 + __popc(rs.unit_mask[u]), cu = (long long)I * wu;
-              if (x < acc + cu) return u * I + (int)((x - acc + wu - 1) / wu);
-              acc += cu;
+            if (x >= C) return U * I;
+            int lo = 0, hi = U - 1;  // the last unit whose offset is <= x
+            while (lo < hi) {
+              const int mid = (lo + hi + 1) >> 1;
+              if (rs.cpre[mid] <= x) lo = mid;
+              else hi = mid - 1;
             }
-            return U * I;
+            const long long wu = kJobW + __popc(rs.unit_mask[lo]);
+            return lo * I + (int)((x - rs.cpre[lo] + wu - 1) / wu);
           };
           const unsigned long long Gu = (unsigned long long)G;
           cur.t = first_from((long long)((unsigned long long)cta * (unsigned long long)C / Gu));
@@ -1292,8 +1310,8 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
             const size_t off = (size_t)j.c0 * rowb;
             mbar_expect_tx(bar, 3 * bytes);
             bulk_g2s(dst, Lw.sh_gate + off, bytes, bar, pol);
-            bulk_g2s(dst + NCH * rowb, Lw.sh_up + off, bytes, bar, pol);
-            bulk_g2s(dst + 2 * NCH * rowb, Lw.sh_down + off, bytes, bar, pol);
+            bulk_g2s(dst + kShN * rowb, Lw.sh_up + off, bytes, bar, pol);
+            bulk_g2s(dst + 2 * kShN * rowb, Lw.sh_down + off, bytes, bar, pol);
           } else if (LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR) {
             // one copy per run of consecutive kept channels (12 KB each)
             const uint32_t cb = 3u * (uint32_t)rowb;
@@ -1354,13 +1372,16 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
     const unsigned long long bar_base = bar_base_s;
     unsigned long long nbar = 0;
 
-    float acc[BMAX][8];
+    // token b's partial output, elements 8 tid + 2 i and 8 tid + 2 i + 1 in
+    // acc[b][i] (fp32 pairs: one packed FMA updates both)
+    float2 acc[BMAX][4];
 #pragma unroll
     for (int b = 0; b < BMAX; ++b)
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[b][i] = 0.f;
+      for (int i = 0; i < 4; ++i) acc[b][i] = make_float2(0.f, 0.f);
     const int H8c = H8;
     const bool has_v = tid < H8;
+    int tcn = 0;  // int4 batch path: routed jobs consumed (tcpart buffer tcn % 2)
     const uint32_t all_tokens = (1u << B) - 1u;
     // tensor-core dots (B = 1, H = 2048): x fragments for the 8 segments
     constexpr bool kMmaDots = (BMAX == 1 && HV == 8);
@@ -1557,9 +1578,197 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
         }
       }
       const uint32_t mask_any = mask0 | mask1;
+      if constexpr (kTcB) {
+        if (j.type == JOB_SHARED || j.type == JOB_ROUTER) {
+          // bf16 rows n at st + n rowb with all tokens: one shared channel
+          // (gate n = 0, up n = 1) or the job's router rows; the same
+          // tensor-core split of H over the warps (no scales: the pairs
+          // {8 w + i, 8 w + i + 4} of the rows themselves)
+          const int tb = tcn & 1;
+          ++tcn;
+          const int nrows = j.type == JOB_SHARED ? 2 : j.n;
+          if (ok) {
+            const int n = lane >> 2, q = lane & 3;
+            const uint4* wr = reinterpret_cast<const uint4*>(st + (size_t)(n < nrows ? n : 0) * rowb) + 2 * q;
+            const uint4* xm = us4 + (size_t)(lane >> 2) * H8c + 2 * q;
+            const bool xin = (lane >> 2) < B, wact = n < nrows;
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int g = 0; g < 4; ++g)
+#pragma unroll
+              for (int s2 = 0; s2 < 2; ++s2) {
+                const int w8 = 8 * (4 * warp + g) + s2;
+                const uint4 v = xin ? xm[w8] : make_uint4(0u, 0u, 0u, 0u);
+                const uint4 wv = wact ? wr[w8] : make_uint4(0u, 0u, 0u, 0u);
+                mma_bf16_16816(d, __byte_perm(v.x, v.z, 0x5410), 0u, __byte_perm(v.x, v.z, 0x7632), 0u,
+                               __byte_perm(wv.x, wv.z, 0x5410), __byte_perm(wv.x, wv.z, 0x7632));
+                mma_bf16_16816(d, __byte_perm(v.y, v.w, 0x5410), 0u, __byte_perm(v.y, v.w, 0x7632), 0u,
+                               __byte_perm(wv.y, wv.w, 0x5410), __byte_perm(wv.y, wv.w, 0x7632));
+              }
+            tcpart[tb][warp][q * 8 + (lane >> 2)] = make_float2(d[0], d[1]);
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&hready[slot]);
+          ok = ok && wait_mb(&hready[slot], ph);
+          if (ok && j.type == JOB_ROUTER) {
+            // warp 0: lane (q = lane / 8, token m = lane % 8) sums rows 2 q
+            // and 2 q + 1 over the warps into the logits
+            if (warp == 0) {
+              float2 v2 = tcpart[tb][0][lane];
+#pragma unroll
+              for (int w = 1; w < kWarps; ++w) {
+                const float2 v = tcpart[tb][w][lane];
+                v2.x += v.x;
+                v2.y += v.y;
+              }
+              const int q = lane >> 3, m = lane & 7;
+              if (m < B) {
+                if (2 * q < j.n) p.logits[(size_t)m * E + j.c0 + 2 * q] = v2.x;
+                if (2 * q + 1 < j.n) p.logits[(size_t)m * E + j.c0 + 2 * q + 1] = v2.y;
+              }
+            }
+          } else if (ok) {
+            if (lane < 8) {
+              float2 gu = tcpart[tb][0][lane];
+#pragma unroll
+              for (int w = 1; w < kWarps; ++w) {
+                const float2 v = tcpart[tb][w][lane];
+                gu.x += v.x;
+                gu.y += v.y;
+              }
+              const float h = lane < B ? silu_f(gu.x) * gu.y : 0.f;
+              hb2[warp][lane] = make_float2(h, h);
+            }
+            __syncwarp();
+            float dv[8];
+            unpack8(reinterpret_cast<const uint4*>(st + 2 * kShN * rowb)[tid], dv);
+            float4* ysb = reinterpret_cast<float4*>(smem + p.off_ysum);
+            for (int b2 = 0; b2 < B; ++b2) {
+              float4* ya = ysb + b2 * (H >> 2) + tid;
+              const float4 y0 = ya[0], y1 = ya[H >> 3];
+              const float2 hh = hb2[warp][b2];
+              const float2 a0 = __ffma2_rn(make_float2(dv[0], dv[1]), hh, make_float2(y0.x, y0.y));
+              const float2 a1 = __ffma2_rn(make_float2(dv[2], dv[3]), hh, make_float2(y0.z, y0.w));
+              const float2 a2 = __ffma2_rn(make_float2(dv[4], dv[5]), hh, make_float2(y1.x, y1.y));
+              const float2 a3 = __ffma2_rn(make_float2(dv[6], dv[7]), hh, make_float2(y1.z, y1.w));
+              ya[0] = make_float4(a0.x, a0.y, a1.x, a1.y);
+              ya[H >> 3] = make_float4(a2.x, a2.y, a3.x, a3.y);
+            }
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&empty[slot]);
+          if (++cslot == p.nstages) { cslot = 0; cph ^= 1u; }
+          ++jc;
+          if (!ok) *(volatile int*)&abort_s = 1;
+          return ok;
+        }
+        if (j.type == JOB_ROUTED) {
+          // 1. warp w: elements 256 w .. 256 w + 255 of the job's 8 rows (row
+          // n = 2 ch + mat) for all 8 tokens. mma D[m][n] (m: token, n: row)
+          // per 64-element group, scaled by the group's scale of row n: lane
+          // (m, q) ends with token m's gate and up partials of channel q.
+          const int tb = tcn & 1;
+          ++tcn;
+          if (ok) {
+            const int n = lane >> 2, q = lane & 3;
+            const uint8_t* wrow = st + (n >> 1) * (H >> 1) + (n & 1) * (NCH * (H >> 1));
+            const uint16_t* sgp = reinterpret_cast<const uint16_t*>(st + 3 * NCH * (H >> 1)) + q * (H >> 6);
+            const uint16_t* sup = sgp + NCH * (H >> 6);
+            // A fragments: token m's elements 8 w + i and 8 w + i + 4 of its
+            // words w = 8 G + 2 q + s, the pairs int4_pair_bf16 makes of the
+            // codes (rows m >= B are zero)
+            const uint4* xm = us4 + (size_t)(lane >> 2) * H8c + 2 * q;
+            const bool xin = (lane >> 2) < B;
+            // one accumulator per group: four independent mma chains
+            float d[4][4];
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              const int G = 4 * warp + g;
+              const uint2 wv = *reinterpret_cast<const uint2*>(wrow + 4 * (8 * G + 2 * q));
+#pragma unroll
+              for (int i = 0; i < 4; ++i) d[g][i] = 0.f;
+#pragma unroll
+              for (int s2 = 0; s2 < 2; ++s2) {
+                const uint32_t w = s2 ? wv.y : wv.x;
+                const uint4 v = xin ? xm[8 * G + s2] : make_uint4(0u, 0u, 0u, 0u);
+                mma_bf16_16816(d[g], __byte_perm(v.x, v.z, 0x5410), 0u, __byte_perm(v.x, v.z, 0x7632), 0u,
+                               int4_pair_bf16(w, 0), int4_pair_bf16(w, 1));
+                mma_bf16_16816(d[g], __byte_perm(v.y, v.w, 0x5410), 0u, __byte_perm(v.y, v.w, 0x7632), 0u,
+                               int4_pair_bf16(w, 2), int4_pair_bf16(w, 3));
+              }
+            }
+            float pg = 0.f, pu = 0.f;
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              pg = fmaf(bf16_to_f(sgp[4 * warp + g]), d[g][0], pg);
+              pu = fmaf(bf16_to_f(sup[4 * warp + g]), d[g][1], pu);
+            }
+            tcpart[tb][warp][q * 8 + n] = make_float2(pg, pu);
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&hready[slot]);
+          // 2. the job's down rows, scaled, while the other warps finish their
+          // dots (codes of channels c >= j.n are stale but finite, and their
+          // h is 0); then every warp: the 32 activations (lane = 8 ch + b)
+          // from the 8 warps' partials, and thread tid's 8 outputs of each
+          // routed token: elements 8 tid .. 8 tid + 3 at float4 slot tid of
+          // the token's first half, 8 tid + 4 .. 8 tid + 7 in its second
+          float2 q2[NCH][4];
+          if (ok) {
+            float sv[8];
+            unpack8(reinterpret_cast<const uint4*>(st + 3 * NCH * (H >> 1) + 2 * NCH * (H >> 5))[tid], sv);
+#pragma unroll
+            for (int c2 = 0; c2 < NCH; ++c2) {
+              float qv[8];
+              int4x8_to_f(reinterpret_cast<const uint32_t*>(st + 2 * NCH * (H >> 1) + c2 * (H >> 1))[tid], qv);
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                q2[c2][i] = __fmul2_rn(make_float2(qv[2 * i], qv[2 * i + 1]), make_float2(sv[2 * i], sv[2 * i + 1]));
+            }
+          }
+          ok = ok && wait_mb(&hready[slot], ph);
+          if (ok) {
+            float2 gu = tcpart[tb][0][lane];
+#pragma unroll
+            for (int w = 1; w < kWarps; ++w) {
+              const float2 v = tcpart[tb][w][lane];
+              gu.x += v.x;
+              gu.y += v.y;
+            }
+            const int ch = lane >> 3, b = lane & 7;
+            float h = 0.f;
+            if (ch < j.n && ((mask0 >> b) & 1u)) h = wts0[b] * silu_f(gu.x) * gu.y;
+            hb2[warp][lane] = make_float2(h, h);
+            __syncwarp();
+            float4* ysb = reinterpret_cast<float4*>(smem + p.off_ysum);
+            for (uint32_t mm = mask0; mm != 0u; mm &= mm - 1u) {
+              const int b2 = __ffs(mm) - 1;
+              float4* ya = ysb + b2 * (H >> 2) + tid;
+              const float4 y0 = ya[0], y1 = ya[H >> 3];
+              float2 a[4] = {make_float2(y0.x, y0.y), make_float2(y0.z, y0.w), make_float2(y1.x, y1.y),
+                             make_float2(y1.z, y1.w)};
+#pragma unroll
+              for (int c2 = 0; c2 < NCH; ++c2) {
+                const float2 hh = hb2[warp][8 * c2 + b2];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) a[i] = __ffma2_rn(q2[c2][i], hh, a[i]);
+              }
+              ya[0] = make_float4(a[0].x, a[0].y, a[1].x, a[1].y);
+              ya[H >> 3] = make_float4(a[2].x, a[2].y, a[3].x, a[3].y);
+            }
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&empty[slot]);
+          if (++cslot == p.nstages) { cslot = 0; cph ^= 1u; }
+          ++jc;
+          if (!ok) *(volatile int*)&abort_s = 1;
+          return ok;
+        }
+      }
       int ch_stride, mat_stride, down_off;
       if (j.type == JOB_ROUTER) { ch_stride = rowb; mat_stride = 0; down_off = 0; }
-      else if (j.type == JOB_SHARED || (LAYOUT == MOE_LAYOUT_PLANAR && WT == MOE_W_BF16)) {
+      else if (j.type == JOB_SHARED) { ch_stride = rowb; mat_stride = kShN * rowb; down_off = 2 * kShN * rowb; }
+      else if (LAYOUT == MOE_LAYOUT_PLANAR && WT == MOE_W_BF16) {
         ch_stride = rowb; mat_stride = NCH * rowb; down_off = 2 * NCH * rowb;
       } else if (LAYOUT == MOE_LAYOUT_CHANNEL_MAJOR) {
         ch_stride = 3 * rowb; mat_stride = rowb; down_off = 2 * rowb;
@@ -1619,7 +1828,8 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
             hbuf[warp][idx] = h;
           }
           __syncwarp();
-          if (has_v) {
+          // (the int4 batch path handles its shared and routed jobs above)
+          if (!kTcB && has_v) {
             if (!int4_rows) {
 #pragma unroll
               for (int ch = 0; ch < NCH; ++ch)
@@ -1631,8 +1841,9 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
                   for (int b = 0; b < BMAX; ++b)
                     if ((m >> b) & 1u) {
                       const float h = hbuf[warp][ch * BMAX + b];
+                      const float2 hh = make_float2(h, h);
 #pragma unroll
-                      for (int i = 0; i < 8; ++i) acc[b][i] = fmaf(h, d[i], acc[b][i]);
+                      for (int i = 0; i < 4; ++i) acc[b][i] = __ffma2_rn(make_float2(d[2 * i], d[2 * i + 1]), hh, acc[b][i]);
                     }
                 }
             } else {
@@ -1652,8 +1863,9 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
                   for (int b = 0; b < BMAX; ++b)
                     if ((mask0 >> b) & 1u) {
                       const float h = hbuf[warp][ch * BMAX + b];
+                      const float2 hh = make_float2(h, h);
 #pragma unroll
-                      for (int i = 0; i < 8; ++i) acc[b][i] = fmaf(h, q[i], acc[b][i]);
+                      for (int i = 0; i < 4; ++i) acc[b][i] = __ffma2_rn(make_float2(q[2 * i], q[2 * i + 1]), hh, acc[b][i]);
                     }
                 }
             }
@@ -1968,6 +2180,33 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
         else rs.unit_w[u][b] = rs.w[b][t % k];
       }
       cbar();
+      // cost offsets of the units (lane l: units 8 l .. 8 l + 7), for the
+      // split of the routed channels over the CTAs
+      if (warp == 0) {
+        const int U = rs.U;
+        int c[8], tot = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int u = 8 * lane + i;
+          c[i] = u < U ? I * (kJobW + __popc(rs.unit_mask[u])) : 0;
+          tot += c[i];
+        }
+        int inc = tot;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int t = __shfl_up_sync(0xffffffffu, inc, o);
+          if (lane >= o) inc += t;
+        }
+        int base = inc - tot;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int u = 8 * lane + i;
+          if (u <= U) rs.cpre[u] = base;
+          base += c[i];
+        }
+        if (lane == 31) rs.cpre[U] = inc;
+      }
+      cbar();
       return bad_s == 0;
       }
     };
@@ -2145,6 +2384,54 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
       return true;
     };
 
+    // Batch > 1 with E <= 256: warp b ranks token b straight from the
+    // workspace logits. Slot s of lane l holds expert 64 (s / 2) + 2 l + s % 2;
+    // each lane sorts its 8 slots best first as key << 32 | ~expert (larger
+    // logit, then lower index) and each of the k rounds takes the best head
+    // over the warp (as in route_warp).
+    auto route_tokens_warp = [&]() {
+      if (warp < B) {
+        const float* lt = p.logits + (size_t)warp * E;
+        unsigned long long v[8];
+#pragma unroll
+        for (int s2 = 0; s2 < 8; ++s2) {
+          const int e = 64 * (s2 >> 1) + 2 * lane + (s2 & 1);
+          v[s2] = e < E ? (((unsigned long long)float_key(__ldcg(lt + e)) << 32) | (unsigned long long)(~(uint32_t)e))
+                        : 0ull;
+        }
+        auto cas = [&](int i, int j2) {
+          const unsigned long long a = v[i], b = v[j2];
+          v[i] = a < b ? b : a;
+          v[j2] = a < b ? a : b;
+        };
+        cas(0, 1); cas(2, 3); cas(4, 5); cas(6, 7);
+        cas(0, 2); cas(1, 3); cas(4, 6); cas(5, 7);
+        cas(1, 2); cas(5, 6);
+        cas(0, 4); cas(1, 5); cas(2, 6); cas(3, 7);
+        cas(2, 4); cas(3, 5);
+        cas(1, 2); cas(3, 4); cas(5, 6);
+        for (int r = 0; r < k; ++r) {
+          const uint32_t hk = (uint32_t)(v[0] >> 32);
+          const uint32_t M = __reduce_max_sync(0xffffffffu, hk);
+          uint32_t tie = __ballot_sync(0xffffffffu, hk == M);
+          if (tie & (tie - 1)) {
+            const uint32_t lo = __reduce_max_sync(0xffffffffu, hk == M ? (uint32_t)v[0] : 0u);
+            tie = __ballot_sync(0xffffffffu, hk == M && (uint32_t)v[0] == lo);
+          }
+          const bool win = lane == __ffs(tie) - 1;
+          if (win) {
+            rs.ids[warp][r] = (int)~(uint32_t)v[0];
+            sel_l[warp][r] = key_float(M);
+          }
+#pragma unroll
+          for (int s2 = 0; s2 < 7; ++s2) v[s2] = win ? v[s2 + 1] : v[s2];
+          v[7] = win ? 0ull : v[7];
+        }
+        __syncwarp();
+        warp_weights(sel_l[warp], k, rs.w[warp]);
+      }
+      cbar();
+    };
     auto route = [&]() {
       if constexpr (BMAX == 1) {
         // two levels: each warp takes the best k of its 1/8 of the experts,
@@ -2444,10 +2731,14 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
             if (tid == 0) okw_s = wait_grid(target) ? 1 : 0;
             cbar();
             if (!okw_s) { if (tid == 0) set_status(ctl, kStatusTimeout); return false; }
-            for (int i = tid; i < B * E; i += kConsumers) lg[i] = __ldcg(p.logits + i);
-            cbar();
-            if (BMAX == 1 && k <= kWarps) { route_b1_small_k(0, l); units_done = true; }
-            else route();
+            if (BMAX > 1 && E <= 256 && k <= 32) {
+              route_tokens_warp();
+            } else {
+              for (int i = tid; i < B * E; i += kConsumers) lg[i] = __ldcg(p.logits + i);
+              cbar();
+              if (BMAX == 1 && k <= kWarps) { route_b1_small_k(0, l); units_done = true; }
+              else route();
+            }
           }
           if (cta == 0 && p.ids_out != nullptr)
             for (int t = tid; t < B * k; t += kConsumers) {
@@ -2521,11 +2812,29 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
         }
         failed = fl;
       } else {
+      // (int4 batch path: once next_job has set this layer's routed range, the
+      // rest of its jobs come straight from the cursor, in next_job's order)
+      int ft = 0, ft1 = 0, fc = 0, fu = 0;
       for (;;) {
-        const JobCursor save = ccur;
-        const bool got = next_job(ccur, j, ready);
-        const bool in_layer = got && j.type != JOB_END && j.layer == l;
-        if (in_layer && j.type == phase) {
+        bool take;
+        JobCursor save;
+        if (kTcB && ft < ft1) {
+          const int n = min(min(NCH - (fc & (NCH - 1)), I - fc), ft1 - ft);
+          j = Job{JOB_ROUTED, l, fu, fc, n};
+          ft += n;
+          fc += n;
+          if (fc >= I) { fc -= I; ++fu; }
+          take = true;
+        } else {
+          save = ccur;
+          const bool got = next_job(ccur, j, ready);
+          take = got && j.type != JOB_END && j.layer == l && j.type == phase;
+          if (kTcB && take && j.type == JOB_ROUTED) {
+            ft = ccur.t; ft1 = ccur.t1; fc = ccur.c; fu = ccur.u;
+            ccur.t = ccur.t1;  // the cursor moves on to the end of the layer
+          }
+        }
+        if (take) {
           if (!consume(j)) { failed = true; break; }
           continue;
         }
@@ -2569,15 +2878,26 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
         float* dst = yacc + 8 * tid;
         red_add_v4(dst, v[0], v[1], v[2], v[3]);
         red_add_v4(dst + 4, v[4], v[5], v[6], v[7]);
+      } else if constexpr (kTcB) {
+        float4* ysb = reinterpret_cast<float4*>(smem + p.off_ysum);
+        for (int b = 0; b < B; ++b) {
+          float4* ya = ysb + b * (H >> 2) + tid;
+          const float4 y0 = ya[0], y1 = ya[H >> 3];
+          float* dst = yacc + (size_t)b * H + 8 * tid;
+          red_add_v4(dst, y0.x, y0.y, y0.z, y0.w);
+          red_add_v4(dst + 4, y1.x, y1.y, y1.z, y1.w);
+          ya[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+          ya[H >> 3] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
       } else if (has_v) {
 #pragma unroll
         for (int b = 0; b < BMAX; ++b)
           if (b < B) {
             float* dst = yacc + (size_t)b * H + 8 * tid;
-            red_add_v4(dst, acc[b][0], acc[b][1], acc[b][2], acc[b][3]);
-            red_add_v4(dst + 4, acc[b][4], acc[b][5], acc[b][6], acc[b][7]);
+            red_add_v4(dst, acc[b][0].x, acc[b][0].y, acc[b][1].x, acc[b][1].y);
+            red_add_v4(dst + 4, acc[b][2].x, acc[b][2].y, acc[b][3].x, acc[b][3].y);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) acc[b][i] = 0.f;
+            for (int i = 0; i < 4; ++i) acc[b][i] = make_float2(0.f, 0.f);
           }
       }
       if (!grid_sync()) { failed = true; if (tid == 0) set_status(ctl, kStatusTimeout); break; }
@@ -2617,8 +2937,21 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
         }
         fast_frags(xv, p.pre_norm != 0);
       } else if constexpr (MODE == MODE_LAYERS) {
-        for (long long i = tid; i < n4; i += kConsumers) {
-          const float4 y4 = __ldcg(reinterpret_cast<const float4*>(yacc) + i);
+        // accumulator loads in flight per thread, then their updates (4 on
+        // the int4 batch path, whose sums left the registers free)
+        constexpr int kEpU = kTcB ? 4 : 1;
+        for (long long i0 = tid; i0 < n4; i0 += kEpU * kConsumers) {
+          float4 yv4[kEpU];
+#pragma unroll
+          for (int u = 0; u < kEpU; ++u) {
+            const long long i = i0 + (long long)u * kConsumers;
+            if (i < n4) yv4[u] = __ldcg(reinterpret_cast<const float4*>(yacc) + i);
+          }
+#pragma unroll
+          for (int u = 0; u < kEpU; ++u) {
+          const long long i = i0 + (long long)u * kConsumers;
+          if (i >= n4) break;
+          const float4 y4 = yv4[u];
           uint2 xv = reinterpret_cast<uint2*>(xs)[i];
           const float x0 = bf16_lo(xv.x) + y4.x, x1 = bf16_hi(xv.x) + y4.y;
           const float x2 = bf16_lo(xv.y) + y4.z, x3 = bf16_hi(xv.y) + y4.w;
@@ -2630,6 +2963,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
             if (yo) reinterpret_cast<float4*>(yo)[i] = y4;
             if (p.x_hist) reinterpret_cast<uint2*>(p.x_hist + (size_t)(l + 1) * B * H)[i] = xv;
             if (l == p.L - 1 && p.x_out) reinterpret_cast<uint2*>(p.x_out)[i] = xv;
+          }
           }
         }
         cbar();

@@ -139,6 +139,31 @@ def test_int4_expert_forward_ragged(M, S):
         assert rel_err(f64(y[b]), yo) <= REL_TOL
 
 
+@pytest.mark.parametrize("B", [2, 5, 8])
+def test_int4_expert_forward_a3b_batches(M, S, a3b_int4, B):
+    # routing given at A3B shapes (H = 2048, I = 768): the tensor-core dots of
+    # the batch path, with fewer than 8 tokens (unused token rows) and tokens
+    # that share experts (ids drawn from 12 of the 128 experts)
+    w, layers = a3b_int4
+    H, E, I, k = w["H"], w["E"], w["I"], w["k"]
+    L = layers[1]
+    desc = int4_desc(M, L, H, E, I, k, router=False)
+    g = torch.Generator().manual_seed(90 + B)
+    pool = torch.randperm(E, generator=g)[:12]
+    ids = torch.stack([pool[torch.randperm(12, generator=g)[:k]] for _ in range(B)]).to(torch.int32).to(DEV)
+    wt = torch.rand((B, k), generator=g).to(DEV)
+    x = S.tokens(B, H, seed=91 + B, device=DEV)
+    ws = M.alloc_workspace(desc, B)
+    y = torch.empty((B, H), dtype=torch.float32, device=DEV)
+    M.moe_expert_forward(desc, x, ids, wt, y, ws)
+    torch.cuda.synchronize()
+    assert M.moe_get_status(ws) == M.MOE_OK
+    HL = HostInt4(L)
+    for b in range(B):
+        yo = O.moe_experts_given(f64(x[b]), HL.expert, ids[b].tolist(), f64(wt[b]))
+        assert rel_err(f64(y[b]), yo) <= REL_TOL, b
+
+
 # ------------------------------------------------------------ channel-sparse
 
 
