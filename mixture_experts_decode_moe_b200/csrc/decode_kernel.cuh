@@ -2077,18 +2077,20 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
     };
 
     // ---- pre-norm: us[b] = bf16(x[b] / sqrt(mean(x[b]^2) + eps)), unit weight
+    // (x is read twice from shared memory, once for the sums of squares and
+    // once to scale, so that no token's values stay live in registers)
     auto normalize_x = [&]() {
       float ss[BMAX];
 #pragma unroll
-      for (int b = 0; b < BMAX; ++b) ss[b] = 0.f;
-      float xv[BMAX][8];
-#pragma unroll
-      for (int b = 0; b < BMAX; ++b)
+      for (int b = 0; b < BMAX; ++b) {
+        ss[b] = 0.f;
         if (b < B && has_v) {
-          unpack8(xs4[b * H8c + tid], xv[b]);
+          float xv[8];
+          unpack8(xs4[b * H8c + tid], xv);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) ss[b] = fmaf(xv[b][i], xv[b][i], ss[b]);
+          for (int i = 0; i < 8; ++i) ss[b] = fmaf(xv[i], xv[i], ss[b]);
         }
+      }
 #pragma unroll
       for (int b = 0; b < BMAX; ++b) {
         const float t = warp_sum(ss[b]);
@@ -2102,11 +2104,13 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
 #pragma unroll
           for (int w = 0; w < kWarps; ++w) t += hbuf[w][b];
           const float sc = rsqrtf(t / (float)H + 1e-6f);
+          float xv[8];
+          unpack8(xs4[b * H8c + tid], xv);
           uint4 o;
-          o.x = uint32_t(f_to_bf16(xv[b][0] * sc)) | (uint32_t(f_to_bf16(xv[b][1] * sc)) << 16);
-          o.y = uint32_t(f_to_bf16(xv[b][2] * sc)) | (uint32_t(f_to_bf16(xv[b][3] * sc)) << 16);
-          o.z = uint32_t(f_to_bf16(xv[b][4] * sc)) | (uint32_t(f_to_bf16(xv[b][5] * sc)) << 16);
-          o.w = uint32_t(f_to_bf16(xv[b][6] * sc)) | (uint32_t(f_to_bf16(xv[b][7] * sc)) << 16);
+          o.x = uint32_t(f_to_bf16(xv[0] * sc)) | (uint32_t(f_to_bf16(xv[1] * sc)) << 16);
+          o.y = uint32_t(f_to_bf16(xv[2] * sc)) | (uint32_t(f_to_bf16(xv[3] * sc)) << 16);
+          o.z = uint32_t(f_to_bf16(xv[4] * sc)) | (uint32_t(f_to_bf16(xv[5] * sc)) << 16);
+          o.w = uint32_t(f_to_bf16(xv[6] * sc)) | (uint32_t(f_to_bf16(xv[7] * sc)) << 16);
           reinterpret_cast<uint4*>(us)[b * H8c + tid] = o;
         }
       cbar();
@@ -2937,9 +2941,9 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
         }
         fast_frags(xv, p.pre_norm != 0);
       } else if constexpr (MODE == MODE_LAYERS) {
-        // accumulator loads in flight per thread, then their updates (4 on
+        // accumulator loads in flight per thread, then their updates (8 on
         // the int4 batch path, whose sums left the registers free)
-        constexpr int kEpU = kTcB ? 4 : 1;
+        constexpr int kEpU = kTcB ? 8 : 1;
         for (long long i0 = tid; i0 < n4; i0 += kEpU * kConsumers) {
           float4 yv4[kEpU];
 #pragma unroll
