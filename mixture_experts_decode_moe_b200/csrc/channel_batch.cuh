@@ -69,7 +69,6 @@ struct ChanBatchParams {
 __global__ void __launch_bounds__(kCbThreads, 1) channel_batch_kernel(const __grid_constant__ ChanBatchParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ uint64_t full[kCbStages], empty[kCbStages];
-  __shared__ int unit_e[kCbMaxUnits];
   __shared__ short unit_of_e[kMaxE];
   __shared__ float wt[kCbMaxUnits][kMaxB];
   __shared__ int tu_e[kMaxK];               // phase A: token's experts, ascending
@@ -255,7 +254,6 @@ __global__ void __launch_bounds__(kCbThreads, 1) channel_batch_kernel(const __gr
         int rk = base + inc - cnt;
         for (uint32_t m = bits; m; m &= m - 1) {
           const int e = wi * 32 + __ffs(m) - 1;
-          unit_e[rk] = e;
           unit_of_e[e] = (short)rk;
           ++rk;
         }

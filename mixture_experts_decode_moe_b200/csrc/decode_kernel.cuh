@@ -563,7 +563,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
   // batch > 1: cost of a routed channel in units of one token's work is
   // kJobW + (tokens routed to its expert): its fetch (and, on the int4 batch
   // path, its tensor-core dots for all tokens at once) plus the per-token work
-  constexpr int kJobW = kTcB ? 3 : 1;
+  constexpr int kJobW = kTcB ? 4 : 1;
   // channels per shared-expert job (bf16 rows): one on the int4 batch path,
   // whose ring stages are sized for int4 jobs
   constexpr int kShN = kTcB ? 1 : NCH;
