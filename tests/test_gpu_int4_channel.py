@@ -68,7 +68,7 @@ def a3b_int4(S):
     return w, layers
 
 
-@pytest.mark.parametrize("B", [1, 8])
+@pytest.mark.parametrize("B", [1, 3, 8])
 def test_int4_layer_a3b_shapes(M, S, a3b_int4, B):
     w, layers = a3b_int4
     H, E, I, k = w["H"], w["E"], w["I"], w["k"]
@@ -137,6 +137,33 @@ def test_int4_expert_forward_ragged(M, S):
     for b in range(B):
         yo = O.moe_experts_given(f64(x[b]), HL.expert, ids[b].tolist(), f64(wt[b]))
         assert rel_err(f64(y[b]), yo) <= REL_TOL
+
+
+def test_int4_layer_batched_tied_router_rows(M, S, a3b_int4):
+    # router rows in identical pairs at A3B shapes (the tensor-core router rows
+    # and the per-warp batch routing): the ids match the oracle exactly
+    w, layers = a3b_int4
+    H, E, I, k = w["H"], w["E"], w["I"], w["k"]
+    R = layers[0]["router"].clone()
+    R[1::2] = R[0::2]
+    L = dict(layers[0], router=R)
+    desc = int4_desc(M, L, H, E, I, k)
+    B = 5
+    x = S.tokens(B, H, seed=S.act_seed(4) + 9, device=DEV)
+    ws = M.alloc_workspace(desc, B)
+    y = torch.empty((B, H), dtype=torch.float32, device=DEV)
+    ids = torch.empty((B, k), dtype=torch.int32, device=DEV)
+    wt = torch.empty((B, k), dtype=torch.float32, device=DEV)
+    M.moe_layer_forward(desc, x, y, ws, ids_out=ids, w_out=wt)
+    torch.cuda.synchronize()
+    assert M.moe_get_status(ws) == M.MOE_OK
+    HL = HostInt4(L)
+    for b in range(B):
+        yo, io, wo, lo, _ = O.moe_layer(f64(x[b]), HL.R, HL.expert, k, shared=HL.shared)
+        got = ids[b].tolist()
+        assert got == [int(v) for v in io], b
+        assert all(got[2 * i] % 2 == 0 and got[2 * i + 1] == got[2 * i] + 1 for i in range(k // 2)), got
+        assert rel_err(f64(y[b]), yo) <= REL_TOL, b
 
 
 @pytest.mark.parametrize("B", [2, 5, 8])

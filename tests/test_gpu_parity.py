@@ -148,6 +148,34 @@ def test_layer_forward_tiny_batched(M, tiny, B):
             assert rel_err(f64(y[b]), yo) <= REL_TOL, (b0, b)
 
 
+def test_layer_forward_batched_tied_router_rows(M, S, tiny):
+    # router rows in identical pairs (2i, 2i + 1): every logit appears twice,
+    # bit-identical on both sides, so each chosen pair must come out lower
+    # index first, and the batch routing must match the oracle exactly
+    w, L, x = tiny
+    H, E, I, k = w["H"], w["E"], w["I"], w["k"]
+    R = L["router"].clone()
+    R[1::2] = R[0::2]
+    Lt = dict(L, router=R)
+    desc = planar_desc(M, Lt, H, E, I, k)
+    B = 3
+    ws = M.alloc_workspace(desc, B)
+    HL = HostLayer(Lt)
+    xb = x[:B].contiguous()
+    y = torch.empty((B, H), dtype=torch.float32, device=DEV)
+    ids = torch.empty((B, k), dtype=torch.int32, device=DEV)
+    wt = torch.empty((B, k), dtype=torch.float32, device=DEV)
+    M.moe_layer_forward(desc, xb, y, ws, ids_out=ids, w_out=wt)
+    torch.cuda.synchronize()
+    assert M.moe_get_status(ws) == M.MOE_OK
+    for b in range(B):
+        yo, io, wo, lo, _ = O.moe_layer(f64(xb[b]), HL.R, HL.expert, k)
+        assert ids[b].tolist() == [int(v) for v in io], b
+        assert ids[b, 0] % 2 == 0 and ids[b, 1] == ids[b, 0] + 1, b
+        assert np.allclose(f64(wt[b]), wo, rtol=1e-5)
+        assert rel_err(f64(y[b]), yo) <= REL_TOL, b
+
+
 def test_expert_forward_given_ids(M, S, tiny):
     w, L, x = tiny
     H, E, I, k = w["H"], w["E"], w["I"], w["k"]
