@@ -142,7 +142,8 @@ bool plan_smem(DecodeParams* p, int static_bytes, bool fast, bool tc_batch) {
   if (budget <= 0) return false;
   const bool cm = p->layout == MOE_LAYOUT_CHANNEL_MAJOR;
   const int x_bytes = (int)align_up((size_t)B * H * 2, 128);
-  const int u_bytes = p->pre_norm ? x_bytes : 0;
+  // u (pre-normed x); the int4 batch path keeps it as 8 token rows of A fragments
+  const int u_bytes = tc_batch ? (int)align_up((size_t)kMaxB * H * 2, 128) : (p->pre_norm ? x_bytes : 0);
   const int lg_bytes = (p->mode == MODE_LAYERS) ? (int)align_up((size_t)B * p->E * 4, 128) : 0;
   // keys: router top-k keys [B*E] and channel-sparse candidates [k*I]
   size_t nkeys = (p->mode == MODE_LAYERS) ? (size_t)B * p->E : 0;

@@ -603,7 +603,9 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
   uint16_t* xs = reinterpret_cast<uint16_t*>(smem + p.off_x);  // residual stream x
   const uint4* xs4 = reinterpret_cast<const uint4*>(xs);
   // MoE input u: RMS-normalised x with the pre-norm, else x itself
-  uint16_t* us = (MODE == MODE_LAYERS && p.pre_norm) ? reinterpret_cast<uint16_t*>(smem + p.off_u) : xs;
+  // u: the pre-normed x (or x itself); on the int4 batch path always its own
+  // buffer, holding u as a table of tensor-core A fragments (build_xfrags)
+  uint16_t* us = (kTcB || (MODE == MODE_LAYERS && p.pre_norm)) ? reinterpret_cast<uint16_t*>(smem + p.off_u) : xs;
   const uint4* us4 = reinterpret_cast<const uint4*>(us);
   float* lg = reinterpret_cast<float*>(smem + p.off_lg);
   uint32_t* keys = reinterpret_cast<uint32_t*>(smem + p.off_keys);
@@ -1590,20 +1592,18 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
           if (ok) {
             const int n = lane >> 2, q = lane & 3;
             const uint4* wr = reinterpret_cast<const uint4*>(st + (size_t)(n < nrows ? n : 0) * rowb) + 2 * q;
-            const uint4* xm = us4 + (size_t)(lane >> 2) * H8c + 2 * q;
-            const bool xin = (lane >> 2) < B, wact = n < nrows;
+            const uint4* xfr = us4 + 256 * warp + lane;  // this warp's A fragments
+            const bool wact = n < nrows;
             float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int g = 0; g < 4; ++g)
 #pragma unroll
               for (int s2 = 0; s2 < 2; ++s2) {
                 const int w8 = 8 * (4 * warp + g) + s2;
-                const uint4 v = xin ? xm[w8] : make_uint4(0u, 0u, 0u, 0u);
+                const uint4 v = xfr[64 * g + 32 * s2];
                 const uint4 wv = wact ? wr[w8] : make_uint4(0u, 0u, 0u, 0u);
-                mma_bf16_16816(d, __byte_perm(v.x, v.z, 0x5410), 0u, __byte_perm(v.x, v.z, 0x7632), 0u,
-                               __byte_perm(wv.x, wv.z, 0x5410), __byte_perm(wv.x, wv.z, 0x7632));
-                mma_bf16_16816(d, __byte_perm(v.y, v.w, 0x5410), 0u, __byte_perm(v.y, v.w, 0x7632), 0u,
-                               __byte_perm(wv.y, wv.w, 0x5410), __byte_perm(wv.y, wv.w, 0x7632));
+                mma_bf16_16816(d, v.x, 0u, v.y, 0u, __byte_perm(wv.x, wv.z, 0x5410), __byte_perm(wv.x, wv.z, 0x7632));
+                mma_bf16_16816(d, v.z, 0u, v.w, 0u, __byte_perm(wv.y, wv.w, 0x5410), __byte_perm(wv.y, wv.w, 0x7632));
               }
             tcpart[tb][warp][q * 8 + (lane >> 2)] = make_float2(d[0], d[1]);
           }
@@ -1674,11 +1674,10 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
             const uint8_t* wrow = st + (n >> 1) * (H >> 1) + (n & 1) * (NCH * (H >> 1));
             const uint16_t* sgp = reinterpret_cast<const uint16_t*>(st + 3 * NCH * (H >> 1)) + q * (H >> 6);
             const uint16_t* sup = sgp + NCH * (H >> 6);
-            // A fragments: token m's elements 8 w + i and 8 w + i + 4 of its
-            // words w = 8 G + 2 q + s, the pairs int4_pair_bf16 makes of the
-            // codes (rows m >= B are zero)
-            const uint4* xm = us4 + (size_t)(lane >> 2) * H8c + 2 * q;
-            const bool xin = (lane >> 2) < B;
+            // A fragments (build_xfrags): token m's elements 8 w + i and
+            // 8 w + i + 4 of its words w = 8 G + 2 q + s, the pairs
+            // int4_pair_bf16 makes of the codes (rows m >= B are zero)
+            const uint4* xfr = us4 + 256 * warp + lane;
             // one accumulator per group: four independent mma chains
             float d[4][4];
 #pragma unroll
@@ -1690,11 +1689,9 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
 #pragma unroll
               for (int s2 = 0; s2 < 2; ++s2) {
                 const uint32_t w = s2 ? wv.y : wv.x;
-                const uint4 v = xin ? xm[8 * G + s2] : make_uint4(0u, 0u, 0u, 0u);
-                mma_bf16_16816(d[g], __byte_perm(v.x, v.z, 0x5410), 0u, __byte_perm(v.x, v.z, 0x7632), 0u,
-                               int4_pair_bf16(w, 0), int4_pair_bf16(w, 1));
-                mma_bf16_16816(d[g], __byte_perm(v.y, v.w, 0x5410), 0u, __byte_perm(v.y, v.w, 0x7632), 0u,
-                               int4_pair_bf16(w, 2), int4_pair_bf16(w, 3));
+                const uint4 v = xfr[64 * g + 32 * s2];
+                mma_bf16_16816(d[g], v.x, 0u, v.y, 0u, int4_pair_bf16(w, 0), int4_pair_bf16(w, 1));
+                mma_bf16_16816(d[g], v.z, 0u, v.w, 0u, int4_pair_bf16(w, 2), int4_pair_bf16(w, 3));
               }
             }
             float pg = 0.f, pu = 0.f;
@@ -2115,7 +2112,60 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
         }
       cbar();
     };
-    if constexpr (MODE == MODE_LAYERS && !kFast)
+    // int4 batch path: u as the tensor-core A fragments, one uint4 per
+    // (warp w, group g, half s, lane) at entry 256 w + 64 g + 32 s + lane: for
+    // lane (m = lane / 4, q = lane % 4) the bf16 pairs {u[m][8 W + i],
+    // u[m][8 W + i + 4]}, i = 0..3, of word W = 8 (4 w + g) + 2 q + s, zero for
+    // m >= B; u = bf16(x * rsqrt(mean(x^2) + eps)) with the pre-norm, else x
+    __shared__ float xsc_s[kMaxB];
+    auto build_xfrags = [&](bool norm) {
+      if constexpr (kTcB) {
+        if (norm) {
+          float ss[BMAX];
+#pragma unroll
+          for (int b = 0; b < BMAX; ++b) {
+            ss[b] = 0.f;
+            if (b < B) {
+              float xv[8];
+              unpack8(xs4[b * H8c + tid], xv);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) ss[b] = fmaf(xv[i], xv[i], ss[b]);
+            }
+          }
+#pragma unroll
+          for (int b = 0; b < BMAX; ++b) {
+            const float t = warp_sum(ss[b]);
+            if (lane == 0) hbuf[warp][b] = t;
+          }
+          cbar();
+          if (tid < B) {
+            float t = 0.f;
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) t += hbuf[w][tid];
+            xsc_s[tid] = rsqrtf(t / (float)H + 1e-6f);
+          }
+          cbar();
+        }
+        uint4* xf4 = reinterpret_cast<uint4*>(us);
+        for (int e = tid; e < 8 * H8c; e += kConsumers) {
+          const int le = e & 31, m = le >> 2;
+          uint4 o = make_uint4(0u, 0u, 0u, 0u);
+          if (m < B) {
+            float xv[8];
+            unpack8(xs4[m * H8c + 8 * (e >> 6) + 2 * (le & 3) + ((e >> 5) & 1)], xv);
+            const float c = norm ? xsc_s[m] : 1.f;
+            uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              ow[i] = uint32_t(f_to_bf16(xv[i] * c)) | (uint32_t(f_to_bf16(xv[i + 4] * c)) << 16);
+          }
+          xf4[e] = o;
+        }
+        cbar();
+      }
+    };
+    if constexpr (kTcB) build_xfrags(MODE == MODE_LAYERS && p.pre_norm);
+    else if constexpr (MODE == MODE_LAYERS && !kFast)
       if (p.pre_norm) normalize_x();
     load_xfrag();
 
@@ -2971,7 +3021,8 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
           }
         }
         cbar();
-        if (p.pre_norm) normalize_x();
+        if constexpr (kTcB) build_xfrags(p.pre_norm != 0);
+        else if (p.pre_norm) normalize_x();
         load_xfrag();
       } else {
         for (long long i = s0 + tid; i < s1; i += kConsumers) {
