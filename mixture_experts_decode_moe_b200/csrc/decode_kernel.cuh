@@ -577,6 +577,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
   __shared__ RouteSmem<BMAX> rs;
   __shared__ int route_ready_s, prod_layer_s[kProducers], abort_s, bad_s, okw_s;
   __shared__ int units_s;  // planar batch 1: layer * 64 + units of its routing published so far
+  __shared__ int bar_l_s;  // last layer whose closing grid barrier the consumers passed
   __shared__ uint32_t ltag_s;  // logit tag of layer 0 in this launch (fast path)
   __shared__ unsigned long long bar_base_s;  // grid-barrier count at launch (a multiple of G)
   __shared__ long long budget_s;  // cycles per bounded wait (the workspace's budget)
@@ -624,6 +625,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
     fence_mbar_init();
     route_ready_s = -1;  // last layer whose routing the consumers published
     units_s = -1;
+    bar_l_s = -1;
     for (int q = 0; q < kProducers; ++q) {
       prod_layer_s[q] = -1;  // last layer whose routed jobs producer q issued
       jp_s[q] = 0;           // jobs producer q has passed (its own ones issued)
@@ -1123,6 +1125,24 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
           next_stage();
         }
       }
+      // the experts predicted for layer l (made in layer l - 1) into L2, once
+      // layer l - 1's closing grid barrier has passed: from then until layer
+      // l's routed copies start, HBM has nothing else to stream
+      if (p.npred > 0 && l > 0) {
+        int okb = 1;
+        if (lane == 0) {
+          const long long tb0 = clock64();
+          while (*(volatile int*)&bar_l_s < l - 1) {
+            if (*(volatile int*)&abort_s || clock64() - tb0 > budget) {
+              okb = 0;
+              break;
+            }
+            __nanosleep(32);
+          }
+        }
+        if (!__shfl_sync(0xffffffffu, okb, 0)) goto producer_done;
+        if (!predict_prefetch(l)) goto producer_done;
+      }
       if (!warp_routes) {
         // routing of layer l (plain polls with short sleeps, then one acquire)
         const long long t0 = clock64();
@@ -1236,12 +1256,6 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
         const uint8_t* sc1 = reinterpret_cast<const uint8_t*>(p.layer[l + 1].scores);
         if (b1 > b0 && ((uintptr_t)sc1 & 15u) == 0) prefetch_l2(sc1 + b0, (uint32_t)(b1 - b0));
       }
-      // every routed copy of layer l is issued: while the layer drains, and
-      // through the barrier, epilogue, router and top-k of layer l + 1 (when
-      // HBM would idle), prefetch this CTA's share of the experts layer
-      // l + 1 is predicted to route to into L2
-      if (p.npred > 0 && l + 1 < p.L)
-        if (!predict_prefetch(l + 1)) goto producer_done;
     }
     } else {
     // producer pi issues the jobs q with q % kProducers == pi; both walk the
@@ -2955,6 +2969,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
           }
       }
       if (!grid_sync()) { failed = true; if (tid == 0) set_status(ctl, kStatusTimeout); break; }
+      if (kFast && tid == 0) st_release_cta(&bar_l_s, l);
       // epilogue: y, residual, outputs (each CTA writes its slice)
       const long long n4 = n4s;
       const long long s0 = ys0, s1 = ys1;
