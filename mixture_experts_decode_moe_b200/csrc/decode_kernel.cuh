@@ -2969,7 +2969,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) decode_kernel(const __grid_con
           }
       }
       if (!grid_sync()) { failed = true; if (tid == 0) set_status(ctl, kStatusTimeout); break; }
-      if (kFast && tid == 0) st_release_cta(&bar_l_s, l);
+      if (kFast && p.npred > 0 && tid == 0) *(volatile int*)&bar_l_s = l;  // (for the expert prefetch)
       // epilogue: y, residual, outputs (each CTA writes its slice)
       const long long n4 = n4s;
       const long long s0 = ys0, s1 = ys1;
